@@ -1,0 +1,755 @@
+// api.cu - the C ABI of libdg.so: argument checks, TMA descriptor set-up,
+// launch planning (split-K, split-KV), the model forward, prefill, the
+// denoising loop and the block commit.  Built as one translation unit so that
+// the per-device error word is shared by every kernel.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/dg.h"
+#include "attn.cuh"
+#include "dg_common.cuh"
+#include "gemm.cuh"
+#include "kvcommit.cuh"
+#include "sampler.cuh"
+
+namespace {
+
+constexpr int kVersion = 1;
+constexpr int kNumSMs = 148;
+
+thread_local char g_last_error[512] = "";
+
+int fail(int status, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_last_error, sizeof(g_last_error), fmt, ap);
+  va_end(ap);
+  return status;
+}
+
+#define DG_CUDA(expr)                                                                     \
+  do {                                                                                    \
+    cudaError_t e_ = (expr);                                                              \
+    if (e_ != cudaSuccess)                                                                \
+      return fail(DG_ERR_CUDA, "%s failed: %s (%s:%d)", #expr, cudaGetErrorString(e_),    \
+                  __FILE__, __LINE__);                                                    \
+  } while (0)
+
+#define DG_TRY(expr)              \
+  do {                            \
+    int s_ = (expr);              \
+    if (s_ != DG_OK) return s_;   \
+  } while (0)
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+inline int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// ---------------------------------------------------------------------------
+// TMA descriptors (driver entry point fetched through the runtime)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D bf16 map over rows of `inner` elements, `row_stride` bytes apart; box
+// {64, box_rows} with 128-byte swizzle (one box row = one 128-byte line).
+int make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+              uint64_t row_stride_bytes, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  if (!aligned16(base) || (row_stride_bytes & 15u))
+    return fail(DG_ERR_ALIGNMENT, "tensor map base %p / stride %llu not 16-byte aligned", base,
+                (unsigned long long)row_stride_bytes);
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {64, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) inner=%llu rows=%llu", (int)r,
+                (unsigned long long)inner, (unsigned long long)rows);
+  return DG_OK;
+}
+
+// ---------------------------------------------------------------------------
+// GEMM
+// ---------------------------------------------------------------------------
+struct GemmPlan {
+  int splits, kb_per_split;
+};
+
+GemmPlan plan_gemm(int M, int N, int K) {
+  const int tiles = (N / dg::gemm::BM) * cdiv(M, dg::gemm::BN);
+  const int kb = K / dg::gemm::BK;
+  int s = std::max(1, kNumSMs / std::max(1, tiles));
+  s = std::min(s, std::max(1, kb / 4));
+  const int kbps = cdiv(kb, s);
+  return GemmPlan{cdiv(kb, kbps), kbps};
+}
+
+bool gemm_attr_done = false;
+
+int launch_gemm(const void* x, const void* w, int M, int N, int K, const GemmPlan& pl, int epi,
+                float* out_f32, __nv_bfloat16* out_bf16, cudaStream_t s) {
+  if (!gemm_attr_done) {
+    DG_CUDA(cudaFuncSetAttribute(dg::gemm::gemm_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dg::gemm::SMEM_BYTES));
+    gemm_attr_done = true;
+  }
+  CUtensorMap tw, tx;
+  DG_TRY(make_tmap(&tw, w, K, N, (uint64_t)K * 2, dg::gemm::BM));
+  DG_TRY(make_tmap(&tx, x, K, M, (uint64_t)K * 2, dg::gemm::BN));
+  dg::gemm::Params p{M, N, K, pl.kb_per_split, epi, out_f32, out_bf16};
+  dim3 grid(N / dg::gemm::BM, cdiv(M, dg::gemm::BN), pl.splits);
+  dg::gemm::gemm_kernel<<<grid, dg::gemm::THREADS, dg::gemm::SMEM_BYTES, s>>>(tw, tx, p);
+  DG_CUDA(cudaGetLastError());
+  return DG_OK;
+}
+
+int launch_reduce(const float* part, int S, int M, int N, int mode, __nv_bfloat16* out_bf16,
+                  float* out_f32, cudaStream_t s) {
+  const size_t n4 = (size_t)M * N / 4;
+  const int blocks = (int)std::min<size_t>(cdiv((int)std::min<size_t>(n4, 1u << 30), 256),
+                                           (size_t)kNumSMs * 8);
+  dg::gemm::reduce_kernel<<<std::max(1, blocks), 256, 0, s>>>(part, S, M, N, mode, out_bf16,
+                                                                out_f32);
+  DG_CUDA(cudaGetLastError());
+  return DG_OK;
+}
+
+// y = x w^T with the given final epilogue, using `part` for split partials.
+// mode: 0 bf16, 1 gelu bf16, 2 residual add fp32 (+ optional RMSNorm into xn).
+int linear(const void* x, const void* w, int M, int N, int K, int mode, void* out, float* part,
+           float eps, __nv_bfloat16* xn_out, cudaStream_t s) {
+  const GemmPlan pl = plan_gemm(M, N, K);
+  const bool norm = (mode == 2 && xn_out != nullptr);
+  if (pl.splits == 1 && !norm) {
+    const int epi = mode == 0 ? dg::gemm::EPI_BF16
+                  : mode == 1 ? dg::gemm::EPI_GELU_BF16
+                              : dg::gemm::EPI_ADD_F32;
+    return launch_gemm(x, w, M, N, K, pl, epi, (float*)out, (__nv_bfloat16*)out, s);
+  }
+  DG_TRY(launch_gemm(x, w, M, N, K, pl, dg::gemm::EPI_STORE_F32, part, nullptr, s));
+  if (norm) {
+    dg::gemm::add_norm_kernel<<<M, dg::gemm::NORM_THREADS, 0, s>>>(part, pl.splits, M, N, eps,
+                                                                    (float*)out, xn_out);
+    DG_CUDA(cudaGetLastError());
+    return DG_OK;
+  }
+  const int rmode = mode == 0 ? dg::gemm::RED_BF16
+                  : mode == 1 ? dg::gemm::RED_GELU_BF16
+                              : dg::gemm::RED_ADD_F32;
+  return launch_reduce(part, pl.splits, M, N, rmode, (__nv_bfloat16*)out, (float*)out, s);
+}
+
+size_t linear_part_bytes(int M, int N, int K) {
+  const GemmPlan pl = plan_gemm(M, N, K);
+  return (size_t)pl.splits * M * N * sizeof(float);
+}
+
+// ---------------------------------------------------------------------------
+// Attention
+// ---------------------------------------------------------------------------
+int attn_splits(int B, int Hq, int Lq, int max_prefix) {
+  const int qtiles = B * Hq * cdiv(Lq, dg::attn::BQ);
+  const int tmax = cdiv(max_prefix, dg::attn::BKV) + cdiv(Lq, dg::attn::BKV);
+  int s = std::max(1, kNumSMs / std::max(1, qtiles));
+  s = std::min(s, std::max(1, tmax / 2));
+  return s;
+}
+
+size_t attn_ws_bytes(int B, int Hq, int Lq, int hd, int max_prefix) {
+  const int S = attn_splits(B, Hq, Lq, max_prefix);
+  if (S == 1) return 0;
+  const size_t rows = (size_t)S * B * Hq * Lq;
+  return align_up(rows * hd * sizeof(float), 256) + align_up(rows * sizeof(float), 256);
+}
+
+bool attn_attr_done[2] = {false, false};
+
+int launch_attn(const void* q, int ldq, const void* k_new, const void* v_new, int ldkv,
+                const void* k_cache, const void* v_cache, const int32_t* cache_len,
+                int max_prefix, int lmax, void* out, int ldo, float* lse, int B, int Hq, int Hkv,
+                int Lq, int hd, float scale, int mask, void* ws, cudaStream_t s) {
+  const int S = attn_splits(B, Hq, Lq, max_prefix);
+  CUtensorMap tq, tkn, tvn, tkc, tvc;
+  DG_TRY(make_tmap(&tq, q, (uint64_t)Hq * hd, (uint64_t)B * Lq, (uint64_t)ldq * 2, 128));
+  DG_TRY(make_tmap(&tkn, k_new, (uint64_t)Hkv * hd, (uint64_t)B * Lq, (uint64_t)ldkv * 2, 128));
+  DG_TRY(make_tmap(&tvn, v_new, (uint64_t)Hkv * hd, (uint64_t)B * Lq, (uint64_t)ldkv * 2, 128));
+  DG_TRY(make_tmap(&tkc, k_cache, hd, (uint64_t)B * Hkv * lmax, (uint64_t)hd * 2, 128));
+  DG_TRY(make_tmap(&tvc, v_cache, hd, (uint64_t)B * Hkv * lmax, (uint64_t)hd * 2, 128));
+  dg::attn::Params p;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.lmax = lmax; p.group = Hq / Hkv;
+  p.n_qtiles = cdiv(Lq, dg::attn::BQ);
+  p.n_splits = S;
+  p.causal = mask == DG_MASK_CAUSAL ? 1 : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.cache_len = cache_len;
+  p.out = (__nv_bfloat16*)out;
+  p.ldo = ldo;
+  p.lse = lse;
+  p.part_o = nullptr;
+  p.part_lse = nullptr;
+  if (S > 1) {
+    const size_t rows = (size_t)S * B * Hq * Lq;
+    p.part_o = (float*)ws;
+    p.part_lse = (float*)((char*)ws + align_up(rows * hd * sizeof(float), 256));
+  }
+  dim3 grid(B * Hq * p.n_qtiles, S);
+  if (hd == 128) {
+    if (!attn_attr_done[1]) {
+      DG_CUDA(cudaFuncSetAttribute(dg::attn::attn_kernel<128>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   dg::attn::Cfg<128>::SMEM_BYTES));
+      attn_attr_done[1] = true;
+    }
+    dg::attn::attn_kernel<128><<<grid, dg::attn::THREADS, dg::attn::Cfg<128>::SMEM_BYTES, s>>>(
+        tq, tkn, tvn, tkc, tvc, p);
+  } else {
+    if (!attn_attr_done[0]) {
+      DG_CUDA(cudaFuncSetAttribute(dg::attn::attn_kernel<64>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   dg::attn::Cfg<64>::SMEM_BYTES));
+      attn_attr_done[0] = true;
+    }
+    dg::attn::attn_kernel<64><<<grid, dg::attn::THREADS, dg::attn::Cfg<64>::SMEM_BYTES, s>>>(
+        tq, tkn, tvn, tkc, tvc, p);
+  }
+  DG_CUDA(cudaGetLastError());
+  if (S > 1) {
+    const int rows = B * Hq * Lq;
+    const int threads = 256;
+    const int blocks = cdiv(rows * 32, threads);
+    if (hd == 128)
+      dg::attn::attn_combine_kernel<128><<<blocks, threads, 0, s>>>(
+          p.part_o, p.part_lse, S, B, Hq, Lq, (__nv_bfloat16*)out, ldo, lse);
+    else
+      dg::attn::attn_combine_kernel<64><<<blocks, threads, 0, s>>>(
+          p.part_o, p.part_lse, S, B, Hq, Lq, (__nv_bfloat16*)out, ldo, lse);
+    DG_CUDA(cudaGetLastError());
+  }
+  return DG_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Sampler
+// ---------------------------------------------------------------------------
+int sample_chunking(int V, int* chunk) {
+  // enough CTAs per row to stream the vocabulary with every SM busy, in
+  // multiples of 4 elements
+  int nchunk = std::max(1, std::min(64, V / 8192));
+  int c = cdiv(V, nchunk);
+  c = (c + 3) / 4 * 4;
+  nchunk = cdiv(V, c);
+  *chunk = c;
+  return nchunk;
+}
+
+size_t sample_ws_bytes(int B, int C, int V) {
+  int chunk;
+  const int nchunk = sample_chunking(V, &chunk);
+  return align_up((size_t)B * C * nchunk * sizeof(dg::RowPartial), 256);
+}
+
+dg::SampleParams make_sample_params(const dg_sampler_cfg& cfg, uint32_t seed, int block,
+                                    const int32_t* step_ptr, int step, int B, int C, int V) {
+  dg::SampleParams p;
+  p.B = B; p.C = C; p.V = V;
+  p.nchunk = sample_chunking(V, &p.chunk);
+  p.seed = seed;
+  p.block = block;
+  p.step_ptr = step_ptr;
+  p.step_val = step;
+  p.max_steps = cfg.max_steps;
+  p.t_start = cfg.t_start;
+  p.t_end = cfg.t_end;
+  p.commit_k = cfg.commit_k;
+  p.log_tau = cfg.renoise_conf > 0.f ? (float)std::log((double)cfg.renoise_conf) : -INFINITY;
+  p.stop_entropy = cfg.stop_entropy;
+  p.policy = cfg.unselected_policy;
+  return p;
+}
+
+int launch_sample(const float* logits, int32_t* tok, uint8_t* committed, int32_t* prev_argmax,
+                  int32_t* seq_status, const dg::SampleParams& p, const dg_step_out* out,
+                  void* ws, cudaStream_t s) {
+  dg::RowPartial* part = (dg::RowPartial*)ws;
+  dg::sample_rowpass_kernel<<<p.B * p.C * p.nchunk, dg::RP_THREADS, 0, s>>>(logits, seq_status,
+                                                                             p, part);
+  DG_CUDA(cudaGetLastError());
+  const int threads = (p.C + 31) / 32 * 32;
+  dg::sample_commit_kernel<<<p.B, threads, 0, s>>>(
+      logits, part, p, tok, committed, prev_argmax, seq_status, out ? out->x_hat : nullptr,
+      out ? out->argmax : nullptr, out ? out->logconf : nullptr, out ? out->entropy : nullptr,
+      out ? out->flags : nullptr);
+  DG_CUDA(cudaGetLastError());
+  return DG_OK;
+}
+
+// ---------------------------------------------------------------------------
+// KV commit
+// ---------------------------------------------------------------------------
+int launch_kv_commit(const void* const* k_blk, const void* const* v_blk, int ld_blk,
+                     void* const* k_cache, void* const* v_cache, const int32_t* cache_len,
+                     int n_layers, int B, int Hkv, int C, int hd, int lmax, cudaStream_t s) {
+  dg::KVTables tab;
+  memset(&tab, 0, sizeof(tab));
+  for (int l = 0; l < n_layers; ++l) {
+    tab.k_blk[l] = (const __nv_bfloat16*)k_blk[l];
+    tab.v_blk[l] = (const __nv_bfloat16*)v_blk[l];
+    tab.k_cache[l] = (__nv_bfloat16*)k_cache[l];
+    tab.v_cache[l] = (__nv_bfloat16*)v_cache[l];
+  }
+  dg::KVParams p{n_layers, B, Hkv, C, hd, lmax, ld_blk, cache_len};
+  const size_t total = (size_t)n_layers * 2 * B * Hkv * C * (hd / 8);
+  const int blocks = (int)std::min<size_t>((total + 255) / 256, (size_t)kNumSMs * 16);
+  dg::kv_commit_kernel<<<std::max(1, blocks), 256, 0, s>>>(tab, p);
+  DG_CUDA(cudaGetLastError());
+  return DG_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Model forward
+// ---------------------------------------------------------------------------
+int check_model(const dg_model* m) {
+  if (!m || !m->embed || !m->unembed || !m->layers)
+    return fail(DG_ERR_INVALID_ARG, "model: null pointer");
+  const dg_model_cfg& c = m->cfg;
+  if (c.d <= 0 || c.n_layers <= 0 || c.n_layers > dg::KV_MAX_LAYERS || c.n_q_heads <= 0 ||
+      c.n_kv_heads <= 0 || c.n_q_heads % c.n_kv_heads != 0 || c.ffn <= 0 || c.vocab <= 0)
+    return fail(DG_ERR_INVALID_ARG, "model: bad configuration");
+  if (c.head_dim != 64 && c.head_dim != 128)
+    return fail(DG_ERR_UNSUPPORTED_SHAPE, "head_dim %d not in {64,128}", c.head_dim);
+  if (c.d % 128 || c.ffn % 128 || c.vocab % 128 || (c.n_q_heads * c.head_dim) % 128 ||
+      ((c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim) % 128)
+    return fail(DG_ERR_UNSUPPORTED_SHAPE,
+                "d, ffn, vocab, Hq*hd and (Hq+2Hkv)*hd must be multiples of 128");
+  if (!aligned16(m->embed) || !aligned16(m->unembed))
+    return fail(DG_ERR_ALIGNMENT, "model: embed/unembed not 16-byte aligned");
+  for (int l = 0; l < c.n_layers; ++l) {
+    const dg_layer_weights& w = m->layers[l];
+    if (!w.w_qkv || !w.w_o || !w.w_up || !w.w_down)
+      return fail(DG_ERR_INVALID_ARG, "model: layer %d has a null weight", l);
+    if (!aligned16(w.w_qkv) || !aligned16(w.w_o) || !aligned16(w.w_up) || !aligned16(w.w_down))
+      return fail(DG_ERR_ALIGNMENT, "model: layer %d weight not 16-byte aligned", l);
+  }
+  return DG_OK;
+}
+
+int check_state(const dg_state* st, const dg_model_cfg& c, bool need_canvas) {
+  if (!st || !st->k_cache || !st->v_cache || !st->cache_len)
+    return fail(DG_ERR_INVALID_ARG, "state: null pointer");
+  if (st->batch <= 0 || st->lmax <= 0) return fail(DG_ERR_INVALID_ARG, "state: bad batch/lmax");
+  if (need_canvas) {
+    if (!st->tok || !st->committed || !st->prev_argmax || !st->seq_status || !st->step)
+      return fail(DG_ERR_INVALID_ARG, "state: null canvas pointer");
+    if (st->canvas <= 0 || st->canvas > 1024)
+      return fail(DG_ERR_UNSUPPORTED_SHAPE, "canvas %d not in [1, 1024]", st->canvas);
+  }
+  for (int l = 0; l < c.n_layers; ++l)
+    if (!st->k_cache[l] || !st->v_cache[l] || !aligned16(st->k_cache[l]) ||
+        !aligned16(st->v_cache[l]))
+      return fail(DG_ERR_ALIGNMENT, "state: cache of layer %d null or misaligned", l);
+  return DG_OK;
+}
+
+// Workspace carve-up for a forward over M = B * Lq rows.
+struct FwdLayout {
+  size_t x, xn, qkv, ao, up, part, attn, logits, spart, flag, total;
+};
+
+FwdLayout fwd_layout(const dg_model_cfg& c, int B, int Lq, int max_prefix, bool logits) {
+  FwdLayout L;
+  const int M = B * Lq;
+  const int nqkv = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim;
+  const int hqd = c.n_q_heads * c.head_dim;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes, 256);
+    return o;
+  };
+  L.x = take((size_t)M * c.d * 4);
+  L.xn = take((size_t)M * c.d * 2);
+  L.qkv = take((size_t)M * nqkv * 2);
+  L.ao = take((size_t)M * hqd * 2);
+  L.up = take((size_t)M * c.ffn * 2);
+  size_t part = 0;
+  part = std::max(part, linear_part_bytes(M, nqkv, c.d));
+  part = std::max(part, linear_part_bytes(M, c.d, hqd));
+  part = std::max(part, linear_part_bytes(M, c.ffn, c.d));
+  part = std::max(part, linear_part_bytes(M, c.d, c.ffn));
+  L.part = take(part);
+  L.attn = take(attn_ws_bytes(B, c.n_q_heads, Lq, c.head_dim, max_prefix));
+  L.logits = take(logits ? (size_t)M * c.vocab * 4 : 0);
+  L.spart = take(logits ? sample_ws_bytes(B, Lq, c.vocab) : 0);
+  L.flag = take(logits ? 16 : 0);
+  L.total = off;
+  return L;
+}
+
+struct Fwd {
+  const dg_model* m;
+  int B, Lq, max_prefix, lmax, mask;
+  const int32_t* cache_len;
+  void* const* k_cache;
+  void* const* v_cache;
+  bool commit_kv;   // write each layer's new K/V into the cache at cache_len
+  bool want_logits;
+  char* ws;
+  FwdLayout L;
+};
+
+int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s) {
+  const dg_model_cfg& c = f.m->cfg;
+  const int M = f.B * f.Lq;
+  const int hd = c.head_dim, hq = c.n_q_heads, hkv = c.n_kv_heads;
+  const int nqkv = (hq + 2 * hkv) * hd;
+  float* x = (float*)(f.ws + f.L.x);
+  __nv_bfloat16* xn = (__nv_bfloat16*)(f.ws + f.L.xn);
+  __nv_bfloat16* qkv = (__nv_bfloat16*)(f.ws + f.L.qkv);
+  __nv_bfloat16* ao = (__nv_bfloat16*)(f.ws + f.L.ao);
+  __nv_bfloat16* up = (__nv_bfloat16*)(f.ws + f.L.up);
+  float* part = (float*)(f.ws + f.L.part);
+  void* aws = f.ws + f.L.attn;
+  const float scale = 1.0f / std::sqrt((float)hd);
+
+  dg::gemm::embed_norm_kernel<<<M, dg::gemm::NORM_THREADS, 0, s>>>(
+      tok, (const __nv_bfloat16*)f.m->embed, c.vocab, c.d, c.eps, x, xn);
+  DG_CUDA(cudaGetLastError());
+  for (int l = 0; l < c.n_layers; ++l) {
+    const dg_layer_weights& w = f.m->layers[l];
+    const bool last = l == c.n_layers - 1;
+    DG_TRY(linear(xn, w.w_qkv, M, nqkv, c.d, 0, qkv, part, c.eps, nullptr, s));
+    if (f.commit_kv) {
+      const void* kb = qkv + hq * hd;
+      const void* vb = qkv + (hq + hkv) * hd;
+      DG_TRY(launch_kv_commit(&kb, &vb, nqkv, &f.k_cache[l], &f.v_cache[l], f.cache_len, 1,
+                              f.B, hkv, f.Lq, hd, f.lmax, s));
+    }
+    if (last && !f.want_logits) break;
+    DG_TRY(launch_attn(qkv, nqkv, qkv + hq * hd, qkv + (hq + hkv) * hd, nqkv, f.k_cache[l],
+                       f.v_cache[l], f.cache_len, f.max_prefix, f.lmax, ao, hq * hd, nullptr,
+                       f.B, hq, hkv, f.Lq, hd, scale, f.mask, aws, s));
+    DG_TRY(linear(ao, w.w_o, M, c.d, hq * hd, 2, x, part, c.eps, xn, s));
+    DG_TRY(linear(xn, w.w_up, M, c.ffn, c.d, 1, up, part, c.eps, nullptr, s));
+    DG_TRY(linear(up, w.w_down, M, c.d, c.ffn, 2, x, part, c.eps, xn, s));
+  }
+  if (f.want_logits) {
+    const GemmPlan pl{1, c.d / dg::gemm::BK};
+    DG_TRY(launch_gemm(xn, f.m->unembed, M, c.vocab, c.d, pl, dg::gemm::EPI_STORE_F32, logits,
+                       nullptr, s));
+  }
+  return DG_OK;
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* dg_status_string(int status) {
+  switch (status) {
+    case DG_OK: return "DG_OK";
+    case DG_ERR_INVALID_ARG: return "DG_ERR_INVALID_ARG";
+    case DG_ERR_UNSUPPORTED_SHAPE: return "DG_ERR_UNSUPPORTED_SHAPE";
+    case DG_ERR_ALIGNMENT: return "DG_ERR_ALIGNMENT";
+    case DG_ERR_WORKSPACE_TOO_SMALL: return "DG_ERR_WORKSPACE_TOO_SMALL";
+    case DG_ERR_CUDA: return "DG_ERR_CUDA";
+    case DG_ERR_TIMEOUT: return "DG_ERR_TIMEOUT";
+    case DG_ERR_DEVICE_CHECK: return "DG_ERR_DEVICE_CHECK";
+    default: return "DG_ERR_UNKNOWN";
+  }
+}
+
+const char* dg_last_error(void) { return g_last_error; }
+
+int dg_version(void) { return kVersion; }
+
+void dg_sampler_defaults(dg_sampler_cfg* cfg) {
+  if (!cfg) return;
+  cfg->max_steps = 48;
+  cfg->t_start = 0.8f;
+  cfg->t_end = 0.4f;
+  cfg->commit_k = 16;
+  cfg->renoise_conf = 0.05f;
+  cfg->stop_entropy = 0.005f;
+  cfg->unselected_policy = DG_UNSELECTED_KEEP;
+}
+
+int dg_check_device_errors(void* stream, uint32_t* code_out) {
+  cudaStream_t s = (cudaStream_t)stream;
+  DG_CUDA(cudaStreamSynchronize(s));
+  uint32_t w[4];
+  DG_CUDA(cudaMemcpyFromSymbol(w, dg::g_err, sizeof(w)));
+  if (code_out) *code_out = w[0];
+  if (w[0] == 0) return DG_OK;
+  const uint32_t zero[4] = {0, 0, 0, 0};
+  DG_CUDA(cudaMemcpyToSymbol(dg::g_err, zero, sizeof(zero)));
+  if (w[0] & dg::ERR_TIMEOUT)
+    return fail(DG_ERR_TIMEOUT, "device wait expired (site 0x%x, detail %u, %u errors)",
+                w[0] & 0xFFFFu, w[2], w[1]);
+  return fail(DG_ERR_DEVICE_CHECK, "device check failed (site 0x%x, detail %u, %u errors)",
+              w[0] & 0xFFFFu, w[2], w[1]);
+}
+
+size_t dg_canvas_attn_workspace_bytes(int B, int Hq, int Hkv, int Lq, int hd, int max_prefix) {
+  (void)Hkv;
+  if (B <= 0 || Hq <= 0 || Lq <= 0 || (hd != 64 && hd != 128) || max_prefix < 0) return 0;
+  return attn_ws_bytes(B, Hq, Lq, hd, max_prefix);
+}
+
+int dg_canvas_attn(const void* q, int ldq, const void* k_new, const void* v_new, int ldkv,
+                   const void* k_cache, const void* v_cache, const int32_t* cache_len,
+                   int max_prefix, int lmax, void* out, int ldo, float* lse, int B, int Hq,
+                   int Hkv, int Lq, int hd, float scale, int mask_mode, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  if (!q || !k_new || !v_new || !k_cache || !v_cache || !cache_len || !out)
+    return fail(DG_ERR_INVALID_ARG, "dg_canvas_attn: null pointer");
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0 || Hq % Hkv || max_prefix < 0 || lmax < 1 ||
+      max_prefix > lmax || (mask_mode != DG_MASK_BIDIR && mask_mode != DG_MASK_CAUSAL))
+    return fail(DG_ERR_INVALID_ARG, "dg_canvas_attn: bad sizes or mask");
+  if (hd != 64 && hd != 128)
+    return fail(DG_ERR_UNSUPPORTED_SHAPE, "dg_canvas_attn: head_dim %d not in {64,128}", hd);
+  if (ldq % 8 || ldkv % 8 || ldo % 8 || ldq < Hq * hd || ldkv < Hkv * hd || ldo < Hq * hd)
+    return fail(DG_ERR_ALIGNMENT, "dg_canvas_attn: leading dimensions");
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) ||
+      !aligned16(v_cache) || !aligned16(out))
+    return fail(DG_ERR_ALIGNMENT, "dg_canvas_attn: pointers must be 16-byte aligned");
+  const size_t need = attn_ws_bytes(B, Hq, Lq, hd, max_prefix);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+    return fail(DG_ERR_WORKSPACE_TOO_SMALL, "dg_canvas_attn: workspace needs %zu bytes", need);
+  return launch_attn(q, ldq, k_new, v_new, ldkv, k_cache, v_cache, cache_len, max_prefix, lmax,
+                     out, ldo, lse, B, Hq, Hkv, Lq, hd, scale, mask_mode, workspace,
+                     (cudaStream_t)stream);
+}
+
+int dg_unembed(const void* h, const void* w_u, float* logits, int M, int d, int V,
+               void* workspace, size_t workspace_bytes, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  if (!h || !w_u || !logits) return fail(DG_ERR_INVALID_ARG, "dg_unembed: null pointer");
+  if (M <= 0 || d <= 0 || V <= 0) return fail(DG_ERR_INVALID_ARG, "dg_unembed: bad sizes");
+  if (V % 128 || d % 64)
+    return fail(DG_ERR_UNSUPPORTED_SHAPE, "dg_unembed: V %% 128 and d %% 64 must be 0");
+  if (!aligned16(h) || !aligned16(w_u) || !aligned16(logits))
+    return fail(DG_ERR_ALIGNMENT, "dg_unembed: pointers must be 16-byte aligned");
+  const GemmPlan pl{1, d / dg::gemm::BK};
+  return launch_gemm(h, w_u, M, V, d, pl, dg::gemm::EPI_STORE_F32, logits, nullptr,
+                     (cudaStream_t)stream);
+}
+
+size_t dg_linear_workspace_bytes(int M, int N, int K) {
+  if (M <= 0 || N <= 0 || K <= 0) return 0;
+  return linear_part_bytes(M, N, K);
+}
+
+int dg_linear(const void* x, const void* w, void* out, int M, int N, int K, int epilogue,
+              void* workspace, size_t workspace_bytes, void* stream) {
+  if (!x || !w || !out) return fail(DG_ERR_INVALID_ARG, "dg_linear: null pointer");
+  if (M <= 0 || N <= 0 || K <= 0 || epilogue < 0 || epilogue > DG_EPI_RESID_F32)
+    return fail(DG_ERR_INVALID_ARG, "dg_linear: bad sizes or epilogue");
+  if (N % 128 || K % 64)
+    return fail(DG_ERR_UNSUPPORTED_SHAPE, "dg_linear: N %% 128 and K %% 64 must be 0");
+  if (!aligned16(x) || !aligned16(w) || !aligned16(out))
+    return fail(DG_ERR_ALIGNMENT, "dg_linear: pointers must be 16-byte aligned");
+  cudaStream_t s = (cudaStream_t)stream;
+  if (epilogue == DG_EPI_F32) {
+    const GemmPlan pl{1, K / dg::gemm::BK};
+    return launch_gemm(x, w, M, N, K, pl, dg::gemm::EPI_STORE_F32, (float*)out, nullptr, s);
+  }
+  const size_t need = linear_part_bytes(M, N, K);
+  const GemmPlan pl = plan_gemm(M, N, K);
+  if (pl.splits > 1 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+    return fail(DG_ERR_WORKSPACE_TOO_SMALL, "dg_linear: workspace needs %zu bytes", need);
+  const int mode = epilogue == DG_EPI_BF16 ? 0 : epilogue == DG_EPI_GELU_BF16 ? 1 : 2;
+  return linear(x, w, M, N, K, mode, out, (float*)workspace, 0.f, nullptr, s);
+}
+
+size_t dg_sample_commit_workspace_bytes(int B, int C, int V) {
+  if (B <= 0 || C <= 0 || V <= 0) return 0;
+  return sample_ws_bytes(B, C, V);
+}
+
+int dg_sample_commit(const float* logits, int32_t* tok, uint8_t* committed,
+                     int32_t* prev_argmax, int32_t* seq_status, const dg_sampler_cfg* cfg,
+                     uint32_t seed, int block, int step, int B, int C, int V,
+                     const dg_step_out* out, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  if (!logits || !tok || !committed || !prev_argmax || !seq_status || !cfg)
+    return fail(DG_ERR_INVALID_ARG, "dg_sample_commit: null pointer");
+  if (B <= 0 || C <= 0 || C > 1024 || V <= 0 || V % 4 || step < 0 || block < 0)
+    return fail(DG_ERR_UNSUPPORTED_SHAPE, "dg_sample_commit: need C <= 1024, V %% 4 == 0");
+  if (cfg->max_steps < 1 || cfg->commit_k < 0 || !(cfg->t_start > 0.f) || !(cfg->t_end > 0.f) ||
+      (cfg->unselected_policy != 0 && cfg->unselected_policy != 1))
+    return fail(DG_ERR_INVALID_ARG, "dg_sample_commit: bad sampler settings");
+  if (!aligned16(logits)) return fail(DG_ERR_ALIGNMENT, "dg_sample_commit: logits alignment");
+  const size_t need = sample_ws_bytes(B, C, V);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return fail(DG_ERR_WORKSPACE_TOO_SMALL, "dg_sample_commit: workspace needs %zu bytes", need);
+  const dg::SampleParams p = make_sample_params(*cfg, seed, block, nullptr, step, B, C, V);
+  return launch_sample(logits, tok, committed, prev_argmax, seq_status, p, out, workspace,
+                       (cudaStream_t)stream);
+}
+
+int dg_kv_block_commit(const void* const* k_blk, const void* const* v_blk, int ld_blk,
+                       void* const* k_cache, void* const* v_cache, int32_t* cache_len,
+                       int n_layers, int B, int Hkv, int C, int hd, int lmax, void* stream) {
+  if (!k_blk || !v_blk || !k_cache || !v_cache || !cache_len)
+    return fail(DG_ERR_INVALID_ARG, "dg_kv_block_commit: null pointer");
+  if (n_layers <= 0 || n_layers > dg::KV_MAX_LAYERS || B <= 0 || Hkv <= 0 || C <= 0 || lmax <= 0)
+    return fail(DG_ERR_INVALID_ARG, "dg_kv_block_commit: bad sizes (n_layers <= %d)",
+                dg::KV_MAX_LAYERS);
+  if (hd % 8 || ld_blk % 8 || ld_blk < Hkv * hd)
+    return fail(DG_ERR_ALIGNMENT, "dg_kv_block_commit: hd and ld_blk must be multiples of 8");
+  for (int l = 0; l < n_layers; ++l)
+    if (!aligned16(k_blk[l]) || !aligned16(v_blk[l]) || !aligned16(k_cache[l]) ||
+        !aligned16(v_cache[l]) || !k_blk[l] || !v_blk[l] || !k_cache[l] || !v_cache[l])
+      return fail(DG_ERR_ALIGNMENT, "dg_kv_block_commit: layer %d pointer null or misaligned", l);
+  cudaStream_t s = (cudaStream_t)stream;
+  DG_TRY(launch_kv_commit(k_blk, v_blk, ld_blk, k_cache, v_cache, cache_len, n_layers, B, Hkv, C,
+                          hd, lmax, s));
+  dg::cache_len_bump_kernel<<<1, 256, 0, s>>>(cache_len, B, C, lmax);
+  DG_CUDA(cudaGetLastError());
+  return DG_OK;
+}
+
+size_t dg_prefill_workspace_bytes(const dg_model_cfg* cfg, int B, int P) {
+  if (!cfg || B <= 0 || P <= 0) return 0;
+  return fwd_layout(*cfg, B, P, 0, false).total;
+}
+
+int dg_prefill(const dg_model* m, dg_state* st, const int32_t* prompt, int P, void* workspace,
+               size_t workspace_bytes, void* stream) {
+  DG_TRY(check_model(m));
+  DG_TRY(check_state(st, m->cfg, false));
+  if (!prompt || P <= 0 || P > st->lmax)
+    return fail(DG_ERR_INVALID_ARG, "dg_prefill: bad prompt (P=%d, lmax=%d)", P, st->lmax);
+  const FwdLayout L = fwd_layout(m->cfg, st->batch, P, 0, false);
+  if (!workspace || workspace_bytes < L.total || !aligned16(workspace))
+    return fail(DG_ERR_WORKSPACE_TOO_SMALL, "dg_prefill: workspace needs %zu bytes", L.total);
+  cudaStream_t s = (cudaStream_t)stream;
+  dg::cache_len_set_kernel<<<1, 256, 0, s>>>(st->cache_len, st->batch, 0);
+  DG_CUDA(cudaGetLastError());
+  Fwd f{m, st->batch, P, 0, st->lmax, DG_MASK_CAUSAL, st->cache_len, st->k_cache,
+        st->v_cache, true, false, (char*)workspace, L};
+  DG_TRY(run_forward(f, prompt, nullptr, s));
+  dg::cache_len_set_kernel<<<1, 256, 0, s>>>(st->cache_len, st->batch, P);
+  DG_CUDA(cudaGetLastError());
+  st->cache_len_host = P;
+  return DG_OK;
+}
+
+size_t dg_denoise_block_workspace_bytes(const dg_model_cfg* cfg, int B, int C, int lmax) {
+  if (!cfg || B <= 0 || C <= 0 || lmax <= 0) return 0;
+  return fwd_layout(*cfg, B, C, lmax, true).total;
+}
+
+int dg_denoise_logits(const dg_model* m, const dg_state* st, float* logits, void* workspace,
+                      size_t workspace_bytes, void* stream) {
+  DG_TRY(check_model(m));
+  DG_TRY(check_state(st, m->cfg, true));
+  if (!logits || !aligned16(logits))
+    return fail(DG_ERR_INVALID_ARG, "dg_denoise_logits: logits null or misaligned");
+  if (st->cache_len_host < 0 || st->cache_len_host > st->lmax)
+    return fail(DG_ERR_INVALID_ARG, "dg_denoise_logits: cache_len_host out of range");
+  const FwdLayout L = fwd_layout(m->cfg, st->batch, st->canvas, st->lmax, true);
+  if (!workspace || workspace_bytes < L.total || !aligned16(workspace))
+    return fail(DG_ERR_WORKSPACE_TOO_SMALL, "dg_denoise_logits: workspace needs %zu bytes",
+                L.total);
+  Fwd f{m, st->batch, st->canvas, st->cache_len_host, st->lmax, DG_MASK_BIDIR, st->cache_len,
+        st->k_cache, st->v_cache, false, true, (char*)workspace, L};
+  return run_forward(f, st->tok, logits, (cudaStream_t)stream);
+}
+
+int dg_denoise_block(const dg_model* m, dg_state* st, const dg_sampler_cfg* cfg, uint32_t seed,
+                     int block, int* steps_taken, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  DG_TRY(check_model(m));
+  DG_TRY(check_state(st, m->cfg, true));
+  if (!cfg || cfg->max_steps < 1 || block < 0)
+    return fail(DG_ERR_INVALID_ARG, "dg_denoise_block: bad sampler settings or block");
+  if (m->cfg.vocab % 4) return fail(DG_ERR_UNSUPPORTED_SHAPE, "vocab must be a multiple of 4");
+  if (st->cache_len_host < 0 || st->cache_len_host + st->canvas > st->lmax)
+    return fail(DG_ERR_INVALID_ARG, "dg_denoise_block: cache full (%d + %d > %d)",
+                st->cache_len_host, st->canvas, st->lmax);
+  const FwdLayout L = fwd_layout(m->cfg, st->batch, st->canvas, st->lmax, true);
+  if (!workspace || workspace_bytes < L.total || !aligned16(workspace))
+    return fail(DG_ERR_WORKSPACE_TOO_SMALL, "dg_denoise_block: workspace needs %zu bytes",
+                L.total);
+  cudaStream_t s = (cudaStream_t)stream;
+  char* ws = (char*)workspace;
+  const int B = st->batch, C = st->canvas, V = m->cfg.vocab;
+  float* logits = (float*)(ws + L.logits);
+  int32_t* running = (int32_t*)(ws + L.flag);
+
+  dg::init_canvas_kernel<<<B, 256, 0, s>>>(B, C, V, seed, block, st->tok, st->committed,
+                                            st->prev_argmax, st->seq_status, st->step);
+  DG_CUDA(cudaGetLastError());
+  Fwd f{m, B, C, st->cache_len_host, st->lmax, DG_MASK_BIDIR, st->cache_len, st->k_cache,
+        st->v_cache, false, true, ws, L};
+  const dg::SampleParams sp = make_sample_params(*cfg, seed, block, st->step, 0, B, C, V);
+  int steps = 0;
+  for (int it = 0; it < cfg->max_steps; ++it) {
+    DG_TRY(run_forward(f, st->tok, logits, s));
+    DG_TRY(launch_sample(logits, st->tok, st->committed, st->prev_argmax, st->seq_status, sp,
+                         nullptr, ws + L.spart, s));
+    dg::step_advance_kernel<<<1, 256, 0, s>>>(B, cfg->max_steps, st->seq_status, st->step,
+                                              running);
+    DG_CUDA(cudaGetLastError());
+    int32_t host_running = 0;
+    DG_CUDA(cudaMemcpyAsync(&host_running, running, sizeof(int32_t), cudaMemcpyDeviceToHost, s));
+    DG_CUDA(cudaStreamSynchronize(s));
+    steps = it + 1;
+    if (!host_running) break;
+  }
+  // causal re-encode of the final block; each layer's K/V goes to rows
+  // [cache_len, cache_len + C), then the length moves on
+  Fwd r{m, B, C, st->cache_len_host, st->lmax, DG_MASK_CAUSAL, st->cache_len, st->k_cache,
+        st->v_cache, true, false, ws, L};
+  DG_TRY(run_forward(r, st->tok, nullptr, s));
+  dg::cache_len_bump_kernel<<<1, 256, 0, s>>>(st->cache_len, B, C, st->lmax);
+  DG_CUDA(cudaGetLastError());
+  st->cache_len_host += C;
+  if (steps_taken) *steps_taken = steps;
+  return DG_OK;
+}
+
+int dg_philox4x32_10(const uint32_t* in, uint32_t* out, int n, void* stream) {
+  if (!in || !out || n < 0) return fail(DG_ERR_INVALID_ARG, "dg_philox4x32_10: bad arguments");
+  if (n == 0) return DG_OK;
+  dg::philox_kernel<<<cdiv(n, 256), 256, 0, (cudaStream_t)stream>>>(in, out, n);
+  DG_CUDA(cudaGetLastError());
+  return DG_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,448 @@
+// attn.cuh - canvas attention on tcgen05 (flash-style, one pass over the keys).
+//
+// Lq new rows of query head h attend to [cached prefix of kv head g ; new
+// rows], g = h / (Hq / Hkv), scale 1/sqrt(hd), no positional encoding; the
+// mask is full over the canvas (denoising) or lower-triangular over the new
+// rows (prefill, block re-encode).  Sources: aiexpert.news "Google's
+// DiffusionGemma Atinge 1.000 Tokens por Segundo", architecture paragraph
+// (bidirectional attention on the 256-token canvas; causal prefill into the
+// KV cache); "DiffusionGemma Guia do Desenvolvedor ...", bullet "Propagacao
+// de Contexto Bidirecional".
+//
+// One CTA = 128 query rows of one head over a contiguous range of 128-key
+// tiles (the key range is split across CTAs when there are too few query
+// tiles to fill the SMs; a combine kernel merges the splits by their
+// log-sum-exp).  Per key tile j:
+//     S_j = Q K_j^T            tcgen05.mma, A = Q (smem), B = K_j (smem), D in TMEM
+//     P_j = 2^(S_j*c - m)      softmax warps: TMEM -> registers -> bf16 -> TMEM
+//     O  += P_j V_j            tcgen05.mma, A = P_j (TMEM), B = V_j (smem, MN-major)
+// S is double-buffered in TMEM so S_{j+1} runs on the tensor core while the
+// softmax warps work on S_j; P_j overwrites S_j in place.  The running max is
+// only raised (and O rescaled) when it grows by more than 2^8, so most tiles
+// need no O round trip; the final 1/l normalisation makes this exact.
+//
+// Warps: 0 = TMA producer, 1 = TMEM owner + MMA issuer, 2..5 = softmax (one
+// query row per thread; warp w owns TMEM lanes 32*(w%4)..+31).
+#pragma once
+
+#include "dg_common.cuh"
+
+namespace dg {
+namespace attn {
+
+constexpr int BQ = 128;
+constexpr int BKV = 128;
+constexpr int THREADS = 192;
+constexpr int TMEM_COLS = 512;  // S0 [0,128), S1 [128,256), O [256, 256+hd)
+constexpr float kRescaleThreshold = 8.0f;
+
+template <int HD>
+struct Cfg {
+  static constexpr int HALVES = HD / 64;
+  static constexpr int Q_BYTES = BQ * HD * 2;
+  static constexpr int T_BYTES = BKV * HD * 2;  // one K or V tile
+  static constexpr int STAGES = HD == 128 ? 2 : 3;
+  static constexpr int SMEM_BYTES = 1024 + Q_BYTES + STAGES * 2 * T_BYTES + 256;
+  static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BQ, BKV, false, false);
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BQ, HD, false, true);
+};
+
+struct Params {
+  int B, Hq, Hkv, Lq, lmax, group;
+  int n_qtiles, n_splits, causal;
+  float scale_log2;          // scale * log2(e)
+  const int32_t* cache_len;  // [B]
+  __nv_bfloat16* out;        // [B, Lq, ldo]
+  int ldo;
+  float* lse;                // [B, Hq, Lq] natural log, or null
+  float* part_o;             // [S, B, Hq, Lq, hd] fp32 (n_splits > 1)
+  float* part_lse;           // [S, B, Hq, Lq]
+};
+
+template <int HD>
+__global__ void __launch_bounds__(THREADS, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kn,
+                const __grid_constant__ CUtensorMap tm_vn,
+                const __grid_constant__ CUtensorMap tm_kc,
+                const __grid_constant__ CUtensorMap tm_vc, Params p) {
+  using CF = Cfg<HD>;
+  constexpr int ST = CF::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sK = sQ + CF::Q_BYTES;             // ST tiles
+  uint8_t* sV = sK + ST * CF::T_BYTES;        // ST tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + ST * CF::T_BYTES);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = q_full + 1;       // [ST]
+  uint64_t* v_full = k_full + ST;      // [ST]
+  uint64_t* kv_empty = v_full + ST;    // [ST]
+  uint64_t* s_full = kv_empty + ST;    // [2]
+  uint64_t* p_full = s_full + 2;       // [2]
+  uint64_t* o_done = p_full + 2;       // one completion per PV (rescale waits)
+  uint64_t* o_final = o_done + 1;      // single completion after the last PV
+  uint64_t* drain = o_final + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+
+  const int warp = warp_id();
+  const int lane = lane_id();
+  const int qt = blockIdx.x % p.n_qtiles;
+  const int bh = blockIdx.x / p.n_qtiles;
+  const int h = bh % p.Hq;
+  const int b = bh / p.Hq;
+  const int g = h / p.group;
+  const int split = blockIdx.y;
+  const int i0 = qt * BQ;
+
+  int L = p.cache_len[b];
+  if (L < 0 || L > p.lmax) {
+    if (threadIdx.x == 0 && split == 0 && qt == 0 && h == 0) raise_error(ERR_CHECK | 0x301, b);
+    L = L < 0 ? 0 : p.lmax;
+  }
+  const int lq_vis = p.causal ? min(p.Lq, i0 + BQ) : p.Lq;
+  const int nP = (L + BKV - 1) / BKV;
+  const int nC = (lq_vis + BKV - 1) / BKV;
+  const int T = nP + nC;
+  const int t_beg = static_cast<int>((static_cast<long long>(T) * split) / p.n_splits);
+  const int t_end = static_cast<int>((static_cast<long long>(T) * (split + 1)) / p.n_splits);
+  const int n = t_end - t_beg;
+
+  if (n <= 0) {
+    // empty key range: this split contributes nothing to the merge
+    if (threadIdx.x < BQ) {
+      const int qrow = i0 + threadIdx.x;
+      if (qrow < p.Lq) {
+        const size_t r = ((static_cast<size_t>(split) * p.B + b) * p.Hq + h) * p.Lq + qrow;
+        p.part_lse[r] = -INFINITY;
+        float4* o = reinterpret_cast<float4*>(p.part_o + r * HD);
+        for (int c = 0; c < HD / 4; ++c) o[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
+    return;
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&s_full[s], 1);
+      mbar_init(&p_full[s], BQ);
+    }
+    mbar_init(o_done, 1);
+    mbar_init(o_final, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_q);
+    tma_prefetch_desc(&tm_kn);
+    tma_prefetch_desc(&tm_vn);
+    tma_prefetch_desc(&tm_kc);
+    tma_prefetch_desc(&tm_vc);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_holder, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_holder;
+  const uint32_t tmem_o = tmem + 256;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      mbar_expect_tx(q_full, CF::Q_BYTES);
+      for (int hf = 0; hf < CF::HALVES; ++hf)
+        tma_load_2d(sQ + hf * (BQ * 128), &tm_q, q_full, h * HD + hf * 64, b * p.Lq + i0);
+      int issued = 0;
+      for (int i = 0; i < n; ++i) {
+        const int st = i % ST;
+        if (i >= ST && !mbar_wait(&kv_empty[st], ((i / ST) - 1) & 1, abort_flag, 0x311)) break;
+        const int t = t_beg + i;
+        const CUtensorMap* mk;
+        const CUtensorMap* mv;
+        int x0, y0;
+        if (t < nP) {
+          mk = &tm_kc;
+          mv = &tm_vc;
+          x0 = 0;
+          y0 = (b * p.Hkv + g) * p.lmax + t * BKV;
+        } else {
+          mk = &tm_kn;
+          mv = &tm_vn;
+          x0 = g * HD;
+          y0 = b * p.Lq + (t - nP) * BKV;
+        }
+        uint8_t* kd = sK + st * CF::T_BYTES;
+        uint8_t* vd = sV + st * CF::T_BYTES;
+        mbar_expect_tx(&k_full[st], CF::T_BYTES);
+        for (int hf = 0; hf < CF::HALVES; ++hf)
+          tma_load_2d(kd + hf * (BKV * 128), mk, &k_full[st], x0 + hf * 64, y0);
+        mbar_expect_tx(&v_full[st], CF::T_BYTES);
+        for (int hf = 0; hf < CF::HALVES; ++hf)
+          tma_load_2d(vd + hf * (BKV * 128), mv, &v_full[st], x0 + hf * 64, y0);
+        issued = i + 1;
+      }
+      if (*abort_flag) {
+        mbar_wait(q_full, 0, nullptr, 0x312);
+        for (int i = max(0, issued - ST); i < issued; ++i) {
+          mbar_wait(&k_full[i % ST], (i / ST) & 1, nullptr, 0x313);
+          mbar_wait(&v_full[i % ST], (i / ST) & 1, nullptr, 0x314);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(q_full, 0, abort_flag, 0x321);
+      const uint32_t q_base = smem_u32(sQ);
+      auto issue_s = [&](int i) -> bool {
+        const int st = i % ST;
+        if (!mbar_wait(&k_full[st], (i / ST) & 1, abort_flag, 0x322)) return false;
+        tc_fence_after();
+        const uint32_t k_base = smem_u32(sK + st * CF::T_BYTES);
+        const uint32_t d = tmem + (i & 1) * 128;
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
+          umma_ss(d, sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(k_base + off, 16, 1024),
+                  CF::IDESC_QK, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(&s_full[i & 1]);
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {
+        const int st = j % ST;
+        if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1, abort_flag, 0x323)) return false;
+        if (!mbar_wait(&v_full[st], (j / ST) & 1, abort_flag, 0x324)) return false;
+        tc_fence_after();
+        const uint32_t v_base = smem_u32(sV + st * CF::T_BYTES);
+        const uint32_t pa = tmem + (j & 1) * 128;
+#pragma unroll
+        for (int kk = 0; kk < BKV / 16; ++kk) {
+          // keys 16kk..16kk+15: rows of the MN-major V tile, 128 B each
+          umma_ts(tmem_o, pa + kk * 8,
+                  sdesc_sw128(v_base + kk * 16 * 128, BKV * 128, 1024), CF::IDESC_PV,
+                  (j > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&kv_empty[st]);
+        umma_commit(o_done);
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int i = 1; ok && i < n; ++i) {
+        ok = issue_s(i);
+        if (ok) ok = issue_pv(i - 1);
+      }
+      if (ok) ok = issue_pv(n - 1);
+      if (ok) umma_commit(o_final);
+      umma_commit(drain);
+      mbar_wait(drain, 0, nullptr, 0x325);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int qrow = i0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    float m = -INFINITY;  // running max in scaled log2 units
+    float l = 0.f;
+    bool ok = true;
+    for (int i = 0; i < n && ok; ++i) {
+      const int sb = i & 1;
+      if (!mbar_wait(&s_full[sb], (i >> 1) & 1, abort_flag, 0x331)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[128];
+      {
+        uint32_t(&c0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+        uint32_t(&c1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+        uint32_t(&c2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[64]);
+        uint32_t(&c3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[96]);
+        const uint32_t base = tmem + sb * 128 + lane_off;
+        tmem_ld32(base + 0, c0);
+        tmem_ld32(base + 32, c1);
+        tmem_ld32(base + 64, c2);
+        tmem_ld32(base + 96, c3);
+        tmem_ld_wait();
+      }
+      // key validity of this tile for this row
+      const int t = t_beg + i;
+      int nvalid;      // keys [0, nvalid) of the tile may be valid
+      int causal_lim;  // canvas key index limit (inclusive) for causal rows
+      bool canvas = t >= nP;
+      if (!canvas) {
+        nvalid = min(BKV, L - t * BKV);
+        causal_lim = 0x7FFFFFFF;
+      } else {
+        const int ck0 = (t - nP) * BKV;
+        nvalid = min(BKV, p.Lq - ck0);
+        causal_lim = p.causal ? (qrow - ck0) : 0x7FFFFFFF;
+      }
+      const int lim = min(nvalid - 1, causal_lim);  // valid keys: [0, lim]
+      float tmax = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; ++c) {
+        const float v = (c <= lim) ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
+        sr[c] = __float_as_uint(v);
+        tmax = fmaxf(tmax, v);
+      }
+      if (tmax > m + kRescaleThreshold || m == -INFINITY) {
+        const float m_new = fmaxf(tmax, m);
+        if (i > 0 && m != -INFINITY) {
+          // O holds PV_0..PV_{i-1}; wait for the last one, then rescale in TMEM
+          if (!mbar_wait(o_done, (i - 1) & 1, abort_flag, 0x332)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const float f = exp2f(m - m_new);
+#pragma unroll
+          for (int c = 0; c < HD / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tmem_o + lane_off + c * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
+            tmem_st32(tmem_o + lane_off + c * 32, o);
+          }
+          tmem_st_wait();
+          l *= f;
+        }
+        m = m_new;
+      }
+      const float mu = (m == -INFINITY) ? 0.f : m;
+      float rs = 0.f;
+      uint32_t pk[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) {
+        const float p0 = exp2f(__uint_as_float(sr[2 * c]) - mu);
+        const float p1 = exp2f(__uint_as_float(sr[2 * c + 1]) - mu);
+        rs += p0 + p1;
+        pk[c] = pack_bf16x2(p0, p1);
+      }
+      l += rs;
+      {
+        uint32_t(&a0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
+        uint32_t(&a1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
+        const uint32_t base = tmem + sb * 128 + lane_off;
+        tmem_st32(base + 0, a0);
+        tmem_st32(base + 32, a1);
+        tmem_st_wait();
+      }
+      tc_fence_before();
+      mbar_arrive(&p_full[sb]);
+    }
+    if (ok && mbar_wait(o_final, 0, abort_flag, 0x333)) {
+      tc_fence_after();
+      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+      const float lse_nat = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      const bool store = qrow < p.Lq;
+      if (p.n_splits == 1) {
+        __nv_bfloat16* orow =
+            p.out + (static_cast<size_t>(b) * p.Lq + qrow) * p.ldo + static_cast<size_t>(h) * HD;
+#pragma unroll
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem_o + lane_off + c * 32, o);
+          tmem_ld_wait();
+          if (store) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+              uint4 w;
+              w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l,
+                                __uint_as_float(o[8 * v + 1]) * inv_l);
+              w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l,
+                                __uint_as_float(o[8 * v + 3]) * inv_l);
+              w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l,
+                                __uint_as_float(o[8 * v + 5]) * inv_l);
+              w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l,
+                                __uint_as_float(o[8 * v + 7]) * inv_l);
+              dst[v] = w;
+            }
+          }
+        }
+        if (store && p.lse) p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Lq + qrow] = lse_nat;
+      } else {
+        const size_t rr = ((static_cast<size_t>(split) * p.B + b) * p.Hq + h) * p.Lq + qrow;
+        float4* dst = reinterpret_cast<float4*>(p.part_o + rr * HD);
+#pragma unroll
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tmem_o + lane_off + c * 32, o);
+          tmem_ld_wait();
+          if (store) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              dst[c * 8 + v] = make_float4(__uint_as_float(o[4 * v]) * inv_l,
+                                           __uint_as_float(o[4 * v + 1]) * inv_l,
+                                           __uint_as_float(o[4 * v + 2]) * inv_l,
+                                           __uint_as_float(o[4 * v + 3]) * inv_l);
+          }
+        }
+        if (store) p.part_lse[rr] = lse_nat;
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+// Merge key-range splits: O = sum_s w_s O_s / sum_s w_s, w_s = exp(lse_s - max).
+// One warp per (b, h, row); lane covers 4 (hd = 128) or 2 (hd = 64) columns.
+template <int HD>
+__global__ void attn_combine_kernel(const float* __restrict__ part_o,
+                                    const float* __restrict__ part_lse, int S, int B, int Hq,
+                                    int Lq, __nv_bfloat16* __restrict__ out, int ldo,
+                                    float* __restrict__ lse) {
+  const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int rows = B * Hq * Lq;
+  if (warp_global >= rows) return;
+  const size_t stride = static_cast<size_t>(rows);
+  float mx = -INFINITY;
+  for (int s = 0; s < S; ++s) mx = fmaxf(mx, part_lse[s * stride + warp_global]);
+  constexpr int PER = HD / 32;
+  float acc[PER];
+#pragma unroll
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
+  float wsum = 0.f;
+  for (int s = 0; s < S; ++s) {
+    const float ls = part_lse[s * stride + warp_global];
+    if (ls == -INFINITY) continue;
+    const float w = expf(ls - mx);
+    wsum += w;
+    const float* src = part_o + (s * stride + warp_global) * HD + lane * PER;
+#pragma unroll
+    for (int e = 0; e < PER; ++e) acc[e] += w * src[e];
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  const int qrow = warp_global % Lq;
+  const int bh = warp_global / Lq;
+  const int h = bh % Hq;
+  const int b = bh / Hq;
+  __nv_bfloat16* dst = out + (static_cast<size_t>(b) * Lq + qrow) * ldo +
+                       static_cast<size_t>(h) * HD + lane * PER;
+#pragma unroll
+  for (int e = 0; e < PER; ++e) dst[e] = __float2bfloat16_rn(acc[e] * inv);
+  if (lse && lane == 0) lse[warp_global] = (wsum > 0.f) ? mx + logf(wsum) : -INFINITY;
+}
+
+}  // namespace attn
+}  // namespace dg

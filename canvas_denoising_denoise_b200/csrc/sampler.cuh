@@ -1,0 +1,402 @@
+// sampler.cuh - the denoising sampler on the GPU.
+//
+// Per step (Google docs page "DiffusionGemma", table "Configuracao de exibicao
+// recomendada": 48-step cap, linear 0.8 -> 0.4 temperature, adaptive stop on
+// mean entropy + two identical predictions; aiexpert.news "Google's
+// DiffusionGemma Atinge 1.000 Tokens por Segundo", architecture paragraph:
+// confident tokens locked each pass, low-confidence ones re-noised):
+//
+//   rowpass   streams the fp32 logits once.  Each CTA reduces one chunk of one
+//             position's vocabulary row to a partial: running max and the
+//             two sums of the online softmax (for logsumexp and entropy), the
+//             raw-logit argmax, and the best Gumbel-perturbed score.
+//   commit    one CTA per sequence, one thread per canvas position: merges the
+//             partials, ranks log confidences for the top-k commit, applies
+//             re-noise / unselected policy / stop rule, updates the canvas.
+//
+// Arithmetic is done in the log2 domain: zl = l * log2(e) / T.  The Gumbel
+// score in that domain is zl - log2(E), E = -ln(u), which orders exactly like
+// z - ln(E).  Ties resolve to the lowest vocabulary index / position.
+#pragma once
+
+#include "dg_common.cuh"
+
+namespace dg {
+
+constexpr uint32_t kTagGumbel = 0;
+constexpr uint32_t kTagRenoise = 1;
+constexpr uint32_t kTagInit = 2;
+
+// Philox4x32-10 (Salmon, Moraes, Dror, Shaw, SC'11): per round two 32x32->64
+// multiplies by the Philox constants; the high halves are XORed with the other
+// two counter words and the round key; the key is bumped by the Weyl constants.
+__host__ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c.x;
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c.z;
+    const uint32_t hi0 = static_cast<uint32_t>(p0 >> 32), lo0 = static_cast<uint32_t>(p0);
+    const uint32_t hi1 = static_cast<uint32_t>(p1 >> 32), lo1 = static_cast<uint32_t>(p1);
+    c = make_uint4(hi1 ^ c.y ^ k.x, lo1, hi0 ^ c.w ^ k.y, lo0);
+    k.x += 0x9E3779B9u;
+    k.y += 0xBB67AE85u;
+  }
+  return c;
+}
+
+__device__ __forceinline__ uint32_t position_word(uint32_t seed, uint32_t b, uint32_t block,
+                                                  uint32_t step, uint32_t pos, uint32_t tag) {
+  return philox4x32_10(make_uint4(0u, (pos & 0xFFFFFFu) | (tag << 24), step, block),
+                       make_uint2(seed, b))
+      .x;
+}
+
+__device__ __forceinline__ int32_t token_from_word(uint32_t r, int vocab) {
+  return static_cast<int32_t>((static_cast<uint64_t>(r) * static_cast<uint32_t>(vocab)) >> 32);
+}
+
+// u = (2 (r >> 9) + 1) 2^-24 in (0, 1), exact in fp32; returns log2(-ln u).
+// logf is accurate to about one ulp over its whole range (including just
+// below 1, where -ln u is tiny), so E keeps its relative accuracy everywhere.
+__device__ __forceinline__ float neg_log2_exponential(uint32_t r) {
+  const float u = __uint2float_rn(((r >> 9) << 1) | 1u) * 5.9604644775390625e-08f;  // 2^-24
+  const float e = -logf(u);
+  return log2f(e);
+}
+
+__device__ __forceinline__ float step_temperature(int step, int max_steps, float t0, float t1) {
+  if (max_steps <= 1) return t0;
+  return t0 + (t1 - t0) * (static_cast<float>(step) / static_cast<float>(max_steps - 1));
+}
+
+struct RowPartial {
+  float m;      // running max of zl
+  float s;      // sum 2^(zl - m)
+  float q;      // sum 2^(zl - m) (zl - m)
+  float amax;   // max raw logit
+  int aidx;     // its index (lowest on ties)
+  float best;   // best Gumbel score, log2 domain
+  int bidx;     // its index (lowest on ties)
+  int pad;
+};
+
+struct SampleParams {
+  int B, C, V;
+  int chunk, nchunk;         // vocabulary chunk per rowpass CTA
+  uint32_t seed;
+  int block;
+  const int32_t* step_ptr;   // device step index, or null: use step_val
+  int step_val;
+  int max_steps;
+  float t_start, t_end;
+  int commit_k;
+  float log_tau;             // ln(renoise_conf), -inf disables re-noise
+  float stop_entropy;
+  int policy;
+};
+
+__device__ __forceinline__ int read_step(const SampleParams& p) {
+  return p.step_ptr ? *p.step_ptr : p.step_val;
+}
+
+__device__ __forceinline__ void merge_softmax(float& m, float& s, float& q, float m2, float s2,
+                                              float q2) {
+  if (m2 == -INFINITY) return;
+  if (m == -INFINITY) {
+    m = m2; s = s2; q = q2;
+    return;
+  }
+  if (m2 > m) {
+    const float d = m - m2, f = exp2f(d);
+    q = f * (q + d * s) + q2;
+    s = f * s + s2;
+    m = m2;
+  } else {
+    const float d = m2 - m, f = exp2f(d);
+    q = q + f * (q2 + d * s2);
+    s = s + f * s2;
+  }
+}
+
+__device__ __forceinline__ void merge_best(float& v, int& i, float v2, int i2) {
+  if (v2 > v || (v2 == v && i2 < i)) {
+    v = v2;
+    i = i2;
+  }
+}
+
+// Grid: B * C * nchunk CTAs of RP_THREADS threads.  Chunk length is a multiple of 4.
+constexpr int RP_THREADS = 256;
+constexpr int RP_UNROLL = 4;
+
+__global__ void __launch_bounds__(RP_THREADS) sample_rowpass_kernel(
+    const float* __restrict__ logits, const int32_t* __restrict__ seq_status, SampleParams p,
+    RowPartial* __restrict__ part) {
+  const int row = blockIdx.x / p.nchunk;
+  const int ck = blockIdx.x - row * p.nchunk;
+  const int b = row / p.C;
+  const int pos = row - b * p.C;
+  if (seq_status[b] != 0) return;
+  const int step = read_step(p);
+  const float T = step_temperature(step, p.max_steps, p.t_start, p.t_end);
+  const float k2 = 1.4426950408889634f / T;  // log2(e) / T
+  const float* x = logits + static_cast<size_t>(row) * p.V;
+  const int v0 = ck * p.chunk;
+  const int v1 = min(p.V, v0 + p.chunk);
+  const uint32_t c1 = (static_cast<uint32_t>(pos) & 0xFFFFFFu) | (kTagGumbel << 24);
+  const uint2 key = make_uint2(p.seed, static_cast<uint32_t>(b));
+
+  float m = -INFINITY, s = 0.f, q = 0.f;
+  float amax = -INFINITY;
+  int aidx = 0x7FFFFFFF;
+  float best = -INFINITY;
+  int bidx = 0x7FFFFFFF;
+
+  for (int base = v0 + threadIdx.x * 4; base < v1; base += RP_THREADS * 4 * RP_UNROLL) {
+    float4 l4[RP_UNROLL];
+#pragma unroll
+    for (int u = 0; u < RP_UNROLL; ++u) {
+      const int v = base + u * RP_THREADS * 4;
+      l4[u] = (v < v1) ? __ldcs(reinterpret_cast<const float4*>(x + v))
+                       : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+    }
+    float bm = -INFINITY;
+#pragma unroll
+    for (int u = 0; u < RP_UNROLL; ++u)
+      bm = fmaxf(bm, fmaxf(fmaxf(l4[u].x, l4[u].y), fmaxf(l4[u].z, l4[u].w)));
+    const float bmz = bm * k2;
+    if (bmz > m) {
+      if (m != -INFINITY) {
+        const float d = m - bmz, f = exp2f(d);
+        q = f * (q + d * s);
+        s = f * s;
+      }
+      m = bmz;
+    }
+#pragma unroll
+    for (int u = 0; u < RP_UNROLL; ++u) {
+      const int v = base + u * RP_THREADS * 4;
+      if (v >= v1) break;
+      const float lv[4] = {l4[u].x, l4[u].y, l4[u].z, l4[u].w};
+      const uint4 r = philox4x32_10(make_uint4(static_cast<uint32_t>(v >> 2), c1,
+                                               static_cast<uint32_t>(step),
+                                               static_cast<uint32_t>(p.block)),
+                                    key);
+      const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float zl = lv[e] * k2;
+        const float t = zl - m;
+        const float w = exp2f(t);
+        s += w;
+        q = fmaf(w, t, q);
+        if (lv[e] > amax) {
+          amax = lv[e];
+          aidx = v + e;
+        }
+        const float score = zl - neg_log2_exponential(rw[e]);
+        if (score > best) {
+          best = score;
+          bidx = v + e;
+        }
+      }
+    }
+  }
+
+  // CTA reduction: warp shuffles, then across warps through shared memory.
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    const float q2 = __shfl_xor_sync(0xffffffffu, q, o);
+    merge_softmax(m, s, q, m2, s2, q2);
+    const float a2 = __shfl_xor_sync(0xffffffffu, amax, o);
+    const int ai2 = __shfl_xor_sync(0xffffffffu, aidx, o);
+    merge_best(amax, aidx, a2, ai2);
+    const float b2 = __shfl_xor_sync(0xffffffffu, best, o);
+    const int bi2 = __shfl_xor_sync(0xffffffffu, bidx, o);
+    merge_best(best, bidx, b2, bi2);
+  }
+  __shared__ RowPartial red[RP_THREADS / 32];
+  const int w = threadIdx.x >> 5;
+  if ((threadIdx.x & 31) == 0) red[w] = RowPartial{m, s, q, amax, aidx, best, bidx, 0};
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    RowPartial r = red[0];
+    for (int i = 1; i < RP_THREADS / 32; ++i) {
+      merge_softmax(r.m, r.s, r.q, red[i].m, red[i].s, red[i].q);
+      merge_best(r.amax, r.aidx, red[i].amax, red[i].aidx);
+      merge_best(r.best, r.bidx, red[i].best, red[i].bidx);
+    }
+    part[blockIdx.x] = r;
+  }
+}
+
+// Grid: B CTAs; blockDim = C rounded up to a multiple of 32 (C <= 1024).
+__global__ void __launch_bounds__(1024) sample_commit_kernel(
+    const float* __restrict__ logits, const RowPartial* __restrict__ part, SampleParams p,
+    int32_t* __restrict__ tok, uint8_t* __restrict__ committed, int32_t* __restrict__ prev_argmax,
+    int32_t* __restrict__ seq_status, int32_t* __restrict__ o_xhat,
+    int32_t* __restrict__ o_argmax, float* __restrict__ o_logconf,
+    float* __restrict__ o_entropy, uint8_t* __restrict__ o_flags) {
+  __shared__ float s_lam[1024];
+  __shared__ uint8_t s_unc[1024];
+  __shared__ float s_red[32];
+  __shared__ int s_flag;
+
+  const int b = blockIdx.x;
+  if (seq_status[b] != 0) return;
+  const int i = threadIdx.x;
+  const bool live = i < p.C;
+  const int step = read_step(p);
+  const float T = step_temperature(step, p.max_steps, p.t_start, p.t_end);
+  const float k2 = 1.4426950408889634f / T;
+  const size_t row = static_cast<size_t>(b) * p.C + i;
+
+  float lam = 0.f, ent = 0.f;
+  int amax_i = -1, xhat = 0, cur = 0;
+  bool was_committed = true;
+  if (live) {
+    const RowPartial* pr = part + row * p.nchunk;
+    float m = pr[0].m, s = pr[0].s, q = pr[0].q, av = pr[0].amax, bv = pr[0].best;
+    int ai = pr[0].aidx, bi = pr[0].bidx;
+    for (int c = 1; c < p.nchunk; ++c) {
+      merge_softmax(m, s, q, pr[c].m, pr[c].s, pr[c].q);
+      merge_best(av, ai, pr[c].amax, pr[c].aidx);
+      merge_best(bv, bi, pr[c].best, pr[c].bidx);
+    }
+    const float l2s = log2f(s);
+    const float lse2 = m + l2s;                          // log2-domain logsumexp
+    ent = 0.69314718055994531f * (l2s - q / s);           // nats
+    amax_i = ai;
+    xhat = bi;
+    cur = tok[row];
+    was_committed = committed[row] != 0;
+    int x = was_committed ? cur : xhat;
+    if (x < 0 || x >= p.V) {
+      raise_error(ERR_CHECK | 0x501, static_cast<uint32_t>(row));
+      x = 0;
+    }
+    const float zl = logits[row * p.V + x] * k2;
+    lam = (zl - lse2) * 0.69314718055994531f;             // natural log confidence
+  }
+
+  // mean entropy (fixed-order reduction), same-prediction test, uncommitted count
+  float hs = live ? ent : 0.f;
+  hs = warp_sum(hs);
+  if ((i & 31) == 0) s_red[i >> 5] = hs;
+  const bool same = !live || (amax_i == prev_argmax[live ? row : 0]);
+  const int all_same = __syncthreads_and(same);
+  const int n_unc = __syncthreads_count(live && !was_committed);
+  if (i == 0) {
+    float tot = 0.f;
+    for (int w = 0; w < (blockDim.x + 31) / 32; ++w) tot += s_red[w];
+    const float mean_h = tot / static_cast<float>(p.C);
+    const bool crit = (mean_h < p.stop_entropy) && step >= 1 && all_same;
+    const bool cap = step >= p.max_steps - 1;
+    s_flag = (crit || cap) ? 1 : 0;
+  }
+  if (live) {
+    s_lam[i] = lam;
+    s_unc[i] = was_committed ? 0 : 1;
+  }
+  __syncthreads();
+  const bool final_step = s_flag != 0;
+
+  // top-k among uncommitted: rank = number of uncommitted positions that beat this one
+  bool selected = false;
+  if (live && !was_committed) {
+    const int k = min(p.commit_k, n_unc);
+    int rank = 0;
+    for (int j = 0; j < p.C; ++j) {
+      if (s_unc[j]) {
+        const float lj = s_lam[j];
+        rank += (lj > lam || (lj == lam && j < i)) ? 1 : 0;
+      }
+    }
+    selected = rank < k;
+  }
+
+  int new_tok = cur;
+  bool new_comm = was_committed;
+  uint8_t flags = 0;
+  if (live) {
+    if (final_step) {
+      if (!was_committed) {
+        new_tok = xhat;
+        flags |= 1;
+      }
+      new_comm = true;
+    } else if (selected) {
+      new_tok = xhat;
+      new_comm = true;
+      flags |= 1;
+    } else if (was_committed) {
+      if (lam < p.log_tau) {
+        new_tok = token_from_word(
+            position_word(p.seed, b, p.block, step, i, kTagRenoise), p.V);
+        new_comm = false;
+        flags |= 2;
+      }
+    } else {
+      new_tok = (p.policy == 0) ? xhat
+                                : token_from_word(position_word(p.seed, b, p.block, step, i,
+                                                                kTagRenoise),
+                                                  p.V);
+    }
+    tok[row] = new_tok;
+    committed[row] = new_comm ? 1 : 0;
+    prev_argmax[row] = amax_i;
+    if (o_xhat) o_xhat[row] = xhat;
+    if (o_argmax) o_argmax[row] = amax_i;
+    if (o_logconf) o_logconf[row] = lam;
+    if (o_entropy) o_entropy[row] = ent;
+    if (o_flags) o_flags[row] = flags;
+  }
+  const int all_comm = __syncthreads_and(!live || new_comm);
+  if (i == 0 && (final_step || all_comm)) seq_status[b] = step + 1;
+}
+
+// Fresh canvas: uniform tokens (tag INIT), nothing committed, no prediction yet.
+__global__ void init_canvas_kernel(int B, int C, int V, uint32_t seed, int block,
+                                   int32_t* __restrict__ tok, uint8_t* __restrict__ committed,
+                                   int32_t* __restrict__ prev_argmax,
+                                   int32_t* __restrict__ seq_status, int32_t* __restrict__ step) {
+  const int b = blockIdx.x;
+  for (int i = threadIdx.x; i < C; i += blockDim.x) {
+    const size_t row = static_cast<size_t>(b) * C + i;
+    tok[row] = token_from_word(position_word(seed, b, block, 0, i, kTagInit), V);
+    committed[row] = 0;
+    prev_argmax[row] = -1;
+  }
+  if (threadIdx.x == 0) seq_status[b] = 0;
+  if (b == 0 && threadIdx.x == 0 && step) *step = 0;
+}
+
+// After a step: advance the step counter and publish whether any sequence runs on.
+__global__ void step_advance_kernel(int B, int max_steps, const int32_t* __restrict__ seq_status,
+                                    int32_t* __restrict__ step, int32_t* __restrict__ running) {
+  int n = 0;
+  for (int b = threadIdx.x; b < B; b += blockDim.x) n += (seq_status[b] == 0) ? 1 : 0;
+  n = __syncthreads_count(n > 0);
+  if (threadIdx.x == 0) {
+    const int s = *step + 1;
+    *step = s;
+    *running = (n > 0 && s < max_steps) ? 1 : 0;
+  }
+}
+
+__global__ void philox_kernel(const uint32_t* __restrict__ in, uint32_t* __restrict__ out,
+                              int n) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const uint32_t* a = in + static_cast<size_t>(i) * 6;
+  const uint4 r = philox4x32_10(make_uint4(a[0], a[1], a[2], a[3]), make_uint2(a[4], a[5]));
+  uint32_t* o = out + static_cast<size_t>(i) * 4;
+  o[0] = r.x;
+  o[1] = r.y;
+  o[2] = r.z;
+  o[3] = r.w;
+}
+
+}  // namespace dg

@@ -1,0 +1,298 @@
+/*
+ * dg.h - C ABI of the B200 canvas-denoising library (libdg.so).
+ *
+ * The library runs the block-autoregressive discrete-diffusion denoising step
+ * of a DiffusionGemma-style model on one NVIDIA B200 (sm_100a):
+ *   - a 256-token canvas attends bidirectionally to itself and to the causal
+ *     KV cache of the committed prefix,
+ *   - is projected to vocabulary logits,
+ *   - is resampled (Philox-keyed Gumbel-max under a linear 0.8 -> 0.4
+ *     temperature schedule, top-k commit, threshold re-noise, adaptive stop),
+ *   - and, once stopped, has its K/V appended to the cache.
+ * Sources: "DiffusionGemma Guia do Desenvolvedor para Decodificacao Paralela a
+ * 1000+ Tokens/s", sections "Difusao de Estado Uniforme" and "Block
+ * Autoregressive Diffusion para Sequencias Longas"; aiexpert.news "Google's
+ * DiffusionGemma Atinge 1.000 Tokens por Segundo", architecture paragraph;
+ * Google docs page "DiffusionGemma", bullet "Arquitetura de
+ * codificador-decodificador" and table "Configuracao de exibicao recomendada".
+ *
+ * Conventions (all entry points):
+ *   - Every function returns an int status (enum dg_status).  DG_OK is 0.
+ *     dg_status_string() names a status; dg_last_error() gives a
+ *     thread-local detail message for the last failure in this thread.
+ *   - No C++ exception crosses this boundary.
+ *   - Ownership: the caller allocates and owns every device buffer.  The
+ *     library never allocates device memory.  Scratch space comes from a
+ *     caller-supplied workspace whose size the *_workspace_bytes() queries
+ *     return.  Host arrays passed in (pointer tables, structs) are read during
+ *     the call only.
+ *   - All device work is enqueued on the caller's stream (a cudaStream_t passed
+ *     as void*; NULL is the legacy default stream) and is asynchronous, except
+ *     where a function says it synchronises.  Results are deterministic: the
+ *     same inputs and seed give the same bits.
+ *   - Argument errors (null pointers, unsupported shapes, misalignment, a too
+ *     small workspace) are detected on the host before any launch and return
+ *     an error with nothing enqueued.
+ *   - Errors found on the device (a bounded wait that expired, a device-side
+ *     bounds check) set a per-device error word instead of faulting.
+ *     dg_check_device_errors() synchronises the stream, reads and clears it.
+ *   - Device pointers must be 16-byte aligned; matrices are row-major with the
+ *     last dimension contiguous.  bf16 means IEEE bfloat16.
+ */
+#ifndef DG_H_
+#define DG_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum dg_status {
+  DG_OK = 0,
+  DG_ERR_INVALID_ARG = 1,
+  DG_ERR_UNSUPPORTED_SHAPE = 2,
+  DG_ERR_ALIGNMENT = 3,
+  DG_ERR_WORKSPACE_TOO_SMALL = 4,
+  DG_ERR_CUDA = 5,
+  DG_ERR_TIMEOUT = 6,
+  DG_ERR_DEVICE_CHECK = 7
+};
+
+/* Attention key masks over [cached prefix ; new rows]. */
+enum dg_mask_mode {
+  DG_MASK_BIDIR = 0,  /* denoising canvas: every prefix key and every new row */
+  DG_MASK_CAUSAL = 1  /* prefill / block re-encode: every prefix key, new rows j <= i */
+};
+
+/* What happens to uncommitted positions that are not selected in a step. */
+enum dg_unselected_policy {
+  DG_UNSELECTED_KEEP = 0,    /* take the step's sample, stay uncommitted (default) */
+  DG_UNSELECTED_RENOISE = 1  /* take a fresh uniform token, stay uncommitted */
+};
+
+/* Epilogues of dg_linear. */
+enum dg_epilogue {
+  DG_EPI_F32 = 0,        /* out fp32 [M,N] = x w^T */
+  DG_EPI_BF16 = 1,       /* out bf16 [M,N] = x w^T */
+  DG_EPI_GELU_BF16 = 2,  /* out bf16 [M,N] = gelu_erf(x w^T) */
+  DG_EPI_RESID_F32 = 3   /* out fp32 [M,N] += x w^T (residual add in place) */
+};
+
+typedef struct dg_model_cfg {
+  int d;           /* model width */
+  int n_layers;
+  int n_q_heads;   /* Hq */
+  int n_kv_heads;  /* Hkv; Hq % Hkv == 0; query head h reads kv head h / (Hq/Hkv) */
+  int head_dim;    /* hd in {64, 128} */
+  int ffn;         /* MLP width F */
+  int vocab;       /* V, a multiple of 128 */
+  float eps;       /* RMSNorm epsilon (the gain is 1) */
+} dg_model_cfg;
+
+/* One layer's bf16 weights, [out_features, in_features] row-major. */
+typedef struct dg_layer_weights {
+  const void* w_qkv;   /* [(Hq + 2 Hkv) hd, d], rows [Q heads | K heads | V heads] */
+  const void* w_o;     /* [d, Hq hd] */
+  const void* w_up;    /* [F, d] */
+  const void* w_down;  /* [d, F] */
+} dg_layer_weights;
+
+typedef struct dg_model {
+  dg_model_cfg cfg;
+  const void* embed;                /* bf16 [V, d] */
+  const void* unembed;              /* bf16 [V, d] (untied) */
+  const dg_layer_weights* layers;   /* host array of cfg.n_layers entries */
+} dg_model;
+
+/* Sampler settings.  dg_sampler_defaults() fills the published values. */
+typedef struct dg_sampler_cfg {
+  int max_steps;        /* step cap per canvas (48) */
+  float t_start;        /* temperature at step 0 (0.8) */
+  float t_end;          /* temperature at step max_steps-1 (0.4) */
+  int commit_k;         /* positions committed per step (16) */
+  float renoise_conf;   /* re-noise committed tokens whose softmax confidence is below (0.05) */
+  float stop_entropy;   /* adaptive stop: mean canvas entropy below, in nats (0.005) */
+  int unselected_policy;/* enum dg_unselected_policy */
+} dg_sampler_cfg;
+
+/* Per-step sampler diagnostics: caller-owned device arrays [B, C]; any may be NULL. */
+typedef struct dg_step_out {
+  int32_t* x_hat;     /* the Gumbel-max sample of each position */
+  int32_t* argmax;    /* argmax of the raw logits (the step's "prediction") */
+  float* logconf;     /* log softmax confidence (tempered) of the token at stake */
+  float* entropy;     /* tempered entropy, nats */
+  uint8_t* flags;     /* bit0: committed this step, bit1: re-noised this step */
+} dg_step_out;
+
+/*
+ * Generation state of a batch of B sequences.  All pointers are device
+ * pointers owned by the caller, except the two host pointer tables.
+ */
+typedef struct dg_state {
+  int batch;              /* B */
+  int lmax;               /* cache capacity in rows */
+  int canvas;             /* C, the canvas length (256) */
+  int cache_len_host;     /* host mirror of the cache length, equal for every sequence */
+  void* const* k_cache;   /* host table [n_layers] of bf16 [B, Hkv, lmax, hd] */
+  void* const* v_cache;   /* host table [n_layers] of bf16 [B, Hkv, lmax, hd] */
+  int32_t* cache_len;     /* [B] rows of the cache in use */
+  int32_t* tok;           /* [B, C] canvas tokens */
+  uint8_t* committed;     /* [B, C] 1 = committed */
+  int32_t* prev_argmax;   /* [B, C] previous step's prediction (-1: none) */
+  int32_t* seq_status;    /* [B] 0 = running; s + 1 once stopped after step s */
+  int32_t* step;          /* [1] current step index of the canvas */
+} dg_state;
+
+const char* dg_status_string(int status);
+const char* dg_last_error(void);
+int dg_version(void);
+void dg_sampler_defaults(dg_sampler_cfg* cfg);
+
+/* Synchronise `stream`, read and clear the device error word.
+ * Returns DG_OK, DG_ERR_TIMEOUT (a bounded wait expired) or DG_ERR_DEVICE_CHECK
+ * (a device-side bounds check failed); *code_out (may be NULL) gets the raw word. */
+int dg_check_device_errors(void* stream, uint32_t* code_out);
+
+/*
+ * dg_canvas_attn - grouped-query attention of Lq new rows over
+ * [cached prefix ; new rows] (the canvas attention of the denoising step, and
+ * the causal attention of prefill and block re-encode).
+ * Source: aiexpert.news architecture paragraph (bidirectional attention on the
+ * canvas, causal prefill into the KV cache); Guia do Desenvolvedor, bullet
+ * "Propagacao de Contexto Bidirecional".
+ *   out[b,i,h,:] = softmax_j(q[b,i,h,:] . key_j * scale) value_j over keys
+ *   j in { prefix rows 0..cache_len[b]-1 of kv head g } U { new rows allowed
+ *   by mask_mode }, g = h / (Hq/Hkv).  No positional encoding.
+ * Layouts (bf16):
+ *   q      [B, Lq, ldq]    head h at columns h*hd .. h*hd+hd-1
+ *   k_new, v_new [B, Lq, ldkv]  kv head g at columns g*hd
+ *   k_cache, v_cache [B, Hkv, lmax, hd]
+ *   out    [B, Lq, ldo]    head h at columns h*hd
+ *   lse    fp32 [B, Hq, Lq] natural-log sum of exp of the scaled scores (may be NULL)
+ *   cache_len: device [B]; every value must be <= max_prefix (host bound used
+ *   to plan the split over keys).
+ * Requires hd in {64,128}, Hq % Hkv == 0, Lq >= 1, lmax >= max_prefix,
+ * ldq/ldkv/ldo multiples of 8.  Workspace: dg_canvas_attn_workspace_bytes().
+ */
+int dg_canvas_attn(const void* q, int ldq, const void* k_new, const void* v_new, int ldkv,
+                   const void* k_cache, const void* v_cache, const int32_t* cache_len,
+                   int max_prefix, int lmax, void* out, int ldo, float* lse,
+                   int B, int Hq, int Hkv, int Lq, int hd, float scale, int mask_mode,
+                   void* workspace, size_t workspace_bytes, void* stream);
+size_t dg_canvas_attn_workspace_bytes(int B, int Hq, int Hkv, int Lq, int hd, int max_prefix);
+
+/*
+ * dg_unembed - vocabulary logits of the normalised final hidden states (the
+ * "diffusion head" of aiexpert.news architecture paragraph; untied).
+ *   logits[m, v] = sum_k h[m, k] w_u[v, k]
+ * h bf16 [M, d]; w_u bf16 [V, d]; logits fp32 [M, V].  V % 128 == 0,
+ * d % 64 == 0.  Needs no workspace (pass NULL, 0).
+ */
+int dg_unembed(const void* h, const void* w_u, float* logits, int M, int d, int V,
+               void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * dg_linear - the layer projections of the stack (QKV, output, MLP up/down):
+ *   y[m, n] = sum_k x[m, k] w[n, k], then the epilogue (enum dg_epilogue).
+ * x bf16 [M, K]; w bf16 [N, K]; out per epilogue.  N % 128 == 0, K % 64 == 0.
+ * Workspace: dg_linear_workspace_bytes() (split-K partial sums).
+ */
+int dg_linear(const void* x, const void* w, void* out, int M, int N, int K, int epilogue,
+              void* workspace, size_t workspace_bytes, void* stream);
+size_t dg_linear_workspace_bytes(int M, int N, int K);
+
+/*
+ * dg_sample_commit - one sampler step over logits [B, C, V] fp32.
+ * Source: Google docs table "Configuracao de exibicao recomendada" (step cap,
+ * linear temperature schedule, adaptive stop on entropy + two identical
+ * predictions); aiexpert.news architecture paragraph (confident tokens locked
+ * per pass, low-confidence positions re-noised); Guia do Desenvolvedor bullet
+ * "Correcao de Erros via Re-Noising".
+ * Per position, with T = t_start + (t_end - t_start) * step / (max_steps - 1)
+ * and z = logits / T: entropy of softmax(z); argmax of the raw logits; the
+ * Gumbel-max sample x_hat = argmax(z + g), g = -ln(-ln u), u from
+ * Philox4x32-10 keyed (seed, b) with counter (v >> 2, pos | 0 << 24, step,
+ * block), word v & 3, u = (2 (r >> 9) + 1) 2^-24; log confidence
+ * lambda = z[x] - logsumexp(z) (x = x_hat if uncommitted, else the current token).
+ * Then: commit the min(k, #uncommitted) uncommitted positions of largest
+ * lambda (ties to the lower position) to x_hat; re-noise committed positions
+ * with lambda < ln(renoise_conf) to a uniform token (Philox tag 1, counter
+ * (0, pos | 1 << 24, step, block), token = (r * V) >> 32) and uncommit them;
+ * unselected uncommitted positions follow unselected_policy.  Stop when every
+ * position is committed, or when mean entropy < stop_entropy and the argmax
+ * equals the previous step's everywhere (step >= 1), or at step max_steps - 1;
+ * the latter two commit every remaining position to x_hat and skip re-noise.
+ * In/out (device): tok, committed, prev_argmax [B, C]; seq_status [B]
+ * (sequences with a nonzero status are left untouched).  out may be NULL.
+ * C <= 1024, V % 4 == 0.  Workspace: dg_sample_commit_workspace_bytes().
+ */
+int dg_sample_commit(const float* logits, int32_t* tok, uint8_t* committed,
+                     int32_t* prev_argmax, int32_t* seq_status, const dg_sampler_cfg* cfg,
+                     uint32_t seed, int block, int step, int B, int C, int V,
+                     const dg_step_out* out, void* workspace, size_t workspace_bytes,
+                     void* stream);
+size_t dg_sample_commit_workspace_bytes(int B, int C, int V);
+
+/*
+ * dg_kv_block_commit - append a finished block's per-layer K/V to the cache
+ * ("Guia do Desenvolvedor", Denoising bullet: when finished, the block is
+ * committed to the KV cache and the next one starts).
+ * For each layer l, sequence b, kv head g, row t < C:
+ *   k_cache[l][b, g, cache_len[b] + t, :] = k_blk[l][(b*C + t)*ld_blk + g*hd ...]
+ * (same for v), then cache_len[b] += C.  Tables k_blk, v_blk, k_cache,
+ * v_cache are host arrays of n_layers device pointers (n_layers <= 128).
+ * A sequence with cache_len[b] + C > lmax is skipped and the device error
+ * word records DG_ERR_DEVICE_CHECK.
+ */
+int dg_kv_block_commit(const void* const* k_blk, const void* const* v_blk, int ld_blk,
+                       void* const* k_cache, void* const* v_cache, int32_t* cache_len,
+                       int n_layers, int B, int Hkv, int C, int hd, int lmax, void* stream);
+
+/*
+ * dg_prefill - causal pass of prompts [B, P] (device int32) through the
+ * model; writes their K/V to cache rows [0, P) and sets cache_len to P
+ * (and st->cache_len_host).  Workspace: dg_prefill_workspace_bytes().
+ */
+int dg_prefill(const dg_model* m, dg_state* st, const int32_t* prompt, int P,
+               void* workspace, size_t workspace_bytes, void* stream);
+size_t dg_prefill_workspace_bytes(const dg_model_cfg* cfg, int B, int P);
+
+/*
+ * dg_denoise_logits - one bidirectional forward of the current canvas
+ * (embedding, layers, final norm, unembedding) over the cached prefix, into
+ * logits fp32 [B, C, V].  The building block of dg_denoise_block, exposed for
+ * parity tests.  Workspace: dg_denoise_block_workspace_bytes().
+ */
+int dg_denoise_logits(const dg_model* m, const dg_state* st, float* logits,
+                      void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * dg_denoise_block - denoise one canvas per sequence to its adaptive stop,
+ * re-encode it causally and commit its K/V (cache_len += C).
+ * Initialises the canvas with uniform tokens (Philox tag 2, counter
+ * (0, pos | 2 << 24, 0, block)), runs sampler steps until every sequence has
+ * stopped (dg_sample_commit semantics), then the causal re-encode and the
+ * block commit.  Synchronises `stream` once per step to read the stop state.
+ * steps_taken (host, may be NULL) receives the largest step count over the batch.
+ * Workspace: dg_denoise_block_workspace_bytes().
+ */
+int dg_denoise_block(const dg_model* m, dg_state* st, const dg_sampler_cfg* cfg, uint32_t seed,
+                     int block, int* steps_taken, void* workspace, size_t workspace_bytes,
+                     void* stream);
+size_t dg_denoise_block_workspace_bytes(const dg_model_cfg* cfg, int B, int C, int lmax);
+
+/*
+ * dg_philox4x32_10 - n independent Philox4x32-10 blocks (Salmon et al., SC'11),
+ * exposed so that the device generator can be checked against known answers.
+ * in: device uint32 [n, 6] = counter words c0..c3 then key words k0, k1;
+ * out: device uint32 [n, 4].
+ */
+int dg_philox4x32_10(const uint32_t* in, uint32_t* out, int n, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DG_H_ */
