@@ -1,0 +1,416 @@
+"""Benchmark: committed tokens/s of the block-autoregressive denoising path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload full|tiny] [--impl reference]
+
+A step is one denoised block per sequence: canvas initialisation, denoising
+steps to the adaptive stop (a random-weight model never reaches the entropy
+stop, so every block runs the 48-step cap), the causal re-encode and the KV
+block commit.  The prompt prefill is outside the timed region, as in the
+metric; the cache length is reset to the prompt length before every step.
+
+Reported (one JSON line from rank 0):
+  value        committed tokens/s over all ranks (each rank an independent
+               replica with its own seed: the path has no data-path exchange)
+  e2e          the same metric through the public API with the prompt copied
+               from pinned host memory and the block's tokens copied back every
+               step (prefill inside the timed region)
+  roofline     the dominant kernel's achieved throughput against the measured peak
+  cpu_baseline the CPU oracle on a bounded sample of the same workload
+With --impl reference the CPU oracle itself is timed on that workload.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "committed tokens/s (B=1, 256-tok canvas)"
+UNIT = "tokens/s"
+CANVAS = 256
+L2_BYTES = 126 * 1024 * 1024
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def workload_spec(name):
+    from canvas_denoising_denoise_b200 import synth
+    w = synth.WORKLOADS[name]
+    return w["model"], w["batch"], w["prompt"]
+
+
+def time_region(fn, steps, stream):
+    import torch
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(steps):
+        fn()
+    end.record(stream)
+    torch.cuda.synchronize()
+    return start.elapsed_time(end) / 1000.0
+
+
+def gemm_roofline(dg, model, shape, batch, peaks, stream):
+    """Achieved TFLOP/s of the tcgen05 GEMM kernel on the unembedding launch.
+
+    The unembedding (M = B*256 tokens, N = vocab, K = d) is the largest single
+    launch of a denoising step; it is timed alone with CUDA events on the
+    benchmark stream, with a buffer larger than L2 written between launches.
+    """
+    import torch
+    M, d, V = batch * CANVAS, shape.d, shape.vocab
+    h = torch.randn((M, d), device="cuda").to(torch.bfloat16)
+    logits = torch.empty((M, V), dtype=torch.float32, device="cuda")
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+    times = []
+    for i in range(8):
+        flush.fill_(float(i))
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        dg.unembed(h, model.w["unembed"], logits, stream=stream)
+        e.record(stream)
+        torch.cuda.synchronize()
+        if i >= 2:
+            times.append(s.elapsed_time(e) / 1000.0)
+    t = statistics.median(times)
+    flops = 2.0 * M * V * d
+    achieved = flops / t / 1e12
+    peak = peaks["bf16_tflops"]
+    return {"kernel": "gemm_kernel (unembedding launch)", "bound": "tensor",
+            "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+            "frac": round(achieved / peak, 4), "traffic": None,
+            "peak_source": f"{peaks['source']} burst bf16",
+            "launch_us": round(t * 1e6, 1), "flops_per_launch": flops}
+
+
+def attn_roofline(dg, shape, batch, prefix, peaks, stream):
+    """Achieved TFLOP/s of canvas attention at the workload's prefix length."""
+    import torch
+    from canvas_denoising_denoise_b200 import synth
+    hq, hkv, hd = shape.n_q_heads, shape.n_kv_heads, shape.head_dim
+    q, kn, vn, kc, vc = synth.make_attn_inputs(batch, hq, hkv, hd, CANVAS, prefix, seed=0,
+                                               device="cuda")
+    cl = torch.full((batch,), prefix, dtype=torch.int32, device="cuda")
+    out = torch.empty((batch, CANVAS, hq * hd), dtype=torch.bfloat16, device="cuda")
+    times = []
+    for i in range(10):
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        dg.canvas_attn(q, kn, vn, kc, vc, cl, prefix, out, n_q_heads=hq, n_kv_heads=hkv,
+                       head_dim=hd, stream=stream)
+        e.record(stream)
+        torch.cuda.synchronize()
+        if i >= 3:
+            times.append(s.elapsed_time(e) / 1000.0)
+    t = statistics.median(times)
+    flops = 4.0 * batch * hq * CANVAS * (prefix + CANVAS) * hd
+    achieved = flops / t / 1e12
+    return {"achieved": round(achieved, 1), "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+            "frac": round(achieved / peaks["bf16_tflops"], 4), "us": round(t * 1e6, 1),
+            "prefix": prefix}
+
+
+def cpu_baseline_sample(w_cpu, shape, prefix, budget_s=30.0):
+    """The CPU oracle on one denoising step of the workload (bounded sample).
+
+    The sample is one bidirectional forward of a 256-token canvas over a
+    `prefix`-row cache plus one sampler step; the cache rows are seeded noise
+    (the oracle's own prefill of a 4096-token prompt would take far longer and
+    is outside the metric anyway).  Tokens/s is extrapolated to a 48-step
+    block with one re-encode pass.
+    """
+    import numpy as np
+    import torch
+    from oracle import model as M
+    from oracle import sampler as S
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count()
+    ocfg = M.ModelCfg(shape.d, shape.n_layers, shape.n_q_heads, shape.n_kv_heads,
+                      shape.head_dim, shape.ffn, shape.vocab, shape.eps)
+    w64 = M.weights_to_f64(w_cpu)
+    g = torch.Generator().manual_seed(5)
+    kc = [torch.randn((shape.n_kv_heads, prefix, shape.head_dim), generator=g).double().numpy()
+          for _ in range(shape.n_layers)]
+    vc = [torch.randn((shape.n_kv_heads, prefix, shape.head_dim), generator=g).double().numpy()
+          for _ in range(shape.n_layers)]
+    tok = S.init_canvas(0, 0, 0, CANVAS, shape.vocab)
+    t0 = time.perf_counter()
+    logits = M.denoise_logits(ocfg, w64, tok, kc, vc, prefix)
+    t_fwd = time.perf_counter() - t0
+    t1 = time.perf_counter()
+    S.sampler_step(S.SamplerCfg(), logits.astype(np.float32), tok, np.zeros(CANVAS, bool), None,
+                   0, 0, 0, 0)
+    t_smp = time.perf_counter() - t1
+    block_s = 48 * (t_fwd + t_smp) + t_fwd
+    return {"value": round(CANVAS / block_s, 4), "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": (f"1 of 48 denoising steps (forward {t_fwd:.1f} s + sampler {t_smp:.1f} s) "
+                       f"at prefix {prefix}, extrapolated to a 48-step block + re-encode; "
+                       f"prefill excluded as in the metric")}
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle timed on the same workload (rank 0 only)."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    import torch
+    from canvas_denoising_denoise_b200 import synth
+    shape, batch, prompt = workload_spec(args.workload)
+    if args.workload == "tiny":
+        w_cpu = synth.make_weights(shape, seed=0)
+    else:
+        w_cpu = synth.make_weights_fast(shape, seed=0, device="cuda" if torch.cuda.is_available()
+                                        else "cpu")
+        w_cpu = {"embed": w_cpu["embed"].cpu(), "unembed": w_cpu["unembed"].cpu(),
+                 "layers": [{k: v.cpu() for k, v in lw.items()} for lw in w_cpu["layers"]]}
+    vals = []
+    for _ in range(max(1, args.steps)):
+        vals.append(cpu_baseline_sample(w_cpu, shape, prompt))
+    v = statistics.median([x["value"] for x in vals])
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(CANVAS / v * 1e3, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "batch": batch, "prompt": prompt,
+                       "canvas": CANVAS},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": vals[0]["cores"],
+                             "kind": "oracle", "sample": vals[0]["sample"]},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="full", choices=["full", "tiny"])
+    ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    import canvas_denoising_denoise_b200 as dg
+    from canvas_denoising_denoise_b200 import synth
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    lib = dg._lib.load()
+    shape, batch, prompt_len = workload_spec(args.workload)
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream()
+
+    # ---------------------------------------------------------------- set-up
+    if args.workload == "tiny":
+        w_cpu = synth.make_weights(shape, seed=0)
+        weights = {"embed": w_cpu["embed"].cuda(), "unembed": w_cpu["unembed"].cuda(),
+                   "layers": [{k: v.cuda() for k, v in lw.items()} for lw in w_cpu["layers"]]}
+    else:
+        weights = synth.make_weights_fast(shape, seed=0, device="cuda")
+    model = dg.DgModel(shape, weights)
+    lmax = prompt_len + CANVAS
+    st = dg.DgState(shape, batch, lmax, CANVAS)
+    prompt = synth.make_prompt(batch, prompt_len, shape.vocab, seed=1 + rank).cuda()
+    ws = dg.Workspace()
+    ws.get(max(dg.denoise_workspace_bytes(model, st),
+               lib.dg_prefill_workspace_bytes(ctypes_ref(model.cfg), batch, prompt_len)))
+    dg.prefill(model, st, prompt, ws=ws)
+    torch.cuda.synchronize()
+    dg.check_device_errors()
+    settings = dg.SamplerSettings()
+    seed = 1000 + rank
+    steps_seen = []
+
+    def block_step():
+        st.cache_len.fill_(prompt_len)
+        st.cache_len_host = prompt_len
+        steps_seen.append(dg.denoise_block(model, st, settings, seed, 0, ws=ws))
+
+    for _ in range(args.warmup):
+        block_step()
+    torch.cuda.synchronize()
+    dg.check_device_errors()
+
+    # ---------------------------------------------------------------- timed
+    clocks = ClockSampler(torch.cuda.current_device())
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    n0 = lib.dg_launch_count()
+    steps_seen.clear()
+    elapsed = time_region(block_step, args.steps, stream)
+    launches = lib.dg_launch_count() - n0
+    clk = clocks.stop()
+    if world > 1:
+        t = torch.tensor([elapsed], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        elapsed = float(t.item())
+        dist.barrier()
+    dg.check_device_errors()
+    tokens = world * batch * CANVAS * args.steps
+    value = tokens / elapsed
+
+    # ---------------------------------------------------------------- end to end
+    host_prompt = synth.make_prompt(batch, prompt_len, shape.vocab, seed=1 + rank).pin_memory()
+    host_out = torch.empty((batch, CANVAS), dtype=torch.int32).pin_memory()
+    dev_prompt = torch.empty_like(prompt)
+
+    def e2e_step():
+        dev_prompt.copy_(host_prompt, non_blocking=True)
+        dg.prefill(model, st, dev_prompt, ws=ws)
+        dg.denoise_block(model, st, settings, seed, 0, ws=ws)
+        host_out.copy_(st.tok, non_blocking=True)
+
+    e2e_step()
+    if world > 1:
+        dist.barrier()
+    e2e_t = time_region(e2e_step, max(1, args.steps // 2), stream)
+    if world > 1:
+        t = torch.tensor([e2e_t], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_t = float(t.item())
+    e2e_val = world * batch * CANVAS * max(1, args.steps // 2) / e2e_t
+
+    # ---------------------------------------------------------------- roofline
+    roof = gemm_roofline(dg, model, shape, batch, peaks, stream)
+    attn = attn_roofline(dg, shape, batch, prompt_len, peaks, stream)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        w_cpu = {"embed": weights["embed"].cpu(), "unembed": weights["unembed"].cpu(),
+                 "layers": [{k: v.cpu() for k, v in lw.items()} for lw in weights["layers"]]}
+        cpu = cpu_baseline_sample(w_cpu, shape, prompt_len)
+        del w_cpu
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(elapsed / args.steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": args.workload, "model": "random-init dense stand-in",
+                       "batch": batch, "prompt": prompt_len, "canvas": CANVAS,
+                       "d": shape.d, "layers": shape.n_layers, "heads": [shape.n_q_heads,
+                                                                         shape.n_kv_heads],
+                       "head_dim": shape.head_dim, "ffn": shape.ffn, "vocab": shape.vocab,
+                       "steps_per_block": steps_seen[-1] if steps_seen else None,
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (3.3 GB of weights streamed per step)"},
+            "roofline": roof,
+            "canvas_attn": attn,
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_val, 2), "unit": UNIT,
+                    "h2d_bytes_per_step": int(host_prompt.numel() * 4),
+                    "d2h_bytes_per_step": int(host_out.numel() * 4),
+                    "includes": "prompt H2D + prefill + denoised block + tokens D2H"},
+            "gpu_launches": int(launches),
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def ctypes_ref(x):
+    import ctypes
+    return ctypes.byref(x)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

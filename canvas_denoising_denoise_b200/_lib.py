@@ -65,6 +65,7 @@ SIGNATURES = {
     "dg_status_string": (c_char_p, [c_int]),
     "dg_last_error": (c_char_p, []),
     "dg_version": (c_int, []),
+    "dg_launch_count": (ctypes.c_ulonglong, []),
     "dg_sampler_defaults": (None, [P(SamplerCfg)]),
     "dg_check_device_errors": (c_int, [c_void_p, P(c_uint32)]),
     "dg_canvas_attn": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_int, c_void_p, c_void_p,

@@ -10,6 +10,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -26,6 +27,8 @@ constexpr int kVersion = 1;
 constexpr int kNumSMs = 148;
 
 thread_local char g_last_error[512] = "";
+std::atomic<unsigned long long> g_launches{0};
+inline void count_launch(unsigned long long n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
 
 int fail(int status, const char* fmt, ...) {
   va_list ap;
@@ -129,6 +132,7 @@ int launch_gemm(const void* x, const void* w, int M, int N, int K, const GemmPla
   dg::gemm::Params p{M, N, K, pl.kb_per_split, epi, out_f32, out_bf16};
   dim3 grid(N / dg::gemm::BM, cdiv(M, dg::gemm::BN), pl.splits);
   dg::gemm::gemm_kernel<<<grid, dg::gemm::THREADS, dg::gemm::SMEM_BYTES, s>>>(tw, tx, p);
+  count_launch();
   DG_CUDA(cudaGetLastError());
   return DG_OK;
 }
@@ -140,6 +144,7 @@ int launch_reduce(const float* part, int S, int M, int N, int mode, __nv_bfloat1
                                            (size_t)kNumSMs * 8);
   dg::gemm::reduce_kernel<<<std::max(1, blocks), 256, 0, s>>>(part, S, M, N, mode, out_bf16,
                                                                 out_f32);
+  count_launch();
   DG_CUDA(cudaGetLastError());
   return DG_OK;
 }
@@ -160,6 +165,7 @@ int linear(const void* x, const void* w, int M, int N, int K, int mode, void* ou
   if (norm) {
     dg::gemm::add_norm_kernel<<<M, dg::gemm::NORM_THREADS, 0, s>>>(part, pl.splits, M, N, eps,
                                                                     (float*)out, xn_out);
+    count_launch();
     DG_CUDA(cudaGetLastError());
     return DG_OK;
   }
@@ -232,6 +238,7 @@ int launch_attn(const void* q, int ldq, const void* k_new, const void* v_new, in
     }
     dg::attn::attn_kernel<128><<<grid, dg::attn::THREADS, dg::attn::Cfg<128>::SMEM_BYTES, s>>>(
         tq, tkn, tvn, tkc, tvc, p);
+    count_launch();
   } else {
     if (!attn_attr_done[0]) {
       DG_CUDA(cudaFuncSetAttribute(dg::attn::attn_kernel<64>,
@@ -241,6 +248,7 @@ int launch_attn(const void* q, int ldq, const void* k_new, const void* v_new, in
     }
     dg::attn::attn_kernel<64><<<grid, dg::attn::THREADS, dg::attn::Cfg<64>::SMEM_BYTES, s>>>(
         tq, tkn, tvn, tkc, tvc, p);
+    count_launch();
   }
   DG_CUDA(cudaGetLastError());
   if (S > 1) {
@@ -253,6 +261,7 @@ int launch_attn(const void* q, int ldq, const void* k_new, const void* v_new, in
     else
       dg::attn::attn_combine_kernel<64><<<blocks, threads, 0, s>>>(
           p.part_o, p.part_lse, S, B, Hq, Lq, (__nv_bfloat16*)out, ldo, lse);
+    count_launch();
     DG_CUDA(cudaGetLastError());
   }
   return DG_OK;
@@ -303,12 +312,14 @@ int launch_sample(const float* logits, int32_t* tok, uint8_t* committed, int32_t
   dg::RowPartial* part = (dg::RowPartial*)ws;
   dg::sample_rowpass_kernel<<<p.B * p.C * p.nchunk, dg::RP_THREADS, 0, s>>>(logits, seq_status,
                                                                              p, part);
+  count_launch();
   DG_CUDA(cudaGetLastError());
   const int threads = (p.C + 31) / 32 * 32;
   dg::sample_commit_kernel<<<p.B, threads, 0, s>>>(
       logits, part, p, tok, committed, prev_argmax, seq_status, out ? out->x_hat : nullptr,
       out ? out->argmax : nullptr, out ? out->logconf : nullptr, out ? out->entropy : nullptr,
       out ? out->flags : nullptr);
+  count_launch();
   DG_CUDA(cudaGetLastError());
   return DG_OK;
 }
@@ -331,6 +342,7 @@ int launch_kv_commit(const void* const* k_blk, const void* const* v_blk, int ld_
   const size_t total = (size_t)n_layers * 2 * B * Hkv * C * (hd / 8);
   const int blocks = (int)std::min<size_t>((total + 255) / 256, (size_t)kNumSMs * 16);
   dg::kv_commit_kernel<<<std::max(1, blocks), 256, 0, s>>>(tab, p);
+  count_launch();
   DG_CUDA(cudaGetLastError());
   return DG_OK;
 }
@@ -443,6 +455,7 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
 
   dg::gemm::embed_norm_kernel<<<M, dg::gemm::NORM_THREADS, 0, s>>>(
       tok, (const __nv_bfloat16*)f.m->embed, c.vocab, c.d, c.eps, x, xn);
+  count_launch();
   DG_CUDA(cudaGetLastError());
   for (int l = 0; l < c.n_layers; ++l) {
     const dg_layer_weights& w = f.m->layers[l];
@@ -494,6 +507,8 @@ const char* dg_status_string(int status) {
 const char* dg_last_error(void) { return g_last_error; }
 
 int dg_version(void) { return kVersion; }
+
+unsigned long long dg_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 void dg_sampler_defaults(dg_sampler_cfg* cfg) {
   if (!cfg) return;
@@ -639,6 +654,7 @@ int dg_kv_block_commit(const void* const* k_blk, const void* const* v_blk, int l
   DG_TRY(launch_kv_commit(k_blk, v_blk, ld_blk, k_cache, v_cache, cache_len, n_layers, B, Hkv, C,
                           hd, lmax, s));
   dg::cache_len_bump_kernel<<<1, 256, 0, s>>>(cache_len, B, C, lmax);
+  count_launch();
   DG_CUDA(cudaGetLastError());
   return DG_OK;
 }
@@ -659,11 +675,13 @@ int dg_prefill(const dg_model* m, dg_state* st, const int32_t* prompt, int P, vo
     return fail(DG_ERR_WORKSPACE_TOO_SMALL, "dg_prefill: workspace needs %zu bytes", L.total);
   cudaStream_t s = (cudaStream_t)stream;
   dg::cache_len_set_kernel<<<1, 256, 0, s>>>(st->cache_len, st->batch, 0);
+  count_launch();
   DG_CUDA(cudaGetLastError());
   Fwd f{m, st->batch, P, 0, st->lmax, DG_MASK_CAUSAL, st->cache_len, st->k_cache,
         st->v_cache, true, false, (char*)workspace, L};
   DG_TRY(run_forward(f, prompt, nullptr, s));
   dg::cache_len_set_kernel<<<1, 256, 0, s>>>(st->cache_len, st->batch, P);
+  count_launch();
   DG_CUDA(cudaGetLastError());
   st->cache_len_host = P;
   return DG_OK;
@@ -714,6 +732,7 @@ int dg_denoise_block(const dg_model* m, dg_state* st, const dg_sampler_cfg* cfg,
 
   dg::init_canvas_kernel<<<B, 256, 0, s>>>(B, C, V, seed, block, st->tok, st->committed,
                                             st->prev_argmax, st->seq_status, st->step);
+  count_launch();
   DG_CUDA(cudaGetLastError());
   Fwd f{m, B, C, st->cache_len_host, st->lmax, DG_MASK_BIDIR, st->cache_len, st->k_cache,
         st->v_cache, false, true, ws, L};
@@ -725,6 +744,7 @@ int dg_denoise_block(const dg_model* m, dg_state* st, const dg_sampler_cfg* cfg,
                          nullptr, ws + L.spart, s));
     dg::step_advance_kernel<<<1, 256, 0, s>>>(B, cfg->max_steps, st->seq_status, st->step,
                                               running);
+    count_launch();
     DG_CUDA(cudaGetLastError());
     int32_t host_running = 0;
     DG_CUDA(cudaMemcpyAsync(&host_running, running, sizeof(int32_t), cudaMemcpyDeviceToHost, s));
@@ -738,6 +758,7 @@ int dg_denoise_block(const dg_model* m, dg_state* st, const dg_sampler_cfg* cfg,
         st->v_cache, true, false, ws, L};
   DG_TRY(run_forward(r, st->tok, nullptr, s));
   dg::cache_len_bump_kernel<<<1, 256, 0, s>>>(st->cache_len, B, C, st->lmax);
+  count_launch();
   DG_CUDA(cudaGetLastError());
   st->cache_len_host += C;
   if (steps_taken) *steps_taken = steps;
@@ -748,6 +769,7 @@ int dg_philox4x32_10(const uint32_t* in, uint32_t* out, int n, void* stream) {
   if (!in || !out || n < 0) return fail(DG_ERR_INVALID_ARG, "dg_philox4x32_10: bad arguments");
   if (n == 0) return DG_OK;
   dg::philox_kernel<<<cdiv(n, 256), 256, 0, (cudaStream_t)stream>>>(in, out, n);
+  count_launch();
   DG_CUDA(cudaGetLastError());
   return DG_OK;
 }

@@ -259,7 +259,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     bool ok = true;
     for (int i = 0; i < n && ok; ++i) {
       const int sb = i & 1;
-      if (!mbar_wait(&s_full[sb], (i >> 1) & 1, abort_flag, 0x331)) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], (i >> 1) & 1, abort_flag, 0x331))) {
         ok = false;
         break;
       }
@@ -298,16 +298,20 @@ __global__ void __launch_bounds__(THREADS, 1)
         sr[c] = __float_as_uint(v);
         tmax = fmaxf(tmax, v);
       }
-      if (tmax > m + kRescaleThreshold || m == -INFINITY) {
+      // The decision is taken per warp: the TMEM loads/stores below are
+      // warp-collective (.sync.aligned) and must see all 32 lanes.  Lanes whose
+      // own max did not move rescale by exactly 1.
+      const bool want = tmax > m + kRescaleThreshold || m == -INFINITY;
+      if (__any_sync(0xffffffffu, want)) {
         const float m_new = fmaxf(tmax, m);
-        if (i > 0 && m != -INFINITY) {
+        if (i > 0) {
           // O holds PV_0..PV_{i-1}; wait for the last one, then rescale in TMEM
-          if (!mbar_wait(o_done, (i - 1) & 1, abort_flag, 0x332)) {
+          if (!__all_sync(0xffffffffu, mbar_wait(o_done, (i - 1) & 1, abort_flag, 0x332))) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const float f = exp2f(m - m_new);
+          const float f = (m == -INFINITY) ? 0.f : exp2f(m - m_new);
 #pragma unroll
           for (int c = 0; c < HD / 32; ++c) {
             uint32_t o[32];
@@ -344,7 +348,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       tc_fence_before();
       mbar_arrive(&p_full[sb]);
     }
-    if (ok && mbar_wait(o_final, 0, abort_flag, 0x333)) {
+    const bool fin = __all_sync(0xffffffffu, ok && mbar_wait(o_final, 0, abort_flag, 0x333));
+    if (fin) {
       tc_fence_after();
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
       const float lse_nat = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;

@@ -147,7 +147,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // epilogue warps 2..5 -> TMEM lane quarter (warp % 4)
       const int quarter = warp & 3;
       const int f = f0 + quarter * 32 + lane;
-      if (mbar_wait(acc_full, 0, abort_flag, 0x105)) {
+      if (__all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, 0x105))) {
         tc_fence_after();
         const uint32_t taddr = tmem_acc + (static_cast<uint32_t>(quarter * 32) << 16);
         for (int c = 0; c < BN / 32; ++c) {
@@ -159,19 +159,26 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int nt = min(32, p.M - tb);
           if (p.epi == EPI_STORE_F32) {
             float* o = p.out_f32 + (static_cast<size_t>(split) * p.M + tb) * p.N + f;
-            for (int j = 0; j < nt; ++j) o[static_cast<size_t>(j) * p.N] = __uint_as_float(r[j]);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nt) o[static_cast<size_t>(j) * p.N] = __uint_as_float(r[j]);
           } else if (p.epi == EPI_ADD_F32) {
             float* o = p.out_f32 + static_cast<size_t>(tb) * p.N + f;
-            for (int j = 0; j < nt; ++j) o[static_cast<size_t>(j) * p.N] += __uint_as_float(r[j]);
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nt) o[static_cast<size_t>(j) * p.N] += __uint_as_float(r[j]);
           } else if (p.epi == EPI_BF16) {
             __nv_bfloat16* o = p.out_bf16 + static_cast<size_t>(tb) * p.N + f;
-            for (int j = 0; j < nt; ++j)
-              o[static_cast<size_t>(j) * p.N] = __float2bfloat16_rn(__uint_as_float(r[j]));
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nt) o[static_cast<size_t>(j) * p.N] = __float2bfloat16_rn(__uint_as_float(r[j]));
           } else {
             __nv_bfloat16* o = p.out_bf16 + static_cast<size_t>(tb) * p.N + f;
-            for (int j = 0; j < nt; ++j)
-              o[static_cast<size_t>(j) * p.N] =
-                  __float2bfloat16_rn(gelu_erf(__uint_as_float(r[j])));
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < nt)
+                o[static_cast<size_t>(j) * p.N] =
+                    __float2bfloat16_rn(gelu_erf(__uint_as_float(r[j])));
           }
         }
       }

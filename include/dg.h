@@ -148,6 +148,8 @@ typedef struct dg_state {
 const char* dg_status_string(int status);
 const char* dg_last_error(void);
 int dg_version(void);
+/* Number of kernels this library has enqueued since it was loaded (all devices). */
+unsigned long long dg_launch_count(void);
 void dg_sampler_defaults(dg_sampler_cfg* cfg);
 
 /* Synchronise `stream`, read and clear the device error word.
