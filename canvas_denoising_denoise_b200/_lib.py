@@ -82,6 +82,9 @@ SIGNATURES = {
                                  c_uint32, c_int, c_int, c_int, c_int, c_int, P(StepOut),
                                  c_void_p, c_size_t, c_void_p]),
     "dg_sample_commit_workspace_bytes": (c_size_t, [c_int, c_int, c_int]),
+    "dg_sample_commit_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                         P(SamplerCfg), c_uint32, c_int, c_int, c_int, c_int,
+                                         c_int, P(StepOut), c_void_p]),
     "dg_kv_block_commit": (c_int, [P(c_void_p), P(c_void_p), c_int, P(c_void_p), P(c_void_p),
                                    c_void_p, c_int, c_int, c_int, c_int, c_int, c_int, c_void_p]),
     "dg_prefill": (c_int, [P(Model), P(State), c_void_p, c_int, c_void_p, c_size_t, c_void_p]),

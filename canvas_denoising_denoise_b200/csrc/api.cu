@@ -483,6 +483,42 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
   return DG_OK;
 }
 
+// ---------------------------------------------------------------------------
+// dg_sample_commit_noalloc: the sampler step with its scratch in a fixed
+// device array instead of a caller-supplied workspace.
+//
+// For callers that cannot allocate device memory: a plugin whose host
+// application owns every device allocation, or code that enqueues work while
+// a stream is being captured, where cudaMalloc is not allowed.  The row
+// partials live in kNoallocScratchBytes of static device memory that every
+// GPU loading this library keeps until the process exits.  Host code may not
+// hand the array's name to a kernel (in host code it is only a stand-in for
+// the device symbol), so the device address is looked up with
+// cudaGetSymbolAddress once per device, with that device current, on the
+// first call there.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoallocScratchBytes = size_t(4) << 20;  // 4 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+int noalloc_scratch(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  DG_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return fail(DG_ERR_INVALID_ARG, "device ordinal %d >= 64", dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || !p)
+      return fail(DG_ERR_CUDA, "cudaGetSymbolAddress(scratch) failed on device %d: %s", dev,
+                  cudaGetErrorString(e));
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return DG_OK;
+}
+
 }  // namespace
 
 // ===========================================================================
@@ -633,6 +669,33 @@ int dg_sample_commit(const float* logits, int32_t* tok, uint8_t* committed,
     return fail(DG_ERR_WORKSPACE_TOO_SMALL, "dg_sample_commit: workspace needs %zu bytes", need);
   const dg::SampleParams p = make_sample_params(*cfg, seed, block, nullptr, step, B, C, V);
   return launch_sample(logits, tok, committed, prev_argmax, seq_status, p, out, workspace,
+                       (cudaStream_t)stream);
+}
+
+int dg_sample_commit_noalloc(const float* logits, int32_t* tok, uint8_t* committed,
+                             int32_t* prev_argmax, int32_t* seq_status, const dg_sampler_cfg* cfg,
+                             uint32_t seed, int block, int step, int B, int C, int V,
+                             const dg_step_out* out, void* stream) {
+  if (!logits || !tok || !committed || !prev_argmax || !seq_status || !cfg)
+    return fail(DG_ERR_INVALID_ARG, "dg_sample_commit_noalloc: null pointer");
+  if (B <= 0 || C <= 0 || C > 1024 || V <= 0 || V % 4 || step < 0 || block < 0)
+    return fail(DG_ERR_UNSUPPORTED_SHAPE,
+                "dg_sample_commit_noalloc: need C <= 1024, V %% 4 == 0");
+  if (cfg->max_steps < 1 || cfg->commit_k < 0 || !(cfg->t_start > 0.f) || !(cfg->t_end > 0.f) ||
+      (cfg->unselected_policy != 0 && cfg->unselected_policy != 1))
+    return fail(DG_ERR_INVALID_ARG, "dg_sample_commit_noalloc: bad sampler settings");
+  if (!aligned16(logits))
+    return fail(DG_ERR_ALIGNMENT, "dg_sample_commit_noalloc: logits alignment");
+  const size_t need = sample_ws_bytes(B, C, V);
+  if (need > kNoallocScratchBytes)
+    return fail(DG_ERR_UNSUPPORTED_SHAPE,
+                "dg_sample_commit_noalloc: B=%d C=%d V=%d needs %zu bytes of scratch, above the "
+                "fixed %zu; use dg_sample_commit with a workspace",
+                B, C, V, need, kNoallocScratchBytes);
+  void* scratch = nullptr;
+  DG_TRY(noalloc_scratch(&scratch));
+  const dg::SampleParams p = make_sample_params(*cfg, seed, block, nullptr, step, B, C, V);
+  return launch_sample(logits, tok, committed, prev_argmax, seq_status, p, out, scratch,
                        (cudaStream_t)stream);
 }
 

@@ -238,6 +238,29 @@ int dg_sample_commit(const float* logits, int32_t* tok, uint8_t* committed,
 size_t dg_sample_commit_workspace_bytes(int B, int C, int V);
 
 /*
+ * dg_sample_commit_noalloc - dg_sample_commit without a workspace argument.
+ * The paper has no counterpart: this is a library convenience.  It serves
+ * callers that cannot allocate device memory - a plugin whose host owns every
+ * device allocation, or code enqueueing work during stream capture, where
+ * cudaMalloc is not permitted.  Its scratch lives in a fixed 4 MiB static
+ * device array that every GPU loading the library keeps until process exit;
+ * nothing is allocated per call (no cudaMalloc, cudaFree or allocating library
+ * routine).  Sizes whose scratch exceeds 4 MiB (dg_sample_commit_workspace_bytes
+ * of B, C, V; e.g. B > 16 at C = 256, V = 262144) return
+ * DG_ERR_UNSUPPORTED_SHAPE.  The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current; make that
+ * first call before any stream capture.  All calls share the one array and it
+ * keeps the last call's contents (every slot read is written earlier in the
+ * same call, so nothing needs clearing); calls that overlap on the GPU - on
+ * different streams, or from different threads - race on it and must be
+ * serialised by the caller.  Arguments and results as dg_sample_commit.
+ */
+int dg_sample_commit_noalloc(const float* logits, int32_t* tok, uint8_t* committed,
+                             int32_t* prev_argmax, int32_t* seq_status, const dg_sampler_cfg* cfg,
+                             uint32_t seed, int block, int step, int B, int C, int V,
+                             const dg_step_out* out, void* stream);
+
+/*
  * dg_kv_block_commit - append a finished block's per-layer K/V to the cache
  * ("Guia do Desenvolvedor", Denoising bullet: when finished, the block is
  * committed to the KV cache and the next one starts).
