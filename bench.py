@@ -262,6 +262,93 @@ def run_reference(args):
     return 0
 
 
+def run_kernel_bench(args):
+    """Single-kernel measurements (CUDA events, warm, L2 flushed between launches).
+
+    --kernel attn     the attention microbench: B=1, Q [32, 256, 128], prefix
+                      K/V [8, L, 128] for L = --prefix (default all of
+                      1024, 4096, 16384, 32768), full mask.
+    --kernel sampler  the sampler sweep: logits [B, 256, 262144] fp32 for
+                      B = --batch, 48 scheduled steps, logits regenerated per
+                      step outside the timed region.
+    --kernel gemm     one projection y = x w^T for --shape M,N,K (bf16 out).
+    """
+    import torch
+    import canvas_denoising_denoise_b200 as dg
+    from canvas_denoising_denoise_b200 import synth
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device="cuda")
+
+    def timed(fn, reps, do_flush=True):
+        ts = []
+        for i in range(reps + 3):
+            if do_flush:
+                flush.fill_(float(i))
+            s = torch.cuda.Event(enable_timing=True)
+            e = torch.cuda.Event(enable_timing=True)
+            s.record(stream)
+            fn()
+            e.record(stream)
+            torch.cuda.synchronize()
+            if i >= 3:
+                ts.append(s.elapsed_time(e) / 1000.0)
+        return statistics.median(ts)
+
+    out = []
+    if args.kernel == "attn":
+        prefixes = [args.prefix] if args.prefix else [1024, 4096, 16384, 32768]
+        B, hq, hkv, hd = 1, 32, 8, 128
+        for L in prefixes:
+            q, kn, vn, kc, vc = synth.make_attn_inputs(B, hq, hkv, hd, CANVAS, L, seed=0,
+                                                       device="cuda")
+            cl = torch.full((B,), L, dtype=torch.int32, device="cuda")
+            o = torch.empty((B, CANVAS, hq * hd), dtype=torch.bfloat16, device="cuda")
+            ws = dg.Workspace()
+            t = timed(lambda: dg.canvas_attn(q, kn, vn, kc, vc, cl, L, o, n_q_heads=hq,
+                                             n_kv_heads=hkv, head_dim=hd, ws=ws), args.steps)
+            fl = 4.0 * B * hq * CANVAS * (L + CANVAS) * hd
+            out.append({"kernel": "canvas_attn", "prefix": L, "us": round(t * 1e6, 2),
+                        "tflops": round(fl / t / 1e12, 1),
+                        "frac_bf16_peak": round(fl / t / 1e12 / peaks["bf16_tflops"], 4)})
+    elif args.kernel == "sampler":
+        B, V = args.batch, 262144
+        settings = dg.SamplerSettings()
+        tok = torch.zeros((B, CANVAS), dtype=torch.int32, device="cuda")
+        com = torch.zeros((B, CANVAS), dtype=torch.uint8, device="cuda")
+        prev = torch.full((B, CANVAS), -1, dtype=torch.int32, device="cuda")
+        stat = torch.zeros(B, dtype=torch.int32, device="cuda")
+        ws = dg.Workspace()
+        ts = []
+        for s_ in range(48):
+            logits = synth.make_sampler_logits(B, CANVAS, V, seed=0, step=s_, device="cuda")
+            ts.append(timed(lambda: dg.sample_commit(logits, tok, com, prev, stat, settings, 0,
+                                                     0, s_, ws=ws), 1, do_flush=False))
+            stat.zero_()  # the sweep runs all 48 scheduled steps
+            del logits
+        t = statistics.median(ts)
+        byts = B * CANVAS * V * 4
+        out.append({"kernel": "sample_commit", "batch": B, "us_per_step": round(t * 1e6, 2),
+                    "gbs": round(byts / t / 1e9, 1),
+                    "frac_hbm_peak": round(byts / t / 1e9 / peaks["hbm_gbs"], 4),
+                    "committed_tokens_per_s": round(16 * B / t, 1)})
+    elif args.kernel == "gemm":
+        M, N, K = (int(x) for x in args.shape.split(","))
+        x = torch.randn((M, K), device="cuda").to(torch.bfloat16)
+        w = (torch.randn((N, K), device="cuda") * K ** -0.5).to(torch.bfloat16)
+        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        ws = dg.Workspace()
+        t = timed(lambda: dg.linear(x, w, y, dg.EPI_BF16, ws=ws), args.steps)
+        fl = 2.0 * M * N * K
+        out.append({"kernel": "linear", "shape": [M, N, K], "us": round(t * 1e6, 2),
+                    "tflops": round(fl / t / 1e12, 1),
+                    "weight_gbs": round(N * K * 2 / t / 1e9, 1)})
+    for o in out:
+        o["peaks"] = peaks["source"]
+        print(json.dumps(o), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -270,7 +357,14 @@ def main():
     ap.add_argument("--workload", default="full", choices=["full", "tiny"])
     ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--kernel", choices=["attn", "sampler", "gemm"], default=None,
+                    help="time one kernel alone instead of the denoising step")
+    ap.add_argument("--prefix", type=int, default=0)
+    ap.add_argument("--batch", type=int, default=1)
+    ap.add_argument("--shape", default="256,8192,2048")
     args = ap.parse_args()
+    if args.kernel:
+        return run_kernel_bench(args)
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":

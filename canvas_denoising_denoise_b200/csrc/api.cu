@@ -107,21 +107,46 @@ struct GemmPlan {
   int splits, kb_per_split;
 };
 
+// Split K over a cluster of S CTAs (a power of two <= 8) when the output
+// tiles alone would leave most SMs idle; each split keeps >= 4 k-blocks.
 GemmPlan plan_gemm(int M, int N, int K) {
   const int tiles = (N / dg::gemm::BM) * cdiv(M, dg::gemm::BN);
   const int kb = K / dg::gemm::BK;
-  int s = std::max(1, kNumSMs / std::max(1, tiles));
-  s = std::min(s, std::max(1, kb / 4));
-  const int kbps = cdiv(kb, s);
-  return GemmPlan{cdiv(kb, kbps), kbps};
+  int s = 1;
+  while (s * 2 <= dg::gemm::MAX_SPLITS && tiles * s * 2 <= kNumSMs && kb % (s * 2) == 0 &&
+         kb / (s * 2) >= 4)
+    s *= 2;
+  return GemmPlan{s, kb / s};
 }
 
 bool gemm_attr_done = false;
 
-int launch_gemm(const void* x, const void* w, int M, int N, int K, const GemmPlan& pl, int epi,
-                float* out_f32, __nv_bfloat16* out_bf16, cudaStream_t s) {
+// Epilogue operands of one GEMM launch (see gemm.cuh).
+struct GemmEpi {
+  int epi = dg::gemm::EPI_F32;
+  float* out_f32 = nullptr;
+  __nv_bfloat16* out_bf16 = nullptr;
+  float* x = nullptr;
+  const float* ssq_in = nullptr;
+  int n_ssq_in = 0;
+  float inv_k = 0.f;
+  float eps = 0.f;
+  float* ssq_out = nullptr;
+};
+
+int launch_gemm(const void* x, const void* w, int M, int N, int K, const GemmPlan& pl,
+                const GemmEpi& e, cudaStream_t s) {
   if (!gemm_attr_done) {
-    DG_CUDA(cudaFuncSetAttribute(dg::gemm::gemm_kernel,
+    DG_CUDA(cudaFuncSetAttribute(dg::gemm::gemm_kernel<1>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dg::gemm::SMEM_BYTES));
+    DG_CUDA(cudaFuncSetAttribute(dg::gemm::gemm_kernel<2>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dg::gemm::SMEM_BYTES));
+    DG_CUDA(cudaFuncSetAttribute(dg::gemm::gemm_kernel<4>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 dg::gemm::SMEM_BYTES));
+    DG_CUDA(cudaFuncSetAttribute(dg::gemm::gemm_kernel<8>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  dg::gemm::SMEM_BYTES));
     gemm_attr_done = true;
@@ -129,55 +154,46 @@ int launch_gemm(const void* x, const void* w, int M, int N, int K, const GemmPla
   CUtensorMap tw, tx;
   DG_TRY(make_tmap(&tw, w, K, N, (uint64_t)K * 2, dg::gemm::BM));
   DG_TRY(make_tmap(&tx, x, K, M, (uint64_t)K * 2, dg::gemm::BN));
-  dg::gemm::Params p{M, N, K, pl.kb_per_split, epi, out_f32, out_bf16};
-  dim3 grid(N / dg::gemm::BM, cdiv(M, dg::gemm::BN), pl.splits);
-  dg::gemm::gemm_kernel<<<grid, dg::gemm::THREADS, dg::gemm::SMEM_BYTES, s>>>(tw, tx, p);
+  dg::gemm::Params p;
+  p.M = M; p.N = N; p.K = K;
+  p.kb_per_split = pl.kb_per_split;
+  p.splits = pl.splits;
+  p.epi = e.epi;
+  p.out_f32 = e.out_f32;
+  p.out_bf16 = e.out_bf16;
+  p.x = e.x;
+  p.ssq_in = e.ssq_in;
+  p.n_ssq_in = e.n_ssq_in;
+  p.inv_k = e.inv_k;
+  p.eps = e.eps;
+  p.ssq_out = e.ssq_out;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(N / dg::gemm::BM, cdiv(M, dg::gemm::BN), pl.splits);
+  cfg.blockDim = dim3(dg::gemm::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = dg::gemm::SMEM_BYTES;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = pl.splits;
+  cfg.attrs = attr;
+  cfg.numAttrs = pl.splits > 1 ? 1 : 0;
+  switch (pl.splits) {
+    case 1: DG_CUDA(cudaLaunchKernelEx(&cfg, dg::gemm::gemm_kernel<1>, tw, tx, p)); break;
+    case 2: DG_CUDA(cudaLaunchKernelEx(&cfg, dg::gemm::gemm_kernel<2>, tw, tx, p)); break;
+    case 4: DG_CUDA(cudaLaunchKernelEx(&cfg, dg::gemm::gemm_kernel<4>, tw, tx, p)); break;
+    case 8: DG_CUDA(cudaLaunchKernelEx(&cfg, dg::gemm::gemm_kernel<8>, tw, tx, p)); break;
+    default: return fail(DG_ERR_UNSUPPORTED_SHAPE, "split count %d", pl.splits);
+  }
   count_launch();
-  DG_CUDA(cudaGetLastError());
   return DG_OK;
 }
 
-int launch_reduce(const float* part, int S, int M, int N, int mode, __nv_bfloat16* out_bf16,
-                  float* out_f32, cudaStream_t s) {
-  const size_t n4 = (size_t)M * N / 4;
-  const int blocks = (int)std::min<size_t>(cdiv((int)std::min<size_t>(n4, 1u << 30), 256),
-                                           (size_t)kNumSMs * 8);
-  dg::gemm::reduce_kernel<<<std::max(1, blocks), 256, 0, s>>>(part, S, M, N, mode, out_bf16,
-                                                                out_f32);
-  count_launch();
-  DG_CUDA(cudaGetLastError());
-  return DG_OK;
-}
-
-// y = x w^T with the given final epilogue, using `part` for split partials.
-// mode: 0 bf16, 1 gelu bf16, 2 residual add fp32 (+ optional RMSNorm into xn).
-int linear(const void* x, const void* w, int M, int N, int K, int mode, void* out, float* part,
-           float eps, __nv_bfloat16* xn_out, cudaStream_t s) {
-  const GemmPlan pl = plan_gemm(M, N, K);
-  const bool norm = (mode == 2 && xn_out != nullptr);
-  if (pl.splits == 1 && !norm) {
-    const int epi = mode == 0 ? dg::gemm::EPI_BF16
-                  : mode == 1 ? dg::gemm::EPI_GELU_BF16
-                              : dg::gemm::EPI_ADD_F32;
-    return launch_gemm(x, w, M, N, K, pl, epi, (float*)out, (__nv_bfloat16*)out, s);
-  }
-  DG_TRY(launch_gemm(x, w, M, N, K, pl, dg::gemm::EPI_STORE_F32, part, nullptr, s));
-  if (norm) {
-    dg::gemm::add_norm_kernel<<<M, dg::gemm::NORM_THREADS, 0, s>>>(part, pl.splits, M, N, eps,
-                                                                    (float*)out, xn_out);
-    count_launch();
-    DG_CUDA(cudaGetLastError());
-    return DG_OK;
-  }
-  const int rmode = mode == 0 ? dg::gemm::RED_BF16
-                  : mode == 1 ? dg::gemm::RED_GELU_BF16
-                              : dg::gemm::RED_ADD_F32;
-  return launch_reduce(part, pl.splits, M, N, rmode, (__nv_bfloat16*)out, (float*)out, s);
-}
-
-size_t linear_part_bytes(int M, int N, int K) {
-  const GemmPlan pl = plan_gemm(M, N, K);
-  return (size_t)pl.splits * M * N * sizeof(float);
+// y = epilogue(x w^T) with the split plan chosen for this shape.
+int linear(const void* x, const void* w, int M, int N, int K, const GemmEpi& e,
+           cudaStream_t s) {
+  return launch_gemm(x, w, M, N, K, plan_gemm(M, N, K), e, s);
 }
 
 // ---------------------------------------------------------------------------
@@ -271,9 +287,9 @@ int launch_attn(const void* q, int ldq, const void* k_new, const void* v_new, in
 // Sampler
 // ---------------------------------------------------------------------------
 int sample_chunking(int V, int* chunk) {
-  // enough CTAs per row to stream the vocabulary with every SM busy, in
+  // chunks of >= 16384 elements (>= 64 per thread), at most 64 per row, in
   // multiples of 4 elements
-  int nchunk = std::max(1, std::min(64, V / 8192));
+  int nchunk = std::max(1, std::min(64, V / 16384));
   int c = cdiv(V, nchunk);
   c = (c + 3) / 4 * 4;
   nchunk = cdiv(V, c);
@@ -394,7 +410,7 @@ int check_state(const dg_state* st, const dg_model_cfg& c, bool need_canvas) {
 
 // Workspace carve-up for a forward over M = B * Lq rows.
 struct FwdLayout {
-  size_t x, xn, qkv, ao, up, part, attn, logits, spart, flag, total;
+  size_t x, xn, qkv, ao, up, ssq_x, ssq_h, attn, logits, spart, flag, total;
 };
 
 FwdLayout fwd_layout(const dg_model_cfg& c, int B, int Lq, int max_prefix, bool logits) {
@@ -413,12 +429,8 @@ FwdLayout fwd_layout(const dg_model_cfg& c, int B, int Lq, int max_prefix, bool 
   L.qkv = take((size_t)M * nqkv * 2);
   L.ao = take((size_t)M * hqd * 2);
   L.up = take((size_t)M * c.ffn * 2);
-  size_t part = 0;
-  part = std::max(part, linear_part_bytes(M, nqkv, c.d));
-  part = std::max(part, linear_part_bytes(M, c.d, hqd));
-  part = std::max(part, linear_part_bytes(M, c.ffn, c.d));
-  part = std::max(part, linear_part_bytes(M, c.d, c.ffn));
-  L.part = take(part);
+  L.ssq_x = take((size_t)(c.d / 128) * M * 4);
+  L.ssq_h = take((size_t)(c.d / 128) * M * 4);
   L.attn = take(attn_ws_bytes(B, c.n_q_heads, Lq, c.head_dim, max_prefix));
   L.logits = take(logits ? (size_t)M * c.vocab * 4 : 0);
   L.spart = take(logits ? sample_ws_bytes(B, Lq, c.vocab) : 0);
@@ -445,22 +457,28 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
   const int hd = c.head_dim, hq = c.n_q_heads, hkv = c.n_kv_heads;
   const int nqkv = (hq + 2 * hkv) * hd;
   float* x = (float*)(f.ws + f.L.x);
-  __nv_bfloat16* xn = (__nv_bfloat16*)(f.ws + f.L.xn);
+  __nv_bfloat16* xb = (__nv_bfloat16*)(f.ws + f.L.xn);  // bf16 copy of the residual stream
   __nv_bfloat16* qkv = (__nv_bfloat16*)(f.ws + f.L.qkv);
   __nv_bfloat16* ao = (__nv_bfloat16*)(f.ws + f.L.ao);
   __nv_bfloat16* up = (__nv_bfloat16*)(f.ws + f.L.up);
-  float* part = (float*)(f.ws + f.L.part);
+  float* ssq_x = (float*)(f.ws + f.L.ssq_x);
+  float* ssq_h = (float*)(f.ws + f.L.ssq_h);
   void* aws = f.ws + f.L.attn;
   const float scale = 1.0f / std::sqrt((float)hd);
+  const int nt = c.d / 128;
 
-  dg::gemm::embed_norm_kernel<<<M, dg::gemm::NORM_THREADS, 0, s>>>(
-      tok, (const __nv_bfloat16*)f.m->embed, c.vocab, c.d, c.eps, x, xn);
+  dg::gemm::embed_kernel<<<M, dg::gemm::EMBED_THREADS, 0, s>>>(
+      tok, (const __nv_bfloat16*)f.m->embed, c.vocab, c.d, M, x, xb, ssq_x);
   count_launch();
   DG_CUDA(cudaGetLastError());
   for (int l = 0; l < c.n_layers; ++l) {
     const dg_layer_weights& w = f.m->layers[l];
     const bool last = l == c.n_layers - 1;
-    DG_TRY(linear(xn, w.w_qkv, M, nqkv, c.d, 0, qkv, part, c.eps, nullptr, s));
+    GemmEpi eq;  // QKV of RMSNorm(x)
+    eq.epi = dg::gemm::EPI_BF16;
+    eq.out_bf16 = qkv;
+    eq.ssq_in = ssq_x; eq.n_ssq_in = nt; eq.inv_k = 1.f / c.d; eq.eps = c.eps;
+    DG_TRY(linear(xb, w.w_qkv, M, nqkv, c.d, eq, s));
     if (f.commit_kv) {
       const void* kb = qkv + hq * hd;
       const void* vb = qkv + (hq + hkv) * hd;
@@ -471,14 +489,27 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
     DG_TRY(launch_attn(qkv, nqkv, qkv + hq * hd, qkv + (hq + hkv) * hd, nqkv, f.k_cache[l],
                        f.v_cache[l], f.cache_len, f.max_prefix, f.lmax, ao, hq * hd, nullptr,
                        f.B, hq, hkv, f.Lq, hd, scale, f.mask, aws, s));
-    DG_TRY(linear(ao, w.w_o, M, c.d, hq * hd, 2, x, part, c.eps, xn, s));
-    DG_TRY(linear(xn, w.w_up, M, c.ffn, c.d, 1, up, part, c.eps, nullptr, s));
-    DG_TRY(linear(up, w.w_down, M, c.d, c.ffn, 2, x, part, c.eps, xn, s));
+    GemmEpi eo;  // h = x + O w_o^T
+    eo.epi = dg::gemm::EPI_RESID;
+    eo.x = x; eo.out_bf16 = xb; eo.ssq_out = ssq_h;
+    DG_TRY(linear(ao, w.w_o, M, c.d, hq * hd, eo, s));
+    GemmEpi eu;  // gelu(RMSNorm(h) w_up^T)
+    eu.epi = dg::gemm::EPI_GELU;
+    eu.out_bf16 = up;
+    eu.ssq_in = ssq_h; eu.n_ssq_in = nt; eu.inv_k = 1.f / c.d; eu.eps = c.eps;
+    DG_TRY(linear(xb, w.w_up, M, c.ffn, c.d, eu, s));
+    GemmEpi ed;  // x = h + u w_down^T
+    ed.epi = dg::gemm::EPI_RESID;
+    ed.x = x; ed.out_bf16 = xb; ed.ssq_out = ssq_x;
+    DG_TRY(linear(up, w.w_down, M, c.d, c.ffn, ed, s));
   }
   if (f.want_logits) {
-    const GemmPlan pl{1, c.d / dg::gemm::BK};
-    DG_TRY(launch_gemm(xn, f.m->unembed, M, c.vocab, c.d, pl, dg::gemm::EPI_STORE_F32, logits,
-                       nullptr, s));
+    GemmEpi el;  // logits of RMSNorm(x)
+    el.epi = dg::gemm::EPI_F32;
+    el.out_f32 = logits;
+    el.ssq_in = ssq_x; el.n_ssq_in = nt; el.inv_k = 1.f / c.d; el.eps = c.eps;
+    DG_TRY(launch_gemm(xb, f.m->unembed, M, c.vocab, c.d, GemmPlan{1, c.d / dg::gemm::BK}, el,
+                       s));
   }
   return DG_OK;
 }
@@ -614,18 +645,23 @@ int dg_unembed(const void* h, const void* w_u, float* logits, int M, int d, int 
     return fail(DG_ERR_UNSUPPORTED_SHAPE, "dg_unembed: V %% 128 and d %% 64 must be 0");
   if (!aligned16(h) || !aligned16(w_u) || !aligned16(logits))
     return fail(DG_ERR_ALIGNMENT, "dg_unembed: pointers must be 16-byte aligned");
-  const GemmPlan pl{1, d / dg::gemm::BK};
-  return launch_gemm(h, w_u, M, V, d, pl, dg::gemm::EPI_STORE_F32, logits, nullptr,
-                     (cudaStream_t)stream);
+  GemmEpi e;
+  e.epi = dg::gemm::EPI_F32;
+  e.out_f32 = logits;
+  return launch_gemm(h, w_u, M, V, d, GemmPlan{1, d / dg::gemm::BK}, e, (cudaStream_t)stream);
 }
 
 size_t dg_linear_workspace_bytes(int M, int N, int K) {
-  if (M <= 0 || N <= 0 || K <= 0) return 0;
-  return linear_part_bytes(M, N, K);
+  (void)M;
+  (void)N;
+  (void)K;
+  return 0;  // split-K partial sums stay in the cluster's shared memory
 }
 
 int dg_linear(const void* x, const void* w, void* out, int M, int N, int K, int epilogue,
               void* workspace, size_t workspace_bytes, void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
   if (!x || !w || !out) return fail(DG_ERR_INVALID_ARG, "dg_linear: null pointer");
   if (M <= 0 || N <= 0 || K <= 0 || epilogue < 0 || epilogue > DG_EPI_RESID_F32)
     return fail(DG_ERR_INVALID_ARG, "dg_linear: bad sizes or epilogue");
@@ -633,17 +669,21 @@ int dg_linear(const void* x, const void* w, void* out, int M, int N, int K, int 
     return fail(DG_ERR_UNSUPPORTED_SHAPE, "dg_linear: N %% 128 and K %% 64 must be 0");
   if (!aligned16(x) || !aligned16(w) || !aligned16(out))
     return fail(DG_ERR_ALIGNMENT, "dg_linear: pointers must be 16-byte aligned");
-  cudaStream_t s = (cudaStream_t)stream;
+  GemmEpi e;
   if (epilogue == DG_EPI_F32) {
-    const GemmPlan pl{1, K / dg::gemm::BK};
-    return launch_gemm(x, w, M, N, K, pl, dg::gemm::EPI_STORE_F32, (float*)out, nullptr, s);
+    e.epi = dg::gemm::EPI_F32;
+    e.out_f32 = (float*)out;
+  } else if (epilogue == DG_EPI_BF16) {
+    e.epi = dg::gemm::EPI_BF16;
+    e.out_bf16 = (__nv_bfloat16*)out;
+  } else if (epilogue == DG_EPI_GELU_BF16) {
+    e.epi = dg::gemm::EPI_GELU;
+    e.out_bf16 = (__nv_bfloat16*)out;
+  } else {
+    e.epi = dg::gemm::EPI_RESID;
+    e.x = (float*)out;
   }
-  const size_t need = linear_part_bytes(M, N, K);
-  const GemmPlan pl = plan_gemm(M, N, K);
-  if (pl.splits > 1 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
-    return fail(DG_ERR_WORKSPACE_TOO_SMALL, "dg_linear: workspace needs %zu bytes", need);
-  const int mode = epilogue == DG_EPI_BF16 ? 0 : epilogue == DG_EPI_GELU_BF16 ? 1 : 2;
-  return linear(x, w, M, N, K, mode, out, (float*)workspace, 0.f, nullptr, s);
+  return linear(x, w, M, N, K, e, (cudaStream_t)stream);
 }
 
 size_t dg_sample_commit_workspace_bytes(int B, int C, int V) {

@@ -36,6 +36,14 @@ constexpr int THREADS = 192;
 constexpr int TMEM_COLS = 512;  // S0 [0,128), S1 [128,256), O [256, 256+hd)
 constexpr float kRescaleThreshold = 8.0f;
 
+// 2^x on the special-function unit (flushes denormal results to zero, which
+// only affects probabilities below 2^-126).
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 template <int HD>
 struct Cfg {
   static constexpr int HALVES = HD / 64;
@@ -291,13 +299,22 @@ __global__ void __launch_bounds__(THREADS, 1)
         causal_lim = p.causal ? (qrow - ck0) : 0x7FFFFFFF;
       }
       const int lim = min(nvalid - 1, causal_lim);  // valid keys: [0, lim]
-      float tmax = -INFINITY;
+      // masking only where some row of this warp has invalid keys
+      if (__any_sync(0xffffffffu, lim < BKV - 1)) {
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const float v = (c <= lim) ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
-        sr[c] = __float_as_uint(v);
-        tmax = fmaxf(tmax, v);
+        for (int c = 0; c < 128; ++c)
+          if (c > lim) sr[c] = __float_as_uint(-INFINITY);
       }
+      // row max of the raw scores (the scale is positive), four chains for ILP
+      float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 128; c += 4) {
+        mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
+        mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
+        mx2 = fmaxf(mx2, __uint_as_float(sr[c + 2]));
+        mx3 = fmaxf(mx3, __uint_as_float(sr[c + 3]));
+      }
+      const float tmax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
       // The decision is taken per warp: the TMEM loads/stores below are
       // warp-collective (.sync.aligned) and must see all 32 lanes.  Lanes whose
       // own max did not move rescale by exactly 1.
@@ -326,16 +343,23 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         m = m_new;
       }
-      const float mu = (m == -INFINITY) ? 0.f : m;
-      float rs = 0.f;
+      const float neg_m = (m == -INFINITY) ? 0.f : -m;
+      float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
       uint32_t pk[64];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float p0 = exp2f(__uint_as_float(sr[2 * c]) - mu);
-        const float p1 = exp2f(__uint_as_float(sr[2 * c + 1]) - mu);
-        rs += p0 + p1;
+      for (int c = 0; c < 64; c += 2) {
+        const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * c]), p.scale_log2, neg_m));
+        const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * c + 1]), p.scale_log2, neg_m));
+        const float p2 = fast_exp2(fmaf(__uint_as_float(sr[2 * c + 2]), p.scale_log2, neg_m));
+        const float p3 = fast_exp2(fmaf(__uint_as_float(sr[2 * c + 3]), p.scale_log2, neg_m));
+        rs0 += p0;
+        rs1 += p1;
+        rs2 += p2;
+        rs3 += p3;
         pk[c] = pack_bf16x2(p0, p1);
+        pk[c + 1] = pack_bf16x2(p2, p3);
       }
+      const float rs = (rs0 + rs1) + (rs2 + rs3);
       l += rs;
       {
         uint32_t(&a0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);

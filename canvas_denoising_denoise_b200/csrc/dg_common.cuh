@@ -83,13 +83,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
                                           uint32_t site) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  while (true) {
+  for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
-    if (abort != nullptr && *abort) return false;
-    if (globaltimer_ns() - t0 > kWaitLimitNs) {
-      raise_error(ERR_TIMEOUT | site, blockIdx.x);
-      if (abort != nullptr) *abort = 1;
-      return false;
+    if ((it & 15u) == 0) {
+      if (abort != nullptr && *abort) return false;
+      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+        raise_error(ERR_TIMEOUT | site, blockIdx.x);
+        if (abort != nullptr) *abort = 1;
+        return false;
+      }
     }
   }
 }

@@ -1,20 +1,34 @@
 // gemm.cuh - the projections of the stack and the unembedding on tcgen05.
 //
-//   y[t, f] = sum_k x[t, k] w[f, k]        x bf16 [M, K] (activations)
-//                                          w bf16 [N, K] (weights, nn.Linear layout)
+//   y[t, f] = rs[t] * sum_k x[t, k] w[f, k]     x bf16 [M, K] (activations)
+//                                               w bf16 [N, K] (weights, [out, in])
 //
-// The weight is the UMMA A operand (M side, 128 output features per tile) and
-// the activations are the B operand (N side, up to 256 tokens per tile): one
-// 128 x 256 x 16 instruction per k-step, the accumulator in TMEM.  At the
-// canvas sizes (256 tokens per sequence) each weight tile is streamed from
-// HBM exactly once and the activations come from L2.  Few output tiles at
-// small widths are spread over the SMs by splitting K; the split partial sums
-// (fp32) are reduced in a fixed order by a separate kernel that also applies
-// the epilogue (bf16 store, GELU, residual add, residual add + RMSNorm).
+// The weight is the UMMA A operand (128 output features per tile) and the
+// tokens are the B operand (up to 256 per tile): one 128 x 256 x 16
+// tcgen05.mma per k-step, fp32 accumulator in TMEM, a 4-stage TMA ring.
 //
-// Warp roles (192 threads): warp 0 issues TMA loads into a ring of stages,
-// warp 1 owns TMEM and one elected lane issues the MMAs, warps 2..5 drain
-// the accumulator (TMEM -> registers -> global).
+// When there are too few output tiles to occupy the SMs (the layer
+// projections of one 256-token canvas), K is split over S CTAs that form one
+// thread-block cluster.  Each CTA stages its partial tile in its own shared
+// memory; after a cluster barrier, CTA r sums token rows [r*256/S, (r+1)*256/S)
+// of all S partials through distributed shared memory and applies the
+// epilogue.  Partial sums never leave the cluster.
+//
+// RMSNorm with unit gain is a per-token scale, so norm(x) w^T = rs * (x w^T)
+// with rs[t] = 1/sqrt(mean_k x[t,k]^2 + eps): the consumer of a normalised
+// input applies rs in its epilogue, computed from per-(128-column tile, token)
+// sums of squares that the producer of x wrote (summed in a fixed order).
+//
+// Epilogues:
+//   EPI_F32    out_f32[t, f]  = rs * acc
+//   EPI_BF16   out_bf16[t, f] = bf16(rs * acc)
+//   EPI_GELU   out_bf16[t, f] = bf16(gelu(rs * acc))            (exact erf)
+//   EPI_RESID  x[t, f] += acc; out_bf16[t, f] = bf16(x[t, f]) (if given);
+//              ssq_out[tile, t] = sum over the tile's 128 f of x[t, f]^2 (if given)
+//
+// Warp roles (192 threads): warp 0 issues TMA loads, warp 1 owns TMEM and one
+// lane issues the MMAs, warps 2..5 move the accumulator TMEM -> shared
+// memory; all six warps run the reduction/epilogue.
 #pragma once
 
 #include "dg_common.cuh"
@@ -30,36 +44,75 @@ constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int STAGES = 4;
 constexpr int THREADS = 192;
+constexpr int WARPS = THREADS / 32;
 constexpr int TMEM_COLS = BN;
-constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + 256;
+constexpr int STAGE_AREA = STAGES * STAGE_BYTES;          // also holds the fp32 tile
+constexpr int TILE_ROW_FLOATS = BM;                       // staged tile: [BN][BM] fp32
+constexpr int SMEM_BYTES = 1024 + STAGE_AREA + BN * 4 + 256;
+constexpr int MAX_SPLITS = 8;
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, false, false);
+static_assert(BN * BM * 4 <= STAGE_AREA, "staged tile must fit in the stage ring");
 
-enum Epi : int {
-  EPI_STORE_F32 = 0,   // out_f32[(split * M + t) * N + f] = acc
-  EPI_BF16 = 1,        // out_bf16[t * N + f] = acc
-  EPI_GELU_BF16 = 2,   // out_bf16[t * N + f] = gelu(acc)
-  EPI_ADD_F32 = 3,     // out_f32[t * N + f] += acc
-};
+enum Epi : int { EPI_F32 = 0, EPI_BF16 = 1, EPI_GELU = 2, EPI_RESID = 3 };
 
 struct Params {
   int M, N, K;
-  int kb_per_split;  // k-blocks (of 64) per split
+  int kb_per_split;        // k-blocks (of 64) per split
+  int splits;              // cluster size along z (1 = no cluster)
   int epi;
-  float* out_f32;
-  __nv_bfloat16* out_bf16;
+  float* out_f32;          // EPI_F32
+  __nv_bfloat16* out_bf16; // EPI_BF16 / EPI_GELU / EPI_RESID (optional there)
+  float* x;                // EPI_RESID residual stream [M, N] fp32, updated in place
+  const float* ssq_in;     // [n_ssq_in, M] sums of squares of the input rows, or null
+  int n_ssq_in;
+  float inv_k;             // 1 / (input width) for the mean
+  float eps;
+  float* ssq_out;          // [N / 128, M] (EPI_RESID), or null
 };
 
 __device__ __forceinline__ float gelu_erf(float x) {
   return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
 }
 
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;"
+               ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+// Remote shared-memory load.  Ordering against the peers' writes comes from
+// the cluster barrier, so no compiler memory clobber is needed here and
+// several loads can be in flight at once.
+__device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr));
+  return v;
+}
+
+template <int S>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                 Params p) {
+  static_assert(S == 1 || S == 2 || S == 4 || S == 8, "split count");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+  float* tile = reinterpret_cast<float*>(smem);  // [BN][BM] after the mainloop
+  float* rowscale = reinterpret_cast<float*>(smem + STAGE_AREA);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGE_AREA + BN * 4);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* drain = acc_full + 1;
@@ -71,9 +124,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int f0 = blockIdx.x * BM;
   const int t0 = blockIdx.y * BN;
   const int split = blockIdx.z;
-  const int kb_total = p.K / BK;
   const int kb_begin = split * p.kb_per_split;
-  const int nkb = min(p.kb_per_split, kb_total - kb_begin);
+  const int nkb = min(p.kb_per_split, p.K / BK - kb_begin);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -98,93 +150,156 @@ __global__ void __launch_bounds__(THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_acc = *tmem_holder;
 
-  if (nkb > 0) {
-    if (warp == 0) {
-      if (lane == 0) {
-        const uint64_t pol_w = l2_policy_evict_first();
-        int issued = 0;
-        for (int kb = 0; kb < nkb; ++kb) {
-          const int st = kb % STAGES;
-          if (kb >= STAGES &&
-              !mbar_wait(&empty[st], ((kb / STAGES) - 1) & 1, abort_flag, 0x101))
-            break;
-          uint8_t* a = smem + st * STAGE_BYTES;
-          uint8_t* bt = a + A_BYTES;
-          mbar_expect_tx(&full[st], STAGE_BYTES);
-          const int kx = (kb_begin + kb) * BK;
-          tma_load_2d_hint(a, &tm_w, &full[st], kx, f0, pol_w);
-          tma_load_2d(bt, &tm_x, &full[st], kx, t0);
-          issued = kb + 1;
-        }
-        if (*abort_flag) {
-          // let every load already in flight land before the CTA exits
-          for (int kb = max(0, issued - STAGES); kb < issued; ++kb)
-            mbar_wait(&full[kb % STAGES], (kb / STAGES) & 1, nullptr, 0x102);
-        }
+  if (warp == 0) {
+    if (lane == 0 && nkb > 0) {
+      const uint64_t pol_w = l2_policy_evict_first();
+      int issued = 0;
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int st = kb % STAGES;
+        if (kb >= STAGES && !mbar_wait(&empty[st], ((kb / STAGES) - 1) & 1, abort_flag, 0x101))
+          break;
+        uint8_t* a = smem + st * STAGE_BYTES;
+        mbar_expect_tx(&full[st], STAGE_BYTES);
+        const int kx = (kb_begin + kb) * BK;
+        tma_load_2d_hint(a, &tm_w, &full[st], kx, f0, pol_w);
+        tma_load_2d(a + A_BYTES, &tm_x, &full[st], kx, t0);
+        issued = kb + 1;
       }
-    } else if (warp == 1) {
-      if (lane == 0) {
-        for (int kb = 0; kb < nkb; ++kb) {
-          const int st = kb % STAGES;
-          if (!mbar_wait(&full[st], (kb / STAGES) & 1, abort_flag, 0x103)) break;
-          tc_fence_after();
-          const uint32_t a_base = smem_u32(smem + st * STAGE_BYTES);
-          const uint32_t b_base = a_base + A_BYTES;
+      if (*abort_flag) {
+        for (int kb = max(0, issued - STAGES); kb < issued; ++kb)
+          mbar_wait(&full[kb % STAGES], (kb / STAGES) & 1, nullptr, 0x102);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && nkb > 0) {
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int st = kb % STAGES;
+        if (!mbar_wait(&full[st], (kb / STAGES) & 1, abort_flag, 0x103)) break;
+        tc_fence_after();
+        const uint32_t a_base = smem_u32(smem + st * STAGE_BYTES);
+        const uint32_t b_base = a_base + A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            const uint64_t ad = sdesc_sw128(a_base + kk * 32, 16, 1024);
-            const uint64_t bd = sdesc_sw128(b_base + kk * 32, 16, 1024);
-            umma_ss(tmem_acc, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
-          }
-          umma_commit(&empty[st]);
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          umma_ss(tmem_acc, sdesc_sw128(a_base + kk * 32, 16, 1024),
+                  sdesc_sw128(b_base + kk * 32, 16, 1024), IDESC, (kb | kk) != 0 ? 1u : 0u);
         }
-        umma_commit(acc_full);
-        // all MMAs of this CTA retire before TMEM is released
-        umma_commit(drain);
-        mbar_wait(drain, 0, nullptr, 0x104);
+        umma_commit(&empty[st]);
+      }
+      umma_commit(acc_full);
+      umma_commit(drain);
+      mbar_wait(drain, 0, nullptr, 0x104);
+    }
+  } else {
+    // warps 2..5: row scales for this tile's tokens while the mainloop runs
+    for (int t = threadIdx.x - 64; t < BN; t += THREADS - 64) {
+      float rs = 1.f;
+      const int tg = t0 + t;
+      if (p.ssq_in != nullptr && tg < p.M) {
+        float acc = 0.f;
+        for (int j = 0; j < p.n_ssq_in; ++j) acc += p.ssq_in[static_cast<size_t>(j) * p.M + tg];
+        rs = rsqrtf(acc * p.inv_k + p.eps);
+      }
+      rowscale[t] = rs;
+    }
+    // TMEM -> registers -> shared tile [token][feature]
+    const bool have_acc =
+        nkb > 0 && __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, 0x105));
+    if (have_acc) {
+      tc_fence_after();
+      const int quarter = warp & 3;
+      const int fl = quarter * 32 + lane;
+      const uint32_t taddr = tmem_acc + (static_cast<uint32_t>(quarter * 32) << 16);
+      for (int c = 0; c < BN / 32; ++c) {
+        if (t0 + c * 32 >= p.M) break;  // warp-uniform
+        uint32_t r[32];
+        tmem_ld32(taddr + c * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          tile[(c * 32 + j) * TILE_ROW_FLOATS + fl] = __uint_as_float(r[j]);
       }
     } else {
-      // epilogue warps 2..5 -> TMEM lane quarter (warp % 4)
-      const int quarter = warp & 3;
-      const int f = f0 + quarter * 32 + lane;
-      if (__all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, 0x105))) {
-        tc_fence_after();
-        const uint32_t taddr = tmem_acc + (static_cast<uint32_t>(quarter * 32) << 16);
-        for (int c = 0; c < BN / 32; ++c) {
-          const int tb = t0 + c * 32;
-          if (tb >= p.M) break;
-          uint32_t r[32];
-          tmem_ld32(taddr + c * 32, r);
-          tmem_ld_wait();
-          const int nt = min(32, p.M - tb);
-          if (p.epi == EPI_STORE_F32) {
-            float* o = p.out_f32 + (static_cast<size_t>(split) * p.M + tb) * p.N + f;
+      // no accumulator (empty split or an abandoned wait): contribute zeros
+      for (int i = threadIdx.x - 64; i < BN * TILE_ROW_FLOATS; i += THREADS - 64) tile[i] = 0.f;
+    }
+  }
+  // every CTA of the cluster has its partial tile in shared memory
+  tc_fence_before();
+  if constexpr (S > 1)
+    cluster_sync();
+  else
+    __syncthreads();
+
+  // ---------------------------------------------------------------- reduce + epilogue
+  // CTA r owns token rows [r*BN/S, (r+1)*BN/S) of the tile.  A warp gathers
+  // MAX_SPLITS float4 per lane per round (S sources x MAX_SPLITS/S rows) so
+  // that the remote loads overlap instead of queueing one by one.
+  constexpr int rows_per = BN / S;
+  constexpr int rows_round = MAX_SPLITS / S;
+  const int r0 = (S > 1 ? static_cast<int>(cluster_rank()) : 0) * rows_per;
+  const uint32_t tile_saddr = smem_u32(tile);
+  for (int rb = warp * rows_round; rb < rows_per; rb += WARPS * rows_round) {
+    float4 v[MAX_SPLITS];
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < nt) o[static_cast<size_t>(j) * p.N] = __uint_as_float(r[j]);
-          } else if (p.epi == EPI_ADD_F32) {
-            float* o = p.out_f32 + static_cast<size_t>(tb) * p.N + f;
+    for (int i = 0; i < MAX_SPLITS; ++i) {
+      const int t = r0 + rb + i / S;
+      const uint32_t off = static_cast<uint32_t>((t * TILE_ROW_FLOATS + lane * 4) * 4);
+      if (rb + i / S < rows_per && t0 + t < p.M) {
+        if constexpr (S > 1)
+          v[i] = ld_dsmem_f4(map_to_rank(tile_saddr + off, i % S));
+        else
+          v[i] = *reinterpret_cast<const float4*>(reinterpret_cast<const uint8_t*>(tile) + off);
+      } else {
+        v[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+    }
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < nt) o[static_cast<size_t>(j) * p.N] += __uint_as_float(r[j]);
-          } else if (p.epi == EPI_BF16) {
-            __nv_bfloat16* o = p.out_bf16 + static_cast<size_t>(tb) * p.N + f;
+    for (int j = 0; j < rows_round; ++j) {
+      const int t = r0 + rb + j;
+      const int tg = t0 + t;
+      if (rb + j >= rows_per || tg >= p.M) break;  // warp-uniform
+      float4 a = v[j * S];
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < nt) o[static_cast<size_t>(j) * p.N] = __float2bfloat16_rn(__uint_as_float(r[j]));
-          } else {
-            __nv_bfloat16* o = p.out_bf16 + static_cast<size_t>(tb) * p.N + f;
-#pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < nt)
-                o[static_cast<size_t>(j) * p.N] =
-                    __float2bfloat16_rn(gelu_erf(__uint_as_float(r[j])));
+      for (int q = 1; q < S; ++q) {
+        const float4 w = v[j * S + q];
+        a.x += w.x; a.y += w.y; a.z += w.z; a.w += w.w;
+      }
+      const int f = f0 + lane * 4;
+      const size_t o = static_cast<size_t>(tg) * p.N + f;
+      if (p.epi == EPI_RESID) {
+        float4* xp = reinterpret_cast<float4*>(p.x + o);
+        float4 xv = *xp;
+        xv.x += a.x; xv.y += a.y; xv.z += a.z; xv.w += a.w;
+        *xp = xv;
+        if (p.out_bf16) {
+          uint2 w;
+          w.x = pack_bf16x2(xv.x, xv.y);
+          w.y = pack_bf16x2(xv.z, xv.w);
+          *reinterpret_cast<uint2*>(p.out_bf16 + o) = w;
+        }
+        if (p.ssq_out) {
+          const float sq = warp_sum(xv.x * xv.x + xv.y * xv.y + xv.z * xv.z + xv.w * xv.w);
+          if (lane == 0) p.ssq_out[static_cast<size_t>(blockIdx.x) * p.M + tg] = sq;
+        }
+      } else {
+        const float rs = rowscale[t];
+        a.x *= rs; a.y *= rs; a.z *= rs; a.w *= rs;
+        if (p.epi == EPI_F32) {
+          *reinterpret_cast<float4*>(p.out_f32 + o) = a;
+        } else {
+          if (p.epi == EPI_GELU) {
+            a.x = gelu_erf(a.x); a.y = gelu_erf(a.y); a.z = gelu_erf(a.z); a.w = gelu_erf(a.w);
           }
+          uint2 w;
+          w.x = pack_bf16x2(a.x, a.y);
+          w.y = pack_bf16x2(a.z, a.w);
+          *reinterpret_cast<uint2*>(p.out_bf16 + o) = w;
         }
       }
     }
   }
-  tc_fence_before();
+  // no CTA leaves while a peer may still read its shared memory
+  if constexpr (S > 1) cluster_sync();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
@@ -192,112 +307,35 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 }
 
-// ---------------------------------------------------------------------------
-// Split-K reductions with the layer epilogues.  part: [S, M, N] fp32.
-// ---------------------------------------------------------------------------
-enum RedMode : int { RED_BF16 = 0, RED_GELU_BF16 = 1, RED_ADD_F32 = 2 };
+// One CTA per token row: x[t] = embed[tok[t]] (fp32), xb[t] = bf16(x[t]),
+// ssq[j, t] = sum of x[t, 128 j .. 128 j + 127]^2.
+constexpr int EMBED_THREADS = 256;
 
-__global__ void reduce_kernel(const float* __restrict__ part, int S, int M, int N, int mode,
-                              __nv_bfloat16* __restrict__ out_bf16, float* __restrict__ out_f32) {
-  const size_t n4 = static_cast<size_t>(M) * N / 4;
-  const size_t stride = static_cast<size_t>(M) * N;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n4;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    float4 a = reinterpret_cast<const float4*>(part)[i];
-    for (int s = 1; s < S; ++s) {
-      const float4 c = reinterpret_cast<const float4*>(part + s * stride)[i];
-      a.x += c.x; a.y += c.y; a.z += c.z; a.w += c.w;
-    }
-    if (mode == RED_ADD_F32) {
-      float4 o = reinterpret_cast<float4*>(out_f32)[i];
-      o.x += a.x; o.y += a.y; o.z += a.z; o.w += a.w;
-      reinterpret_cast<float4*>(out_f32)[i] = o;
-    } else {
-      if (mode == RED_GELU_BF16) {
-        a.x = gelu_erf(a.x); a.y = gelu_erf(a.y); a.z = gelu_erf(a.z); a.w = gelu_erf(a.w);
-      }
-      uint2 v;
-      v.x = pack_bf16x2(a.x, a.y);
-      v.y = pack_bf16x2(a.z, a.w);
-      reinterpret_cast<uint2*>(out_bf16)[i] = v;
-    }
-  }
-}
-
-// One CTA per token row: x[t] (+)= sum_s part[s][t], then xn[t] = bf16(x[t] / rms(x[t])).
-// With S == 0 only the normalisation runs.
-constexpr int NORM_THREADS = 256;
-
-__global__ void __launch_bounds__(NORM_THREADS) add_norm_kernel(
-    const float* __restrict__ part, int S, int M, int N, float eps, float* __restrict__ x,
-    __nv_bfloat16* __restrict__ xn) {
-  const int t = blockIdx.x;
-  const size_t stride = static_cast<size_t>(M) * N;
-  float* xr = x + static_cast<size_t>(t) * N;
-  float ss = 0.f;
-  for (int c = threadIdx.x * 4; c < N; c += NORM_THREADS * 4) {
-    float4 a = *reinterpret_cast<float4*>(xr + c);
-    for (int s = 0; s < S; ++s) {
-      const float4 d = *reinterpret_cast<const float4*>(part + s * stride +
-                                                        static_cast<size_t>(t) * N + c);
-      a.x += d.x; a.y += d.y; a.z += d.z; a.w += d.w;
-    }
-    if (S > 0) *reinterpret_cast<float4*>(xr + c) = a;
-    ss += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
-  }
-  __shared__ float red[NORM_THREADS / 32];
-  ss = warp_sum(ss);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
-  __syncthreads();
-  float tot = 0.f;
-  for (int w = 0; w < NORM_THREADS / 32; ++w) tot += red[w];
-  const float inv = rsqrtf(tot / static_cast<float>(N) + eps);
-  __nv_bfloat16* xo = xn + static_cast<size_t>(t) * N;
-  for (int c = threadIdx.x * 4; c < N; c += NORM_THREADS * 4) {
-    const float4 a = *reinterpret_cast<const float4*>(xr + c);
-    uint2 v;
-    v.x = pack_bf16x2(a.x * inv, a.y * inv);
-    v.y = pack_bf16x2(a.z * inv, a.w * inv);
-    *reinterpret_cast<uint2*>(xo + c) = v;
-  }
-}
-
-// One CTA per token row: x[t] = embed[tok[t]] (fp32), xn[t] = bf16(rmsnorm(x[t])).
-__global__ void __launch_bounds__(NORM_THREADS) embed_norm_kernel(
-    const int32_t* __restrict__ tok, const __nv_bfloat16* __restrict__ embed, int V, int d,
-    float eps, float* __restrict__ x, __nv_bfloat16* __restrict__ xn) {
+__global__ void __launch_bounds__(EMBED_THREADS) embed_kernel(
+    const int32_t* __restrict__ tok, const __nv_bfloat16* __restrict__ embed, int V, int d, int M,
+    float* __restrict__ x, __nv_bfloat16* __restrict__ xb, float* __restrict__ ssq) {
   const int t = blockIdx.x;
   int id = tok[t];
   if (id < 0 || id >= V) {
-    raise_error(ERR_CHECK | 0x201, static_cast<uint32_t>(t));
+    if (threadIdx.x == 0) raise_error(ERR_CHECK | 0x201, static_cast<uint32_t>(t));
     id = 0;
   }
   const __nv_bfloat16* e = embed + static_cast<size_t>(id) * d;
   float* xr = x + static_cast<size_t>(t) * d;
-  float ss = 0.f;
-  for (int c = threadIdx.x * 4; c < d; c += NORM_THREADS * 4) {
+  __nv_bfloat16* br = xb + static_cast<size_t>(t) * d;
+  // a warp covers 128 columns (one ssq tile) per iteration: lane -> 4 columns
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int j = warp; j < d / 128; j += EMBED_THREADS / 32) {
+    const int c = j * 128 + lane * 4;
     const uint2 raw = *reinterpret_cast<const uint2*>(e + c);
+    *reinterpret_cast<uint2*>(br + c) = raw;
     const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
     const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
     const float4 a = make_float4(__low2float(lo), __high2float(lo), __low2float(hi),
                                  __high2float(hi));
     *reinterpret_cast<float4*>(xr + c) = a;
-    ss += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
-  }
-  __shared__ float red[NORM_THREADS / 32];
-  ss = warp_sum(ss);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
-  __syncthreads();
-  float tot = 0.f;
-  for (int w = 0; w < NORM_THREADS / 32; ++w) tot += red[w];
-  const float inv = rsqrtf(tot / static_cast<float>(d) + eps);
-  __nv_bfloat16* xo = xn + static_cast<size_t>(t) * d;
-  for (int c = threadIdx.x * 4; c < d; c += NORM_THREADS * 4) {
-    const float4 a = *reinterpret_cast<const float4*>(xr + c);
-    uint2 v;
-    v.x = pack_bf16x2(a.x * inv, a.y * inv);
-    v.y = pack_bf16x2(a.z * inv, a.w * inv);
-    *reinterpret_cast<uint2*>(xo + c) = v;
+    const float sq = warp_sum(a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w);
+    if (lane == 0) ssq[static_cast<size_t>(j) * M + t] = sq;
   }
 }
 

@@ -55,13 +55,33 @@ __device__ __forceinline__ int32_t token_from_word(uint32_t r, int vocab) {
   return static_cast<int32_t>((static_cast<uint64_t>(r) * static_cast<uint32_t>(vocab)) >> 32);
 }
 
-// u = (2 (r >> 9) + 1) 2^-24 in (0, 1), exact in fp32; returns log2(-ln u).
-// logf is accurate to about one ulp over its whole range (including just
-// below 1, where -ln u is tiny), so E keeps its relative accuracy everywhere.
-__device__ __forceinline__ float neg_log2_exponential(uint32_t r) {
-  const float u = __uint2float_rn(((r >> 9) << 1) | 1u) * 5.9604644775390625e-08f;  // 2^-24
-  const float e = -logf(u);
-  return log2f(e);
+__device__ __forceinline__ float sfu_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+__device__ __forceinline__ float sfu_log2(float x) {
+  float y;
+  asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// Exponential variate E = -ln(u) of the draw word r, u = (2 (r >> 9) + 1) 2^-24.
+// u is built exactly from the bits: 1 + (r >> 9) 2^-23 is an fp32 in [1, 2), and
+// subtracting 1 - 2^-24 (representable) is exact; w = 1 - u is exact too.
+// Away from u = 1 the special-function log2 is accurate to ~2^-22 absolute, i.e.
+// ~3e-6 relative in E for u <= 15/16.  For w = 1 - u <= 1/16 the series
+// -ln(1 - w) = w + w^2/2 + ... + w^6/6 (truncation < 1e-8 relative) is used.
+__device__ __forceinline__ float exp_variate(uint32_t r) {
+  const float f = __uint_as_float(0x3F800000u | (r >> 9));
+  const float u = f - 0.999999940395355224609375f;  // f - (1 - 2^-24)
+  const float w = 1.0f - u;
+  const float e_log = sfu_log2(u) * -0.693147180559945309f;
+  const float e_ser =
+      w * fmaf(w, fmaf(w, fmaf(w, fmaf(w, fmaf(w, 0.16666667f, 0.2f), 0.25f), 0.33333334f), 0.5f),
+               1.0f);
+  return w <= 0.0625f ? e_ser : e_log;
 }
 
 __device__ __forceinline__ float step_temperature(int step, int max_steps, float t0, float t1) {
@@ -126,6 +146,14 @@ __device__ __forceinline__ void merge_best(float& v, int& i, float v2, int i2) {
 }
 
 // Grid: B * C * nchunk CTAs of RP_THREADS threads.  Chunk length is a multiple of 4.
+//
+// Per element, in the log2 domain with m the running maximum:
+//   pe = 2^(l k2 - m)         one FFMA + one ex2 (shared by the softmax sums)
+//   E  = -ln(u)               Philox word -> exponential variate
+// The Gumbel-max sample argmax_v (z_v - ln E_v) equals argmax_v pe_v / E_v (the
+// exponential race), so within a thread the best is kept as (pb, Eb) and
+// compared by cross-multiplication; pb rescales with the running maximum.  The
+// thread's best is turned into the score l k2 - log2(E) only for the merges.
 constexpr int RP_THREADS = 256;
 constexpr int RP_UNROLL = 4;
 
@@ -149,7 +177,7 @@ __global__ void __launch_bounds__(RP_THREADS) sample_rowpass_kernel(
   float m = -INFINITY, s = 0.f, q = 0.f;
   float amax = -INFINITY;
   int aidx = 0x7FFFFFFF;
-  float best = -INFINITY;
+  float pb = 0.f, eb = 1.f, lb = -INFINITY;  // best of the race: pe, E, raw logit
   int bidx = 0x7FFFFFFF;
 
   for (int base = v0 + threadIdx.x * 4; base < v1; base += RP_THREADS * 4 * RP_UNROLL) {
@@ -164,15 +192,29 @@ __global__ void __launch_bounds__(RP_THREADS) sample_rowpass_kernel(
 #pragma unroll
     for (int u = 0; u < RP_UNROLL; ++u)
       bm = fmaxf(bm, fmaxf(fmaxf(l4[u].x, l4[u].y), fmaxf(l4[u].z, l4[u].w)));
+    if (bm > amax) {
+      // new raw maximum in this batch: first index holding it (ascending order)
+      amax = bm;
+#pragma unroll
+      for (int u = RP_UNROLL - 1; u >= 0; --u) {
+        const int v = base + u * RP_THREADS * 4;
+        if (l4[u].w == bm) aidx = v + 3;
+        if (l4[u].z == bm) aidx = v + 2;
+        if (l4[u].y == bm) aidx = v + 1;
+        if (l4[u].x == bm) aidx = v;
+      }
+    }
     const float bmz = bm * k2;
     if (bmz > m) {
       if (m != -INFINITY) {
-        const float d = m - bmz, f = exp2f(d);
+        const float d = m - bmz, f = sfu_exp2(d);
         q = f * (q + d * s);
-        s = f * s;
+        s *= f;
+        pb *= f;
       }
       m = bmz;
     }
+    const float neg_m = -m;
 #pragma unroll
     for (int u = 0; u < RP_UNROLL; ++u) {
       const int v = base + u * RP_THREADS * 4;
@@ -185,23 +227,21 @@ __global__ void __launch_bounds__(RP_THREADS) sample_rowpass_kernel(
       const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const float zl = lv[e] * k2;
-        const float t = zl - m;
-        const float w = exp2f(t);
-        s += w;
-        q = fmaf(w, t, q);
-        if (lv[e] > amax) {
-          amax = lv[e];
-          aidx = v + e;
-        }
-        const float score = zl - neg_log2_exponential(rw[e]);
-        if (score > best) {
-          best = score;
+        const float t = fmaf(lv[e], k2, neg_m);
+        const float pe = sfu_exp2(t);
+        s += pe;
+        q = fmaf(pe, t, q);
+        const float ev = exp_variate(rw[e]);
+        if (pe * eb > pb * ev) {
+          pb = pe;
+          eb = ev;
+          lb = lv[e];
           bidx = v + e;
         }
       }
     }
   }
+  float best = (bidx == 0x7FFFFFFF) ? -INFINITY : lb * k2 - sfu_log2(eb);
 
   // CTA reduction: warp shuffles, then across warps through shared memory.
 #pragma unroll

@@ -246,7 +246,7 @@ size_t dg_sample_commit_workspace_bytes(int B, int C, int V);
  * device array that every GPU loading the library keeps until process exit;
  * nothing is allocated per call (no cudaMalloc, cudaFree or allocating library
  * routine).  Sizes whose scratch exceeds 4 MiB (dg_sample_commit_workspace_bytes
- * of B, C, V; e.g. B > 16 at C = 256, V = 262144) return
+ * of B, C, V; e.g. B > 32 at C = 256, V = 262144) return
  * DG_ERR_UNSUPPORTED_SHAPE.  The first call on a device looks up the array's
  * device address (cudaGetSymbolAddress) with that device current; make that
  * first call before any stream capture.  All calls share the one array and it
