@@ -9,7 +9,9 @@
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
+#include <cstdlib>
 #include <cstring>
+#include <utility>
 #include <atomic>
 #include <mutex>
 #include <vector>
@@ -29,6 +31,45 @@ constexpr int kNumSMs = 148;
 thread_local char g_last_error[512] = "";
 std::atomic<unsigned long long> g_launches{0};
 inline void count_launch(unsigned long long n = 1) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+// Programmatic dependent launch is on unless DG_PDL=0 is set in the environment.
+bool pdl_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("DG_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
+// Launch with programmatic stream serialization (the kernel must call
+// griddep_wait before touching its predecessors' data) and an optional
+// cluster shape along z.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t s, int cluster_z, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  int n = 0;
+  if (pdl_enabled()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  if (cluster_z > 1) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = 1;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = cluster_z;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
 
 int fail(int status, const char* fmt, ...) {
   va_list ap;
@@ -104,19 +145,30 @@ int make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
 // GEMM
 // ---------------------------------------------------------------------------
 struct GemmPlan {
-  int splits, kb_per_split;
+  int splits, kb_per_split, bn;
 };
 
-// Split K over a cluster of S CTAs (a power of two <= 8) when the output
-// tiles alone would leave most SMs idle; each split keeps >= 4 k-blocks.
+// Choose the token tile (128 or 256) and the K split (cluster of 1, 2 or 4)
+// that puts the most CTAs on the SMs in a single wave, preferring fewer splits
+// and then wider tiles; each split keeps >= 4 k-blocks.  Shapes with more
+// tiles than SMs use 256-token tiles without splitting.
 GemmPlan plan_gemm(int M, int N, int K) {
-  const int tiles = (N / dg::gemm::BM) * cdiv(M, dg::gemm::BN);
   const int kb = K / dg::gemm::BK;
-  int s = 1;
-  while (s * 2 <= dg::gemm::MAX_SPLITS && tiles * s * 2 <= kNumSMs && kb % (s * 2) == 0 &&
-         kb / (s * 2) >= 4)
-    s *= 2;
-  return GemmPlan{s, kb / s};
+  const int ft = N / dg::gemm::BM;
+  GemmPlan best{1, kb, 256};
+  int best_ctas = -1;
+  for (int s : {1, 2, 4}) {
+    for (int bn : {256, 128}) {
+      if (kb % s || kb / s < 4) continue;
+      const int ctas = ft * cdiv(M, bn) * s;
+      if (ctas > kNumSMs) continue;
+      if (ctas > best_ctas) {
+        best = GemmPlan{s, kb / s, bn};
+        best_ctas = ctas;
+      }
+    }
+  }
+  return best;
 }
 
 bool gemm_attr_done = false;
@@ -132,28 +184,36 @@ struct GemmEpi {
   float inv_k = 0.f;
   float eps = 0.f;
   float* ssq_out = nullptr;
+  unsigned long long* trace = nullptr;
 };
+
+template <int S, int BN>
+cudaError_t launch_gemm_t(dim3 grid, cudaStream_t s, const CUtensorMap& tw, const CUtensorMap& tx,
+                          const dg::gemm::Params& p) {
+  return launch_ex(dg::gemm::gemm_kernel<S, BN>, grid, dim3(dg::gemm::THREADS),
+                   dg::gemm::SMEM_BYTES, s, S, tw, tx, p);
+}
+
+template <int S, int BN>
+cudaError_t gemm_set_attr() {
+  return cudaFuncSetAttribute(dg::gemm::gemm_kernel<S, BN>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize, dg::gemm::SMEM_BYTES);
+}
 
 int launch_gemm(const void* x, const void* w, int M, int N, int K, const GemmPlan& pl,
                 const GemmEpi& e, cudaStream_t s) {
   if (!gemm_attr_done) {
-    DG_CUDA(cudaFuncSetAttribute(dg::gemm::gemm_kernel<1>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 dg::gemm::SMEM_BYTES));
-    DG_CUDA(cudaFuncSetAttribute(dg::gemm::gemm_kernel<2>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 dg::gemm::SMEM_BYTES));
-    DG_CUDA(cudaFuncSetAttribute(dg::gemm::gemm_kernel<4>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 dg::gemm::SMEM_BYTES));
-    DG_CUDA(cudaFuncSetAttribute(dg::gemm::gemm_kernel<8>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 dg::gemm::SMEM_BYTES));
+    DG_CUDA((gemm_set_attr<1, 256>()));
+    DG_CUDA((gemm_set_attr<2, 256>()));
+    DG_CUDA((gemm_set_attr<4, 256>()));
+    DG_CUDA((gemm_set_attr<1, 128>()));
+    DG_CUDA((gemm_set_attr<2, 128>()));
+    DG_CUDA((gemm_set_attr<4, 128>()));
     gemm_attr_done = true;
   }
   CUtensorMap tw, tx;
   DG_TRY(make_tmap(&tw, w, K, N, (uint64_t)K * 2, dg::gemm::BM));
-  DG_TRY(make_tmap(&tx, x, K, M, (uint64_t)K * 2, dg::gemm::BN));
+  DG_TRY(make_tmap(&tx, x, K, M, (uint64_t)K * 2, pl.bn));
   dg::gemm::Params p;
   p.M = M; p.N = N; p.K = K;
   p.kb_per_split = pl.kb_per_split;
@@ -167,25 +227,25 @@ int launch_gemm(const void* x, const void* w, int M, int N, int K, const GemmPla
   p.inv_k = e.inv_k;
   p.eps = e.eps;
   p.ssq_out = e.ssq_out;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(N / dg::gemm::BM, cdiv(M, dg::gemm::BN), pl.splits);
-  cfg.blockDim = dim3(dg::gemm::THREADS, 1, 1);
-  cfg.dynamicSmemBytes = dg::gemm::SMEM_BYTES;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = pl.splits;
-  cfg.attrs = attr;
-  cfg.numAttrs = pl.splits > 1 ? 1 : 0;
-  switch (pl.splits) {
-    case 1: DG_CUDA(cudaLaunchKernelEx(&cfg, dg::gemm::gemm_kernel<1>, tw, tx, p)); break;
-    case 2: DG_CUDA(cudaLaunchKernelEx(&cfg, dg::gemm::gemm_kernel<2>, tw, tx, p)); break;
-    case 4: DG_CUDA(cudaLaunchKernelEx(&cfg, dg::gemm::gemm_kernel<4>, tw, tx, p)); break;
-    case 8: DG_CUDA(cudaLaunchKernelEx(&cfg, dg::gemm::gemm_kernel<8>, tw, tx, p)); break;
-    default: return fail(DG_ERR_UNSUPPORTED_SHAPE, "split count %d", pl.splits);
+  p.trace = e.trace;
+  const dim3 grid(N / dg::gemm::BM, cdiv(M, pl.bn), pl.splits);
+  cudaError_t err = cudaErrorInvalidValue;
+  if (pl.bn == 256) {
+    switch (pl.splits) {
+      case 1: err = launch_gemm_t<1, 256>(grid, s, tw, tx, p); break;
+      case 2: err = launch_gemm_t<2, 256>(grid, s, tw, tx, p); break;
+      case 4: err = launch_gemm_t<4, 256>(grid, s, tw, tx, p); break;
+    }
+  } else if (pl.bn == 128) {
+    switch (pl.splits) {
+      case 1: err = launch_gemm_t<1, 128>(grid, s, tw, tx, p); break;
+      case 2: err = launch_gemm_t<2, 128>(grid, s, tw, tx, p); break;
+      case 4: err = launch_gemm_t<4, 128>(grid, s, tw, tx, p); break;
+    }
   }
+  if (err != cudaSuccess)
+    return fail(DG_ERR_CUDA, "gemm launch (S=%d, BN=%d) failed: %s", pl.splits, pl.bn,
+                cudaGetErrorString(err));
   count_launch();
   return DG_OK;
 }
@@ -252,8 +312,8 @@ int launch_attn(const void* q, int ldq, const void* k_new, const void* v_new, in
                                    dg::attn::Cfg<128>::SMEM_BYTES));
       attn_attr_done[1] = true;
     }
-    dg::attn::attn_kernel<128><<<grid, dg::attn::THREADS, dg::attn::Cfg<128>::SMEM_BYTES, s>>>(
-        tq, tkn, tvn, tkc, tvc, p);
+    DG_CUDA(launch_ex(dg::attn::attn_kernel<128>, grid, dim3(dg::attn::THREADS),
+                      dg::attn::Cfg<128>::SMEM_BYTES, s, 1, tq, tkn, tvn, tkc, tvc, p));
     count_launch();
   } else {
     if (!attn_attr_done[0]) {
@@ -262,8 +322,8 @@ int launch_attn(const void* q, int ldq, const void* k_new, const void* v_new, in
                                    dg::attn::Cfg<64>::SMEM_BYTES));
       attn_attr_done[0] = true;
     }
-    dg::attn::attn_kernel<64><<<grid, dg::attn::THREADS, dg::attn::Cfg<64>::SMEM_BYTES, s>>>(
-        tq, tkn, tvn, tkc, tvc, p);
+    DG_CUDA(launch_ex(dg::attn::attn_kernel<64>, grid, dim3(dg::attn::THREADS),
+                      dg::attn::Cfg<64>::SMEM_BYTES, s, 1, tq, tkn, tvn, tkc, tvc, p));
     count_launch();
   }
   DG_CUDA(cudaGetLastError());
@@ -272,11 +332,13 @@ int launch_attn(const void* q, int ldq, const void* k_new, const void* v_new, in
     const int threads = 256;
     const int blocks = cdiv(rows * 32, threads);
     if (hd == 128)
-      dg::attn::attn_combine_kernel<128><<<blocks, threads, 0, s>>>(
-          p.part_o, p.part_lse, S, B, Hq, Lq, (__nv_bfloat16*)out, ldo, lse);
+      DG_CUDA(launch_ex(dg::attn::attn_combine_kernel<128>, dim3(blocks), dim3(threads), 0, s, 1,
+                        (const float*)p.part_o, (const float*)p.part_lse, S, B, Hq, Lq,
+                        (__nv_bfloat16*)out, ldo, lse));
     else
-      dg::attn::attn_combine_kernel<64><<<blocks, threads, 0, s>>>(
-          p.part_o, p.part_lse, S, B, Hq, Lq, (__nv_bfloat16*)out, ldo, lse);
+      DG_CUDA(launch_ex(dg::attn::attn_combine_kernel<64>, dim3(blocks), dim3(threads), 0, s, 1,
+                        (const float*)p.part_o, (const float*)p.part_lse, S, B, Hq, Lq,
+                        (__nv_bfloat16*)out, ldo, lse));
     count_launch();
     DG_CUDA(cudaGetLastError());
   }
@@ -326,17 +388,16 @@ int launch_sample(const float* logits, int32_t* tok, uint8_t* committed, int32_t
                   int32_t* seq_status, const dg::SampleParams& p, const dg_step_out* out,
                   void* ws, cudaStream_t s) {
   dg::RowPartial* part = (dg::RowPartial*)ws;
-  dg::sample_rowpass_kernel<<<p.B * p.C * p.nchunk, dg::RP_THREADS, 0, s>>>(logits, seq_status,
-                                                                             p, part);
+  DG_CUDA(launch_ex(dg::sample_rowpass_kernel, dim3(p.B * p.C * p.nchunk), dim3(dg::RP_THREADS),
+                    0, s, 1, logits, (const int32_t*)seq_status, p, part));
   count_launch();
-  DG_CUDA(cudaGetLastError());
   const int threads = (p.C + 31) / 32 * 32;
-  dg::sample_commit_kernel<<<p.B, threads, 0, s>>>(
-      logits, part, p, tok, committed, prev_argmax, seq_status, out ? out->x_hat : nullptr,
-      out ? out->argmax : nullptr, out ? out->logconf : nullptr, out ? out->entropy : nullptr,
-      out ? out->flags : nullptr);
+  DG_CUDA(launch_ex(dg::sample_commit_kernel, dim3(p.B), dim3(threads), 0, s, 1, logits,
+                    (const dg::RowPartial*)part, p, tok, committed, prev_argmax, seq_status,
+                    out ? out->x_hat : (int32_t*)nullptr, out ? out->argmax : (int32_t*)nullptr,
+                    out ? out->logconf : (float*)nullptr, out ? out->entropy : (float*)nullptr,
+                    out ? out->flags : (uint8_t*)nullptr));
   count_launch();
-  DG_CUDA(cudaGetLastError());
   return DG_OK;
 }
 
@@ -467,8 +528,8 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
   const float scale = 1.0f / std::sqrt((float)hd);
   const int nt = c.d / 128;
 
-  dg::gemm::embed_kernel<<<M, dg::gemm::EMBED_THREADS, 0, s>>>(
-      tok, (const __nv_bfloat16*)f.m->embed, c.vocab, c.d, M, x, xb, ssq_x);
+  DG_CUDA(launch_ex(dg::gemm::embed_kernel, dim3(M), dim3(dg::gemm::EMBED_THREADS), 0, s, 1, tok,
+                    (const __nv_bfloat16*)f.m->embed, c.vocab, c.d, M, x, xb, ssq_x));
   count_launch();
   DG_CUDA(cudaGetLastError());
   for (int l = 0; l < c.n_layers; ++l) {
@@ -508,7 +569,7 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
     el.epi = dg::gemm::EPI_F32;
     el.out_f32 = logits;
     el.ssq_in = ssq_x; el.n_ssq_in = nt; el.inv_k = 1.f / c.d; el.eps = c.eps;
-    DG_TRY(launch_gemm(xb, f.m->unembed, M, c.vocab, c.d, GemmPlan{1, c.d / dg::gemm::BK}, el,
+    DG_TRY(launch_gemm(xb, f.m->unembed, M, c.vocab, c.d, GemmPlan{1, c.d / dg::gemm::BK, 256}, el,
                        s));
   }
   return DG_OK;
@@ -648,7 +709,7 @@ int dg_unembed(const void* h, const void* w_u, float* logits, int M, int d, int 
   GemmEpi e;
   e.epi = dg::gemm::EPI_F32;
   e.out_f32 = logits;
-  return launch_gemm(h, w_u, M, V, d, GemmPlan{1, d / dg::gemm::BK}, e, (cudaStream_t)stream);
+  return launch_gemm(h, w_u, M, V, d, GemmPlan{1, d / dg::gemm::BK, 256}, e, (cudaStream_t)stream);
 }
 
 size_t dg_linear_workspace_bytes(int M, int N, int K) {

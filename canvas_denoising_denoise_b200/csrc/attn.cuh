@@ -104,6 +104,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int split = blockIdx.y;
   const int i0 = qt * BQ;
 
+  griddep_wait();
+  griddep_launch();
   int L = p.cache_len[b];
   if (L < 0 || L > p.lmax) {
     if (threadIdx.x == 0 && split == 0 && qt == 0 && h == 0) raise_error(ERR_CHECK | 0x301, b);
@@ -440,6 +442,8 @@ __global__ void attn_combine_kernel(const float* __restrict__ part_o,
                                     const float* __restrict__ part_lse, int S, int B, int Hq,
                                     int Lq, __nv_bfloat16* __restrict__ out, int ldo,
                                     float* __restrict__ lse) {
+  griddep_wait();
+  griddep_launch();
   const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
   const int rows = B * Hq * Lq;

@@ -37,6 +37,17 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 // microseconds; two seconds means something upstream never arrived.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start before its predecessor finishes; it must call
+// griddep_wait() before reading anything an earlier kernel wrote (or writing
+// anything an earlier kernel reads).  griddep_launch() lets the successor be
+// scheduled once every CTA of this grid has issued it.  Both are no-ops for a
+// normally ordered launch.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -37,21 +37,25 @@ namespace dg {
 namespace gemm {
 
 constexpr int BM = 128;  // output features per tile (UMMA M)
-constexpr int BN = 256;  // tokens per tile (UMMA N)
 constexpr int BK = 64;   // K per stage: one 128-byte swizzle row of bf16
 constexpr int A_BYTES = BM * BK * 2;
-constexpr int B_BYTES = BN * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int STAGES = 4;
 constexpr int THREADS = 192;
 constexpr int WARPS = THREADS / 32;
-constexpr int TMEM_COLS = BN;
-constexpr int STAGE_AREA = STAGES * STAGE_BYTES;          // also holds the fp32 tile
+constexpr int RING_BYTES = 192 * 1024;                    // TMA stage ring (also holds the fp32 tile)
 constexpr int TILE_ROW_FLOATS = BM;                       // staged tile: [BN][BM] fp32
-constexpr int SMEM_BYTES = 1024 + STAGE_AREA + BN * 4 + 256;
+constexpr int SMEM_BYTES = 1024 + RING_BYTES + 256 * 4 + 256;
 constexpr int MAX_SPLITS = 8;
-constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, false, false);
-static_assert(BN * BM * 4 <= STAGE_AREA, "staged tile must fit in the stage ring");
+
+// BN: tokens per tile (UMMA N), 128 or 256.
+template <int BN>
+struct TileCfg {
+  static constexpr int B_BYTES = BN * BK * 2;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int STAGES = RING_BYTES / STAGE_BYTES;  // 4 (BN 256) or 6 (BN 128)
+  static constexpr int TMEM_COLS = BN;
+  static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, false, false);
+  static_assert(BN * BM * 4 <= RING_BYTES, "staged tile must fit in the stage ring");
+};
 
 enum Epi : int { EPI_F32 = 0, EPI_BF16 = 1, EPI_GELU = 2, EPI_RESID = 3 };
 
@@ -68,7 +72,16 @@ struct Params {
   float inv_k;             // 1 / (input width) for the mean
   float eps;
   float* ssq_out;          // [N / 128, M] (EPI_RESID), or null
+  unsigned long long* trace;  // optional [grid, 8] %globaltimer stamps of the phases
 };
+
+__device__ __forceinline__ void trace_stamp(const Params& p, int slot) {
+  if (p.trace) {
+    const size_t cta = (static_cast<size_t>(blockIdx.z) * gridDim.y + blockIdx.y) * gridDim.x +
+                       blockIdx.x;
+    p.trace[cta * 8 + slot] = globaltimer_ns();
+  }
+}
 
 __device__ __forceinline__ float gelu_erf(float x) {
   return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
@@ -102,17 +115,21 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
   return v;
 }
 
-template <int S>
+template <int S, int BN>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                 Params p) {
   static_assert(S == 1 || S == 2 || S == 4 || S == 8, "split count");
+  using TC = TileCfg<BN>;
+  constexpr int STAGES = TC::STAGES;
+  constexpr int STAGE_BYTES = TC::STAGE_BYTES;
+  constexpr int TMEM_COLS = TC::TMEM_COLS;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   float* tile = reinterpret_cast<float*>(smem);  // [BN][BM] after the mainloop
-  float* rowscale = reinterpret_cast<float*>(smem + STAGE_AREA);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGE_AREA + BN * 4);
+  float* rowscale = reinterpret_cast<float*>(smem + RING_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + RING_BYTES + 256 * 4);
   uint64_t* empty = full + STAGES;
   uint64_t* acc_full = empty + STAGES;
   uint64_t* drain = acc_full + 1;
@@ -128,6 +145,7 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int nkb = min(p.kb_per_split, p.K / BK - kb_begin);
 
   if (threadIdx.x == 0) {
+    trace_stamp(p, 0);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -149,15 +167,27 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_acc = *tmem_holder;
+  if (threadIdx.x == 0) trace_stamp(p, 1);
 
+  griddep_launch();
   if (warp == 0) {
     if (lane == 0 && nkb > 0) {
       const uint64_t pol_w = l2_policy_evict_first();
-      int issued = 0;
-      for (int kb = 0; kb < nkb; ++kb) {
+      // the weights are never written by another kernel: the first stages'
+      // weight tiles are requested before waiting on the predecessor
+      const int pre = min(STAGES, nkb);
+      for (int kb = 0; kb < pre; ++kb) {
+        mbar_expect_tx(&full[kb], STAGE_BYTES);
+        tma_load_2d_hint(smem + kb * STAGE_BYTES, &tm_w, &full[kb], (kb_begin + kb) * BK, f0,
+                         pol_w);
+      }
+      griddep_wait();
+      for (int kb = 0; kb < pre; ++kb)
+        tma_load_2d(smem + kb * STAGE_BYTES + A_BYTES, &tm_x, &full[kb], (kb_begin + kb) * BK, t0);
+      int issued = pre;
+      for (int kb = pre; kb < nkb; ++kb) {
         const int st = kb % STAGES;
-        if (kb >= STAGES && !mbar_wait(&empty[st], ((kb / STAGES) - 1) & 1, abort_flag, 0x101))
-          break;
+        if (!mbar_wait(&empty[st], ((kb / STAGES) - 1) & 1, abort_flag, 0x101)) break;
         uint8_t* a = smem + st * STAGE_BYTES;
         mbar_expect_tx(&full[st], STAGE_BYTES);
         const int kx = (kb_begin + kb) * BK;
@@ -169,27 +199,33 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int kb = max(0, issued - STAGES); kb < issued; ++kb)
           mbar_wait(&full[kb % STAGES], (kb / STAGES) & 1, nullptr, 0x102);
       }
+    } else {
+      griddep_wait();
     }
   } else if (warp == 1) {
+    griddep_wait();
     if (lane == 0 && nkb > 0) {
       for (int kb = 0; kb < nkb; ++kb) {
         const int st = kb % STAGES;
         if (!mbar_wait(&full[st], (kb / STAGES) & 1, abort_flag, 0x103)) break;
+        if (kb == 0) trace_stamp(p, 2);
         tc_fence_after();
         const uint32_t a_base = smem_u32(smem + st * STAGE_BYTES);
         const uint32_t b_base = a_base + A_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk) {
           umma_ss(tmem_acc, sdesc_sw128(a_base + kk * 32, 16, 1024),
-                  sdesc_sw128(b_base + kk * 32, 16, 1024), IDESC, (kb | kk) != 0 ? 1u : 0u);
+                  sdesc_sw128(b_base + kk * 32, 16, 1024), TC::IDESC, (kb | kk) != 0 ? 1u : 0u);
         }
         umma_commit(&empty[st]);
       }
+      trace_stamp(p, 3);
       umma_commit(acc_full);
       umma_commit(drain);
       mbar_wait(drain, 0, nullptr, 0x104);
     }
   } else {
+    griddep_wait();
     // warps 2..5: row scales for this tile's tokens while the mainloop runs
     for (int t = threadIdx.x - 64; t < BN; t += THREADS - 64) {
       float rs = 1.f;
@@ -205,18 +241,23 @@ __global__ void __launch_bounds__(THREADS, 1)
     const bool have_acc =
         nkb > 0 && __all_sync(0xffffffffu, mbar_wait(acc_full, 0, abort_flag, 0x105));
     if (have_acc) {
+      if (threadIdx.x == 64) trace_stamp(p, 4);
       tc_fence_after();
       const int quarter = warp & 3;
       const int fl = quarter * 32 + lane;
       const uint32_t taddr = tmem_acc + (static_cast<uint32_t>(quarter * 32) << 16);
-      for (int c = 0; c < BN / 32; ++c) {
+      for (int c = 0; c < BN / 32; c += 2) {
         if (t0 + c * 32 >= p.M) break;  // warp-uniform
-        uint32_t r[32];
-        tmem_ld32(taddr + c * 32, r);
+        uint32_t r0[32], r1[32];
+        tmem_ld32(taddr + c * 32, r0);
+        tmem_ld32(taddr + c * 32 + 32, r1);
         tmem_ld_wait();
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          tile[(c * 32 + j) * TILE_ROW_FLOATS + fl] = __uint_as_float(r[j]);
+          tile[(c * 32 + j) * TILE_ROW_FLOATS + fl] = __uint_as_float(r0[j]);
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          tile[(c * 32 + 32 + j) * TILE_ROW_FLOATS + fl] = __uint_as_float(r1[j]);
       }
     } else {
       // no accumulator (empty split or an abandoned wait): contribute zeros
@@ -229,6 +270,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     cluster_sync();
   else
     __syncthreads();
+  if (threadIdx.x == 0) trace_stamp(p, 5);
 
   // ---------------------------------------------------------------- reduce + epilogue
   // CTA r owns token rows [r*BN/S, (r+1)*BN/S) of the tile.  A warp gathers
@@ -298,9 +340,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
   }
+  if (threadIdx.x == 0) trace_stamp(p, 6);
   // no CTA leaves while a peer may still read its shared memory
   if constexpr (S > 1) cluster_sync();
   __syncthreads();
+  if (threadIdx.x == 0) trace_stamp(p, 7);
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_acc, TMEM_COLS);
@@ -314,6 +358,8 @@ constexpr int EMBED_THREADS = 256;
 __global__ void __launch_bounds__(EMBED_THREADS) embed_kernel(
     const int32_t* __restrict__ tok, const __nv_bfloat16* __restrict__ embed, int V, int d, int M,
     float* __restrict__ x, __nv_bfloat16* __restrict__ xb, float* __restrict__ ssq) {
+  griddep_wait();
+  griddep_launch();
   const int t = blockIdx.x;
   int id = tok[t];
   if (id < 0 || id >= V) {

@@ -160,6 +160,8 @@ constexpr int RP_UNROLL = 4;
 __global__ void __launch_bounds__(RP_THREADS) sample_rowpass_kernel(
     const float* __restrict__ logits, const int32_t* __restrict__ seq_status, SampleParams p,
     RowPartial* __restrict__ part) {
+  griddep_wait();
+  griddep_launch();
   const int row = blockIdx.x / p.nchunk;
   const int ck = blockIdx.x - row * p.nchunk;
   const int b = row / p.C;
@@ -284,6 +286,8 @@ __global__ void __launch_bounds__(1024) sample_commit_kernel(
   __shared__ float s_red[32];
   __shared__ int s_flag;
 
+  griddep_wait();
+  griddep_launch();
   const int b = blockIdx.x;
   if (seq_status[b] != 0) return;
   const int i = threadIdx.x;
