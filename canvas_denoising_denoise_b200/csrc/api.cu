@@ -259,16 +259,21 @@ int linear(const void* x, const void* w, int M, int N, int K, const GemmEpi& e,
 // ---------------------------------------------------------------------------
 // Attention
 // ---------------------------------------------------------------------------
-int attn_splits(int B, int Hq, int Lq, int max_prefix) {
-  const int qtiles = B * Hq * cdiv(Lq, dg::attn::BQ);
+// CTAs before splitting the key range: pairs of 128-row query tiles per kv head.
+int attn_pairs(int Hq, int Hkv, int Lq) {
+  return cdiv((Hq / Hkv) * cdiv(Lq, dg::attn::BQ), 2);
+}
+
+int attn_splits(int B, int Hq, int Hkv, int Lq, int max_prefix) {
+  const int units = B * Hkv * attn_pairs(Hq, Hkv, Lq);
   const int tmax = cdiv(max_prefix, dg::attn::BKV) + cdiv(Lq, dg::attn::BKV);
-  int s = std::max(1, kNumSMs / std::max(1, qtiles));
+  int s = std::max(1, kNumSMs / std::max(1, units));
   s = std::min(s, std::max(1, tmax / 2));
   return s;
 }
 
-size_t attn_ws_bytes(int B, int Hq, int Lq, int hd, int max_prefix) {
-  const int S = attn_splits(B, Hq, Lq, max_prefix);
+size_t attn_ws_bytes(int B, int Hq, int Hkv, int Lq, int hd, int max_prefix) {
+  const int S = attn_splits(B, Hq, Hkv, Lq, max_prefix);
   if (S == 1) return 0;
   const size_t rows = (size_t)S * B * Hq * Lq;
   return align_up(rows * hd * sizeof(float), 256) + align_up(rows * sizeof(float), 256);
@@ -280,7 +285,7 @@ int launch_attn(const void* q, int ldq, const void* k_new, const void* v_new, in
                 const void* k_cache, const void* v_cache, const int32_t* cache_len,
                 int max_prefix, int lmax, void* out, int ldo, float* lse, int B, int Hq, int Hkv,
                 int Lq, int hd, float scale, int mask, void* ws, cudaStream_t s) {
-  const int S = attn_splits(B, Hq, Lq, max_prefix);
+  const int S = attn_splits(B, Hq, Hkv, Lq, max_prefix);
   CUtensorMap tq, tkn, tvn, tkc, tvc;
   DG_TRY(make_tmap(&tq, q, (uint64_t)Hq * hd, (uint64_t)B * Lq, (uint64_t)ldq * 2, 128));
   DG_TRY(make_tmap(&tkn, k_new, (uint64_t)Hkv * hd, (uint64_t)B * Lq, (uint64_t)ldkv * 2, 128));
@@ -289,7 +294,8 @@ int launch_attn(const void* q, int ldq, const void* k_new, const void* v_new, in
   DG_TRY(make_tmap(&tvc, v_cache, hd, (uint64_t)B * Hkv * lmax, (uint64_t)hd * 2, 128));
   dg::attn::Params p;
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.lmax = lmax; p.group = Hq / Hkv;
-  p.n_qtiles = cdiv(Lq, dg::attn::BQ);
+  p.n_rt = cdiv(Lq, dg::attn::BQ);
+  p.n_pairs = attn_pairs(Hq, Hkv, Lq);
   p.n_splits = S;
   p.causal = mask == DG_MASK_CAUSAL ? 1 : 0;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -304,7 +310,7 @@ int launch_attn(const void* q, int ldq, const void* k_new, const void* v_new, in
     p.part_o = (float*)ws;
     p.part_lse = (float*)((char*)ws + align_up(rows * hd * sizeof(float), 256));
   }
-  dim3 grid(B * Hq * p.n_qtiles, S);
+  dim3 grid(B * Hkv * p.n_pairs, S);
   if (hd == 128) {
     if (!attn_attr_done[1]) {
       DG_CUDA(cudaFuncSetAttribute(dg::attn::attn_kernel<128>,
@@ -492,7 +498,7 @@ FwdLayout fwd_layout(const dg_model_cfg& c, int B, int Lq, int max_prefix, bool 
   L.up = take((size_t)M * c.ffn * 2);
   L.ssq_x = take((size_t)(c.d / 128) * M * 4);
   L.ssq_h = take((size_t)(c.d / 128) * M * 4);
-  L.attn = take(attn_ws_bytes(B, c.n_q_heads, Lq, c.head_dim, max_prefix));
+  L.attn = take(attn_ws_bytes(B, c.n_q_heads, c.n_kv_heads, Lq, c.head_dim, max_prefix));
   L.logits = take(logits ? (size_t)M * c.vocab * 4 : 0);
   L.spart = take(logits ? sample_ws_bytes(B, Lq, c.vocab) : 0);
   L.flag = take(logits ? 16 : 0);
@@ -666,9 +672,10 @@ int dg_check_device_errors(void* stream, uint32_t* code_out) {
 }
 
 size_t dg_canvas_attn_workspace_bytes(int B, int Hq, int Hkv, int Lq, int hd, int max_prefix) {
-  (void)Hkv;
-  if (B <= 0 || Hq <= 0 || Lq <= 0 || (hd != 64 && hd != 128) || max_prefix < 0) return 0;
-  return attn_ws_bytes(B, Hq, Lq, hd, max_prefix);
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || Lq <= 0 || (hd != 64 && hd != 128) ||
+      max_prefix < 0)
+    return 0;
+  return attn_ws_bytes(B, Hq, Hkv, Lq, hd, max_prefix);
 }
 
 int dg_canvas_attn(const void* q, int ldq, const void* k_new, const void* v_new, int ldkv,
@@ -688,7 +695,7 @@ int dg_canvas_attn(const void* q, int ldq, const void* k_new, const void* v_new,
   if (!aligned16(q) || !aligned16(k_new) || !aligned16(v_new) || !aligned16(k_cache) ||
       !aligned16(v_cache) || !aligned16(out))
     return fail(DG_ERR_ALIGNMENT, "dg_canvas_attn: pointers must be 16-byte aligned");
-  const size_t need = attn_ws_bytes(B, Hq, Lq, hd, max_prefix);
+  const size_t need = attn_ws_bytes(B, Hq, Hkv, Lq, hd, max_prefix);
   if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
     return fail(DG_ERR_WORKSPACE_TOO_SMALL, "dg_canvas_attn: workspace needs %zu bytes", need);
   return launch_attn(q, ldq, k_new, v_new, ldkv, k_cache, v_cache, cache_len, max_prefix, lmax,

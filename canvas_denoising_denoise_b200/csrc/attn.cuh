@@ -9,20 +9,22 @@
 // KV cache); "DiffusionGemma Guia do Desenvolvedor ...", bullet "Propagacao
 // de Contexto Bidirecional".
 //
-// One CTA = 128 query rows of one head over a contiguous range of 128-key
-// tiles (the key range is split across CTAs when there are too few query
-// tiles to fill the SMs; a combine kernel merges the splits by their
-// log-sum-exp).  Per key tile j:
-//     S_j = Q K_j^T            tcgen05.mma, A = Q (smem), B = K_j (smem), D in TMEM
-//     P_j = 2^(S_j*c - m)      softmax warps: TMEM -> registers -> bf16 -> TMEM
-//     O  += P_j V_j            tcgen05.mma, A = P_j (TMEM), B = V_j (smem, MN-major)
-// S is double-buffered in TMEM so S_{j+1} runs on the tensor core while the
-// softmax warps work on S_j; P_j overwrites S_j in place.  The running max is
-// only raised (and O rescaled) when it grows by more than 2^8, so most tiles
-// need no O round trip; the final 1/l normalisation makes this exact.
+// One CTA = two 128-row query tiles that share a kv head, over a contiguous
+// range of 128-key tiles (the key range is split across CTAs when there are
+// too few query tiles to fill the SMs; a combine kernel merges the splits by
+// their log-sum-exp).  Per key tile j and query tile X in {A, B}:
+//     S_X = Q_X K_j^T          tcgen05.mma, A = Q_X (smem), B = K_j (smem), D in TMEM
+//     P_X = 2^(S_X*c - m_X)    softmax warpgroup X: TMEM -> registers -> bf16 -> TMEM
+//     O_X += P_X V_j           tcgen05.mma, A = P_X (TMEM), B = V_j (smem, MN-major)
+// Each K/V tile is loaded once for both query tiles.  The two softmax
+// warpgroups ping-pong: while one works, the tensor core runs the other
+// tile's MMAs.  P_X overwrites S_X in place.  The running max is only raised
+// (and O rescaled) when it grows by more than 2^8, so most tiles need no O
+// round trip; the final 1/l normalisation makes this exact.
 //
-// Warps: 0 = TMA producer, 1 = TMEM owner + MMA issuer, 2..5 = softmax (one
-// query row per thread; warp w owns TMEM lanes 32*(w%4)..+31).
+// Warps: 0 = TMA producer, 1 = TMEM owner + MMA issuer, 2..5 = softmax of
+// tile A, 6..9 = softmax of tile B (one query row per thread; warp w owns
+// TMEM lanes 32*(w%4)..+31).
 #pragma once
 
 #include "dg_common.cuh"
@@ -32,8 +34,8 @@ namespace attn {
 
 constexpr int BQ = 128;
 constexpr int BKV = 128;
-constexpr int THREADS = 192;
-constexpr int TMEM_COLS = 512;  // S0 [0,128), S1 [128,256), O [256, 256+hd)
+constexpr int THREADS = 320;    // warp 0 TMA, warp 1 MMA, warps 2-5 softmax A, warps 6-9 softmax B
+constexpr int TMEM_COLS = 512;  // S_A [0,128) S_B [128,256) O_A [256,384) O_B [384,512)
 constexpr float kRescaleThreshold = 8.0f;
 
 // 2^x on the special-function unit (flushes denormal results to zero, which
@@ -50,14 +52,16 @@ struct Cfg {
   static constexpr int Q_BYTES = BQ * HD * 2;
   static constexpr int T_BYTES = BKV * HD * 2;  // one K or V tile
   static constexpr int STAGES = HD == 128 ? 2 : 3;
-  static constexpr int SMEM_BYTES = 1024 + Q_BYTES + STAGES * 2 * T_BYTES + 256;
+  static constexpr int SMEM_BYTES = 1024 + 2 * Q_BYTES + STAGES * 2 * T_BYTES + 256;
   static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BQ, BKV, false, false);
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BQ, HD, false, true);
 };
 
 struct Params {
   int B, Hq, Hkv, Lq, lmax, group;
-  int n_qtiles, n_splits, causal;
+  int n_rt;        // 128-row tiles per head
+  int n_pairs;     // CTAs (per kv head and split) = ceil(group * n_rt / 2)
+  int n_splits, causal;
   float scale_log2;          // scale * log2(e)
   const int32_t* cache_len;  // [B]
   __nv_bfloat16* out;        // [B, Lq, ldo]
@@ -67,6 +71,13 @@ struct Params {
   float* part_lse;           // [S, B, Hq, Lq]
 };
 
+// One CTA = two 128-row query tiles that read the same kv head (the query
+// tiles of a kv head are ordered row tile first, so a pair shares its row
+// tile whenever the group size is even), over one contiguous range of
+// 128-key tiles.  The tensor core alternates [PV_A(j), S_A(j+1)] and
+// [PV_B(j), S_B(j+1)] so that one softmax warpgroup works while the other
+// tile's MMAs run.  S_X(j+1) is issued after PV_X(j), so once S_X(j+1) is
+// complete, O_X is stable and may be rescaled in TMEM.
 template <int HD>
 __global__ void __launch_bounds__(THREADS, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kn,
@@ -78,40 +89,48 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + CF::Q_BYTES;             // ST tiles
-  uint8_t* sV = sK + ST * CF::T_BYTES;        // ST tiles
+  uint8_t* sQ = smem;                          // [2][Q_BYTES]
+  uint8_t* sK = sQ + 2 * CF::Q_BYTES;          // ST tiles
+  uint8_t* sV = sK + ST * CF::T_BYTES;         // ST tiles
   uint64_t* bars = reinterpret_cast<uint64_t*>(sV + ST * CF::T_BYTES);
   uint64_t* q_full = bars;
   uint64_t* k_full = q_full + 1;       // [ST]
   uint64_t* v_full = k_full + ST;      // [ST]
   uint64_t* kv_empty = v_full + ST;    // [ST]
-  uint64_t* s_full = kv_empty + ST;    // [2]
-  uint64_t* p_full = s_full + 2;       // [2]
-  uint64_t* o_done = p_full + 2;       // one completion per PV (rescale waits)
-  uint64_t* o_final = o_done + 1;      // single completion after the last PV
+  uint64_t* s_full = kv_empty + ST;    // [2] per tile
+  uint64_t* p_full = s_full + 2;       // [2] per tile
+  uint64_t* o_final = p_full + 2;      // after the last PV of both tiles
   uint64_t* drain = o_final + 1;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
   const int warp = warp_id();
   const int lane = lane_id();
-  const int qt = blockIdx.x % p.n_qtiles;
-  const int bh = blockIdx.x / p.n_qtiles;
-  const int h = bh % p.Hq;
-  const int b = bh / p.Hq;
-  const int g = h / p.group;
+  const int pi = blockIdx.x % p.n_pairs;
+  const int g = (blockIdx.x / p.n_pairs) % p.Hkv;
+  const int b = blockIdx.x / (p.n_pairs * p.Hkv);
   const int split = blockIdx.y;
-  const int i0 = qt * BQ;
+  const int nq = p.group * p.n_rt;  // query tiles of this kv head
+  int hX[2], i0X[2];
+  bool vX[2];
+#pragma unroll
+  for (int X = 0; X < 2; ++X) {
+    const int qi = 2 * pi + X;
+    vX[X] = qi < nq;
+    const int qq = vX[X] ? qi : 2 * pi;
+    hX[X] = g * p.group + qq % p.group;
+    i0X[X] = (qq / p.group) * BQ;
+  }
 
   griddep_wait();
   griddep_launch();
   int L = p.cache_len[b];
   if (L < 0 || L > p.lmax) {
-    if (threadIdx.x == 0 && split == 0 && qt == 0 && h == 0) raise_error(ERR_CHECK | 0x301, b);
+    if (threadIdx.x == 0 && split == 0 && pi == 0 && g == 0) raise_error(ERR_CHECK | 0x301, b);
     L = L < 0 ? 0 : p.lmax;
   }
-  const int lq_vis = p.causal ? min(p.Lq, i0 + BQ) : p.Lq;
+  const int i0max = max(i0X[0], vX[1] ? i0X[1] : 0);
+  const int lq_vis = p.causal ? min(p.Lq, i0max + BQ) : p.Lq;
   const int nP = (L + BKV - 1) / BKV;
   const int nC = (lq_vis + BKV - 1) / BKV;
   const int T = nP + nC;
@@ -121,10 +140,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (n <= 0) {
     // empty key range: this split contributes nothing to the merge
-    if (threadIdx.x < BQ) {
-      const int qrow = i0 + threadIdx.x;
+    for (int X = 0; X < 2; ++X) {
+      if (!vX[X] || threadIdx.x >= BQ) continue;
+      const int qrow = i0X[X] + threadIdx.x;
       if (qrow < p.Lq) {
-        const size_t r = ((static_cast<size_t>(split) * p.B + b) * p.Hq + h) * p.Lq + qrow;
+        const size_t r = ((static_cast<size_t>(split) * p.B + b) * p.Hq + hX[X]) * p.Lq + qrow;
         p.part_lse[r] = -INFINITY;
         float4* o = reinterpret_cast<float4*>(p.part_o + r * HD);
         for (int c = 0; c < HD / 4; ++c) o[c] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -144,7 +164,6 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(&s_full[s], 1);
       mbar_init(&p_full[s], BQ);
     }
-    mbar_init(o_done, 1);
     mbar_init(o_final, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -165,14 +184,16 @@ __global__ void __launch_bounds__(THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_holder;
-  const uint32_t tmem_o = tmem + 256;
+  const bool vB = vX[1];
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      mbar_expect_tx(q_full, CF::Q_BYTES);
-      for (int hf = 0; hf < CF::HALVES; ++hf)
-        tma_load_2d(sQ + hf * (BQ * 128), &tm_q, q_full, h * HD + hf * 64, b * p.Lq + i0);
+      mbar_expect_tx(q_full, CF::Q_BYTES * (vB ? 2 : 1));
+      for (int X = 0; X < (vB ? 2 : 1); ++X)
+        for (int hf = 0; hf < CF::HALVES; ++hf)
+          tma_load_2d(sQ + X * CF::Q_BYTES + hf * (BQ * 128), &tm_q, q_full,
+                      hX[X] * HD + hf * 64, b * p.Lq + i0X[X]);
       int issued = 0;
       for (int i = 0; i < n; ++i) {
         const int st = i % ST;
@@ -215,168 +236,174 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (lane == 0) {
       bool ok = mbar_wait(q_full, 0, abort_flag, 0x321);
       const uint32_t q_base = smem_u32(sQ);
-      auto issue_s = [&](int i) -> bool {
-        const int st = i % ST;
-        if (!mbar_wait(&k_full[st], (i / ST) & 1, abort_flag, 0x322)) return false;
-        tc_fence_after();
-        const uint32_t k_base = smem_u32(sK + st * CF::T_BYTES);
-        const uint32_t d = tmem + (i & 1) * 128;
+      auto issue_s = [&](int X, int i) {
+        const uint32_t k_base = smem_u32(sK + (i % ST) * CF::T_BYTES);
+        const uint32_t qb = q_base + X * CF::Q_BYTES;
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-          umma_ss(d, sdesc_sw128(q_base + off, 16, 1024), sdesc_sw128(k_base + off, 16, 1024),
-                  CF::IDESC_QK, kk > 0 ? 1u : 0u);
+          umma_ss(tmem + X * 128, sdesc_sw128(qb + off, 16, 1024),
+                  sdesc_sw128(k_base + off, 16, 1024), CF::IDESC_QK, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&s_full[i & 1]);
-        return true;
+        umma_commit(&s_full[X]);
       };
-      auto issue_pv = [&](int j) -> bool {
-        const int st = j % ST;
-        if (!mbar_wait(&p_full[j & 1], (j >> 1) & 1, abort_flag, 0x323)) return false;
-        if (!mbar_wait(&v_full[st], (j / ST) & 1, abort_flag, 0x324)) return false;
+      auto issue_pv = [&](int X, int j) -> bool {
+        if (!mbar_wait(&p_full[X], j & 1, abort_flag, 0x323)) return false;
         tc_fence_after();
-        const uint32_t v_base = smem_u32(sV + st * CF::T_BYTES);
-        const uint32_t pa = tmem + (j & 1) * 128;
+        const uint32_t v_base = smem_u32(sV + (j % ST) * CF::T_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk) {
-          // keys 16kk..16kk+15: rows of the MN-major V tile, 128 B each
-          umma_ts(tmem_o, pa + kk * 8,
+        for (int kk = 0; kk < BKV / 16; ++kk)
+          umma_ts(tmem + 256 + X * 128, tmem + X * 128 + kk * 8,
                   sdesc_sw128(v_base + kk * 16 * 128, BKV * 128, 1024), CF::IDESC_PV,
                   (j > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(&kv_empty[st]);
-        umma_commit(o_done);
         return true;
       };
-      if (ok) ok = issue_s(0);
-      for (int i = 1; ok && i < n; ++i) {
-        ok = issue_s(i);
-        if (ok) ok = issue_pv(i - 1);
+      if (ok) ok = mbar_wait(&k_full[0], 0, abort_flag, 0x322);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0, 0);
+        if (vB) issue_s(1, 0);
       }
-      if (ok) ok = issue_pv(n - 1);
+      for (int j = 0; ok && j < n; ++j) {
+        ok = mbar_wait(&v_full[j % ST], (j / ST) & 1, abort_flag, 0x324);
+        if (ok) ok = issue_pv(0, j);
+        const bool more = j + 1 < n;
+        if (ok && more) {
+          ok = mbar_wait(&k_full[(j + 1) % ST], ((j + 1) / ST) & 1, abort_flag, 0x322);
+          if (ok) {
+            tc_fence_after();
+            issue_s(0, j + 1);
+          }
+        }
+        if (ok && vB) ok = issue_pv(1, j);
+        if (ok) umma_commit(&kv_empty[j % ST]);
+        if (ok && vB && more) issue_s(1, j + 1);
+      }
       if (ok) umma_commit(o_final);
       umma_commit(drain);
       mbar_wait(drain, 0, nullptr, 0x325);
     }
   } else {
-    // ------------------------------------------------------------ softmax
+    // ------------------------------------------------------------ softmax (tile X)
+    const int X = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
-    const int qrow = i0 + r;
+    const int qrow = i0X[X] + r;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem + X * 128 + lane_off;
+    const uint32_t tO = tmem + 256 + X * 128 + lane_off;
     float m = -INFINITY;  // running max in scaled log2 units
     float l = 0.f;
-    bool ok = true;
-    for (int i = 0; i < n && ok; ++i) {
-      const int sb = i & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[sb], (i >> 1) & 1, abort_flag, 0x331))) {
+    bool ok = vX[X];
+    for (int j = 0; j < n && ok; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[X], j & 1, abort_flag, 0x331))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      uint32_t sr[128];
-      {
-        uint32_t(&c0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
-        uint32_t(&c1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-        uint32_t(&c2)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[64]);
-        uint32_t(&c3)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[96]);
-        const uint32_t base = tmem + sb * 128 + lane_off;
-        tmem_ld32(base + 0, c0);
-        tmem_ld32(base + 32, c1);
-        tmem_ld32(base + 64, c2);
-        tmem_ld32(base + 96, c3);
-        tmem_ld_wait();
-      }
-      // key validity of this tile for this row
-      const int t = t_beg + i;
-      int nvalid;      // keys [0, nvalid) of the tile may be valid
-      int causal_lim;  // canvas key index limit (inclusive) for causal rows
-      bool canvas = t >= nP;
-      if (!canvas) {
-        nvalid = min(BKV, L - t * BKV);
-        causal_lim = 0x7FFFFFFF;
+      // key validity of this tile for this row: keys [0, lim] may be valid
+      const int t = t_beg + j;
+      int lim;
+      if (t < nP) {
+        lim = min(BKV, L - t * BKV) - 1;
       } else {
         const int ck0 = (t - nP) * BKV;
-        nvalid = min(BKV, p.Lq - ck0);
-        causal_lim = p.causal ? (qrow - ck0) : 0x7FFFFFFF;
+        lim = min(BKV, p.Lq - ck0) - 1;
+        if (p.causal) lim = min(lim, qrow - ck0);
       }
-      const int lim = min(nvalid - 1, causal_lim);  // valid keys: [0, lim]
-      // masking only where some row of this warp has invalid keys
-      if (__any_sync(0xffffffffu, lim < BKV - 1)) {
-#pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c > lim) sr[c] = __float_as_uint(-INFINITY);
-      }
-      // row max of the raw scores (the scale is positive), four chains for ILP
+      const bool masked = __any_sync(0xffffffffu, lim < BKV - 1);
+      // pass 1: row max of the raw scores (the scale is positive)
       float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; c += 4) {
-        mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
-        mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
-        mx2 = fmaxf(mx2, __uint_as_float(sr[c + 2]));
-        mx3 = fmaxf(mx3, __uint_as_float(sr[c + 3]));
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t sa[32], sb[32];
+        tmem_ld32(tS + h2 * 64, sa);
+        tmem_ld32(tS + h2 * 64 + 32, sb);
+        tmem_ld_wait();
+        if (masked) {
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            if (h2 * 64 + c > lim) sa[c] = __float_as_uint(-INFINITY);
+            if (h2 * 64 + 32 + c > lim) sb[c] = __float_as_uint(-INFINITY);
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 32; c += 2) {
+          mx0 = fmaxf(mx0, __uint_as_float(sa[c]));
+          mx1 = fmaxf(mx1, __uint_as_float(sa[c + 1]));
+          mx2 = fmaxf(mx2, __uint_as_float(sb[c]));
+          mx3 = fmaxf(mx3, __uint_as_float(sb[c + 1]));
+        }
       }
       const float tmax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
-      // The decision is taken per warp: the TMEM loads/stores below are
-      // warp-collective (.sync.aligned) and must see all 32 lanes.  Lanes whose
-      // own max did not move rescale by exactly 1.
+      // Raise the running max only when it grows by more than 2^8 (the final
+      // 1/l keeps this exact).  Decided per warp: TMEM accesses are
+      // warp-collective.  PV_X(j-1) is complete because S_X(j) is.
       const bool want = tmax > m + kRescaleThreshold || m == -INFINITY;
       if (__any_sync(0xffffffffu, want)) {
         const float m_new = fmaxf(tmax, m);
-        if (i > 0) {
-          // O holds PV_0..PV_{i-1}; wait for the last one, then rescale in TMEM
-          if (!__all_sync(0xffffffffu, mbar_wait(o_done, (i - 1) & 1, abort_flag, 0x332))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const float f = (m == -INFINITY) ? 0.f : exp2f(m - m_new);
+        if (j > 0) {
+          const float f = (m == -INFINITY) ? 0.f : fast_exp2(m - m_new);
 #pragma unroll
           for (int c = 0; c < HD / 32; ++c) {
             uint32_t o[32];
-            tmem_ld32(tmem_o + lane_off + c * 32, o);
+            tmem_ld32(tO + c * 32, o);
             tmem_ld_wait();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * f);
-            tmem_st32(tmem_o + lane_off + c * 32, o);
+            tmem_st32(tO + c * 32, o);
           }
-          tmem_st_wait();
           l *= f;
         }
         m = m_new;
       }
       const float neg_m = (m == -INFINITY) ? 0.f : -m;
       float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
-      uint32_t pk[64];
+      // pass 2: re-read S in halves, exponentiate, pack P over the consumed columns
 #pragma unroll
-      for (int c = 0; c < 64; c += 2) {
-        const float p0 = fast_exp2(fmaf(__uint_as_float(sr[2 * c]), p.scale_log2, neg_m));
-        const float p1 = fast_exp2(fmaf(__uint_as_float(sr[2 * c + 1]), p.scale_log2, neg_m));
-        const float p2 = fast_exp2(fmaf(__uint_as_float(sr[2 * c + 2]), p.scale_log2, neg_m));
-        const float p3 = fast_exp2(fmaf(__uint_as_float(sr[2 * c + 3]), p.scale_log2, neg_m));
-        rs0 += p0;
-        rs1 += p1;
-        rs2 += p2;
-        rs3 += p3;
-        pk[c] = pack_bf16x2(p0, p1);
-        pk[c + 1] = pack_bf16x2(p2, p3);
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t sa[64];
+        {
+          uint32_t(&c0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sa[0]);
+          uint32_t(&c1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sa[32]);
+          tmem_ld32(tS + h2 * 64, c0);
+          tmem_ld32(tS + h2 * 64 + 32, c1);
+          tmem_ld_wait();
+        }
+        if (masked) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (h2 * 64 + c > lim) sa[c] = __float_as_uint(-INFINITY);
+        }
+#pragma unroll
+        for (int q2 = 0; q2 < 2; ++q2) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; c += 2) {
+            const int k0 = q2 * 32 + 2 * c;
+            const float p0 = fast_exp2(fmaf(__uint_as_float(sa[k0]), p.scale_log2, neg_m));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(sa[k0 + 1]), p.scale_log2, neg_m));
+            const float p2 = fast_exp2(fmaf(__uint_as_float(sa[k0 + 2]), p.scale_log2, neg_m));
+            const float p3 = fast_exp2(fmaf(__uint_as_float(sa[k0 + 3]), p.scale_log2, neg_m));
+            rs0 += p0;
+            rs1 += p1;
+            rs2 += p2;
+            rs3 += p3;
+            pk[c] = pack_bf16x2(p0, p1);
+            pk[c + 1] = pack_bf16x2(p2, p3);
+          }
+          tmem_st16(tS + h2 * 32 + q2 * 16, pk);
+        }
       }
-      const float rs = (rs0 + rs1) + (rs2 + rs3);
-      l += rs;
-      {
-        uint32_t(&a0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[0]);
-        uint32_t(&a1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&pk[32]);
-        const uint32_t base = tmem + sb * 128 + lane_off;
-        tmem_st32(base + 0, a0);
-        tmem_st32(base + 32, a1);
-        tmem_st_wait();
-      }
+      l += (rs0 + rs1) + (rs2 + rs3);
+      tmem_st_wait();
       tc_fence_before();
-      mbar_arrive(&p_full[sb]);
+      mbar_arrive(&p_full[X]);
     }
     const bool fin = __all_sync(0xffffffffu, ok && mbar_wait(o_final, 0, abort_flag, 0x333));
     if (fin) {
       tc_fence_after();
+      const int h = hX[X];
       const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
       const float lse_nat = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
       const bool store = qrow < p.Lq;
@@ -386,7 +413,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int c = 0; c < HD / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(tmem_o + lane_off + c * 32, o);
+          tmem_ld32(tO + c * 32, o);
           tmem_ld_wait();
           if (store) {
             uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
@@ -412,7 +439,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int c = 0; c < HD / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(tmem_o + lane_off + c * 32, o);
+          tmem_ld32(tO + c * 32, o);
           tmem_ld_wait();
           if (store) {
 #pragma unroll
