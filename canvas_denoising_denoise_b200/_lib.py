@@ -3,7 +3,8 @@ import ctypes
 import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "libdg.so")
+# DG_LIB_PATH selects another build of the library (e.g. a tuning variant)
+LIB_PATH = os.environ.get("DG_LIB_PATH") or os.path.join(HERE, "libdg.so")
 
 c_int = ctypes.c_int
 c_float = ctypes.c_float

@@ -228,7 +228,7 @@ int launch_gemm(const void* x, const void* w, int M, int N, int K, const GemmPla
   p.eps = e.eps;
   p.ssq_out = e.ssq_out;
   p.trace = e.trace;
-  const dim3 grid(N / dg::gemm::BM, cdiv(M, pl.bn), pl.splits);
+  const dim3 grid(cdiv(M, pl.bn), N / dg::gemm::BM, pl.splits);
   cudaError_t err = cudaErrorInvalidValue;
   if (pl.bn == 256) {
     switch (pl.splits) {
@@ -265,18 +265,25 @@ int attn_pairs(int Hq, int Hkv, int Lq) {
 }
 
 int attn_splits(int B, int Hq, int Hkv, int Lq, int max_prefix) {
+  static const int forced = [] {
+    const char* e = getenv("DG_ATTN_SPLITS");  // tuning override
+    return e ? atoi(e) : 0;
+  }();
   const int units = B * Hkv * attn_pairs(Hq, Hkv, Lq);
+  if (forced > 0)
+    return std::min({forced, dg::attn::MAX_SPLITS,
+                     std::max(1, cdiv(max_prefix, dg::attn::BKV) + cdiv(Lq, dg::attn::BKV))});
   const int tmax = cdiv(max_prefix, dg::attn::BKV) + cdiv(Lq, dg::attn::BKV);
   int s = std::max(1, kNumSMs / std::max(1, units));
   s = std::min(s, std::max(1, tmax / 2));
-  return s;
+  return std::min(s, dg::attn::MAX_SPLITS);
 }
 
 size_t attn_ws_bytes(int B, int Hq, int Hkv, int Lq, int hd, int max_prefix) {
   const int S = attn_splits(B, Hq, Hkv, Lq, max_prefix);
   if (S == 1) return 0;
   const size_t rows = (size_t)S * B * Hq * Lq;
-  return align_up(rows * hd * sizeof(float), 256) + align_up(rows * sizeof(float), 256);
+  return align_up(rows * hd * 2, 256) + align_up(rows * sizeof(float), 256);
 }
 
 bool attn_attr_done[2] = {false, false};
@@ -307,8 +314,8 @@ int launch_attn(const void* q, int ldq, const void* k_new, const void* v_new, in
   p.part_lse = nullptr;
   if (S > 1) {
     const size_t rows = (size_t)S * B * Hq * Lq;
-    p.part_o = (float*)ws;
-    p.part_lse = (float*)((char*)ws + align_up(rows * hd * sizeof(float), 256));
+    p.part_o = (__nv_bfloat16*)ws;
+    p.part_lse = (float*)((char*)ws + align_up(rows * hd * 2, 256));
   }
   dim3 grid(B * Hkv * p.n_pairs, S);
   if (hd == 128) {
@@ -339,11 +346,11 @@ int launch_attn(const void* q, int ldq, const void* k_new, const void* v_new, in
     const int blocks = cdiv(rows * 32, threads);
     if (hd == 128)
       DG_CUDA(launch_ex(dg::attn::attn_combine_kernel<128>, dim3(blocks), dim3(threads), 0, s, 1,
-                        (const float*)p.part_o, (const float*)p.part_lse, S, B, Hq, Lq,
+                        (const __nv_bfloat16*)p.part_o, (const float*)p.part_lse, S, B, Hq, Lq,
                         (__nv_bfloat16*)out, ldo, lse));
     else
       DG_CUDA(launch_ex(dg::attn::attn_combine_kernel<64>, dim3(blocks), dim3(threads), 0, s, 1,
-                        (const float*)p.part_o, (const float*)p.part_lse, S, B, Hq, Lq,
+                        (const __nv_bfloat16*)p.part_o, (const float*)p.part_lse, S, B, Hq, Lq,
                         (__nv_bfloat16*)out, ldo, lse));
     count_launch();
     DG_CUDA(cudaGetLastError());

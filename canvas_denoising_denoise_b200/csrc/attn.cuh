@@ -34,7 +34,7 @@ namespace attn {
 
 constexpr int BQ = 128;
 constexpr int BKV = 128;
-constexpr int THREADS = 320;    // warp 0 TMA, warp 1 MMA, warps 2-5 softmax A, warps 6-9 softmax B
+constexpr int THREADS = 320;  // warp 0 TMA, warp 1 MMA, warps 2-5 softmax A, warps 6-9 softmax B
 constexpr int TMEM_COLS = 512;  // S_A [0,128) S_B [128,256) O_A [256,384) O_B [384,512)
 constexpr float kRescaleThreshold = 8.0f;
 
@@ -67,9 +67,10 @@ struct Params {
   __nv_bfloat16* out;        // [B, Lq, ldo]
   int ldo;
   float* lse;                // [B, Hq, Lq] natural log, or null
-  float* part_o;             // [S, B, Hq, Lq, hd] fp32 (n_splits > 1)
+  __nv_bfloat16* part_o;     // [S, B, Hq, Lq, hd] bf16 (n_splits > 1)
   float* part_lse;           // [S, B, Hq, Lq]
 };
+
 
 // One CTA = two 128-row query tiles that read the same kv head (the query
 // tiles of a kv head are ordered row tile first, so a pair shares its row
@@ -146,8 +147,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (qrow < p.Lq) {
         const size_t r = ((static_cast<size_t>(split) * p.B + b) * p.Hq + hX[X]) * p.Lq + qrow;
         p.part_lse[r] = -INFINITY;
-        float4* o = reinterpret_cast<float4*>(p.part_o + r * HD);
-        for (int c = 0; c < HD / 4; ++c) o[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+        uint4* o = reinterpret_cast<uint4*>(p.part_o + r * HD);
+        for (int c = 0; c < HD / 8; ++c) o[c] = make_uint4(0u, 0u, 0u, 0u);
       }
     }
     return;
@@ -359,7 +360,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       const float neg_m = (m == -INFINITY) ? 0.f : -m;
       float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
-      // pass 2: re-read S in halves, exponentiate, pack P over the consumed columns
+      // pass 2: re-read S in halves, exponentiate, pack P (bf16 pairs) over
+      // the consumed columns
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
         uint32_t sa[64];
@@ -401,56 +403,60 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_arrive(&p_full[X]);
     }
     const bool fin = __all_sync(0xffffffffu, ok && mbar_wait(o_final, 0, abort_flag, 0x333));
+    // Stage O_X (fp32, 1/l applied) in the K/V ring, which is idle once the
+    // last PV has completed: row r at [X][r][HD] with its 16-byte chunks
+    // XOR-swizzled by (r & 7) so that both the row-per-thread writes and the
+    // row-per-warp reads are bank-conflict free.  Then each warp writes whole
+    // rows: coalesced stores instead of one 16-byte piece per row per lane.
+    float* stage = reinterpret_cast<float*>(sK) + X * (BQ * HD);
+    const int h = hX[X];
+    const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+    const float lse_nat = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
     if (fin) {
       tc_fence_after();
-      const int h = hX[X];
-      const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
-      const float lse_nat = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
-      const bool store = qrow < p.Lq;
-      if (p.n_splits == 1) {
-        __nv_bfloat16* orow =
-            p.out + (static_cast<size_t>(b) * p.Lq + qrow) * p.ldo + static_cast<size_t>(h) * HD;
 #pragma unroll
-        for (int c = 0; c < HD / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
-          tmem_ld_wait();
-          if (store) {
-            uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+      for (int c = 0; c < HD / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + c * 32, o);
+        tmem_ld_wait();
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              uint4 w;
-              w.x = pack_bf16x2(__uint_as_float(o[8 * v + 0]) * inv_l,
-                                __uint_as_float(o[8 * v + 1]) * inv_l);
-              w.y = pack_bf16x2(__uint_as_float(o[8 * v + 2]) * inv_l,
-                                __uint_as_float(o[8 * v + 3]) * inv_l);
-              w.z = pack_bf16x2(__uint_as_float(o[8 * v + 4]) * inv_l,
-                                __uint_as_float(o[8 * v + 5]) * inv_l);
-              w.w = pack_bf16x2(__uint_as_float(o[8 * v + 6]) * inv_l,
-                                __uint_as_float(o[8 * v + 7]) * inv_l);
-              dst[v] = w;
-            }
+        for (int v = 0; v < 8; ++v) {
+          const int chunk = (c * 8 + v) ^ (r & 7);
+          reinterpret_cast<float4*>(stage + r * HD)[chunk] =
+              make_float4(__uint_as_float(o[4 * v]) * inv_l, __uint_as_float(o[4 * v + 1]) * inv_l,
+                          __uint_as_float(o[4 * v + 2]) * inv_l,
+                          __uint_as_float(o[4 * v + 3]) * inv_l);
+        }
+      }
+      if (qrow < p.Lq) {
+        if (p.n_splits == 1) {
+          if (p.lse) p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Lq + qrow] = lse_nat;
+        } else {
+          p.part_lse[((static_cast<size_t>(split) * p.B + b) * p.Hq + h) * p.Lq + qrow] = lse_nat;
+        }
+      }
+    }
+    // the four warps of this tile's warpgroup meet here (named barrier 1 + X)
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + X), "r"(BQ) : "memory");
+    if (fin) {
+      constexpr int CPR = HD / 4;  // 16-byte chunks per row
+      for (int rr = quarter; rr < BQ; rr += 4) {
+        const int qr = i0X[X] + rr;
+        if (qr >= p.Lq) break;
+        for (int cc = lane; cc < CPR; cc += 32) {
+          const float4 v = reinterpret_cast<const float4*>(stage + rr * HD)[cc ^ (rr & 7)];
+          uint2 w;
+          w.x = pack_bf16x2(v.x, v.y);
+          w.y = pack_bf16x2(v.z, v.w);
+          if (p.n_splits == 1) {
+            *reinterpret_cast<uint2*>(p.out + (static_cast<size_t>(b) * p.Lq + qr) * p.ldo +
+                                      static_cast<size_t>(h) * HD + cc * 4) = w;
+          } else {
+            const size_t row =
+                ((static_cast<size_t>(split) * p.B + b) * p.Hq + h) * p.Lq + qr;
+            *reinterpret_cast<uint2*>(p.part_o + row * HD + cc * 4) = w;
           }
         }
-        if (store && p.lse) p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Lq + qrow] = lse_nat;
-      } else {
-        const size_t rr = ((static_cast<size_t>(split) * p.B + b) * p.Hq + h) * p.Lq + qrow;
-        float4* dst = reinterpret_cast<float4*>(p.part_o + rr * HD);
-#pragma unroll
-        for (int c = 0; c < HD / 32; ++c) {
-          uint32_t o[32];
-          tmem_ld32(tO + c * 32, o);
-          tmem_ld_wait();
-          if (store) {
-#pragma unroll
-            for (int v = 0; v < 8; ++v)
-              dst[c * 8 + v] = make_float4(__uint_as_float(o[4 * v]) * inv_l,
-                                           __uint_as_float(o[4 * v + 1]) * inv_l,
-                                           __uint_as_float(o[4 * v + 2]) * inv_l,
-                                           __uint_as_float(o[4 * v + 3]) * inv_l);
-          }
-        }
-        if (store) p.part_lse[rr] = lse_nat;
       }
     }
   }
@@ -463,9 +469,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // Merge key-range splits: O = sum_s w_s O_s / sum_s w_s, w_s = exp(lse_s - max).
-// One warp per (b, h, row); lane covers 4 (hd = 128) or 2 (hd = 64) columns.
+// One warp per (b, h, row): lane s holds split s's weight (S <= 32), and the
+// split rows are loaded in batches of 8 so that the loads overlap.
+constexpr int MAX_SPLITS = 32;
+
 template <int HD>
-__global__ void attn_combine_kernel(const float* __restrict__ part_o,
+__global__ void attn_combine_kernel(const __nv_bfloat16* __restrict__ part_o,
                                     const float* __restrict__ part_lse, int S, int B, int Hq,
                                     int Lq, __nv_bfloat16* __restrict__ out, int ldo,
                                     float* __restrict__ lse) {
@@ -476,21 +485,43 @@ __global__ void attn_combine_kernel(const float* __restrict__ part_o,
   const int rows = B * Hq * Lq;
   if (warp_global >= rows) return;
   const size_t stride = static_cast<size_t>(rows);
-  float mx = -INFINITY;
-  for (int s = 0; s < S; ++s) mx = fmaxf(mx, part_lse[s * stride + warp_global]);
+  const float ls = lane < S ? part_lse[lane * stride + warp_global] : -INFINITY;
+  float mx = ls;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const float w = (ls == -INFINITY || mx == -INFINITY) ? 0.f : expf(ls - mx);
+  const float wsum = warp_sum(w);
   constexpr int PER = HD / 32;
   float acc[PER];
 #pragma unroll
   for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  float wsum = 0.f;
-  for (int s = 0; s < S; ++s) {
-    const float ls = part_lse[s * stride + warp_global];
-    if (ls == -INFINITY) continue;
-    const float w = expf(ls - mx);
-    wsum += w;
-    const float* src = part_o + (s * stride + warp_global) * HD + lane * PER;
+  for (int s0 = 0; s0 < S; s0 += 8) {
+    float v[8][PER];
 #pragma unroll
-    for (int e = 0; e < PER; ++e) acc[e] += w * src[e];
+    for (int k = 0; k < 8; ++k) {
+      if (s0 + k < S) {
+        const __nv_bfloat16* src = part_o + ((s0 + k) * stride + warp_global) * HD + lane * PER;
+        if constexpr (PER == 4) {
+          const uint2 t = *reinterpret_cast<const uint2*>(src);
+          const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&t.x);
+          const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&t.y);
+          v[k][0] = __low2float(lo); v[k][1] = __high2float(lo);
+          v[k][2] = __low2float(hi); v[k][3] = __high2float(hi);
+        } else {
+          const uint32_t t = *reinterpret_cast<const uint32_t*>(src);
+          const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&t);
+          v[k][0] = __low2float(lo); v[k][1] = __high2float(lo);
+        }
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float wk = __shfl_sync(0xffffffffu, w, (s0 + k) & 31);
+      if (s0 + k < S && wk > 0.f) {
+#pragma unroll
+        for (int e = 0; e < PER; ++e) acc[e] += wk * v[k][e];
+      }
+    }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
   const int qrow = warp_global % Lq;
@@ -499,8 +530,14 @@ __global__ void attn_combine_kernel(const float* __restrict__ part_o,
   const int b = bh / Hq;
   __nv_bfloat16* dst = out + (static_cast<size_t>(b) * Lq + qrow) * ldo +
                        static_cast<size_t>(h) * HD + lane * PER;
-#pragma unroll
-  for (int e = 0; e < PER; ++e) dst[e] = __float2bfloat16_rn(acc[e] * inv);
+  if constexpr (PER == 4) {
+    uint2 wv;
+    wv.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    wv.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+    *reinterpret_cast<uint2*>(dst) = wv;
+  } else {
+    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  }
   if (lse && lane == 0) lse[warp_global] = (wsum > 0.f) ? mx + logf(wsum) : -INFINITY;
 }
 

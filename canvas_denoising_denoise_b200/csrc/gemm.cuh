@@ -138,8 +138,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int warp = warp_id();
   const int lane = lane_id();
-  const int f0 = blockIdx.x * BM;
-  const int t0 = blockIdx.y * BN;
+  // token tile fastest: the CTAs that share a weight tile start together, so
+  // the second reader finds it in L2
+  const int t0 = blockIdx.x * BN;
+  const int f0 = blockIdx.y * BM;
   const int split = blockIdx.z;
   const int kb_begin = split * p.kb_per_split;
   const int nkb = min(p.kb_per_split, p.K / BK - kb_begin);
@@ -172,7 +174,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   griddep_launch();
   if (warp == 0) {
     if (lane == 0 && nkb > 0) {
-      const uint64_t pol_w = l2_policy_evict_first();
+      // weights are streamed once: evict them first unless another token tile
+      // of this launch reads the same weight tile
+      const uint64_t pol_w = gridDim.x > 1 ? l2_policy_evict_normal() : l2_policy_evict_first();
       // the weights are never written by another kernel: the first stages'
       // weight tiles are requested before waiting on the predecessor
       const int pre = min(STAGES, nkb);
@@ -321,7 +325,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         if (p.ssq_out) {
           const float sq = warp_sum(xv.x * xv.x + xv.y * xv.y + xv.z * xv.z + xv.w * xv.w);
-          if (lane == 0) p.ssq_out[static_cast<size_t>(blockIdx.x) * p.M + tg] = sq;
+          if (lane == 0) p.ssq_out[static_cast<size_t>(blockIdx.y) * p.M + tg] = sq;
         }
       } else {
         const float rs = rowscale[t];
