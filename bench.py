@@ -141,6 +141,31 @@ def time_region(fn, steps, stream):
     return start.elapsed_time(end) / 1000.0
 
 
+def captured_traffic(profile, sources):
+    """DRAM bytes per launch from a committed ncu summary, or None when the
+    kernel sources changed since the capture (hash recorded in the summary)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", profile)
+    if not os.path.exists(path):
+        return None
+    h = hashlib.sha256()
+    for src in sources:
+        with open(os.path.join(ROOT, "canvas_denoising_denoise_b200", "csrc", src), "rb") as f:
+            h.update(f.read())
+    fields = {}
+    with open(path) as f:
+        for line in f:
+            if ":" in line and not line.startswith(("#", "|", " ")):
+                k, v = line.split(":", 1)
+                fields[k.strip()] = v.strip()
+    if fields.get("kernel_sources_sha256_16") != h.hexdigest()[:16]:
+        return None
+    try:
+        return int(fields["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
 def gemm_roofline(dg, model, shape, batch, peaks, stream):
     """Achieved TFLOP/s of the tcgen05 GEMM kernel on the unembedding launch.
 
@@ -170,7 +195,10 @@ def gemm_roofline(dg, model, shape, batch, peaks, stream):
     peak = peaks["bf16_tflops"]
     return {"kernel": "gemm_kernel (unembedding launch)", "bound": "tensor",
             "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-            "frac": round(achieved / peak, 4), "traffic": None,
+            "frac": round(achieved / peak, 4),
+            "traffic": (captured_traffic("gemm_unembed_full.md", ["gemm.cuh", "dg_common.cuh"])
+                        if batch == 1 else None),
+            "algorithmic_bytes": int(V * d * 2 + M * V * 4 + M * d * 2),
             "peak_source": f"{peaks['source']} burst bf16",
             "launch_us": round(t * 1e6, 1), "flops_per_launch": flops}
 
@@ -350,6 +378,20 @@ def run_kernel_bench(args):
                     "gbs": round(byts / t / 1e9, 1),
                     "frac_hbm_peak": round(byts / t / 1e9 / peaks["hbm_gbs"], 4),
                     "committed_tokens_per_s": round(16 * B / t, 1)})
+    elif args.kernel == "unembed":
+        # the unembedding launch of the full workload: logits [256, 262144] fp32
+        M, d, V = 256 * args.batch, 2048, 262144
+        h = torch.randn((M, d), device="cuda").to(torch.bfloat16)
+        w = (torch.randn((V, d), device="cuda") * 0.02).to(torch.bfloat16)
+        lg = torch.empty((M, V), dtype=torch.float32, device="cuda")
+        t = timed(lambda: dg.unembed(h, w, lg), args.steps)
+        fl = 2.0 * M * V * d
+        byts = V * d * 2 + M * V * 4 + M * d * 2
+        out.append({"kernel": "unembed", "shape": [M, V, d], "us": round(t * 1e6, 2),
+                    "tflops": round(fl / t / 1e12, 1),
+                    "frac_bf16_peak": round(fl / t / 1e12 / peaks["bf16_tflops"], 4),
+                    "gbs": round(byts / t / 1e9, 1),
+                    "frac_hbm_peak": round(byts / t / 1e9 / peaks["hbm_gbs"], 4)})
     elif args.kernel == "gemm":
         M, N, K = (int(x) for x in args.shape.split(","))
         x = torch.randn((M, K), device="cuda").to(torch.bfloat16)
@@ -375,7 +417,7 @@ def main():
     ap.add_argument("--workload", default="full", choices=["full", "tiny"])
     ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["attn", "sampler", "gemm"], default=None,
+    ap.add_argument("--kernel", choices=["attn", "sampler", "gemm", "unembed"], default=None,
                     help="time one kernel alone instead of the denoising step")
     ap.add_argument("--prefix", type=int, default=0)
     ap.add_argument("--batch", type=int, default=1)
