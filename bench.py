@@ -102,10 +102,21 @@ class ClockSampler:
 
 
 def dist_env():
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return rank, world, local
+    from canvas_denoising_denoise_b200 import replicas
+    e = replicas.rank_env()
+    return e.rank, e.world, e.local
+
+
+def workload_config(name, world, steps_per_block=None):
+    """The `config` object of both arms' JSON lines."""
+    shape, batch, prompt = workload_spec(name)
+    return {"workload": name, "model": "random-init dense stand-in", "batch": batch,
+            "prompt": prompt, "canvas": CANVAS, "d": shape.d, "layers": shape.n_layers,
+            "heads": [shape.n_q_heads, shape.n_kv_heads], "head_dim": shape.head_dim,
+            "ffn": shape.ffn, "vocab": shape.vocab, "steps_per_block": steps_per_block,
+            "parallelism": f"replicas x{world}",
+            "l2": ("inputs larger than L2 (3.3 GB of weights streamed per step)"
+                   if shape.vocab * shape.d * 2 > L2_BYTES else "weights fit in L2")}
 
 
 def workload_spec(name):
@@ -297,8 +308,7 @@ def run_reference(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(CANVAS / v * 1e3, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
-            "config": {"workload": args.workload, "batch": batch, "prompt": prompt,
-                       "canvas": CANVAS},
+            "config": workload_config(args.workload, world, 48),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": vals[0]["cores"],
                              "kind": "oracle", "sample": vals[0]["sample"]},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -432,16 +442,15 @@ def main():
         return run_reference(args)
 
     import torch
-    import torch.distributed as dist
 
     import canvas_denoising_denoise_b200 as dg
-    from canvas_denoising_denoise_b200 import synth
+    from canvas_denoising_denoise_b200 import replicas, synth
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        replicas.init("nccl", timeout_s=120)
+    seeds = replicas.replica_seeds(rank)
     lib = dg._lib.load()
     shape, batch, prompt_len = workload_spec(args.workload)
     peaks = load_peaks()
@@ -457,7 +466,7 @@ def main():
     model = dg.DgModel(shape, weights)
     lmax = prompt_len + CANVAS
     st = dg.DgState(shape, batch, lmax, CANVAS)
-    prompt = synth.make_prompt(batch, prompt_len, shape.vocab, seed=1 + rank).cuda()
+    prompt = synth.make_prompt(batch, prompt_len, shape.vocab, seed=seeds.prompt).cuda()
     ws = dg.Workspace()
     ws.get(max(dg.denoise_workspace_bytes(model, st),
                lib.dg_prefill_workspace_bytes(ctypes_ref(model.cfg), batch, prompt_len)))
@@ -465,7 +474,7 @@ def main():
     torch.cuda.synchronize()
     dg.check_device_errors()
     settings = dg.SamplerSettings()
-    seed = 1000 + rank
+    seed = seeds.sampler
     steps_seen = []
 
     def block_step():
@@ -480,8 +489,7 @@ def main():
 
     # ---------------------------------------------------------------- timed
     clocks = ClockSampler(torch.cuda.current_device())
-    if world > 1:
-        dist.barrier()
+    replicas.barrier(world)
     torch.cuda.synchronize()
     clocks.start()
     time.sleep(0.3)
@@ -490,17 +498,13 @@ def main():
     elapsed = time_region(block_step, args.steps, stream)
     launches = lib.dg_launch_count() - n0
     clk = clocks.stop()
-    if world > 1:
-        t = torch.tensor([elapsed], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        elapsed = float(t.item())
-        dist.barrier()
+    elapsed = replicas.max_over_ranks(elapsed, world)
+    replicas.barrier(world)
     dg.check_device_errors()
-    tokens = world * batch * CANVAS * args.steps
-    value = tokens / elapsed
+    value = replicas.whole_job_rate(batch * CANVAS * args.steps, world, elapsed)
 
     # ---------------------------------------------------------------- end to end
-    host_prompt = synth.make_prompt(batch, prompt_len, shape.vocab, seed=1 + rank).pin_memory()
+    host_prompt = synth.make_prompt(batch, prompt_len, shape.vocab, seed=seeds.prompt).pin_memory()
     host_out = torch.empty((batch, CANVAS), dtype=torch.int32).pin_memory()
     dev_prompt = torch.empty_like(prompt)
 
@@ -511,14 +515,10 @@ def main():
         host_out.copy_(st.tok, non_blocking=True)
 
     e2e_step()
-    if world > 1:
-        dist.barrier()
+    replicas.barrier(world)
     e2e_t = time_region(e2e_step, max(1, args.steps // 2), stream)
-    if world > 1:
-        t = torch.tensor([e2e_t], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_t = float(t.item())
-    e2e_val = world * batch * CANVAS * max(1, args.steps // 2) / e2e_t
+    e2e_t = replicas.max_over_ranks(e2e_t, world)
+    e2e_val = replicas.whole_job_rate(batch * CANVAS * max(1, args.steps // 2), world, e2e_t)
 
     # ---------------------------------------------------------------- roofline
     roof = gemm_roofline(dg, model, shape, batch, peaks, stream)
@@ -537,14 +537,8 @@ def main():
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(elapsed / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": args.workload, "model": "random-init dense stand-in",
-                       "batch": batch, "prompt": prompt_len, "canvas": CANVAS,
-                       "d": shape.d, "layers": shape.n_layers, "heads": [shape.n_q_heads,
-                                                                         shape.n_kv_heads],
-                       "head_dim": shape.head_dim, "ffn": shape.ffn, "vocab": shape.vocab,
-                       "steps_per_block": steps_seen[-1] if steps_seen else None,
-                       "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (3.3 GB of weights streamed per step)"},
+            "config": workload_config(args.workload, world,
+                                      steps_seen[-1] if steps_seen else None),
             "roofline": roof,
             "canvas_attn": attn,
             "cpu_baseline": cpu,
@@ -556,9 +550,7 @@ def main():
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    replicas.finish(world)
     return 0
 
 
