@@ -21,6 +21,7 @@
 #include "dg_common.cuh"
 #include "gemm.cuh"
 #include "kvcommit.cuh"
+#include "unembed.cuh"
 #include "sampler.cuh"
 
 namespace {
@@ -45,8 +46,8 @@ bool pdl_enabled() {
 // griddep_wait before touching its predecessors' data) and an optional
 // cluster shape along z.
 template <typename... KArgs, typename... Args>
-cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
-                      cudaStream_t s, int cluster_z, Args&&... args) {
+cudaError_t launch_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                           cudaStream_t s, dim3 cluster, Args&&... args) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -59,16 +60,23 @@ cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
     attr[n].val.programmaticStreamSerializationAllowed = 1;
     ++n;
   }
-  if (cluster_z > 1) {
+  if (cluster.x * cluster.y * cluster.z > 1) {
     attr[n].id = cudaLaunchAttributeClusterDimension;
-    attr[n].val.clusterDim.x = 1;
-    attr[n].val.clusterDim.y = 1;
-    attr[n].val.clusterDim.z = cluster_z;
+    attr[n].val.clusterDim.x = cluster.x;
+    attr[n].val.clusterDim.y = cluster.y;
+    attr[n].val.clusterDim.z = cluster.z;
     ++n;
   }
   cfg.attrs = attr;
   cfg.numAttrs = n;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t s, int cluster_z, Args&&... args) {
+  return launch_cluster(kernel, grid, block, smem, s, dim3(1, 1, cluster_z),
+                        std::forward<Args>(args)...);
 }
 
 int fail(int status, const char* fmt, ...) {
@@ -254,6 +262,41 @@ int launch_gemm(const void* x, const void* w, int M, int N, int K, const GemmPla
 int linear(const void* x, const void* w, int M, int N, int K, const GemmEpi& e,
            cudaStream_t s) {
   return launch_gemm(x, w, M, N, K, plan_gemm(M, N, K), e, s);
+}
+
+// logits = rs * (h w_u^T).  Vocabularies that are a multiple of 256 run on
+// the persistent CTA-pair kernel (unembed.cuh); others on the single-CTA GEMM.
+bool unembed_attr_done = false;
+
+int launch_unembed(const void* h, const void* w_u, float* logits, int M, int d, int V,
+                   const float* ssq_in, int n_ssq_in, float inv_k, float eps, cudaStream_t s) {
+  namespace ue = dg::unembed;
+  if (V % ue::TILE_V != 0) {
+    GemmEpi e;
+    e.epi = dg::gemm::EPI_F32;
+    e.out_f32 = logits;
+    e.ssq_in = ssq_in; e.n_ssq_in = n_ssq_in; e.inv_k = inv_k; e.eps = eps;
+    return launch_gemm(h, w_u, M, V, d, GemmPlan{1, d / dg::gemm::BK, 256}, e, s);
+  }
+  if (!unembed_attr_done) {
+    DG_CUDA(cudaFuncSetAttribute(ue::unembed_pair_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, ue::SMEM_BYTES));
+    unembed_attr_done = true;
+  }
+  CUtensorMap tw, tx;
+  DG_TRY(make_tmap(&tw, w_u, d, V, (uint64_t)d * 2, ue::HALF_V));
+  DG_TRY(make_tmap(&tx, h, d, M, (uint64_t)d * 2, ue::HALF_T));
+  ue::Params p;
+  p.M = M; p.N = V; p.K = d;
+  p.n_ttiles = cdiv(M, ue::TILE_T);
+  p.n_tiles = (V / ue::TILE_V) * p.n_ttiles;
+  p.n_pairs = std::min(kNumSMs / 2, p.n_tiles);
+  p.logits = logits;
+  p.ssq_in = ssq_in; p.n_ssq_in = n_ssq_in; p.inv_k = inv_k; p.eps = eps;
+  DG_CUDA(launch_cluster(ue::unembed_pair_kernel, dim3(2 * p.n_pairs), dim3(ue::THREADS),
+                         ue::SMEM_BYTES, s, dim3(2, 1, 1), tw, tx, p));
+  count_launch();
+  return DG_OK;
 }
 
 // ---------------------------------------------------------------------------
@@ -578,12 +621,9 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
     DG_TRY(linear(up, w.w_down, M, c.d, c.ffn, ed, s));
   }
   if (f.want_logits) {
-    GemmEpi el;  // logits of RMSNorm(x)
-    el.epi = dg::gemm::EPI_F32;
-    el.out_f32 = logits;
-    el.ssq_in = ssq_x; el.n_ssq_in = nt; el.inv_k = 1.f / c.d; el.eps = c.eps;
-    DG_TRY(launch_gemm(xb, f.m->unembed, M, c.vocab, c.d, GemmPlan{1, c.d / dg::gemm::BK, 256}, el,
-                       s));
+    // logits of RMSNorm(x)
+    DG_TRY(launch_unembed(xb, f.m->unembed, logits, M, c.d, c.vocab, ssq_x, nt, 1.f / c.d, c.eps,
+                          s));
   }
   return DG_OK;
 }
@@ -720,10 +760,7 @@ int dg_unembed(const void* h, const void* w_u, float* logits, int M, int d, int 
     return fail(DG_ERR_UNSUPPORTED_SHAPE, "dg_unembed: V %% 128 and d %% 64 must be 0");
   if (!aligned16(h) || !aligned16(w_u) || !aligned16(logits))
     return fail(DG_ERR_ALIGNMENT, "dg_unembed: pointers must be 16-byte aligned");
-  GemmEpi e;
-  e.epi = dg::gemm::EPI_F32;
-  e.out_f32 = logits;
-  return launch_gemm(h, w_u, M, V, d, GemmPlan{1, d / dg::gemm::BK, 256}, e, (cudaStream_t)stream);
+  return launch_unembed(h, w_u, logits, M, d, V, nullptr, 0, 0.f, 0.f, (cudaStream_t)stream);
 }
 
 size_t dg_linear_workspace_bytes(int M, int N, int K) {

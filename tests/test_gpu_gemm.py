@@ -45,7 +45,13 @@ def test_linear_epilogues(Mr, N, K, epi):
     assert_close(out, want, rel_l2=5e-3, max_abs=3e-2, what=f"{epi} {Mr}x{N}x{K}")
 
 
-@pytest.mark.parametrize("Mr,d,V", [(256, 256, 512), (256, 2048, 4096), (131, 512, 1024)])
+# V % 256 == 0 runs on CTA pairs (256 x 256 tiles, persistent, double-buffered
+# accumulators); V = 384 on the single-CTA GEMM.  600 and 1024 rows span
+# several token tiles (600 with a ragged one); V = 65536 gives each pair
+# several tiles, so both accumulator buffers are reused.
+@pytest.mark.parametrize("Mr,d,V", [(256, 256, 512), (256, 2048, 4096), (131, 512, 1024),
+                                    (256, 256, 384), (600, 512, 2048), (1024, 256, 8192),
+                                    (256, 512, 65536), (1, 64, 256)])
 def test_unembed_against_oracle(Mr, d, V):
     import canvas_denoising_denoise_b200 as dg
     h = rand_bf16(Mr, d, seed=4)
