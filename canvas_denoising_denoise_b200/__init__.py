@@ -6,7 +6,8 @@ kernels.  There is no CPU fallback: every call needs the built library and a
 CUDA device, and raises otherwise.
 
 Functions take torch tensors and pass their device pointers:
-    canvas_attn, unembed, linear, sample_commit, kv_block_commit, philox
+    canvas_attn, unembed, linear, sample_commit, unembed_sample_commit, kv_block_commit,
+    philox
 Objects:
     DgModel   weights + configuration (dg_model)
     DgState   KV caches and canvas state of a batch (dg_state)
@@ -20,7 +21,8 @@ from . import _lib
 from ._lib import (EPI_BF16, EPI_F32, EPI_GELU_BF16, EPI_RESID_F32, MASK_BIDIR, MASK_CAUSAL,
                    UNSELECTED_KEEP, UNSELECTED_RENOISE, DgError)
 
-__all__ = ["canvas_attn", "unembed", "linear", "sample_commit", "kv_block_commit", "philox",
+__all__ = ["canvas_attn", "unembed", "linear", "sample_commit", "unembed_sample_commit",
+           "kv_block_commit", "philox",
            "DgModel", "DgState", "SamplerSettings", "prefill", "denoise_logits", "denoise_block",
            "check_device_errors", "Workspace", "DgError", "MASK_BIDIR", "MASK_CAUSAL",
            "EPI_F32", "EPI_BF16", "EPI_GELU_BF16", "EPI_RESID_F32", "UNSELECTED_KEEP",
@@ -170,6 +172,28 @@ def sample_commit(logits, tok, committed, prev_argmax, seq_status, settings, see
                                     _ptr(seq_status), ctypes.byref(settings.c), seed, block, step,
                                     B, C, V, ctypes.byref(so) if so is not None else None,
                                     wp, wn, _stream(stream)))
+
+
+def unembed_sample_commit(h, w_u, tok, committed, prev_argmax, seq_status, settings, seed,
+                          block, step, out=None, ws=None, stream=None):
+    """The unembedding h[B*C, d] @ w_u[V, d]^T fused with one sampler step.
+
+    Same canvas updates and outputs as sample_commit on those logits; the
+    logits are never written.  V % 256 == 0.
+    """
+    _need_contig(h, w_u, tok, committed, prev_argmax, seq_status)
+    lib = _lib.load()
+    B, C = tok.shape
+    V, d = w_u.shape
+    so = None
+    if out is not None:
+        so = _lib.StepOut(*[(out[k].data_ptr() if out.get(k) is not None else None)
+                            for k in ("x_hat", "argmax", "logconf", "entropy", "flags")])
+    wp, wn = _ws(ws).args(lib.dg_unembed_sample_commit_workspace_bytes(B, C, V))
+    _lib.check(lib.dg_unembed_sample_commit(
+        _ptr(h), _ptr(w_u), d, _ptr(tok), _ptr(committed), _ptr(prev_argmax), _ptr(seq_status),
+        ctypes.byref(settings.c), seed, block, step, B, C, V,
+        ctypes.byref(so) if so is not None else None, wp, wn, _stream(stream)))
 
 
 def kv_block_commit(k_blk, v_blk, k_cache, v_cache, cache_len, *, n_kv_heads, head_dim,

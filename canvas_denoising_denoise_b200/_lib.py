@@ -83,6 +83,11 @@ SIGNATURES = {
                                  c_uint32, c_int, c_int, c_int, c_int, c_int, P(StepOut),
                                  c_void_p, c_size_t, c_void_p]),
     "dg_sample_commit_workspace_bytes": (c_size_t, [c_int, c_int, c_int]),
+    "dg_unembed_sample_commit": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p,
+                                         c_void_p, P(SamplerCfg), c_uint32, c_int, c_int, c_int,
+                                         c_int, c_int, P(StepOut), c_void_p, c_size_t,
+                                         c_void_p]),
+    "dg_unembed_sample_commit_workspace_bytes": (c_size_t, [c_int, c_int, c_int]),
     "dg_sample_commit_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                          P(SamplerCfg), c_uint32, c_int, c_int, c_int, c_int,
                                          c_int, P(StepOut), c_void_p]),

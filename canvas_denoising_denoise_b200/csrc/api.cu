@@ -271,7 +271,7 @@ bool unembed_attr_done = false;
 int launch_unembed(const void* h, const void* w_u, float* logits, int M, int d, int V,
                    const float* ssq_in, int n_ssq_in, float inv_k, float eps, cudaStream_t s) {
   namespace ue = dg::unembed;
-  if (V % ue::TILE_V != 0) {
+  if (V % ue::TILE != 0) {
     GemmEpi e;
     e.epi = dg::gemm::EPI_F32;
     e.out_f32 = logits;
@@ -284,16 +284,17 @@ int launch_unembed(const void* h, const void* w_u, float* logits, int M, int d, 
     unembed_attr_done = true;
   }
   CUtensorMap tw, tx;
-  DG_TRY(make_tmap(&tw, w_u, d, V, (uint64_t)d * 2, ue::HALF_V));
-  DG_TRY(make_tmap(&tx, h, d, M, (uint64_t)d * 2, ue::HALF_T));
+  DG_TRY(make_tmap(&tw, w_u, d, V, (uint64_t)d * 2, ue::HALF));
+  DG_TRY(make_tmap(&tx, h, d, M, (uint64_t)d * 2, ue::HALF));
   ue::Params p;
   p.M = M; p.N = V; p.K = d;
-  p.n_ttiles = cdiv(M, ue::TILE_T);
-  p.n_tiles = (V / ue::TILE_V) * p.n_ttiles;
+  p.n_ttiles = cdiv(M, ue::TILE);
+  p.n_tiles = (V / ue::TILE) * p.n_ttiles;
   p.n_pairs = std::min(kNumSMs / 2, p.n_tiles);
   p.logits = logits;
   p.ssq_in = ssq_in; p.n_ssq_in = n_ssq_in; p.inv_k = inv_k; p.eps = eps;
-  DG_CUDA(launch_cluster(ue::unembed_pair_kernel, dim3(2 * p.n_pairs), dim3(ue::THREADS),
+  DG_CUDA(launch_cluster(ue::unembed_pair_kernel, dim3(2 * p.n_pairs),
+                         dim3(ue::threads_for(ue::STORE_EPI_WARPS)),
                          ue::SMEM_BYTES, s, dim3(2, 1, 1), tw, tx, p));
   count_launch();
   return DG_OK;
@@ -449,7 +450,81 @@ int launch_sample(const float* logits, int32_t* tok, uint8_t* committed, int32_t
   count_launch();
   const int threads = (p.C + 31) / 32 * 32;
   DG_CUDA(launch_ex(dg::sample_commit_kernel, dim3(p.B), dim3(threads), 0, s, 1, logits,
-                    (const dg::RowPartial*)part, p, tok, committed, prev_argmax, seq_status,
+                    (const dg::RowPartial*)part, (const dg::RowStats*)nullptr, p, tok, committed, prev_argmax, seq_status,
+                    out ? out->x_hat : (int32_t*)nullptr, out ? out->argmax : (int32_t*)nullptr,
+                    out ? out->logconf : (float*)nullptr, out ? out->entropy : (float*)nullptr,
+                    out ? out->flags : (uint8_t*)nullptr));
+  count_launch();
+  return DG_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Unembedding fused with the sampler step (vocabularies that are a multiple
+// of 256): unembed_sample_kernel -> sample_merge_kernel -> sample_commit_kernel
+// ---------------------------------------------------------------------------
+struct FusedPlan {
+  int n_ttiles, segs, n_pairs, nparts;
+};
+
+// As many vocabulary segments per token tile as keep one wave of CTA pairs.
+FusedPlan plan_fused(int M, int V) {
+  FusedPlan f;
+  f.n_ttiles = cdiv(M, dg::unembed::TILE);
+  f.segs = std::max(1, std::min(V / dg::unembed::TILE, (kNumSMs / 2) / f.n_ttiles));
+  f.n_pairs = f.segs * f.n_ttiles;
+  f.nparts = 2 * f.segs;  // two column halves per segment
+  return f;
+}
+
+size_t fused_ws_bytes(int B, int C, int V) {
+  const int M = B * C;
+  const FusedPlan f = plan_fused(M, V);
+  return align_up((size_t)M * f.nparts * sizeof(dg::FusedPartial), 256) +
+         align_up((size_t)M * sizeof(dg::RowStats), 256);
+}
+
+bool fused_attr_done = false;
+
+int launch_unembed_sample(const void* h, const void* w_u, int d, const float* ssq_in,
+                          int n_ssq_in, float inv_k, float eps, int32_t* tok,
+                          uint8_t* committed, int32_t* prev_argmax, int32_t* seq_status,
+                          const dg::SampleParams& sp, const dg_step_out* out, void* ws,
+                          cudaStream_t s) {
+  namespace ue = dg::unembed;
+  const int M = sp.B * sp.C, V = sp.V;
+  const FusedPlan f = plan_fused(M, V);
+  if (!fused_attr_done) {
+    DG_CUDA(cudaFuncSetAttribute(ue::unembed_sample_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, ue::SMEM_BYTES));
+    fused_attr_done = true;
+  }
+  dg::FusedPartial* part = (dg::FusedPartial*)ws;
+  dg::RowStats* stats = (dg::RowStats*)((char*)ws + align_up((size_t)M * f.nparts *
+                                                             sizeof(dg::FusedPartial), 256));
+  CUtensorMap tx, tw;
+  DG_TRY(make_tmap(&tx, h, d, M, (uint64_t)d * 2, ue::HALF));
+  DG_TRY(make_tmap(&tw, w_u, d, V, (uint64_t)d * 2, ue::HALF));
+  ue::SampleFusedParams p;
+  p.M = M; p.N = V; p.K = d;
+  p.n_vtiles = V / ue::TILE;
+  p.segs = f.segs;
+  p.n_pairs = f.n_pairs;
+  p.ssq_in = ssq_in; p.n_ssq_in = n_ssq_in; p.inv_k = inv_k; p.eps = eps;
+  p.sp = sp;
+  p.tok = tok;
+  p.part = part;
+  DG_CUDA(launch_cluster(ue::unembed_sample_kernel, dim3(2 * f.n_pairs),
+                         dim3(ue::threads_for(ue::SAMPLE_EPI_WARPS)), ue::SMEM_BYTES, s,
+                         dim3(2, 1, 1), tx, tw, p));
+  count_launch();
+  DG_CUDA(launch_ex(dg::sample_merge_kernel, dim3(cdiv(M, dg::MERGE_WARPS)),
+                    dim3(dg::MERGE_WARPS * 32), 0, s, 1, (const dg::FusedPartial*)part, f.nparts,
+                    (const uint8_t*)committed, sp, stats));
+  count_launch();
+  const int threads = (sp.C + 31) / 32 * 32;
+  DG_CUDA(launch_ex(dg::sample_commit_kernel, dim3(sp.B), dim3(threads), 0, s, 1,
+                    (const float*)nullptr, (const dg::RowPartial*)nullptr,
+                    (const dg::RowStats*)stats, sp, tok, committed, prev_argmax, seq_status,
                     out ? out->x_hat : (int32_t*)nullptr, out ? out->argmax : (int32_t*)nullptr,
                     out ? out->logconf : (float*)nullptr, out ? out->entropy : (float*)nullptr,
                     out ? out->flags : (uint8_t*)nullptr));
@@ -550,7 +625,10 @@ FwdLayout fwd_layout(const dg_model_cfg& c, int B, int Lq, int max_prefix, bool 
   L.ssq_h = take((size_t)(c.d / 128) * M * 4);
   L.attn = take(attn_ws_bytes(B, c.n_q_heads, c.n_kv_heads, Lq, c.head_dim, max_prefix));
   L.logits = take(logits ? (size_t)M * c.vocab * 4 : 0);
-  L.spart = take(logits ? sample_ws_bytes(B, Lq, c.vocab) : 0);
+  L.spart = take(logits ? std::max(sample_ws_bytes(B, Lq, c.vocab),
+                                    c.vocab % dg::unembed::TILE == 0
+                                        ? fused_ws_bytes(B, Lq, c.vocab) : (size_t)0)
+                         : 0);
   L.flag = take(logits ? 16 : 0);
   L.total = off;
   return L;
@@ -563,9 +641,10 @@ struct Fwd {
   void* const* k_cache;
   void* const* v_cache;
   bool commit_kv;   // write each layer's new K/V into the cache at cache_len
-  bool want_logits;
+  bool want_logits;  // run the whole stack and (unless unembed_elsewhere) the unembedding
   char* ws;
   FwdLayout L;
+  bool unembed_elsewhere = false;  // the caller fuses the unembedding into its sampler step
 };
 
 int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s) {
@@ -620,7 +699,7 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
     ed.x = x; ed.out_bf16 = xb; ed.ssq_out = ssq_x;
     DG_TRY(linear(up, w.w_down, M, c.d, c.ffn, ed, s));
   }
-  if (f.want_logits) {
+  if (f.want_logits && !f.unembed_elsewhere) {
     // logits of RMSNorm(x)
     DG_TRY(launch_unembed(xb, f.m->unembed, logits, M, c.d, c.vocab, ssq_x, nt, 1.f / c.d, c.eps,
                           s));
@@ -824,6 +903,36 @@ int dg_sample_commit(const float* logits, int32_t* tok, uint8_t* committed,
                        (cudaStream_t)stream);
 }
 
+size_t dg_unembed_sample_commit_workspace_bytes(int B, int C, int V) {
+  if (B <= 0 || C <= 0 || V <= 0 || V % dg::unembed::TILE) return 0;
+  return fused_ws_bytes(B, C, V);
+}
+
+int dg_unembed_sample_commit(const void* h, const void* w_u, int d, int32_t* tok,
+                             uint8_t* committed, int32_t* prev_argmax, int32_t* seq_status,
+                             const dg_sampler_cfg* cfg, uint32_t seed, int block, int step,
+                             int B, int C, int V, const dg_step_out* out, void* workspace,
+                             size_t workspace_bytes, void* stream) {
+  if (!h || !w_u || !tok || !committed || !prev_argmax || !seq_status || !cfg)
+    return fail(DG_ERR_INVALID_ARG, "dg_unembed_sample_commit: null pointer");
+  if (B <= 0 || C <= 0 || C > 1024 || V <= 0 || V % dg::unembed::TILE || d <= 0 || d % 64 ||
+      step < 0 || block < 0)
+    return fail(DG_ERR_UNSUPPORTED_SHAPE,
+                "dg_unembed_sample_commit: need C <= 1024, V %% 256 == 0, d %% 64 == 0");
+  if (cfg->max_steps < 1 || cfg->commit_k < 0 || !(cfg->t_start > 0.f) || !(cfg->t_end > 0.f) ||
+      (cfg->unselected_policy != 0 && cfg->unselected_policy != 1))
+    return fail(DG_ERR_INVALID_ARG, "dg_unembed_sample_commit: bad sampler settings");
+  if (!aligned16(h) || !aligned16(w_u))
+    return fail(DG_ERR_ALIGNMENT, "dg_unembed_sample_commit: pointers must be 16-byte aligned");
+  const size_t need = fused_ws_bytes(B, C, V);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return fail(DG_ERR_WORKSPACE_TOO_SMALL,
+                "dg_unembed_sample_commit: workspace needs %zu bytes", need);
+  const dg::SampleParams p = make_sample_params(*cfg, seed, block, nullptr, step, B, C, V);
+  return launch_unembed_sample(h, w_u, d, nullptr, 0, 0.f, 0.f, tok, committed, prev_argmax,
+                               seq_status, p, out, workspace, (cudaStream_t)stream);
+}
+
 int dg_sample_commit_noalloc(const float* logits, int32_t* tok, uint8_t* committed,
                              int32_t* prev_argmax, int32_t* seq_status, const dg_sampler_cfg* cfg,
                              uint32_t seed, int block, int step, int B, int C, int V,
@@ -953,10 +1062,21 @@ int dg_denoise_block(const dg_model* m, dg_state* st, const dg_sampler_cfg* cfg,
         st->v_cache, false, true, ws, L};
   const dg::SampleParams sp = make_sample_params(*cfg, seed, block, st->step, 0, B, C, V);
   int steps = 0;
+  // with a vocabulary of 256-entry tiles the sampler's row pass runs inside
+  // the unembedding and the logits never reach memory
+  const bool fused = V % dg::unembed::TILE == 0;
+  Fwd fl = f;
+  fl.unembed_elsewhere = fused;
   for (int it = 0; it < cfg->max_steps; ++it) {
-    DG_TRY(run_forward(f, st->tok, logits, s));
-    DG_TRY(launch_sample(logits, st->tok, st->committed, st->prev_argmax, st->seq_status, sp,
-                         nullptr, ws + L.spart, s));
+    DG_TRY(run_forward(fl, st->tok, logits, s));
+    if (fused)
+      DG_TRY(launch_unembed_sample(ws + L.xn, m->unembed, m->cfg.d, (const float*)(ws + L.ssq_x),
+                                   m->cfg.d / 128, 1.f / m->cfg.d, m->cfg.eps, st->tok,
+                                   st->committed, st->prev_argmax, st->seq_status, sp, nullptr,
+                                   ws + L.spart, s));
+    else
+      DG_TRY(launch_sample(logits, st->tok, st->committed, st->prev_argmax, st->seq_status, sp,
+                           nullptr, ws + L.spart, s));
     dg::step_advance_kernel<<<1, 256, 0, s>>>(B, cfg->max_steps, st->seq_status, st->step,
                                               running);
     count_launch();

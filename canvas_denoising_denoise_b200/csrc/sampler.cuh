@@ -100,6 +100,125 @@ struct RowPartial {
   int pad;
 };
 
+// Row pass partial of the fused unembedding: as RowPartial, plus the raw
+// logit of the Gumbel winner and of the current canvas token (NaN when that
+// token lies outside the partial's vocabulary range).
+struct FusedPartial {
+  float m, s, q, amax;
+  int aidx;
+  float best;
+  int bidx;
+  float lx;
+  float lcur;
+  int pad;
+};
+
+// Merged per-position statistics that the commit step consumes.
+struct RowStats {
+  float lam;   // natural log confidence of the token at stake
+  float ent;   // tempered entropy, nats
+  int amax;    // raw-logit argmax
+  int xhat;    // Gumbel-max sample
+};
+
+// Row pass state of one thread over an ascending run of vocabulary entries.
+// Per element, in the log2 domain with m the running maximum:
+//   pe = 2^(l k2 - m)         one FFMA + one ex2 (shared by the softmax sums)
+//   E  = -ln(u)               Philox word -> exponential variate
+// The Gumbel-max sample argmax_v (z_v - ln E_v) equals argmax_v pe_v / E_v (the
+// exponential race), so the best is kept as (pb, Eb) and compared by
+// cross-multiplication; pb rescales with the running maximum.  It becomes the
+// score l k2 - log2(E) only for the merges.
+struct RowState {
+  float m, s, q;        // running max of zl, sum 2^(zl - m), sum 2^(zl - m) (zl - m)
+  float amax;           // max raw logit
+  int aidx;             // its index (lowest on ties)
+  float pb, eb, lb;     // race leader: pe, E, raw logit
+  int bidx;             // its index (lowest on ties)
+  float lcur;           // raw logit of the current token, NaN until seen
+
+  __device__ __forceinline__ void reset() {
+    m = -INFINITY; s = 0.f; q = 0.f;
+    amax = -INFINITY; aidx = 0x7FFFFFFF;
+    pb = 0.f; eb = 1.f; lb = -INFINITY; bidx = 0x7FFFFFFF;
+    lcur = __int_as_float(0x7FC00000);
+  }
+
+  // G groups of 4 consecutive entries, group g starting at vg[g] (a multiple
+  // of 4, ascending in g); only groups [0, n_valid) are counted (the others
+  // hold -inf).  The Philox words of group g are counter (vg[g] / 4, c1, step,
+  // block), key `key`.
+  template <int G, bool TRACK_CUR>
+  __device__ __forceinline__ void update(const float (&l)[4 * G], const int (&vg)[G],
+                                         int n_valid, int cur, float k2, uint32_t c1,
+                                         uint32_t step, uint32_t block, uint2 key) {
+    float bm = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < 4 * G; ++i) bm = fmaxf(bm, l[i]);
+    if (bm > amax) {
+      // new raw maximum in this batch: first index holding it (ascending order)
+      amax = bm;
+#pragma unroll
+      for (int g = G - 1; g >= 0; --g)
+#pragma unroll
+        for (int e = 3; e >= 0; --e)
+          if (l[4 * g + e] == bm) aidx = vg[g] + e;
+    }
+    const float bmz = bm * k2;
+    if (bmz > m) {
+      if (m != -INFINITY) {
+        const float d = m - bmz, f = sfu_exp2(d);
+        q = f * (q + d * s);
+        s *= f;
+        pb *= f;
+      }
+      m = bmz;
+    }
+    const float neg_m = -m;
+#pragma unroll
+    for (int g = 0; g < G; ++g) {
+      if (g >= n_valid) break;
+      const uint4 r = philox4x32_10(
+          make_uint4(static_cast<uint32_t>(vg[g] >> 2), c1, step, block), key);
+      const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float lv = l[4 * g + e];
+        const float t = fmaf(lv, k2, neg_m);
+        const float pe = sfu_exp2(t);
+        s += pe;
+        q = fmaf(pe, t, q);
+        const float ev = exp_variate(rw[e]);
+        if (pe * eb > pb * ev) {
+          pb = pe;
+          eb = ev;
+          lb = lv;
+          bidx = vg[g] + e;
+        }
+        if (TRACK_CUR && vg[g] + e == cur) lcur = lv;
+      }
+    }
+  }
+
+  // 32 consecutive entries starting at v0 (a multiple of 4)
+  __device__ __forceinline__ void update32(const float (&l)[32], int v0, int cur, float k2,
+                                           uint32_t c1, uint32_t step, uint32_t block,
+                                           uint2 key) {
+    int vg[8];
+#pragma unroll
+    for (int g = 0; g < 8; ++g) vg[g] = v0 + 4 * g;
+    update<8, true>(l, vg, 8, cur, k2, c1, step, block, key);
+  }
+
+  __device__ __forceinline__ float best_score(float k2) const {
+    return (bidx == 0x7FFFFFFF) ? -INFINITY : lb * k2 - sfu_log2(eb);
+  }
+
+  __device__ __forceinline__ FusedPartial partial(float k2) const {
+    return FusedPartial{m, s, q, amax, aidx, best_score(k2), bidx, lb, lcur, 0};
+  }
+};
+
 struct SampleParams {
   int B, C, V;
   int chunk, nchunk;         // vocabulary chunk per rowpass CTA
@@ -145,15 +264,8 @@ __device__ __forceinline__ void merge_best(float& v, int& i, float v2, int i2) {
   }
 }
 
-// Grid: B * C * nchunk CTAs of RP_THREADS threads.  Chunk length is a multiple of 4.
-//
-// Per element, in the log2 domain with m the running maximum:
-//   pe = 2^(l k2 - m)         one FFMA + one ex2 (shared by the softmax sums)
-//   E  = -ln(u)               Philox word -> exponential variate
-// The Gumbel-max sample argmax_v (z_v - ln E_v) equals argmax_v pe_v / E_v (the
-// exponential race), so within a thread the best is kept as (pb, Eb) and
-// compared by cross-multiplication; pb rescales with the running maximum.  The
-// thread's best is turned into the score l k2 - log2(E) only for the merges.
+// Grid: B * C * nchunk CTAs of RP_THREADS threads.  Chunk length is a multiple
+// of 4.  Each thread runs a RowState over its interleaved groups of 4.
 constexpr int RP_THREADS = 256;
 constexpr int RP_UNROLL = 4;
 
@@ -176,74 +288,30 @@ __global__ void __launch_bounds__(RP_THREADS) sample_rowpass_kernel(
   const uint32_t c1 = (static_cast<uint32_t>(pos) & 0xFFFFFFu) | (kTagGumbel << 24);
   const uint2 key = make_uint2(p.seed, static_cast<uint32_t>(b));
 
-  float m = -INFINITY, s = 0.f, q = 0.f;
-  float amax = -INFINITY;
-  int aidx = 0x7FFFFFFF;
-  float pb = 0.f, eb = 1.f, lb = -INFINITY;  // best of the race: pe, E, raw logit
-  int bidx = 0x7FFFFFFF;
-
+  RowState st;
+  st.reset();
   for (int base = v0 + threadIdx.x * 4; base < v1; base += RP_THREADS * 4 * RP_UNROLL) {
-    float4 l4[RP_UNROLL];
+    float l[4 * RP_UNROLL];
+    int vg[RP_UNROLL];
+    int n_valid = 0;
 #pragma unroll
     for (int u = 0; u < RP_UNROLL; ++u) {
       const int v = base + u * RP_THREADS * 4;
-      l4[u] = (v < v1) ? __ldcs(reinterpret_cast<const float4*>(x + v))
-                       : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      vg[u] = v;
+      const float4 l4 = (v < v1) ? __ldcs(reinterpret_cast<const float4*>(x + v))
+                                 : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      l[4 * u] = l4.x;
+      l[4 * u + 1] = l4.y;
+      l[4 * u + 2] = l4.z;
+      l[4 * u + 3] = l4.w;
+      n_valid += (v < v1) ? 1 : 0;
     }
-    float bm = -INFINITY;
-#pragma unroll
-    for (int u = 0; u < RP_UNROLL; ++u)
-      bm = fmaxf(bm, fmaxf(fmaxf(l4[u].x, l4[u].y), fmaxf(l4[u].z, l4[u].w)));
-    if (bm > amax) {
-      // new raw maximum in this batch: first index holding it (ascending order)
-      amax = bm;
-#pragma unroll
-      for (int u = RP_UNROLL - 1; u >= 0; --u) {
-        const int v = base + u * RP_THREADS * 4;
-        if (l4[u].w == bm) aidx = v + 3;
-        if (l4[u].z == bm) aidx = v + 2;
-        if (l4[u].y == bm) aidx = v + 1;
-        if (l4[u].x == bm) aidx = v;
-      }
-    }
-    const float bmz = bm * k2;
-    if (bmz > m) {
-      if (m != -INFINITY) {
-        const float d = m - bmz, f = sfu_exp2(d);
-        q = f * (q + d * s);
-        s *= f;
-        pb *= f;
-      }
-      m = bmz;
-    }
-    const float neg_m = -m;
-#pragma unroll
-    for (int u = 0; u < RP_UNROLL; ++u) {
-      const int v = base + u * RP_THREADS * 4;
-      if (v >= v1) break;
-      const float lv[4] = {l4[u].x, l4[u].y, l4[u].z, l4[u].w};
-      const uint4 r = philox4x32_10(make_uint4(static_cast<uint32_t>(v >> 2), c1,
-                                               static_cast<uint32_t>(step),
-                                               static_cast<uint32_t>(p.block)),
-                                    key);
-      const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float t = fmaf(lv[e], k2, neg_m);
-        const float pe = sfu_exp2(t);
-        s += pe;
-        q = fmaf(pe, t, q);
-        const float ev = exp_variate(rw[e]);
-        if (pe * eb > pb * ev) {
-          pb = pe;
-          eb = ev;
-          lb = lv[e];
-          bidx = v + e;
-        }
-      }
-    }
+    st.update<RP_UNROLL, false>(l, vg, n_valid, -1, k2, c1, static_cast<uint32_t>(step),
+                                static_cast<uint32_t>(p.block), key);
   }
-  float best = (bidx == 0x7FFFFFFF) ? -INFINITY : lb * k2 - sfu_log2(eb);
+  float m = st.m, s = st.s, q = st.q, amax = st.amax;
+  int aidx = st.aidx, bidx = st.bidx;
+  float best = st.best_score(k2);
 
   // CTA reduction: warp shuffles, then across warps through shared memory.
 #pragma unroll
@@ -274,9 +342,75 @@ __global__ void __launch_bounds__(RP_THREADS) sample_rowpass_kernel(
   }
 }
 
+// Merge of the fused unembedding's partials: one warp per position.  Lane j
+// merges partials j, j + 32, ... in order, then lanes merge pairwise (xor
+// pattern) and lane 0's result is used, so the order is fixed.
+constexpr int MERGE_WARPS = 8;
+
+__global__ void __launch_bounds__(MERGE_WARPS * 32) sample_merge_kernel(
+    const FusedPartial* __restrict__ part, int nparts, const uint8_t* __restrict__ committed,
+    SampleParams p, RowStats* __restrict__ stats) {
+  griddep_wait();
+  griddep_launch();
+  const int row = blockIdx.x * MERGE_WARPS + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= p.B * p.C) return;  // warp-uniform
+  const int step = read_step(p);
+  const float k2 = 1.4426950408889634f / step_temperature(step, p.max_steps, p.t_start, p.t_end);
+  const FusedPartial* pr = part + static_cast<size_t>(row) * nparts;
+  float m = -INFINITY, s = 0.f, q = 0.f, av = -INFINITY, bv = -INFINITY;
+  float lx = 0.f, lcur = __int_as_float(0x7FC00000);
+  int ai = 0x7FFFFFFF, bi = 0x7FFFFFFF;
+  for (int j = lane; j < nparts; j += 32) {
+    const FusedPartial f = pr[j];
+    merge_softmax(m, s, q, f.m, f.s, f.q);
+    merge_best(av, ai, f.amax, f.aidx);
+    const int b_before = bi;
+    merge_best(bv, bi, f.best, f.bidx);
+    if (bi != b_before) lx = f.lx;
+    if (!isnan(f.lcur)) lcur = f.lcur;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float m2 = __shfl_xor_sync(0xffffffffu, m, o);
+    const float s2 = __shfl_xor_sync(0xffffffffu, s, o);
+    const float q2 = __shfl_xor_sync(0xffffffffu, q, o);
+    merge_softmax(m, s, q, m2, s2, q2);
+    const float a2 = __shfl_xor_sync(0xffffffffu, av, o);
+    const int ai2 = __shfl_xor_sync(0xffffffffu, ai, o);
+    merge_best(av, ai, a2, ai2);
+    const float b2 = __shfl_xor_sync(0xffffffffu, bv, o);
+    const int bi2 = __shfl_xor_sync(0xffffffffu, bi, o);
+    const float lx2 = __shfl_xor_sync(0xffffffffu, lx, o);
+    const int b_before = bi;
+    merge_best(bv, bi, b2, bi2);
+    if (bi != b_before) lx = lx2;
+    const float lc2 = __shfl_xor_sync(0xffffffffu, lcur, o);
+    if (isnan(lcur)) lcur = lc2;
+  }
+  if (lane == 0) {
+    const float l2s = log2f(s);
+    const float lse2 = m + l2s;  // log2-domain logsumexp
+    float lat = lx;
+    if (committed[row] != 0) {
+      lat = lcur;
+      if (isnan(lcur)) {  // the current token is not a vocabulary entry
+        raise_error(ERR_CHECK | 0x502, static_cast<uint32_t>(row));
+        lat = lse2 / k2;
+      }
+    }
+    stats[row] = RowStats{(lat * k2 - lse2) * 0.69314718055994531f,
+                          0.69314718055994531f * (l2s - q / s), ai, bi};
+  }
+}
+
 // Grid: B CTAs; blockDim = C rounded up to a multiple of 32 (C <= 1024).
+// Per-position statistics come either from the row pass partials (`part`,
+// nchunk per position, and the logit at stake read from `logits`) or, when
+// `stats` is given, from the fused unembedding's merged statistics.
 __global__ void __launch_bounds__(1024) sample_commit_kernel(
-    const float* __restrict__ logits, const RowPartial* __restrict__ part, SampleParams p,
+    const float* __restrict__ logits, const RowPartial* __restrict__ part,
+    const RowStats* __restrict__ stats, SampleParams p,
     int32_t* __restrict__ tok, uint8_t* __restrict__ committed, int32_t* __restrict__ prev_argmax,
     int32_t* __restrict__ seq_status, int32_t* __restrict__ o_xhat,
     int32_t* __restrict__ o_argmax, float* __restrict__ o_logconf,
@@ -300,7 +434,15 @@ __global__ void __launch_bounds__(1024) sample_commit_kernel(
   float lam = 0.f, ent = 0.f;
   int amax_i = -1, xhat = 0, cur = 0;
   bool was_committed = true;
-  if (live) {
+  if (live && stats != nullptr) {
+    const RowStats rs = stats[row];
+    lam = rs.lam;
+    ent = rs.ent;
+    amax_i = rs.amax;
+    xhat = rs.xhat;
+    cur = tok[row];
+    was_committed = committed[row] != 0;
+  } else if (live) {
     const RowPartial* pr = part + row * p.nchunk;
     float m = pr[0].m, s = pr[0].s, q = pr[0].q, av = pr[0].amax, bv = pr[0].best;
     int ai = pr[0].aidx, bi = pr[0].bidx;

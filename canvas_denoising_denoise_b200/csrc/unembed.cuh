@@ -1,4 +1,5 @@
-// unembed.cuh - the unembedding on CTA pairs:
+// unembed.cuh - the unembedding on CTA pairs, alone or fused with the sampler's
+// row pass.
 //
 //   logits[t, v] = rs[t] * sum_k h[t, k] W_U[v, k]     h bf16 [M, K], W_U bf16 [V, K]
 //
@@ -8,60 +9,70 @@
 //
 // The vocabulary is far larger than the 148 SMs, so one persistent grid of
 // CTA pairs walks 256 (vocabulary) x 256 (token) output tiles.  A pair tile is
-// one cta_group::2 MMA chain: each CTA stages 128 vocabulary rows of W_U and
-// 128 tokens of h per k-block, and the pair's MMA (M = 256, N = 256, issued by
-// the even CTA) reads both CTAs' halves.  Compared with one CTA per 128 x 256
-// tile this halves the activation bytes every SM pulls in per weight byte:
-// with 256 tokens the activation tile is as large as the weight tile, so the
-// single-CTA form moves three bytes through each SM per weight byte and the
-// pair form two.
+// one cta_group::2 MMA chain: each CTA stages 128 rows of each operand per
+// k-block and the pair's MMA (M = 256, N = 256, issued by the even CTA) reads
+// both CTAs' halves.  Compared with one CTA per 128 x 256 tile this halves the
+// activation bytes every SM pulls in per weight byte: with 256 tokens the
+// activation tile is as large as the weight tile, so the single-CTA form moves
+// three bytes through each SM per weight byte and the pair form two.
 //
-// The accumulator is double-buffered in TMEM (2 x 256 columns), so the store
-// of tile i (fp32 logits straight from registers, 128 contiguous bytes per
-// warp store) overlaps the MMAs of tile i + 1.
+// The accumulator is double-buffered in TMEM (2 x 256 columns), so the
+// epilogue of tile i overlaps the MMAs of tile i + 1.
 //
-// Roles, 192 threads per CTA: warp 0 issues the TMA loads (both CTAs, each
-// into its own ring, completion counted on the even CTA's barrier); warp 1
-// owns TMEM and, in the even CTA, one lane issues the MMAs; warps 2..5 read
-// this CTA's 128 accumulator rows (vocabulary entries) and store the logits.
+// Two epilogues share the pipeline:
+//   unembed_pair_kernel    A = W_U, B = h: TMEM lanes are vocabulary entries;
+//                          fp32 logits stored straight from registers (a warp
+//                          store covers 128 contiguous bytes of one token row).
+//   unembed_sample_kernel  A = h, B = W_U: TMEM lanes are tokens, so a thread
+//                          sees one token's vocabulary values and runs the
+//                          sampler's row pass on them in registers - online
+//                          softmax sums, raw-logit argmax, Gumbel race - across
+//                          all the tiles of its pair.  The logits never reach
+//                          memory; each (token, pair segment) leaves one
+//                          partial for the merge.
+//
+// Roles: warp 0 issues the TMA loads (both CTAs, each into its own ring,
+// completion counted on the even CTA's barrier); warp 1 owns TMEM and, in the
+// even CTA, one lane issues the MMAs; the epilogue warps (2 ..) read this
+// CTA's 128 accumulator lanes.
 #pragma once
 
 #include "dg_common.cuh"
+#include "sampler.cuh"
 
 namespace dg {
 namespace unembed {
 
-constexpr int TILE_V = 256;               // vocabulary rows per pair tile (MMA M)
-constexpr int HALF_V = TILE_V / 2;        // ... per CTA
-constexpr int TILE_T = 256;               // tokens per pair tile (MMA N)
-constexpr int HALF_T = TILE_T / 2;        // ... per CTA
+constexpr int TILE = 256;                 // rows of each operand per pair tile (MMA M and N)
+constexpr int HALF = TILE / 2;            // ... per CTA
 constexpr int BK = 64;                    // one 128-byte swizzle row of bf16
-constexpr int A_BYTES = HALF_V * BK * 2;  // 16 KB
-constexpr int B_BYTES = HALF_T * BK * 2;  // 16 KB
+constexpr int A_BYTES = HALF * BK * 2;    // 16 KB
+constexpr int B_BYTES = HALF * BK * 2;    // 16 KB
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int STAGES = 6;
 constexpr int RING_BYTES = STAGES * STAGE_BYTES;  // 192 KB
-constexpr int ACC_COLS = TILE_T;                  // fp32 columns per accumulator buffer
+constexpr int ACC_COLS = TILE;                    // fp32 columns per accumulator buffer
 constexpr int TMEM_COLS = 2 * ACC_COLS;           // two buffers: all 512 columns
-constexpr int THREADS = 192;
-constexpr int EPI_THREADS = 128;
 constexpr int SMEM_BYTES = 1024 + RING_BYTES + 256;
-constexpr uint32_t IDESC = idesc_bf16_f32(TILE_V, TILE_T, false, false);
+constexpr uint32_t IDESC = idesc_bf16_f32(TILE, TILE, false, false);
 
-struct Params {
-  int M, N, K;
-  int n_ttiles;          // token tiles: ceil(M / 256)
-  int n_tiles;           // (N / 256) * n_ttiles pair tiles, token tile fastest
-  int n_pairs;           // CTA pairs in the grid
-  float* logits;         // [M, N] fp32
-  const float* ssq_in;   // [n_ssq_in, M] or null (rs = 1)
-  int n_ssq_in;
-  float inv_k, eps;
-};
+// Epilogue warps: 4 for the logits store, 8 for the fused sampler (two warps
+// per TMEM lane quarter, each taking half of a tile's columns).
+constexpr int STORE_EPI_WARPS = 4;
+constexpr int SAMPLE_EPI_WARPS = 8;
+__host__ __device__ constexpr int threads_for(int epi_warps) { return 64 + 32 * epi_warps; }
 
-__global__ void __launch_bounds__(THREADS, 1)
-    unembed_pair_kernel(const __grid_constant__ CUtensorMap tm_w,
-                        const __grid_constant__ CUtensorMap tm_x, Params p) {
+// ---------------------------------------------------------------------------
+// Shared pipeline.  Sched: count (tiles of this pair), nkb, a_row(li),
+// b_row(li) (pair-level row origins; CTA r takes rows origin + 128 r).
+// Epi (epilogue warps): start() once the predecessor kernels have finished,
+// prepare(li) before the tile's accumulator is ready, consume(li, taddr, col0,
+// ncols) once it is, finish() after the last tile.
+// ---------------------------------------------------------------------------
+template <int EPI_WARPS, class Sched, class Epi>
+__device__ __forceinline__ void pair_pipeline(const CUtensorMap* tm_a, const CUtensorMap* tm_b,
+                                              uint64_t pol_a, uint64_t pol_b, const Sched& sc,
+                                              Epi& epi) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -76,11 +87,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int warp = warp_id();
   const int lane = lane_id();
   const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs
-  const uint32_t peer = rank ^ 1u;
-  const int pair = static_cast<int>(blockIdx.x >> 1);
-  const int nkb = p.K / BK;
-  const int my_tiles = pair < p.n_tiles ? (p.n_tiles - 1 - pair) / p.n_pairs + 1 : 0;
-  const int total_kb = my_tiles * nkb;
+  const int nkb = sc.nkb;
+  const int total_kb = sc.count * nkb;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -89,39 +97,32 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 2 * (EPI_THREADS / 32));
+      mbar_init(&acc_empty[b], 2 * EPI_WARPS);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tm_w);
-    tma_prefetch_desc(&tm_x);
+    tma_prefetch_desc(tm_a);
+    tma_prefetch_desc(tm_b);
   }
   // both CTAs' barriers exist before either CTA signals the other's
   cluster_arrive_wait();
 
-  const uint32_t abort_peer = cluster_addr(const_cast<int*>(abort_flag), peer);
+  const uint32_t abort_peer = cluster_addr(const_cast<int*>(abort_flag), rank ^ 1u);
   const uint32_t full_even = cluster_addr(full, 0);
-  const uint64_t pol_w = l2_policy_evict_first();  // streamed once
-  const uint64_t pol_x = l2_policy_evict_last();   // re-read by every pair
+  const int roff = static_cast<int>(rank) * HALF;
 
-  // k-block g of this pair's walk: tile index and coordinates
-  auto tile_of = [&](int li) { return pair + li * p.n_pairs; };
-  auto issue_w = [&](int g) {
+  auto issue_a = [&](int g) {
     const int st = g % STAGES;
-    const int j = tile_of(g / nkb);
-    const int v0 = (j / p.n_ttiles) * TILE_V + static_cast<int>(rank) * HALF_V;
-    tma_load_2d_pair(smem + st * STAGE_BYTES, &tm_w, full_even + st * 8, (g % nkb) * BK, v0,
-                     pol_w);
+    tma_load_2d_pair(smem + st * STAGE_BYTES, tm_a, full_even + st * 8, (g % nkb) * BK,
+                     sc.a_row(g / nkb) + roff, pol_a);
   };
-  auto issue_x = [&](int g) {
+  auto issue_b = [&](int g) {
     const int st = g % STAGES;
-    const int j = tile_of(g / nkb);
-    const int t0 = (j % p.n_ttiles) * TILE_T + static_cast<int>(rank) * HALF_T;
-    tma_load_2d_pair(smem + st * STAGE_BYTES + A_BYTES, &tm_x, full_even + st * 8,
-                     (g % nkb) * BK, t0, pol_x);
+    tma_load_2d_pair(smem + st * STAGE_BYTES + A_BYTES, tm_b, full_even + st * 8,
+                     (g % nkb) * BK, sc.b_row(g / nkb) + roff, pol_b);
   };
 
   // The weights are never written by another kernel: the first stages' weight
@@ -130,12 +131,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0 && lane == 0) {
     for (int g = 0; g < pre; ++g) {
       if (rank == 0) mbar_expect_tx(&full[g], 2 * STAGE_BYTES);
-      issue_w(g);
+      if (Sched::kAIsWeight) issue_a(g); else issue_b(g);
     }
   }
   griddep_wait();
+  if (warp >= 2) epi.start();
   if (warp == 0 && lane == 0)
-    for (int g = 0; g < pre; ++g) issue_x(g);
+    for (int g = 0; g < pre; ++g) {
+      if (Sched::kAIsWeight) issue_b(g); else issue_a(g);
+    }
   // TMEM is taken only once every earlier kernel has finished, so a CTA that
   // holds it never waits on a predecessor
   if (warp == 1) {
@@ -156,8 +160,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!mbar_wait_pair(&empty[st], ((g / STAGES) - 1) & 1, abort_flag, abort_peer, 0x301))
           break;
         if (rank == 0) mbar_expect_tx(&full[st], 2 * STAGE_BYTES);
-        issue_w(g);
-        issue_x(g);
+        issue_a(g);
+        issue_b(g);
       }
       if (*abort_flag && rank == 0) {
         // let the loads in flight land before the CTA can exit
@@ -169,7 +173,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (rank == 0 && lane == 0 && total_kb > 0) {
       int g = 0;
       bool ok = true;
-      for (int li = 0; li < my_tiles && ok; ++li) {
+      for (int li = 0; li < sc.count && ok; ++li) {
         const int b = li & 1;
         if (li >= 2 &&
             !mbar_wait_pair(&acc_empty[b], ((li >> 1) - 1) & 1, abort_flag, abort_peer, 0x303))
@@ -198,53 +202,31 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_wait(drain, 0, nullptr, 0x306);
     }
   } else {
-    // warps 2..5: TMEM lane quarter (warp % 4) = this CTA's vocabulary rows.
-    // The warps work independently (no barrier among them), so one that gives
-    // up after an expired wait cannot strand the others.
+    // Epilogue warps, TMEM lane quarter warp % 4; with 8 warps the second four
+    // take the upper half of each tile's columns.  The warps work
+    // independently (no barrier among them), so one that gives up after an
+    // expired wait cannot strand the others.
+    const int e = warp - 2;
     const int quarter = warp & 3;
+    constexpr int NCOLS = ACC_COLS / (EPI_WARPS / 4);
+    const int col0 = (e / 4) * NCOLS;
     const uint32_t acc_empty_even = cluster_addr(acc_empty, 0);
-    for (int li = 0; li < my_tiles; ++li) {
+    for (int li = 0; li < sc.count; ++li) {
       const int b = li & 1;
-      const int j = tile_of(li);
-      const int tb = (j % p.n_ttiles) * TILE_T;
-      const int v = (j / p.n_ttiles) * TILE_V + static_cast<int>(rank) * HALF_V + quarter * 32 +
-                    lane;
-      // row scale of token tb + 32 c + lane, for every chunk c, while the MMAs run
-      float rs[TILE_T / 32];
-#pragma unroll
-      for (int c = 0; c < TILE_T / 32; ++c) {
-        rs[c] = 1.f;
-        const int tg = tb + c * 32 + lane;
-        if (p.ssq_in != nullptr && tg < p.M) {
-          float acc = 0.f;
-          for (int q = 0; q < p.n_ssq_in; ++q) acc += p.ssq_in[static_cast<size_t>(q) * p.M + tg];
-          rs[c] = rsqrtf(acc * p.inv_k + p.eps);
-        }
-      }
+      epi.prepare(li);
       if (!__all_sync(0xffffffffu,
                       mbar_wait_pair(&acc_full[b], (li >> 1) & 1, abort_flag, abort_peer, 0x305)))
         break;
       tc_fence_after();
-      const uint32_t taddr =
-          tmem + static_cast<uint32_t>(b * ACC_COLS) + (static_cast<uint32_t>(quarter * 32) << 16);
-#pragma unroll
-      for (int c = 0; c < TILE_T / 32; ++c) {
-        if (tb + c * 32 >= p.M) break;  // warp-uniform
-        uint32_t r[32];
-        tmem_ld32(taddr + c * 32, r);
-        tmem_ld_wait();
-        float* out = p.logits + static_cast<size_t>(tb + c * 32) * p.N + v;
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float sc = __shfl_sync(0xffffffffu, rs[c], i);
-          if (tb + c * 32 + i < p.M) out[static_cast<size_t>(i) * p.N] = __uint_as_float(r[i]) * sc;
-        }
-      }
+      epi.consume(li, tmem + static_cast<uint32_t>(b * ACC_COLS + col0) +
+                          (static_cast<uint32_t>(quarter * 32) << 16),
+                  col0, NCOLS);
       // this warp's reads of buffer b are complete: the MMAs may overwrite it
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(acc_empty_even + b * 8);
     }
+    epi.finish();
   }
 
   // every MMA has completed (each CTA saw its last acc_full) and every remote
@@ -255,6 +237,190 @@ __global__ void __launch_bounds__(THREADS, 1)
     tc_fence_after();
     tmem_dealloc_pair(tmem, TMEM_COLS);
   }
+}
+
+// Row scale of token t (1 without sums of squares).
+__device__ __forceinline__ float row_scale(const float* ssq_in, int n_ssq_in, int M, int t,
+                                           float inv_k, float eps) {
+  if (ssq_in == nullptr || t >= M) return 1.f;
+  float acc = 0.f;
+  for (int q = 0; q < n_ssq_in; ++q) acc += ssq_in[static_cast<size_t>(q) * M + t];
+  return rsqrtf(acc * inv_k + eps);
+}
+
+// ---------------------------------------------------------------------------
+// Logits to memory.
+// ---------------------------------------------------------------------------
+struct Params {
+  int M, N, K;
+  int n_ttiles;          // token tiles: ceil(M / 256)
+  int n_tiles;           // (N / 256) * n_ttiles pair tiles, token tile fastest
+  int n_pairs;           // CTA pairs in the grid
+  float* logits;         // [M, N] fp32
+  const float* ssq_in;   // [n_ssq_in, M] or null (rs = 1)
+  int n_ssq_in;
+  float inv_k, eps;
+};
+
+struct StoreSched {
+  static constexpr bool kAIsWeight = true;
+  int count, nkb, pair, n_pairs, n_ttiles;
+  __device__ int tile(int li) const { return pair + li * n_pairs; }
+  __device__ int a_row(int li) const { return (tile(li) / n_ttiles) * TILE; }  // vocabulary
+  __device__ int b_row(int li) const { return (tile(li) % n_ttiles) * TILE; }  // tokens
+};
+
+struct StoreEpi {
+  const Params* p;
+  const StoreSched* sc;
+  uint32_t rank;
+  int quarter, lane;
+  float rs[TILE / 32];  // scale of token (tile base + 32 c + lane)
+
+  __device__ void start() {}
+  __device__ void prepare(int li) {
+    const int tb = sc->b_row(li);
+#pragma unroll
+    for (int c = 0; c < TILE / 32; ++c)
+      rs[c] = row_scale(p->ssq_in, p->n_ssq_in, p->M, tb + c * 32 + lane, p->inv_k, p->eps);
+  }
+  __device__ void consume(int li, uint32_t taddr, int col0, int ncols) {
+    (void)col0;
+    (void)ncols;
+    const int tb = sc->b_row(li);
+    const int v = sc->a_row(li) + static_cast<int>(rank) * HALF + quarter * 32 + lane;
+#pragma unroll
+    for (int c = 0; c < TILE / 32; ++c) {
+      if (tb + c * 32 >= p->M) break;  // warp-uniform
+      uint32_t r[32];
+      tmem_ld32(taddr + c * 32, r);
+      tmem_ld_wait();
+      float* out = p->logits + static_cast<size_t>(tb + c * 32) * p->N + v;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float sc_i = __shfl_sync(0xffffffffu, rs[c], i);
+        if (tb + c * 32 + i < p->M) out[static_cast<size_t>(i) * p->N] = __uint_as_float(r[i]) * sc_i;
+      }
+    }
+  }
+  __device__ void finish() {}
+};
+
+__global__ void __launch_bounds__(threads_for(STORE_EPI_WARPS), 1)
+    unembed_pair_kernel(const __grid_constant__ CUtensorMap tm_w,
+                        const __grid_constant__ CUtensorMap tm_x, Params p) {
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  StoreSched sc;
+  sc.nkb = p.K / BK;
+  sc.pair = pair;
+  sc.n_pairs = p.n_pairs;
+  sc.n_ttiles = p.n_ttiles;
+  sc.count = pair < p.n_tiles ? (p.n_tiles - 1 - pair) / p.n_pairs + 1 : 0;
+  StoreEpi epi;
+  epi.p = &p;
+  epi.sc = &sc;
+  epi.rank = cluster_ctarank();
+  epi.quarter = warp_id() & 3;
+  epi.lane = lane_id();
+  pair_pipeline<STORE_EPI_WARPS>(&tm_w, &tm_x, l2_policy_evict_first(), l2_policy_evict_last(),
+                                 sc, epi);
+}
+
+// ---------------------------------------------------------------------------
+// Unembedding fused with the sampler's row pass.
+//
+// Pair p works on token tile p / segs and on the contiguous vocabulary range
+// [seg * V / segs, (seg + 1) * V / segs) (in 256-entry tiles), seg = p % segs.
+// A thread of an epilogue warp owns one token and one half of each tile's
+// columns; it keeps the row pass state of sampler.cuh across the range and
+// writes one FusedPartial at the end, slot (token, 2 seg + half).
+// ---------------------------------------------------------------------------
+struct SampleFusedParams {
+  int M, N, K;            // tokens, vocabulary, width
+  int n_vtiles;           // N / 256
+  int segs;               // pairs per token tile
+  int n_pairs;            // segs * ceil(M / 256)
+  const float* ssq_in;
+  int n_ssq_in;
+  float inv_k, eps;
+  SampleParams sp;        // sampler settings (B, C, V = N, seed, block, step, temperature)
+  const int32_t* tok;     // [M] current canvas tokens
+  FusedPartial* part;     // [M, 2 * segs]
+};
+
+struct SampleSched {
+  static constexpr bool kAIsWeight = false;
+  int count, nkb, tt, vt0;
+  __device__ int a_row(int li) const { (void)li; return tt * TILE; }   // tokens
+  __device__ int b_row(int li) const { return (vt0 + li) * TILE; }     // vocabulary
+};
+
+struct SampleEpi {
+  const SampleFusedParams* p;
+  const SampleSched* sc;
+  int t;            // token row (global), may be >= M in a ragged tile
+  int slot;
+  int cur;          // current canvas token (its logit is recorded)
+  float k2, rs;
+  uint32_t c1, step, block;
+  uint2 key;
+  RowState st;
+
+  int seg;
+
+  __device__ void start() {
+    const uint32_t rank = cluster_ctarank();
+    const int warp = warp_id(), lane = lane_id();
+    const int e = warp - 2;
+    t = sc->tt * TILE + static_cast<int>(rank) * HALF + (warp & 3) * 32 + lane;
+    slot = 2 * seg + e / 4;
+    const bool valid = t < p->M;
+    const int b = valid ? t / p->sp.C : 0;
+    const int pos = valid ? t - b * p->sp.C : 0;
+    cur = valid ? p->tok[t] : -1;
+    const int s = read_step(p->sp);
+    step = static_cast<uint32_t>(s);
+    block = static_cast<uint32_t>(p->sp.block);
+    k2 = 1.4426950408889634f / step_temperature(s, p->sp.max_steps, p->sp.t_start, p->sp.t_end);
+    rs = row_scale(p->ssq_in, p->n_ssq_in, p->M, t, p->inv_k, p->eps);
+    c1 = (static_cast<uint32_t>(pos) & 0xFFFFFFu) | (kTagGumbel << 24);
+    key = make_uint2(p->sp.seed, static_cast<uint32_t>(b));
+    st.reset();
+  }
+  __device__ void prepare(int li) { (void)li; }
+  __device__ void consume(int li, uint32_t taddr, int col0, int ncols) {
+    const int vbase = sc->b_row(li) + col0;
+    for (int c = 0; c < ncols; c += 32) {
+      uint32_t r[32];
+      tmem_ld32(taddr + c, r);
+      tmem_ld_wait();
+      float l[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) l[i] = __uint_as_float(r[i]) * rs;
+      st.update32(l, vbase + c, cur, k2, c1, step, block, key);
+    }
+  }
+  __device__ void finish() {
+    if (t < p->M) p->part[static_cast<size_t>(t) * (2 * p->segs) + slot] = st.partial(k2);
+  }
+};
+
+__global__ void __launch_bounds__(threads_for(SAMPLE_EPI_WARPS), 1)
+    unembed_sample_kernel(const __grid_constant__ CUtensorMap tm_x,
+                          const __grid_constant__ CUtensorMap tm_w, SampleFusedParams p) {
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  const int seg = pair % p.segs;
+  SampleSched sc;
+  sc.nkb = p.K / BK;
+  sc.tt = pair / p.segs;
+  sc.vt0 = static_cast<int>((static_cast<long long>(seg) * p.n_vtiles) / p.segs);
+  sc.count = static_cast<int>((static_cast<long long>(seg + 1) * p.n_vtiles) / p.segs) - sc.vt0;
+  SampleEpi epi;
+  epi.p = &p;
+  epi.sc = &sc;
+  epi.seg = seg;
+  pair_pipeline<SAMPLE_EPI_WARPS>(&tm_x, &tm_w, l2_policy_evict_last(), l2_policy_evict_first(),
+                                  sc, epi);
 }
 
 }  // namespace unembed

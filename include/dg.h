@@ -238,6 +238,24 @@ int dg_sample_commit(const float* logits, int32_t* tok, uint8_t* committed,
 size_t dg_sample_commit_workspace_bytes(int B, int C, int V);
 
 /*
+ * dg_unembed_sample_commit - dg_unembed followed by dg_sample_commit, fused:
+ * the logits h w_u^T are formed tile by tile on the tensor cores and reduced
+ * to the sampler's per-position statistics in registers, so they never reach
+ * memory.  Same sources, definitions and in/out state as dg_sample_commit,
+ * with logits[b, i, v] = sum_k h[b*C + i, k] w_u[v, k].
+ * h bf16 [B*C, d] (already normalised); w_u bf16 [V, d].  V % 256 == 0,
+ * d % 64 == 0, C <= 1024.  Workspace: dg_unembed_sample_commit_workspace_bytes().
+ * The statistics are merged in a different order than dg_sample_commit's,
+ * so sums agree to rounding and decisions agree except at near-ties.
+ */
+int dg_unembed_sample_commit(const void* h, const void* w_u, int d, int32_t* tok,
+                             uint8_t* committed, int32_t* prev_argmax, int32_t* seq_status,
+                             const dg_sampler_cfg* cfg, uint32_t seed, int block, int step,
+                             int B, int C, int V, const dg_step_out* out, void* workspace,
+                             size_t workspace_bytes, void* stream);
+size_t dg_unembed_sample_commit_workspace_bytes(int B, int C, int V);
+
+/*
  * dg_sample_commit_noalloc - dg_sample_commit without a workspace argument.
  * The paper has no counterpart: this is a library convenience.  It serves
  * callers that cannot allocate device memory - a plugin whose host owns every
