@@ -326,6 +326,8 @@ def run_kernel_bench(args):
                       B = --batch, 48 scheduled steps, logits regenerated per
                       step outside the timed region.
     --kernel gemm     one projection y = x w^T for --shape M,N,K (bf16 out).
+    --kernel unembed  the unembedding alone, logits to memory.
+    --kernel fused    the unembedding fused with a sampler step, and unfused.
     """
     import torch
     import canvas_denoising_denoise_b200 as dg
@@ -402,6 +404,39 @@ def run_kernel_bench(args):
                     "frac_bf16_peak": round(fl / t / 1e12 / peaks["bf16_tflops"], 4),
                     "gbs": round(byts / t / 1e9, 1),
                     "frac_hbm_peak": round(byts / t / 1e9 / peaks["hbm_gbs"], 4)})
+    elif args.kernel == "fused":
+        # the unembedding fused with one sampler step (fused kernel + merge +
+        # commit) against the unfused pair (unembedding, then sample_commit)
+        B, d, V = args.batch, 2048, 262144
+        M = B * CANVAS
+        h = torch.randn((M, d), device="cuda").to(torch.bfloat16)
+        w = (torch.randn((V, d), device="cuda") * 0.02).to(torch.bfloat16)
+        settings = dg.SamplerSettings()
+        tok = torch.zeros((B, CANVAS), dtype=torch.int32, device="cuda")
+        com = torch.zeros((B, CANVAS), dtype=torch.uint8, device="cuda")
+        prev = torch.full((B, CANVAS), -1, dtype=torch.int32, device="cuda")
+        stat = torch.zeros(B, dtype=torch.int32, device="cuda")
+        lg = torch.empty((B, CANVAS, V), dtype=torch.float32, device="cuda")
+        ws = dg.Workspace()
+
+        def fused():
+            stat.zero_()
+            dg.unembed_sample_commit(h, w, tok, com, prev, stat, settings, 0, 0, 5, ws=ws)
+
+        def unfused():
+            stat.zero_()
+            dg.unembed(h, w, lg.view(M, V))
+            dg.sample_commit(lg, tok, com, prev, stat, settings, 0, 0, 5, ws=ws)
+
+        fl = 2.0 * M * V * d
+        for name, fn in (("unembed_sample_commit (fused)", fused),
+                         ("unembed + sample_commit", unfused)):
+            t = timed(fn, args.steps)
+            out.append({"kernel": name, "shape": [M, V, d], "us": round(t * 1e6, 2),
+                        "tflops": round(fl / t / 1e12, 1),
+                        "frac_bf16_peak": round(fl / t / 1e12 / peaks["bf16_tflops"], 4),
+                        "weight_gbs": round(V * d * 2 / t / 1e9, 1),
+                        "frac_hbm_peak": round(V * d * 2 / t / 1e9 / peaks["hbm_gbs"], 4)})
     elif args.kernel == "gemm":
         M, N, K = (int(x) for x in args.shape.split(","))
         x = torch.randn((M, K), device="cuda").to(torch.bfloat16)
@@ -427,7 +462,8 @@ def main():
     ap.add_argument("--workload", default="full", choices=["full", "tiny"])
     ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["attn", "sampler", "gemm", "unembed"], default=None,
+    ap.add_argument("--kernel", choices=["attn", "sampler", "gemm", "unembed", "fused"],
+                    default=None,
                     help="time one kernel alone instead of the denoising step")
     ap.add_argument("--prefix", type=int, default=0)
     ap.add_argument("--batch", type=int, default=1)
