@@ -83,3 +83,37 @@ def test_unembed_full_vocab_sampled_rows():
     dg.unembed(h, w, again)
     torch.cuda.synchronize()
     assert torch.equal(again, logits)
+
+
+def test_gelu_epilogue_matches_exact_gelu_to_the_bf16_step():
+    """Identity weights make the accumulator equal the input, so each output is
+    bf16(gelu(x)) of one bf16 x; the epilogue's erf (Abramowitz & Stegun 7.1.26,
+    error <= 1.5e-7) must give the bf16 rounding of the exact GELU except within
+    a hair of a rounding boundary, and never more than one bf16 step away."""
+    import canvas_denoising_denoise_b200 as dg
+    n = 128
+    g = torch.Generator().manual_seed(8)
+    x = (torch.rand((1024, n), generator=g) * 12 - 6).to(torch.bfloat16)
+    w = torch.eye(n, dtype=torch.bfloat16)
+    out = torch.empty((1024, n), dtype=torch.bfloat16, device="cuda")
+    dg.linear(x.cuda(), w.cuda(), out, dg.EPI_GELU_BF16)
+    torch.cuda.synchronize()
+    exact = M.gelu(to64(x))                        # fp64, exact erf
+    want = torch.from_numpy(exact).to(torch.bfloat16)
+    got = out.cpu()
+    diff = got != want
+    # a mismatch is allowed only where the exact value lies within the erf
+    # error (plus fp32 rounding) of the midpoint between want and its bf16
+    # neighbour on the side of the exact value, and only by that one step
+    ex = torch.from_numpy(exact)
+    wi = want.view(torch.int16).int()
+    away = ex.abs() > want.double().abs()            # exact beyond want in magnitude
+    nb = (wi + torch.where(away, 1, -1)).short().view(torch.bfloat16)
+    mid = (want.double() + nb.double()) / 2
+    near = (ex - mid).abs() <= 1e-6 + 1e-6 * ex.abs()
+    assert not (diff & ~near).any(), int((diff & ~near).sum())
+    assert torch.equal(got[diff], nb[diff])
+    # where the output is not tiny the absolute error is a negligible fraction
+    # of the bf16 step, so mismatches (midpoint cases) must be rare
+    big = ex.abs() >= 1e-2
+    assert int((diff & big).sum()) <= 0.01 * int(big.sum())
