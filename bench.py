@@ -177,41 +177,78 @@ def captured_traffic(profile, sources):
         return None
 
 
-def gemm_roofline(dg, model, shape, batch, peaks, stream):
-    """Achieved TFLOP/s of the tcgen05 GEMM kernel on the unembedding launch.
-
-    The unembedding (M = B*256 tokens, N = vocab, K = d) is the largest single
-    launch of a denoising step; it is timed alone with CUDA events on the
-    benchmark stream, with a buffer larger than L2 written between launches.
-    """
+def timed_alone(fn, stream, reps=8, warm=2):
+    """Median CUDA-event time of fn() on `stream`, L2 flushed (read-only) before each call."""
     import torch
-    M, d, V = batch * CANVAS, shape.d, shape.vocab
-    h = torch.randn((M, d), device="cuda").to(torch.bfloat16)
-    logits = torch.empty((M, V), dtype=torch.float32, device="cuda")
     flush = L2Flush()
     times = []
-    for i in range(8):
+    for i in range(reps + warm):
         flush()
         s = torch.cuda.Event(enable_timing=True)
         e = torch.cuda.Event(enable_timing=True)
         s.record(stream)
-        dg.unembed(h, model.w["unembed"], logits, stream=stream)
+        fn()
         e.record(stream)
         torch.cuda.synchronize()
-        if i >= 2:
+        if i >= warm:
             times.append(s.elapsed_time(e) / 1000.0)
-    t = statistics.median(times)
-    flops = 2.0 * M * V * d
+    return statistics.median(times)
+
+
+def gemm_roofline(dg, model, shape, batch, peaks, stream):
+    """The dominant kernel: the layer projection GEMM (gemm_kernel), on its
+    largest launch of a denoising step, the MLP down projection
+    (M = B*256 tokens, N = d, K = F; at B = 1 gemm_kernel<4,128>, 128 CTAs).
+
+    Timed alone with CUDA events on the benchmark stream after a read-only L2
+    flush, with the workload's own weights; FLOP-based against the burst bf16
+    peak (at 256 tokens the launch sits at the ridge: 256 FLOP per weight byte).
+    """
+    import torch
+    M, N, K = batch * CANVAS, shape.d, shape.ffn
+    w = model.w["layers"][shape.n_layers - 1]["w_down"]
+    x = torch.randn((M, K), device="cuda").to(torch.bfloat16)
+    out = torch.zeros((M, N), dtype=torch.float32, device="cuda")
+    ws = dg.Workspace()
+    t = timed_alone(lambda: dg.linear(x, w, out, dg.EPI_RESID_F32, ws=ws, stream=stream), stream)
+    flops = 2.0 * M * N * K
     achieved = flops / t / 1e12
     peak = peaks["bf16_tflops"]
-    return {"kernel": "gemm_kernel (unembedding launch)", "bound": "tensor",
-            "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+    return {"kernel": "gemm_kernel (MLP down projection launch)", "shape": [M, N, K],
+            "bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4),
-            "traffic": (captured_traffic("gemm_unembed_full.md", ["gemm.cuh", "dg_common.cuh"])
+            "traffic": (captured_traffic("gemm_mlp_down_full.md", ["gemm.cuh", "dg_common.cuh"])
                         if batch == 1 else None),
-            "algorithmic_bytes": int(V * d * 2 + M * V * 4 + M * d * 2),
+            "algorithmic_bytes": int(N * K * 2 + M * K * 2 + M * N * 4 * 2),
+            "hbm_frac": round((N * K * 2 + M * K * 2 + M * N * 8) / t / 1e9 / peaks["hbm_gbs"], 4),
             "peak_source": f"{peaks['source']} burst bf16",
-            "launch_us": round(t * 1e6, 1), "flops_per_launch": flops}
+            "launch_us": round(t * 1e6, 2), "flops_per_launch": flops}
+
+
+def sampler_step_roofline(dg, model, shape, batch, peaks, stream):
+    """The unembedding fused with one sampler step (fused kernel + merge +
+    commit): 2*M*V*d FLOP; the vocabulary matrix (V*d*2 bytes) is read once."""
+    import torch
+    M, d, V = batch * CANVAS, shape.d, shape.vocab
+    h = torch.randn((M, d), device="cuda").to(torch.bfloat16)
+    tok = torch.zeros((batch, CANVAS), dtype=torch.int32, device="cuda")
+    com = torch.zeros((batch, CANVAS), dtype=torch.uint8, device="cuda")
+    prev = torch.full((batch, CANVAS), -1, dtype=torch.int32, device="cuda")
+    stat = torch.zeros(batch, dtype=torch.int32, device="cuda")
+    ws = dg.Workspace()
+    settings = dg.SamplerSettings()
+
+    def step():
+        stat.zero_()
+        dg.unembed_sample_commit(h, model.w["unembed"], tok, com, prev, stat, settings, 0, 0, 5,
+                                 ws=ws, stream=stream)
+    t = timed_alone(step, stream)
+    flops = 2.0 * M * V * d
+    return {"kernel": "unembed_sample_kernel + merge + commit", "shape": [M, V, d],
+            "achieved": round(flops / t / 1e12, 1), "peak": peaks["bf16_tflops"],
+            "unit": "TFLOP/s", "frac": round(flops / t / 1e12 / peaks["bf16_tflops"], 4),
+            "hbm_frac": round(V * d * 2 / t / 1e9 / peaks["hbm_gbs"], 4),
+            "us": round(t * 1e6, 1)}
 
 
 def attn_roofline(dg, shape, batch, prefix, peaks, stream):
@@ -441,11 +478,16 @@ def run_kernel_bench(args):
         M, N, K = (int(x) for x in args.shape.split(","))
         x = torch.randn((M, K), device="cuda").to(torch.bfloat16)
         w = (torch.randn((N, K), device="cuda") * K ** -0.5).to(torch.bfloat16)
-        y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+        epi = {"bf16": dg.EPI_BF16, "gelu": dg.EPI_GELU_BF16, "f32": dg.EPI_F32,
+               "resid": dg.EPI_RESID_F32}[args.epi]
+        y = (torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+             if args.epi in ("bf16", "gelu") else torch.zeros((M, N), dtype=torch.float32,
+                                                                device="cuda"))
         ws = dg.Workspace()
-        t = timed(lambda: dg.linear(x, w, y, dg.EPI_BF16, ws=ws), args.steps)
+        t = timed(lambda: dg.linear(x, w, y, epi, ws=ws), args.steps)
         fl = 2.0 * M * N * K
-        out.append({"kernel": "linear", "shape": [M, N, K], "us": round(t * 1e6, 2),
+        out.append({"kernel": "linear", "epilogue": args.epi, "shape": [M, N, K],
+                    "us": round(t * 1e6, 2),
                     "tflops": round(fl / t / 1e12, 1),
                     "weight_gbs": round(N * K * 2 / t / 1e9, 1)})
     for o in out:
@@ -468,6 +510,8 @@ def main():
     ap.add_argument("--prefix", type=int, default=0)
     ap.add_argument("--batch", type=int, default=1)
     ap.add_argument("--shape", default="256,8192,2048")
+    ap.add_argument("--epi", default="bf16", choices=["bf16", "gelu", "f32", "resid"],
+                    help="epilogue for --kernel gemm")
     ap.add_argument("--heads", default="32,8", help="query,kv heads for --kernel attn")
     args = ap.parse_args()
     if args.kernel:
@@ -559,6 +603,8 @@ def main():
     # ---------------------------------------------------------------- roofline
     roof = gemm_roofline(dg, model, shape, batch, peaks, stream)
     attn = attn_roofline(dg, shape, batch, prompt_len, peaks, stream)
+    samp = (sampler_step_roofline(dg, model, shape, batch, peaks, stream)
+            if shape.vocab % 256 == 0 else None)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -577,6 +623,7 @@ def main():
                                       steps_seen[-1] if steps_seen else None),
             "roofline": roof,
             "canvas_attn": attn,
+            "unembed_sample": samp,
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_val, 2), "unit": UNIT,
                     "h2d_bytes_per_step": int(host_prompt.numel() * 4),

@@ -46,12 +46,16 @@ constexpr int TILE_ROW_FLOATS = BM;                       // staged tile: [BN][B
 constexpr int SMEM_BYTES = 1024 + RING_BYTES + 256 * 4 + 256;
 constexpr int MAX_SPLITS = 8;
 
-// BN: tokens per tile (UMMA N), 128 or 256.
+// BN: tokens per tile (UMMA N), 128 or 256.  A stage holds KPS k-blocks (the
+// k-blocks' A tiles, then their B tiles): each stage costs a fixed share of
+// the pipeline's round trip whatever its size, so at BN = 128 two k-blocks per
+// stage (3 stages of 64 KB) stream faster than one (6 stages of 32 KB).
 template <int BN>
 struct TileCfg {
   static constexpr int B_BYTES = BN * BK * 2;
-  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-  static constexpr int STAGES = RING_BYTES / STAGE_BYTES;  // 4 (BN 256) or 6 (BN 128)
+  static constexpr int KPS = BN == 128 ? 2 : 1;
+  static constexpr int STAGE_BYTES = KPS * (A_BYTES + B_BYTES);
+  static constexpr int STAGES = RING_BYTES / STAGE_BYTES;  // 4 (BN 256) or 3 (BN 128)
   static constexpr int TMEM_COLS = BN;
   static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, false, false);
   static_assert(BN * BM * 4 <= RING_BYTES, "staged tile must fit in the stage ring");
@@ -194,36 +198,48 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (threadIdx.x == 0) trace_stamp(p, 1);
 
   griddep_launch();
+  constexpr int KPS = TC::KPS;
+  const int nst = (nkb + KPS - 1) / KPS;  // stages of this split
+  // k-blocks in stage q (the last one may be short)
+  auto stage_kbs = [&](int q) { return min(KPS, nkb - q * KPS); };
   if (warp == 0) {
     if (lane == 0 && nkb > 0) {
       // weights are streamed once: evict them first unless another token tile
       // of this launch reads the same weight tile
       const uint64_t pol_w = gridDim.x > 1 ? l2_policy_evict_normal() : l2_policy_evict_first();
+      auto load_w = [&](int q) {
+        uint8_t* a = smem + (q % STAGES) * STAGE_BYTES;
+        for (int j = 0; j < stage_kbs(q); ++j)
+          tma_load_2d_hint(a + j * A_BYTES, &tm_w, &full[q % STAGES],
+                           (kb_begin + q * KPS + j) * BK, f0, pol_w);
+      };
+      auto load_x = [&](int q) {
+        uint8_t* b = smem + (q % STAGES) * STAGE_BYTES + KPS * A_BYTES;
+        for (int j = 0; j < stage_kbs(q); ++j)
+          tma_load_2d(b + j * TC::B_BYTES, &tm_x, &full[q % STAGES], (kb_begin + q * KPS + j) * BK,
+                      t0);
+      };
       // the weights are never written by another kernel: the first stages'
       // weight tiles are requested before waiting on the predecessor
-      const int pre = min(STAGES, nkb);
-      for (int kb = 0; kb < pre; ++kb) {
-        mbar_expect_tx(&full[kb], STAGE_BYTES);
-        tma_load_2d_hint(smem + kb * STAGE_BYTES, &tm_w, &full[kb], (kb_begin + kb) * BK, f0,
-                         pol_w);
+      const int pre = min(STAGES, nst);
+      for (int q = 0; q < pre; ++q) {
+        mbar_expect_tx(&full[q], stage_kbs(q) * (A_BYTES + TC::B_BYTES));
+        load_w(q);
       }
       griddep_wait();
-      for (int kb = 0; kb < pre; ++kb)
-        tma_load_2d(smem + kb * STAGE_BYTES + A_BYTES, &tm_x, &full[kb], (kb_begin + kb) * BK, t0);
+      for (int q = 0; q < pre; ++q) load_x(q);
       int issued = pre;
-      for (int kb = pre; kb < nkb; ++kb) {
-        const int st = kb % STAGES;
-        if (!mbar_wait(&empty[st], ((kb / STAGES) - 1) & 1, abort_flag, 0x101)) break;
-        uint8_t* a = smem + st * STAGE_BYTES;
-        mbar_expect_tx(&full[st], STAGE_BYTES);
-        const int kx = (kb_begin + kb) * BK;
-        tma_load_2d_hint(a, &tm_w, &full[st], kx, f0, pol_w);
-        tma_load_2d(a + A_BYTES, &tm_x, &full[st], kx, t0);
-        issued = kb + 1;
+      for (int q = pre; q < nst; ++q) {
+        const int st = q % STAGES;
+        if (!mbar_wait(&empty[st], ((q / STAGES) - 1) & 1, abort_flag, 0x101)) break;
+        mbar_expect_tx(&full[st], stage_kbs(q) * (A_BYTES + TC::B_BYTES));
+        load_w(q);
+        load_x(q);
+        issued = q + 1;
       }
       if (*abort_flag) {
-        for (int kb = max(0, issued - STAGES); kb < issued; ++kb)
-          mbar_wait(&full[kb % STAGES], (kb / STAGES) & 1, nullptr, 0x102);
+        for (int q = max(0, issued - STAGES); q < issued; ++q)
+          mbar_wait(&full[q % STAGES], (q / STAGES) & 1, nullptr, 0x102);
       }
     } else {
       griddep_wait();
@@ -231,17 +247,20 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp == 1) {
     griddep_wait();
     if (lane == 0 && nkb > 0) {
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int st = kb % STAGES;
-        if (!mbar_wait(&full[st], (kb / STAGES) & 1, abort_flag, 0x103)) break;
-        if (kb == 0) trace_stamp(p, 2);
+      for (int q = 0; q < nst; ++q) {
+        const int st = q % STAGES;
+        if (!mbar_wait(&full[st], (q / STAGES) & 1, abort_flag, 0x103)) break;
+        if (q == 0) trace_stamp(p, 2);
         tc_fence_after();
         const uint32_t a_base = smem_u32(smem + st * STAGE_BYTES);
-        const uint32_t b_base = a_base + A_BYTES;
+        const uint32_t b_base = a_base + KPS * A_BYTES;
+        for (int j = 0; j < stage_kbs(q); ++j) {
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk) {
-          umma_ss(tmem_acc, sdesc_sw128(a_base + kk * 32, 16, 1024),
-                  sdesc_sw128(b_base + kk * 32, 16, 1024), TC::IDESC, (kb | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < BK / 16; ++kk) {
+            umma_ss(tmem_acc, sdesc_sw128(a_base + j * A_BYTES + kk * 32, 16, 1024),
+                    sdesc_sw128(b_base + j * TC::B_BYTES + kk * 32, 16, 1024), TC::IDESC,
+                    (q | j | kk) != 0 ? 1u : 0u);
+          }
         }
         umma_commit(&empty[st]);
       }
