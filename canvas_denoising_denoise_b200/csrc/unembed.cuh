@@ -48,18 +48,18 @@ constexpr int HALF = TILE / 2;            // ... per CTA
 constexpr int BK = 64;                    // one 128-byte swizzle row of bf16
 constexpr int A_BYTES = HALF * BK * 2;    // 16 KB
 constexpr int B_BYTES = HALF * BK * 2;    // 16 KB
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int STAGES = 6;
-constexpr int RING_BYTES = STAGES * STAGE_BYTES;  // 192 KB
+constexpr int RING_BYTES = 6 * (A_BYTES + B_BYTES);  // 192 KB of TMA stages
 constexpr int ACC_COLS = TILE;                    // fp32 columns per accumulator buffer
 constexpr int TMEM_COLS = 2 * ACC_COLS;           // two buffers: all 512 columns
 constexpr int SMEM_BYTES = 1024 + RING_BYTES + 256;
 constexpr uint32_t IDESC = idesc_bf16_f32(TILE, TILE, false, false);
 
-// Epilogue warps: 4 for the logits store, 8 for the fused sampler (two warps
-// per TMEM lane quarter, each taking half of a tile's columns).
+// Epilogue warps: 4 for the logits store, 12 for the fused sampler (three
+// warps per TMEM lane quarter, each taking a third of a tile's columns: the
+// row pass is a long dependent chain per element, and more warps hide it).
 constexpr int STORE_EPI_WARPS = 4;
-constexpr int SAMPLE_EPI_WARPS = 8;
+constexpr int SAMPLE_EPI_WARPS = 12;
+constexpr int SAMPLE_SLOTS = SAMPLE_EPI_WARPS / 4;  // partials per (token, segment)
 __host__ __device__ constexpr int threads_for(int epi_warps) { return 64 + 32 * epi_warps; }
 
 // ---------------------------------------------------------------------------
@@ -69,10 +69,15 @@ __host__ __device__ constexpr int threads_for(int epi_warps) { return 64 + 32 * 
 // prepare(li) before the tile's accumulator is ready, consume(li, taddr, col0,
 // ncols) once it is, finish() after the last tile.
 // ---------------------------------------------------------------------------
-template <int EPI_WARPS, class Sched, class Epi>
+template <int EPI_WARPS, int KPS, class Sched, class Epi>
 __device__ __forceinline__ void pair_pipeline(const CUtensorMap* tm_a, const CUtensorMap* tm_b,
                                               uint64_t pol_a, uint64_t pol_b, const Sched& sc,
                                               Epi& epi) {
+  // A stage holds KPS consecutive k-blocks (their A tiles, then their B
+  // tiles), so each row of a weight tile is requested KPS * 128 contiguous
+  // bytes at a time.  sc.nkb is a multiple of KPS.
+  constexpr int STAGE_BYTES = KPS * (A_BYTES + B_BYTES);
+  constexpr int STAGES = RING_BYTES / STAGE_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -88,7 +93,8 @@ __device__ __forceinline__ void pair_pipeline(const CUtensorMap* tm_a, const CUt
   const int lane = lane_id();
   const uint32_t rank = cluster_ctarank();  // 0: issues the MMAs
   const int nkb = sc.nkb;
-  const int total_kb = sc.count * nkb;
+  const int nstg = nkb / KPS;              // stages per tile
+  const int total_stg = sc.count * nstg;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -114,20 +120,24 @@ __device__ __forceinline__ void pair_pipeline(const CUtensorMap* tm_a, const CUt
   const uint32_t full_even = cluster_addr(full, 0);
   const int roff = static_cast<int>(rank) * HALF;
 
+  // stage g of this pair's walk: tile g / nstg, k-blocks KPS * (g % nstg) + j
   auto issue_a = [&](int g) {
     const int st = g % STAGES;
-    tma_load_2d_pair(smem + st * STAGE_BYTES, tm_a, full_even + st * 8, (g % nkb) * BK,
-                     sc.a_row(g / nkb) + roff, pol_a);
+    for (int j = 0; j < KPS; ++j)
+      tma_load_2d_pair(smem + st * STAGE_BYTES + j * A_BYTES, tm_a, full_even + st * 8,
+                       (KPS * (g % nstg) + j) * BK, sc.a_row(g / nstg) + roff, pol_a);
   };
   auto issue_b = [&](int g) {
     const int st = g % STAGES;
-    tma_load_2d_pair(smem + st * STAGE_BYTES + A_BYTES, tm_b, full_even + st * 8,
-                     (g % nkb) * BK, sc.b_row(g / nkb) + roff, pol_b);
+    for (int j = 0; j < KPS; ++j)
+      tma_load_2d_pair(smem + st * STAGE_BYTES + KPS * A_BYTES + j * B_BYTES, tm_b,
+                       full_even + st * 8, (KPS * (g % nstg) + j) * BK,
+                       sc.b_row(g / nstg) + roff, pol_b);
   };
 
   // The weights are never written by another kernel: the first stages' weight
   // tiles are requested before waiting on the predecessor.
-  const int pre = min(STAGES, total_kb);
+  const int pre = min(STAGES, total_stg);
   if (warp == 0 && lane == 0) {
     for (int g = 0; g < pre; ++g) {
       if (rank == 0) mbar_expect_tx(&full[g], 2 * STAGE_BYTES);
@@ -155,7 +165,7 @@ __device__ __forceinline__ void pair_pipeline(const CUtensorMap* tm_a, const CUt
   if (warp == 0) {
     if (lane == 0) {
       int g = pre;
-      for (; g < total_kb; ++g) {
+      for (; g < total_stg; ++g) {
         const int st = g % STAGES;
         if (!mbar_wait_pair(&empty[st], ((g / STAGES) - 1) & 1, abort_flag, abort_peer, 0x301))
           break;
@@ -170,7 +180,7 @@ __device__ __forceinline__ void pair_pipeline(const CUtensorMap* tm_a, const CUt
       }
     }
   } else if (warp == 1) {
-    if (rank == 0 && lane == 0 && total_kb > 0) {
+    if (rank == 0 && lane == 0 && total_stg > 0) {
       int g = 0;
       bool ok = true;
       for (int li = 0; li < sc.count && ok; ++li) {
@@ -180,7 +190,7 @@ __device__ __forceinline__ void pair_pipeline(const CUtensorMap* tm_a, const CUt
           break;
         tc_fence_after();
         const uint32_t d = tmem + static_cast<uint32_t>(b * ACC_COLS);
-        for (int kb = 0; kb < nkb; ++kb, ++g) {
+        for (int q = 0; q < nstg; ++q, ++g) {
           const int st = g % STAGES;
           if (!mbar_wait_pair(&full[st], (g / STAGES) & 1, abort_flag, abort_peer, 0x304)) {
             ok = false;
@@ -188,11 +198,14 @@ __device__ __forceinline__ void pair_pipeline(const CUtensorMap* tm_a, const CUt
           }
           tc_fence_after();
           const uint32_t a_base = smem_u32(smem + st * STAGE_BYTES);
-          const uint32_t b_base = a_base + A_BYTES;
+          const uint32_t b_base = a_base + KPS * A_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk)
-            umma_ss_pair(d, sdesc_sw128(a_base + kk * 32, 16, 1024),
-                         sdesc_sw128(b_base + kk * 32, 16, 1024), IDESC, (kb | kk) != 0 ? 1u : 0u);
+          for (int j = 0; j < KPS; ++j)
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+              umma_ss_pair(d, sdesc_sw128(a_base + j * A_BYTES + kk * 32, 16, 1024),
+                           sdesc_sw128(b_base + j * B_BYTES + kk * 32, 16, 1024), IDESC,
+                           (q | j | kk) != 0 ? 1u : 0u);
           umma_commit_pair(&empty[st], 0x3);
         }
         if (ok) umma_commit_pair(&acc_full[b], 0x3);
@@ -202,14 +215,18 @@ __device__ __forceinline__ void pair_pipeline(const CUtensorMap* tm_a, const CUt
       mbar_wait(drain, 0, nullptr, 0x306);
     }
   } else {
-    // Epilogue warps, TMEM lane quarter warp % 4; with 8 warps the second four
-    // take the upper half of each tile's columns.  The warps work
+    // Epilogue warps, TMEM lane quarter warp % 4; with more than four, the
+    // warps of a quarter split each tile's columns.  The warps work
     // independently (no barrier among them), so one that gives up after an
     // expired wait cannot strand the others.
     const int e = warp - 2;
     const int quarter = warp & 3;
-    constexpr int NCOLS = ACC_COLS / (EPI_WARPS / 4);
-    const int col0 = (e / 4) * NCOLS;
+    // warps per lane quarter split the tile's 32-column chunks as evenly as
+    // possible: warp set k takes chunks [k C / W, (k + 1) C / W)
+    constexpr int WPQ = EPI_WARPS / 4;
+    constexpr int CHUNKS = ACC_COLS / 32;
+    const int col0 = ((e / 4) * CHUNKS / WPQ) * 32;
+    const int ncols = (((e / 4) + 1) * CHUNKS / WPQ) * 32 - col0;
     const uint32_t acc_empty_even = cluster_addr(acc_empty, 0);
     for (int li = 0; li < sc.count; ++li) {
       const int b = li & 1;
@@ -220,7 +237,7 @@ __device__ __forceinline__ void pair_pipeline(const CUtensorMap* tm_a, const CUt
       tc_fence_after();
       epi.consume(li, tmem + static_cast<uint32_t>(b * ACC_COLS + col0) +
                           (static_cast<uint32_t>(quarter * 32) << 16),
-                  col0, NCOLS);
+                  col0, ncols);
       // this warp's reads of buffer b are complete: the MMAs may overwrite it
       tc_fence_before();
       __syncwarp();
@@ -306,6 +323,7 @@ struct StoreEpi {
   __device__ void finish() {}
 };
 
+template <int KPS>
 __global__ void __launch_bounds__(threads_for(STORE_EPI_WARPS), 1)
     unembed_pair_kernel(const __grid_constant__ CUtensorMap tm_w,
                         const __grid_constant__ CUtensorMap tm_x, Params p) {
@@ -322,7 +340,7 @@ __global__ void __launch_bounds__(threads_for(STORE_EPI_WARPS), 1)
   epi.rank = cluster_ctarank();
   epi.quarter = warp_id() & 3;
   epi.lane = lane_id();
-  pair_pipeline<STORE_EPI_WARPS>(&tm_w, &tm_x, l2_policy_evict_first(), l2_policy_evict_last(),
+  pair_pipeline<STORE_EPI_WARPS, KPS>(&tm_w, &tm_x, l2_policy_evict_first(), l2_policy_evict_last(),
                                  sc, epi);
 }
 
@@ -331,9 +349,9 @@ __global__ void __launch_bounds__(threads_for(STORE_EPI_WARPS), 1)
 //
 // Pair p works on token tile p / segs and on the contiguous vocabulary range
 // [seg * V / segs, (seg + 1) * V / segs) (in 256-entry tiles), seg = p % segs.
-// A thread of an epilogue warp owns one token and one half of each tile's
+// A thread of an epilogue warp owns one token and one third of each tile's
 // columns; it keeps the row pass state of sampler.cuh across the range and
-// writes one FusedPartial at the end, slot (token, 2 seg + half).
+// writes one FusedPartial at the end, slot (token, 3 seg + third).
 // ---------------------------------------------------------------------------
 struct SampleFusedParams {
   int M, N, K;            // tokens, vocabulary, width
@@ -345,7 +363,7 @@ struct SampleFusedParams {
   float inv_k, eps;
   SampleParams sp;        // sampler settings (B, C, V = N, seed, block, step, temperature)
   const int32_t* tok;     // [M] current canvas tokens
-  FusedPartial* part;     // [M, 2 * segs]
+  FusedPartial* part;     // [M, SAMPLE_SLOTS * segs]
 };
 
 struct SampleSched {
@@ -373,7 +391,7 @@ struct SampleEpi {
     const int warp = warp_id(), lane = lane_id();
     const int e = warp - 2;
     t = sc->tt * TILE + static_cast<int>(rank) * HALF + (warp & 3) * 32 + lane;
-    slot = 2 * seg + e / 4;
+    slot = SAMPLE_SLOTS * seg + e / 4;
     const bool valid = t < p->M;
     const int b = valid ? t / p->sp.C : 0;
     const int pos = valid ? t - b * p->sp.C : 0;
@@ -401,10 +419,11 @@ struct SampleEpi {
     }
   }
   __device__ void finish() {
-    if (t < p->M) p->part[static_cast<size_t>(t) * (2 * p->segs) + slot] = st.partial(k2);
+    if (t < p->M) p->part[static_cast<size_t>(t) * (SAMPLE_SLOTS * p->segs) + slot] = st.partial(k2);
   }
 };
 
+template <int KPS>
 __global__ void __launch_bounds__(threads_for(SAMPLE_EPI_WARPS), 1)
     unembed_sample_kernel(const __grid_constant__ CUtensorMap tm_x,
                           const __grid_constant__ CUtensorMap tm_w, SampleFusedParams p) {
@@ -419,7 +438,7 @@ __global__ void __launch_bounds__(threads_for(SAMPLE_EPI_WARPS), 1)
   epi.p = &p;
   epi.sc = &sc;
   epi.seg = seg;
-  pair_pipeline<SAMPLE_EPI_WARPS>(&tm_x, &tm_w, l2_policy_evict_last(), l2_policy_evict_first(),
+  pair_pipeline<SAMPLE_EPI_WARPS, KPS>(&tm_x, &tm_w, l2_policy_evict_last(), l2_policy_evict_first(),
                                   sc, epi);
 }
 
