@@ -38,6 +38,13 @@ Readings (each listed in the design notes):
   Unselected uncommitted positions take x_hat and stay uncommitted (policy
       "keep"), or a fresh uniform token (policy "renoise").
   "Prediction" in stop rule (B) = the argmax of the raw logits at every position.
+  Entropy-bounded selection (same settings table, row "Selecao de token":
+      entropy limit 0.1, the lowest-entropy tokens are selected so that the
+      mutual-information bound stays below the limit), used instead of the
+      fixed k when selection = SELECT_ENTROPY: order U by entropy (ties to the
+      lower position) and commit the longest prefix whose summed entropy is
+      <= entropy_bound; at least the first position is committed, so that
+      every step makes progress.
   Stop after step s when any of: every position is committed after the step;
       (A) and (B) with s >= 1; s = max_steps - 1.  On an (A)/(B) or step-cap
       stop every still-uncommitted position takes x_hat and is committed, and
@@ -53,6 +60,9 @@ from .philox import (TAG_GUMBEL, TAG_INIT, TAG_RENOISE, position_word, token_fro
 POLICY_KEEP = 0
 POLICY_RENOISE = 1
 
+SELECT_TOP_K = 0     # the k uncommitted positions of largest confidence
+SELECT_ENTROPY = 1   # lowest-entropy prefix within the entropy bound
+
 
 @dataclass(frozen=True)
 class SamplerCfg:
@@ -63,6 +73,8 @@ class SamplerCfg:
     renoise_conf: float = 0.05
     stop_entropy: float = 0.005
     unselected_policy: int = POLICY_KEEP
+    selection: int = SELECT_TOP_K
+    entropy_bound: float = 0.1
 
 
 def temperature(cfg, step):
@@ -159,9 +171,18 @@ def sampler_step(cfg, logits, tok, committed, prev_argmax, step, seed, b, block,
     lam = np.where(committed, z_tok - lse, z_x - lse)
 
     uncommitted = np.flatnonzero(~committed)
-    k = min(cfg.commit_k, uncommitted.size)
-    # Largest lambda first, ties to the lower position.
-    order = sorted(uncommitted.tolist(), key=lambda i: (-lam[i], i))
+    if cfg.selection == SELECT_ENTROPY:
+        # Lowest entropy first, ties to the lower position; the longest prefix
+        # whose entropies sum to at most the bound, and never an empty one.
+        order = sorted(uncommitted.tolist(), key=lambda i: (ent[i], i))
+        csum = np.cumsum([ent[i] for i in order])
+        k = int(np.count_nonzero(csum <= cfg.entropy_bound))
+        if uncommitted.size > 0:
+            k = max(k, 1)
+    else:
+        k = min(cfg.commit_k, uncommitted.size)
+        # Largest lambda first, ties to the lower position.
+        order = sorted(uncommitted.tolist(), key=lambda i: (-lam[i], i))
     chosen = np.array(order[:k], dtype=np.int64)
     commit_mask = np.zeros(C, dtype=bool)
     commit_mask[chosen] = True
@@ -200,11 +221,22 @@ def sampler_step(cfg, logits, tok, committed, prev_argmax, step, seed, b, block,
     near = {}
     near["gumbel"] = np.array([s.gumbel_gap < tie_margin for s in stats])
     near["argmax"] = np.array([s.argmax_gap < tie_margin for s in stats])
-    lam_u = np.sort(lam[uncommitted])[::-1]
     boundary = np.zeros(C, dtype=bool)
-    if 0 < k < uncommitted.size and (lam_u[k - 1] - lam_u[k]) < tie_margin:
-        edge = 0.5 * (lam_u[k - 1] + lam_u[k])
-        boundary[uncommitted[np.abs(lam[uncommitted] - edge) < tie_margin]] = True
+    if cfg.selection == SELECT_ENTROPY:
+        # the cut moves if an entropy sum straddles the bound, or if the last
+        # selected and first unselected entropies nearly tie
+        if 0 < k < uncommitted.size:
+            e_in, e_out = ent[order[k - 1]], ent[order[k]]
+            near_cut = (abs(csum[k] - cfg.entropy_bound) < tie_margin or
+                        abs(csum[k - 1] - cfg.entropy_bound) < tie_margin or
+                        (e_out - e_in) < tie_margin)
+            if near_cut:
+                boundary[np.array(order[k - 1:k + 1], dtype=np.int64)] = True
+    else:
+        lam_u = np.sort(lam[uncommitted])[::-1]
+        if 0 < k < uncommitted.size and (lam_u[k - 1] - lam_u[k]) < tie_margin:
+            edge = 0.5 * (lam_u[k - 1] + lam_u[k])
+            boundary[uncommitted[np.abs(lam[uncommitted] - edge) < tie_margin]] = True
     near["commit_boundary"] = boundary
     near["renoise"] = committed & (np.abs(lam - log_tau) < tie_margin)
     near["stop"] = abs(mean_h - cfg.stop_entropy) < tie_margin

@@ -233,3 +233,76 @@ def test_canvas_init_uniform_and_keyed():
     assert a.min() >= 0 and a.max() < 512
     assert not np.array_equal(a, b) and not np.array_equal(a, c)
     assert a[0] == P.token_from_word(P.position_word(0, 0, 0, 0, 0, P.TAG_INIT), 512)
+
+
+def two_outcome_logits(ps, T, V=4):
+    """Rows whose tempered softmax is (p, 1 - p, 0, ...): z = (ln p, ln(1 - p), -inf...)."""
+    rows = np.full((len(ps), V), -1e30)
+    for i, p in enumerate(ps):
+        rows[i, 0] = T * math.log(p)
+        rows[i, 1] = T * math.log1p(-p)
+    return rows
+
+
+def binary_entropy(p):
+    return -p * math.log(p) - (1 - p) * math.log1p(-p)
+
+
+def test_entropy_bounded_selection_worked_example():
+    """GDocs table row "Selecao de token" (entropy limit 0.1), worked by hand.
+
+    Six positions with two-outcome softmaxes p = 0.99, 0.5, 0.999, 0.98,
+    0.995, 0.9 have entropies 0.0560, 0.6931, 0.0079, 0.0980, 0.0314,
+    0.3251 nats.  In increasing entropy: positions 2, 4, 0, 3, 5, 1 with
+    running sums 0.0079, 0.0393, 0.0953, 0.1933, ...  The bound 0.1 admits
+    the first three: positions {2, 4, 0} are committed, the rest are not.
+    """
+    ss = sampler_settings()
+    c = cfg(selection=S.SELECT_ENTROPY, entropy_bound=ss["select_entropy"], renoise_conf=0.0)
+    step = 5
+    ps = [0.99, 0.5, 0.999, 0.98, 0.995, 0.9]
+    logits = two_outcome_logits(ps, S.temperature(c, step))
+    r = S.sampler_step(c, logits, np.zeros(6, dtype=int), np.zeros(6, dtype=bool), None, step,
+                       seed=0, b=0, block=0)
+    for p, h in zip(ps, r.entropy):
+        assert h == pytest.approx(binary_entropy(p), abs=1e-12)
+    assert sorted(np.flatnonzero(r.commit_mask).tolist()) == [0, 2, 4]
+
+
+def test_entropy_bounded_selection_always_progresses_and_skips_committed():
+    """All entropies above the bound: exactly the lowest-entropy uncommitted
+    position is committed; committed positions are never reselected."""
+    c = cfg(selection=S.SELECT_ENTROPY, renoise_conf=0.0)
+    step = 2
+    ps = [0.9, 0.8, 0.7, 0.95, 0.6]          # entropies 0.325 .. 0.673, all > 0.1
+    logits = two_outcome_logits(ps, S.temperature(c, step))
+    committed = np.array([False, False, False, True, False])  # 0.95 is the lowest, but committed
+    r = S.sampler_step(c, logits, np.zeros(5, dtype=int), committed, None, step, seed=0, b=0,
+                       block=0)
+    assert np.flatnonzero(r.commit_mask).tolist() == [0]  # p = 0.9 is the lowest uncommitted
+
+
+def test_entropy_bounded_selection_invariants_on_random_rows():
+    """The committed set is a prefix of the entropy order of U whose sum is
+    within the bound unless it is a single position, and the next position
+    would break the bound."""
+    rng = np.random.default_rng(7)
+    C, V = 48, 64
+    sharp = rng.random(C) < 0.5
+    logits = rng.normal(size=(C, V))
+    logits[sharp, rng.integers(0, V, size=sharp.sum())] += rng.uniform(8, 30, size=sharp.sum())
+    committed = rng.random(C) < 0.2
+    c = cfg(selection=S.SELECT_ENTROPY, renoise_conf=0.0)
+    r = S.sampler_step(c, logits, rng.integers(0, V, size=C), committed, None, 4, seed=3, b=0,
+                       block=0)
+    chosen = np.flatnonzero(r.commit_mask)
+    unc = np.flatnonzero(~committed)
+    assert len(chosen) >= 1 and not np.any(committed[chosen])
+    worst_in = max(r.entropy[chosen])
+    rest = np.setdiff1d(unc, chosen)
+    assert rest.size == 0 or min(r.entropy[rest]) >= worst_in
+    total = float(np.sum(r.entropy[chosen]))
+    assert len(chosen) == 1 or total <= c.entropy_bound
+    if rest.size:
+        assert total + min(r.entropy[rest]) > c.entropy_bound
+    assert len(chosen) > 1  # the sharp rows have tiny entropies: several fit
