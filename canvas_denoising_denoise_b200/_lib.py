@@ -46,7 +46,7 @@ class Model(ctypes.Structure):
 class SamplerCfg(ctypes.Structure):
     _fields_ = [("max_steps", c_int), ("t_start", c_float), ("t_end", c_float),
                 ("commit_k", c_int), ("renoise_conf", c_float), ("stop_entropy", c_float),
-                ("unselected_policy", c_int)]
+                ("unselected_policy", c_int), ("selection", c_int), ("entropy_bound", c_float)]
 
 
 class StepOut(ctypes.Structure):

@@ -424,6 +424,14 @@ size_t sample_ws_bytes(int B, int C, int V) {
   return align_up((size_t)B * C * nchunk * sizeof(dg::RowPartial), 256);
 }
 
+bool sampler_cfg_ok(const dg_sampler_cfg& c) {
+  return c.max_steps >= 1 && c.commit_k >= 0 && c.t_start > 0.f && c.t_end > 0.f &&
+         (c.unselected_policy == DG_UNSELECTED_KEEP ||
+          c.unselected_policy == DG_UNSELECTED_RENOISE) &&
+         (c.selection == DG_SELECT_TOP_K || c.selection == DG_SELECT_ENTROPY) &&
+         c.entropy_bound >= 0.f;
+}
+
 dg::SampleParams make_sample_params(const dg_sampler_cfg& cfg, uint32_t seed, int block,
                                     const int32_t* step_ptr, int step, int B, int C, int V) {
   dg::SampleParams p;
@@ -440,6 +448,8 @@ dg::SampleParams make_sample_params(const dg_sampler_cfg& cfg, uint32_t seed, in
   p.log_tau = cfg.renoise_conf > 0.f ? (float)std::log((double)cfg.renoise_conf) : -INFINITY;
   p.stop_entropy = cfg.stop_entropy;
   p.policy = cfg.unselected_policy;
+  p.selection = cfg.selection;
+  p.entropy_bound = cfg.entropy_bound;
   return p;
 }
 
@@ -787,6 +797,8 @@ void dg_sampler_defaults(dg_sampler_cfg* cfg) {
   cfg->renoise_conf = 0.05f;
   cfg->stop_entropy = 0.005f;
   cfg->unselected_policy = DG_UNSELECTED_KEEP;
+  cfg->selection = DG_SELECT_TOP_K;
+  cfg->entropy_bound = 0.1f;
 }
 
 int dg_check_device_errors(void* stream, uint32_t* code_out) {
@@ -899,8 +911,7 @@ int dg_sample_commit(const float* logits, int32_t* tok, uint8_t* committed,
     return fail(DG_ERR_INVALID_ARG, "dg_sample_commit: null pointer");
   if (B <= 0 || C <= 0 || C > 1024 || V <= 0 || V % 4 || step < 0 || block < 0)
     return fail(DG_ERR_UNSUPPORTED_SHAPE, "dg_sample_commit: need C <= 1024, V %% 4 == 0");
-  if (cfg->max_steps < 1 || cfg->commit_k < 0 || !(cfg->t_start > 0.f) || !(cfg->t_end > 0.f) ||
-      (cfg->unselected_policy != 0 && cfg->unselected_policy != 1))
+  if (!sampler_cfg_ok(*cfg))
     return fail(DG_ERR_INVALID_ARG, "dg_sample_commit: bad sampler settings");
   if (!aligned16(logits)) return fail(DG_ERR_ALIGNMENT, "dg_sample_commit: logits alignment");
   const size_t need = sample_ws_bytes(B, C, V);
@@ -927,8 +938,7 @@ int dg_unembed_sample_commit(const void* h, const void* w_u, int d, int32_t* tok
       step < 0 || block < 0)
     return fail(DG_ERR_UNSUPPORTED_SHAPE,
                 "dg_unembed_sample_commit: need C <= 1024, V %% 256 == 0, d %% 64 == 0");
-  if (cfg->max_steps < 1 || cfg->commit_k < 0 || !(cfg->t_start > 0.f) || !(cfg->t_end > 0.f) ||
-      (cfg->unselected_policy != 0 && cfg->unselected_policy != 1))
+  if (!sampler_cfg_ok(*cfg))
     return fail(DG_ERR_INVALID_ARG, "dg_unembed_sample_commit: bad sampler settings");
   if (!aligned16(h) || !aligned16(w_u))
     return fail(DG_ERR_ALIGNMENT, "dg_unembed_sample_commit: pointers must be 16-byte aligned");
@@ -950,8 +960,7 @@ int dg_sample_commit_noalloc(const float* logits, int32_t* tok, uint8_t* committ
   if (B <= 0 || C <= 0 || C > 1024 || V <= 0 || V % 4 || step < 0 || block < 0)
     return fail(DG_ERR_UNSUPPORTED_SHAPE,
                 "dg_sample_commit_noalloc: need C <= 1024, V %% 4 == 0");
-  if (cfg->max_steps < 1 || cfg->commit_k < 0 || !(cfg->t_start > 0.f) || !(cfg->t_end > 0.f) ||
-      (cfg->unselected_policy != 0 && cfg->unselected_policy != 1))
+  if (!sampler_cfg_ok(*cfg))
     return fail(DG_ERR_INVALID_ARG, "dg_sample_commit_noalloc: bad sampler settings");
   if (!aligned16(logits))
     return fail(DG_ERR_ALIGNMENT, "dg_sample_commit_noalloc: logits alignment");
@@ -1046,7 +1055,7 @@ int dg_denoise_block(const dg_model* m, dg_state* st, const dg_sampler_cfg* cfg,
                      void* stream) {
   DG_TRY(check_model(m));
   DG_TRY(check_state(st, m->cfg, true));
-  if (!cfg || cfg->max_steps < 1 || block < 0)
+  if (!cfg || !sampler_cfg_ok(*cfg) || block < 0)
     return fail(DG_ERR_INVALID_ARG, "dg_denoise_block: bad sampler settings or block");
   if (m->cfg.vocab % 4) return fail(DG_ERR_UNSUPPORTED_SHAPE, "vocab must be a multiple of 4");
   if (st->cache_len_host < 0 || st->cache_len_host + st->canvas > st->lmax)

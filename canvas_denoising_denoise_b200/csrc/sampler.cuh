@@ -232,6 +232,8 @@ struct SampleParams {
   float log_tau;             // ln(renoise_conf), -inf disables re-noise
   float stop_entropy;
   int policy;
+  int selection;             // 0: top commit_k by confidence, 1: entropy-bounded
+  float entropy_bound;
 };
 
 __device__ __forceinline__ int read_step(const SampleParams& p) {
@@ -416,6 +418,7 @@ __global__ void __launch_bounds__(1024) sample_commit_kernel(
     int32_t* __restrict__ o_argmax, float* __restrict__ o_logconf,
     float* __restrict__ o_entropy, uint8_t* __restrict__ o_flags) {
   __shared__ float s_lam[1024];
+  __shared__ float s_ent[1024];
   __shared__ uint8_t s_unc[1024];
   __shared__ float s_red[32];
   __shared__ int s_flag;
@@ -484,14 +487,31 @@ __global__ void __launch_bounds__(1024) sample_commit_kernel(
   }
   if (live) {
     s_lam[i] = lam;
+    s_ent[i] = ent;
     s_unc[i] = was_committed ? 0 : 1;
   }
   __syncthreads();
   const bool final_step = s_flag != 0;
 
-  // top-k among uncommitted: rank = number of uncommitted positions that beat this one
   bool selected = false;
-  if (live && !was_committed) {
+  if (live && !was_committed && p.selection == 1) {
+    // entropy-bounded: rank by (entropy, position) among the uncommitted; the
+    // selection is the ranked prefix whose entropies sum to <= the bound, and
+    // at least rank 0 (the sum is taken in fp64: order-independent)
+    int rank = 0;
+    double csum = static_cast<double>(ent);
+    for (int j = 0; j < p.C; ++j) {
+      if (s_unc[j] && j != i) {
+        const float ej = s_ent[j];
+        if (ej < ent || (ej == ent && j < i)) {
+          ++rank;
+          csum += static_cast<double>(ej);
+        }
+      }
+    }
+    selected = rank == 0 || csum <= static_cast<double>(p.entropy_bound);
+  } else if (live && !was_committed) {
+    // top-k among uncommitted: rank = number of uncommitted positions that beat this one
     const int k = min(p.commit_k, n_unc);
     int rank = 0;
     for (int j = 0; j < p.C; ++j) {

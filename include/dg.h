@@ -106,6 +106,15 @@ typedef struct dg_model {
   const dg_layer_weights* layers;   /* host array of cfg.n_layers entries */
 } dg_model;
 
+/* Which uncommitted positions a step commits.
+ * DG_SELECT_TOP_K: the commit_k of largest log confidence (aiexpert.news
+ *   architecture paragraph: 15-20 confident tokens locked per pass).
+ * DG_SELECT_ENTROPY: Google docs table "Configuracao de exibicao recomendada",
+ *   row "Selecao de token" (entropy limit 0.1): the uncommitted positions in
+ *   increasing entropy (ties to the lower position), as long as their summed
+ *   entropy stays <= entropy_bound, and at least the first one. */
+enum dg_selection { DG_SELECT_TOP_K = 0, DG_SELECT_ENTROPY = 1 };
+
 /* Sampler settings.  dg_sampler_defaults() fills the published values. */
 typedef struct dg_sampler_cfg {
   int max_steps;        /* step cap per canvas (48) */
@@ -115,6 +124,8 @@ typedef struct dg_sampler_cfg {
   float renoise_conf;   /* re-noise committed tokens whose softmax confidence is below (0.05) */
   float stop_entropy;   /* adaptive stop: mean canvas entropy below, in nats (0.005) */
   int unselected_policy;/* enum dg_unselected_policy */
+  int selection;        /* enum dg_selection (DG_SELECT_TOP_K) */
+  float entropy_bound;  /* DG_SELECT_ENTROPY: summed-entropy limit, nats (0.1) */
 } dg_sampler_cfg;
 
 /* Per-step sampler diagnostics: caller-owned device arrays [B, C]; any may be NULL. */
@@ -219,7 +230,8 @@ size_t dg_linear_workspace_bytes(int M, int N, int K);
  * block), word v & 3, u = (2 (r >> 9) + 1) 2^-24; log confidence
  * lambda = z[x] - logsumexp(z) (x = x_hat if uncommitted, else the current token).
  * Then: commit the min(k, #uncommitted) uncommitted positions of largest
- * lambda (ties to the lower position) to x_hat; re-noise committed positions
+ * lambda (ties to the lower position) to x_hat (or, with selection =
+ * DG_SELECT_ENTROPY, the entropy-bounded prefix described at enum dg_selection); re-noise committed positions
  * with lambda < ln(renoise_conf) to a uniform token (Philox tag 1, counter
  * (0, pos | 1 << 24, step, block), token = (r * V) >> 32) and uncommit them;
  * unselected uncommitted positions follow unselected_policy.  Stop when every

@@ -111,3 +111,26 @@ def test_fused_matches_unfused_at_full_vocab():
         if ps.gumbel_gap >= 1e-4:
             assert f["x_hat"][0, pos] == ps.x_hat
         np.testing.assert_allclose(f["entropy"][0, pos], ps.entropy, rtol=1e-4, atol=2e-4)
+
+
+def test_fused_step_entropy_bounded_selection():
+    """The fused path with DG_SELECT_ENTROPY against the oracle."""
+    import canvas_denoising_denoise_b200 as dg
+    B, C, V, d, step = 1, 256, 1024, 256, 12
+    h, w, tok, committed, prev = make_case(B, C, V, d, seed=4242, commit_frac=0.2)
+    # sharpen half the rows: adding 18 w_t / |w_t|^2 to h raises logit t by 18
+    g = torch.Generator().manual_seed(5)
+    rows = torch.randperm(C, generator=g)[: C // 2]
+    targets = torch.randint(0, V, (rows.numel(),), generator=g)
+    hf = h.float()
+    wf = w.float()
+    hf[rows] += 18.0 * wf[targets] / wf[targets].norm(dim=1, keepdim=True) ** 2
+    h = hf.to(torch.bfloat16)
+    settings = dg.SamplerSettings(selection=1, entropy_bound=0.1)
+    gres = run("fused", h, w, tok, committed, prev, settings, 13, 3, step)
+    logits = (h.double() @ w.double().T).float().numpy().reshape(B, C, V)
+    counters = {"near_gumbel": 0, "near_renoise": 0, "skipped_sequences": 0}
+    r = S.sampler_step(S.SamplerCfg(selection=S.SELECT_ENTROPY, entropy_bound=0.1), logits[0],
+                       tok[0], committed[0], prev[0], step, 13, 0, 3)
+    compare(gres, r, 0, committed[0], counters)
+    assert int(r.commit_mask.sum()) > 1
