@@ -30,7 +30,11 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-METRIC = "committed tokens/s (B=1, 256-tok canvas)"
+METRIC = "committed tokens/s (B=1, 256-tok canvas); canvas-attn % of BF16 tensor peak"
+
+
+def metric_name(batch):
+    return METRIC.replace("B=1", f"B={batch}")
 UNIT = "tokens/s"
 CANVAS = 256
 L2_BYTES = 126 * 1024 * 1024
@@ -123,6 +127,11 @@ def workload_spec(name):
     from canvas_denoising_denoise_b200 import synth
     w = synth.WORKLOADS[name]
     return w["model"], w["batch"], w["prompt"]
+
+
+def workload_blocks(name):
+    from canvas_denoising_denoise_b200 import synth
+    return synth.WORKLOADS[name]["blocks"]
 
 
 class L2Flush:
@@ -341,7 +350,8 @@ def run_reference(args):
     for _ in range(max(1, args.steps)):
         vals.append(cpu_baseline_sample(w_cpu, shape, prompt))
     v = statistics.median([x["value"] for x in vals])
-    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": world,
+    line = {"impl": "reference", "metric": metric_name(batch), "value": v, "unit": UNIT,
+            "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(CANVAS / v * 1e3, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic",
@@ -501,7 +511,9 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=5)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--workload", default="full", choices=["full", "tiny"])
+    ap.add_argument("--workload", default="full", choices=["full", "tiny", "long_b1", "long_b8"],
+                    help="full: one canvas after a 4096-token prompt (the headline); long_b*: "
+                         "8 canvases after a 2048-token prompt at B = 1 / 8")
     ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel", choices=["attn", "sampler", "gemm", "unembed", "fused"],
@@ -544,7 +556,8 @@ def main():
     else:
         weights = synth.make_weights_fast(shape, seed=0, device="cuda")
     model = dg.DgModel(shape, weights)
-    lmax = prompt_len + CANVAS
+    blocks = workload_blocks(args.workload)
+    lmax = prompt_len + CANVAS * blocks
     st = dg.DgState(shape, batch, lmax, CANVAS)
     prompt = synth.make_prompt(batch, prompt_len, shape.vocab, seed=seeds.prompt).cuda()
     ws = dg.Workspace()
@@ -558,9 +571,11 @@ def main():
     steps_seen = []
 
     def block_step():
+        # the generation of `blocks` canvases after the prompt
         st.cache_len.fill_(prompt_len)
         st.cache_len_host = prompt_len
-        steps_seen.append(dg.denoise_block(model, st, settings, seed, 0, ws=ws))
+        for blk in range(blocks):
+            steps_seen.append(dg.denoise_block(model, st, settings, seed, blk, ws=ws))
 
     for _ in range(args.warmup):
         block_step()
@@ -581,7 +596,7 @@ def main():
     elapsed = replicas.max_over_ranks(elapsed, world)
     replicas.barrier(world)
     dg.check_device_errors()
-    value = replicas.whole_job_rate(batch * CANVAS * args.steps, world, elapsed)
+    value = replicas.whole_job_rate(batch * CANVAS * blocks * args.steps, world, elapsed)
 
     # ---------------------------------------------------------------- end to end
     host_prompt = synth.make_prompt(batch, prompt_len, shape.vocab, seed=seeds.prompt).pin_memory()
@@ -591,14 +606,16 @@ def main():
     def e2e_step():
         dev_prompt.copy_(host_prompt, non_blocking=True)
         dg.prefill(model, st, dev_prompt, ws=ws)
-        dg.denoise_block(model, st, settings, seed, 0, ws=ws)
-        host_out.copy_(st.tok, non_blocking=True)
+        for blk in range(blocks):
+            dg.denoise_block(model, st, settings, seed, blk, ws=ws)
+            host_out.copy_(st.tok, non_blocking=True)
 
     e2e_step()
     replicas.barrier(world)
     e2e_t = time_region(e2e_step, max(1, args.steps // 2), stream)
     e2e_t = replicas.max_over_ranks(e2e_t, world)
-    e2e_val = replicas.whole_job_rate(batch * CANVAS * max(1, args.steps // 2), world, e2e_t)
+    e2e_val = replicas.whole_job_rate(batch * CANVAS * blocks * max(1, args.steps // 2), world,
+                                      e2e_t)
 
     # ---------------------------------------------------------------- roofline
     roof = gemm_roofline(dg, model, shape, batch, peaks, stream)
@@ -615,7 +632,7 @@ def main():
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": round(value, 2), "unit": UNIT, "n_gpus": world,
+            "metric": metric_name(batch), "value": round(value, 2), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(elapsed / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
@@ -627,7 +644,7 @@ def main():
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_val, 2), "unit": UNIT,
                     "h2d_bytes_per_step": int(host_prompt.numel() * 4),
-                    "d2h_bytes_per_step": int(host_out.numel() * 4),
+                    "d2h_bytes_per_step": int(host_out.numel() * 4 * blocks),
                     "includes": "prompt H2D + prefill + denoised block + tokens D2H"},
             "gpu_launches": int(launches),
             "clocks": clk,
