@@ -14,6 +14,8 @@ Modules:
   sampler  temperature schedule, per-position statistics, Gumbel-max sample,
            top-k commit, threshold re-noise, adaptive stop.
   loop     the block-autoregressive loop composed from the two.
+  fp8      e4m3 encoding from the format's definition, per-row / per-tensor
+           scaling, and the FP8 unembedding's logits.
 
 Parity status: every function is pinned by a test under tests/ against the
 pages' fixed settings, closed forms, library routines or invariants, except
