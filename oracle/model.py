@@ -31,6 +31,11 @@ Weight layout (nn.Linear convention, [out_features, in_features]):
     w_o     [d, Hq hd]
     w_up    [F, d]          w_down  [d, F]
 
+FP8 unembedding (optional, ``e4m3_unembed=True``; a reading: the pages quote
+FP8 checkpoints but fix no recipe): the final normalised hidden state, stored
+as bfloat16, is quantised to e4m3 per token and the unembedding per tensor
+(oracle.fp8), and the logits are the scaled products of the codes.
+
 Storage rounding: with ``bf16_storage=True`` (default) the oracle rounds to
 bfloat16 at the points where the product stores bfloat16 tensors - the
 normalised GEMM inputs, Q/K/V (hence the KV cache), the attention output and
@@ -41,6 +46,8 @@ from dataclasses import dataclass
 
 import numpy as np
 from scipy.special import erf
+
+from . import fp8
 
 
 @dataclass(frozen=True)
@@ -156,8 +163,17 @@ def layer_forward(cfg, w, x, k_pre, v_pre, causal, bf16_storage=True, skip_tail=
     return x_out, k_new, v_new
 
 
+def unembed_e4m3(hn, w_unembed):
+    """FP8 logits of normalised hidden states hn [Lq, d]: per-token e4m3 codes and
+    scales of hn, one e4m3 scale for the unembedding, products of the decoded
+    codes summed in fp64 and scaled."""
+    hq, hs = fp8.quantize_rows(hn)
+    wq, ws = fp8.quantize_tensor(w_unembed)
+    return fp8.unembed_logits(hq, hs, wq, ws).astype(np.float64)
+
+
 def forward(cfg, weights, tokens, k_cache, v_cache, prefix_len, causal,
-            bf16_storage=True, want_logits=True):
+            bf16_storage=True, want_logits=True, e4m3_unembed=False):
     """Run the stack over new rows of one sequence.
 
     tokens [Lq] int; k_cache/v_cache: per layer [Hkv, >=prefix_len, hd] arrays.
@@ -176,6 +192,8 @@ def forward(cfg, weights, tokens, k_cache, v_cache, prefix_len, causal,
     if not want_logits:
         return None, kv
     hn = _r(rmsnorm(x, cfg.eps), bf16_storage)
+    if e4m3_unembed:
+        return unembed_e4m3(hn, weights["unembed"]), kv
     logits = hn @ weights["unembed"].T
     return logits, kv
 
@@ -203,10 +221,11 @@ def prefill(cfg, weights, prompt, k_cache, v_cache, bf16_storage=True):
     return commit_kv(k_cache, v_cache, kv, 0)
 
 
-def denoise_logits(cfg, weights, canvas, k_cache, v_cache, prefix_len, bf16_storage=True):
+def denoise_logits(cfg, weights, canvas, k_cache, v_cache, prefix_len, bf16_storage=True,
+                   e4m3_unembed=False):
     """Bidirectional pass of the canvas over the cached prefix -> logits [C, V]."""
     logits, _ = forward(cfg, weights, canvas, k_cache, v_cache, prefix_len, causal=False,
-                        bf16_storage=bf16_storage, want_logits=True)
+                        bf16_storage=bf16_storage, want_logits=True, e4m3_unembed=e4m3_unembed)
     return logits
 
 

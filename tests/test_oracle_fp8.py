@@ -65,3 +65,41 @@ def test_unembed_logits_equal_the_dequantised_product():
     assert np.allclose(got, want, rtol=1e-6, atol=1e-7)
     # and close to the unquantised product (3 mantissa bits on each side)
     assert np.linalg.norm(got - h @ w.T) <= 0.08 * np.linalg.norm(h @ w.T)
+
+
+def test_unembed_e4m3_one_hot_hidden_state():
+    """hn = c e_j: its codes are 448 at j (scale c/448), so logit v is exactly c times
+    the e4m3-rounded w[v, j] (the weight's own scale times its decoded code)."""
+    from oracle import model as M
+    rng = np.random.default_rng(3)
+    w = rng.normal(scale=0.05, size=(64, 32))
+    c, j = 1.5, 7
+    hn = np.zeros((1, 32))
+    hn[0, j] = c
+    wq, ws = fp8.quantize_tensor(w)
+    q_w = np.float64(ws) * fp8.decode(wq)
+    got = M.unembed_e4m3(hn, w)
+    np.testing.assert_array_equal(got[0], (c * q_w[:, j]).astype(np.float32))
+    # a transposed or mis-scaled operand breaks it
+    assert not np.allclose(got[0], c * w[:, j] * 2)
+
+
+def test_unembed_e4m3_within_the_format_error_bound():
+    """Each e4m3 operand of a normal-range value carries a relative error of at most
+    2^-4 (half a step of a 3-bit mantissa); below 2^-6 scale units the error is at
+    most 2^-10 absolute.  So |fp8 - exact| <= sum_k (2^-4 + 2^-4 + 2^-8) |h_k w_k| plus
+    the subnormal slack, and the error is not zero (the path does quantise)."""
+    from oracle import model as M
+    rng = np.random.default_rng(4)
+    h = rng.normal(size=(16, 128))
+    w = rng.normal(scale=0.02, size=(96, 128))
+    got = M.unembed_e4m3(h, w)
+    exact = h @ w.T
+    hs = np.abs(h).max(axis=1) / 448.0
+    ws = np.abs(w).max() / 448.0
+    rel = 2.0 ** -4 * 2 + 2.0 ** -8
+    sub = 2.0 ** -10 * (hs[:, None] * (np.abs(w).sum(axis=1)[None, :])
+                        + ws * np.abs(h).sum(axis=1)[:, None])
+    bound = rel * (np.abs(h) @ np.abs(w).T) + sub + 1e-6 * np.abs(exact)
+    assert np.all(np.abs(got - exact) <= bound)
+    assert np.abs(got - exact).max() > 0
