@@ -114,7 +114,7 @@ def dist_env():
 def workload_config(name, world, steps_per_block=None):
     """The `config` object of both arms' JSON lines."""
     shape, batch, prompt = workload_spec(name)
-    return {"workload": name, "model": "random-init dense stand-in", "batch": batch,
+    return {"workload": name, "weights": "random-init dense stand-in", "batch": batch,
             "prompt": prompt, "canvas": CANVAS, "d": shape.d, "layers": shape.n_layers,
             "heads": [shape.n_q_heads, shape.n_kv_heads], "head_dim": shape.head_dim,
             "ffn": shape.ffn, "vocab": shape.vocab, "steps_per_block": steps_per_block,
@@ -247,16 +247,31 @@ def sampler_step_roofline(dg, model, shape, batch, peaks, stream):
     ws = dg.Workspace()
     settings = dg.SamplerSettings()
 
-    def step():
-        stat.zero_()
-        dg.unembed_sample_commit(h, model.w["unembed"], tok, com, prev, stat, settings, 0, 0, 5,
-                                 ws=ws, stream=stream)
+    if model.unembed_q is not None:
+        # e4m3 operands: the per-token quantisation of h is part of the step
+        hq = torch.empty((M, d), dtype=torch.uint8, device="cuda")
+        hs = torch.empty(M, dtype=torch.float32, device="cuda")
+
+        def step():
+            stat.zero_()
+            dg.quantize_e4m3(h, hq, hs, per_row=True, stream=stream)
+            dg.unembed_sample_commit_e4m3(hq, hs, model.unembed_q, model.unembed_scale, tok, com,
+                                          prev, stat, settings, 0, 0, 5, ws=ws, stream=stream)
+        # the recipe's nominal fp8 : bf16 dense ratio (4.5 : 2.25) times the measured bf16 peak
+        peak, wbytes, kname = 2.0 * peaks["bf16_tflops"], V * d, "quantize + e4m3 fused step"
+    else:
+        def step():
+            stat.zero_()
+            dg.unembed_sample_commit(h, model.w["unembed"], tok, com, prev, stat, settings, 0,
+                                     0, 5, ws=ws, stream=stream)
+        peak, wbytes, kname = peaks["bf16_tflops"], V * d * 2, \
+            "unembed_sample_kernel + merge + commit"
     t = timed_alone(step, stream)
     flops = 2.0 * M * V * d
-    return {"kernel": "unembed_sample_kernel + merge + commit", "shape": [M, V, d],
-            "achieved": round(flops / t / 1e12, 1), "peak": peaks["bf16_tflops"],
-            "unit": "TFLOP/s", "frac": round(flops / t / 1e12 / peaks["bf16_tflops"], 4),
-            "hbm_frac": round(V * d * 2 / t / 1e9 / peaks["hbm_gbs"], 4),
+    return {"kernel": kname, "shape": [M, V, d],
+            "achieved": round(flops / t / 1e12, 1), "peak": round(peak, 1),
+            "unit": "TFLOP/s", "frac": round(flops / t / 1e12 / peak, 4),
+            "hbm_frac": round(wbytes / t / 1e9 / peaks["hbm_gbs"], 4),
             "us": round(t * 1e6, 1)}
 
 
@@ -475,15 +490,35 @@ def run_kernel_bench(args):
             dg.unembed(h, w, lg.view(M, V))
             dg.sample_commit(lg, tok, com, prev, stat, settings, 0, 0, 5, ws=ws)
 
+        hq = torch.empty((M, d), dtype=torch.uint8, device="cuda")
+        hs = torch.empty(M, dtype=torch.float32, device="cuda")
+        wq = torch.empty((V, d), dtype=torch.uint8, device="cuda")
+        wsc = torch.empty(1, dtype=torch.float32, device="cuda")
+        dg.quantize_e4m3(w, wq, wsc, per_row=False)
+
+        def quant():
+            dg.quantize_e4m3(h, hq, hs, per_row=True)
+
+        def fused_e4m3():
+            stat.zero_()
+            dg.unembed_sample_commit_e4m3(hq, hs, wq, wsc, tok, com, prev, stat, settings, 0, 0,
+                                          5, ws=ws)
+
         fl = 2.0 * M * V * d
-        for name, fn in (("unembed_sample_commit (fused)", fused),
-                         ("unembed + sample_commit", unfused)):
+        for name, fn, wbytes, peak in (
+                ("unembed_sample_commit (fused)", fused, V * d * 2, peaks["bf16_tflops"]),
+                ("unembed + sample_commit", unfused, V * d * 2, peaks["bf16_tflops"]),
+                ("unembed_sample_commit_e4m3 (fused)", fused_e4m3, V * d,
+                 2.0 * peaks["bf16_tflops"]),
+                ("quantize_e4m3 per token", quant, M * d * 3, None)):
             t = timed(fn, args.steps)
-            out.append({"kernel": name, "shape": [M, V, d], "us": round(t * 1e6, 2),
-                        "tflops": round(fl / t / 1e12, 1),
-                        "frac_bf16_peak": round(fl / t / 1e12 / peaks["bf16_tflops"], 4),
-                        "weight_gbs": round(V * d * 2 / t / 1e9, 1),
-                        "frac_hbm_peak": round(V * d * 2 / t / 1e9 / peaks["hbm_gbs"], 4)})
+            row = {"kernel": name, "shape": [M, V, d], "us": round(t * 1e6, 2),
+                   "weight_gbs": round(wbytes / t / 1e9, 1),
+                   "frac_hbm_peak": round(wbytes / t / 1e9 / peaks["hbm_gbs"], 4)}
+            if peak:
+                row.update(tflops=round(fl / t / 1e12, 1),
+                           frac_tensor_peak=round(fl / t / 1e12 / peak, 4))
+            out.append(row)
     elif args.kernel == "gemm":
         M, N, K = (int(x) for x in args.shape.split(","))
         x = torch.randn((M, K), device="cuda").to(torch.bfloat16)
@@ -525,6 +560,8 @@ def main():
     ap.add_argument("--epi", default="bf16", choices=["bf16", "gelu", "f32", "resid"],
                     help="epilogue for --kernel gemm")
     ap.add_argument("--heads", default="32,8", help="query,kv heads for --kernel attn")
+    ap.add_argument("--fp8-unembed", action="store_true",
+                    help="run the unembedding + sampler step on e4m3 operands")
     args = ap.parse_args()
     if args.kernel:
         return run_kernel_bench(args)
@@ -555,7 +592,7 @@ def main():
                    "layers": [{k: v.cuda() for k, v in lw.items()} for lw in w_cpu["layers"]]}
     else:
         weights = synth.make_weights_fast(shape, seed=0, device="cuda")
-    model = dg.DgModel(shape, weights)
+    model = dg.DgModel(shape, weights, fp8_unembed=args.fp8_unembed)
     blocks = workload_blocks(args.workload)
     lmax = prompt_len + CANVAS * blocks
     st = dg.DgState(shape, batch, lmax, CANVAS)
@@ -635,9 +672,11 @@ def main():
             "metric": metric_name(batch), "value": round(value, 2), "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(elapsed / args.steps * 1e3, 3), "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": workload_config(args.workload, world,
-                                      steps_seen[-1] if steps_seen else None),
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16+e4m3-unembed" if args.fp8_unembed else "bf16", "data": "synthetic",
+            "config": dict(workload_config(args.workload, world,
+                                           steps_seen[-1] if steps_seen else None),
+                           unembed="e4m3" if args.fp8_unembed else "bf16"),
             "roofline": roof,
             "canvas_attn": attn,
             "unembed_sample": samp,

@@ -7,6 +7,7 @@ CUDA device, and raises otherwise.
 
 Functions take torch tensors and pass their device pointers:
     canvas_attn, unembed, linear, sample_commit, unembed_sample_commit, kv_block_commit,
+    quantize_e4m3, unembed_e4m3, unembed_sample_commit_e4m3,
     philox
 Objects:
     DgModel   weights + configuration (dg_model)
@@ -22,6 +23,7 @@ from ._lib import (EPI_BF16, EPI_F32, EPI_GELU_BF16, EPI_RESID_F32, MASK_BIDIR, 
                    UNSELECTED_KEEP, UNSELECTED_RENOISE, DgError)
 
 __all__ = ["canvas_attn", "unembed", "linear", "sample_commit", "unembed_sample_commit",
+           "quantize_e4m3", "unembed_e4m3", "unembed_sample_commit_e4m3",
            "kv_block_commit", "philox",
            "DgModel", "DgState", "SamplerSettings", "prefill", "denoise_logits", "denoise_block",
            "check_device_errors", "Workspace", "DgError", "MASK_BIDIR", "MASK_CAUSAL",
@@ -196,6 +198,42 @@ def unembed_sample_commit(h, w_u, tok, committed, prev_argmax, seq_status, setti
         ctypes.byref(so) if so is not None else None, wp, wn, _stream(stream)))
 
 
+def quantize_e4m3(x, out, scales, per_row=True, stream=None):
+    """bf16 x[R, C] -> e4m3 codes out[R, C] (uint8) and fp32 scales ([R] per row, else [1])."""
+    _need_contig(x, out, scales)
+    R, C = x.shape
+    _lib.check(_lib.load().dg_quantize_e4m3(_ptr(x), R, C, 1 if per_row else 0, _ptr(out),
+                                            _ptr(scales), _stream(stream)))
+
+
+def unembed_e4m3(h_q, h_scale, w_q, w_scale, logits, stream=None):
+    """logits[M, V] = h_scale[m] w_scale (h_q[M, d] . w_q[V, d]) on e4m3 codes."""
+    _need_contig(h_q, h_scale, w_q, w_scale, logits)
+    M, d = h_q.shape
+    V = w_q.shape[0]
+    _lib.check(_lib.load().dg_unembed_e4m3(_ptr(h_q), _ptr(h_scale), _ptr(w_q), _ptr(w_scale),
+                                           _ptr(logits), M, d, V, _stream(stream)))
+
+
+def unembed_sample_commit_e4m3(h_q, h_scale, w_q, w_scale, tok, committed, prev_argmax,
+                               seq_status, settings, seed, block, step, out=None, ws=None,
+                               stream=None):
+    """unembed_sample_commit with the logits of unembed_e4m3."""
+    _need_contig(h_q, h_scale, w_q, w_scale, tok, committed, prev_argmax, seq_status)
+    lib = _lib.load()
+    B, C = tok.shape
+    V, d = w_q.shape
+    so = None
+    if out is not None:
+        so = _lib.StepOut(*[(out[k].data_ptr() if out.get(k) is not None else None)
+                            for k in ("x_hat", "argmax", "logconf", "entropy", "flags")])
+    wp, wn = _ws(ws).args(lib.dg_unembed_sample_commit_workspace_bytes(B, C, V))
+    _lib.check(lib.dg_unembed_sample_commit_e4m3(
+        _ptr(h_q), _ptr(h_scale), _ptr(w_q), _ptr(w_scale), d, _ptr(tok), _ptr(committed),
+        _ptr(prev_argmax), _ptr(seq_status), ctypes.byref(settings.c), seed, block, step, B, C,
+        V, ctypes.byref(so) if so is not None else None, wp, wn, _stream(stream)))
+
+
 def kv_block_commit(k_blk, v_blk, k_cache, v_cache, cache_len, *, n_kv_heads, head_dim,
                     stream=None):
     """Append per-layer block K/V ([B, C, ld] views) to the caches; cache_len += C."""
@@ -220,9 +258,13 @@ def philox(inp, out, stream=None):
 
 
 class DgModel:
-    """Model weights (bf16 device tensors, [out, in]) and their dg_model view."""
+    """Model weights (bf16 device tensors, [out, in]) and their dg_model view.
 
-    def __init__(self, shape, weights):
+    fp8_unembed=True also keeps an e4m3 copy of the unembedding (one tensor
+    scale), which the denoising loop's unembedding + sampler step then uses.
+    """
+
+    def __init__(self, shape, weights, fp8_unembed=False):
         self.shape = shape
         self.w = weights
         n = shape.n_layers
@@ -232,8 +274,16 @@ class DgModel:
                                                 lw["w_up"].data_ptr(), lw["w_down"].data_ptr())
         self.cfg = _lib.ModelCfg(shape.d, shape.n_layers, shape.n_q_heads, shape.n_kv_heads,
                                  shape.head_dim, shape.ffn, shape.vocab, shape.eps)
+        self.unembed_q = self.unembed_scale = None
+        if fp8_unembed:
+            wu = weights["unembed"]
+            self.unembed_q = torch.empty(wu.shape, dtype=torch.uint8, device=wu.device)
+            self.unembed_scale = torch.empty(1, dtype=torch.float32, device=wu.device)
+            quantize_e4m3(wu, self.unembed_q, self.unembed_scale, per_row=False)
         self.c = _lib.Model(self.cfg, weights["embed"].data_ptr(), weights["unembed"].data_ptr(),
-                            ctypes.cast(self._layers, ctypes.POINTER(_lib.LayerWeights)))
+                            ctypes.cast(self._layers, ctypes.POINTER(_lib.LayerWeights)),
+                            self.unembed_q.data_ptr() if fp8_unembed else None,
+                            self.unembed_scale.data_ptr() if fp8_unembed else None)
 
 
 class DgState:

@@ -40,7 +40,8 @@ class LayerWeights(ctypes.Structure):
 
 class Model(ctypes.Structure):
     _fields_ = [("cfg", ModelCfg), ("embed", c_void_p), ("unembed", c_void_p),
-                ("layers", P(LayerWeights))]
+                ("layers", P(LayerWeights)), ("unembed_e4m3", c_void_p),
+                ("unembed_scale", c_void_p)]
 
 
 class SamplerCfg(ctypes.Structure):
@@ -88,6 +89,14 @@ SIGNATURES = {
                                          c_int, c_int, P(StepOut), c_void_p, c_size_t,
                                          c_void_p]),
     "dg_unembed_sample_commit_workspace_bytes": (c_size_t, [c_int, c_int, c_int]),
+    "dg_quantize_e4m3": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]),
+    "dg_unembed_e4m3": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int,
+                                c_int, c_void_p]),
+    "dg_unembed_sample_commit_e4m3": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int,
+                                              c_void_p, c_void_p, c_void_p, c_void_p,
+                                              P(SamplerCfg), c_uint32, c_int, c_int, c_int,
+                                              c_int, c_int, P(StepOut), c_void_p, c_size_t,
+                                              c_void_p]),
     "dg_sample_commit_noalloc": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                          P(SamplerCfg), c_uint32, c_int, c_int, c_int, c_int,
                                          c_int, P(StepOut), c_void_p]),

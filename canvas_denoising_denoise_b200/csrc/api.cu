@@ -21,6 +21,7 @@
 #include "dg_common.cuh"
 #include "gemm.cuh"
 #include "kvcommit.cuh"
+#include "quant.cuh"
 #include "unembed.cuh"
 #include "sampler.cuh"
 
@@ -149,6 +150,33 @@ int make_tmap(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
   return DG_OK;
 }
 
+// The same for 8-bit elements: box {128, box_rows} (one 128-byte line per row).
+int make_tmap_u8(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows,
+                 uint64_t row_stride_bytes, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  if (!aligned16(base) || (row_stride_bytes & 15u))
+    return fail(DG_ERR_ALIGNMENT, "tensor map base %p / stride %llu not 16-byte aligned", base,
+                (unsigned long long)row_stride_bytes);
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {row_stride_bytes};
+  cuuint32_t box[2] = {128, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(DG_ERR_CUDA, "cuTensorMapEncodeTiled (u8) failed (%d) inner=%llu rows=%llu",
+                (int)r, (unsigned long long)inner, (unsigned long long)rows);
+  return DG_OK;
+}
+
+// Dequantisation scales of e4m3 unembedding operands (null: bf16 operands).
+struct Fp8Scales {
+  const float* tok;  // [M] per-token scale of the activations
+  const float* w;    // the weight tensor's scale (device scalar)
+};
+
 // ---------------------------------------------------------------------------
 // GEMM
 // ---------------------------------------------------------------------------
@@ -269,9 +297,10 @@ int linear(const void* x, const void* w, int M, int N, int K, const GemmEpi& e,
 bool unembed_attr_done = false;
 
 int launch_unembed(const void* h, const void* w_u, float* logits, int M, int d, int V,
-                   const float* ssq_in, int n_ssq_in, float inv_k, float eps, cudaStream_t s) {
+                   const float* ssq_in, int n_ssq_in, float inv_k, float eps, cudaStream_t s,
+                   const Fp8Scales* f8 = nullptr) {
   namespace ue = dg::unembed;
-  if (V % ue::TILE != 0) {
+  if (f8 == nullptr && V % ue::TILE != 0) {
     GemmEpi e;
     e.epi = dg::gemm::EPI_F32;
     e.out_f32 = logits;
@@ -279,13 +308,20 @@ int launch_unembed(const void* h, const void* w_u, float* logits, int M, int d, 
     return launch_gemm(h, w_u, M, V, d, GemmPlan{1, d / dg::gemm::BK, 256}, e, s);
   }
   if (!unembed_attr_done) {
-    DG_CUDA(cudaFuncSetAttribute(ue::unembed_pair_kernel<1>,
+    DG_CUDA(cudaFuncSetAttribute(ue::unembed_pair_kernel<1, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, ue::SMEM_BYTES));
+    DG_CUDA(cudaFuncSetAttribute(ue::unembed_pair_kernel<1, true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, ue::SMEM_BYTES));
     unembed_attr_done = true;
   }
   CUtensorMap tw, tx;
-  DG_TRY(make_tmap(&tw, w_u, d, V, (uint64_t)d * 2, ue::HALF));
-  DG_TRY(make_tmap(&tx, h, d, M, (uint64_t)d * 2, ue::HALF));
+  if (f8) {
+    DG_TRY(make_tmap_u8(&tw, w_u, d, V, (uint64_t)d, ue::HALF));
+    DG_TRY(make_tmap_u8(&tx, h, d, M, (uint64_t)d, ue::HALF));
+  } else {
+    DG_TRY(make_tmap(&tw, w_u, d, V, (uint64_t)d * 2, ue::HALF));
+    DG_TRY(make_tmap(&tx, h, d, M, (uint64_t)d * 2, ue::HALF));
+  }
   ue::Params p;
   p.M = M; p.N = V; p.K = d;
   p.n_ttiles = cdiv(M, ue::TILE);
@@ -293,9 +329,12 @@ int launch_unembed(const void* h, const void* w_u, float* logits, int M, int d, 
   p.n_pairs = std::min(kNumSMs / 2, p.n_tiles);
   p.logits = logits;
   p.ssq_in = ssq_in; p.n_ssq_in = n_ssq_in; p.inv_k = inv_k; p.eps = eps;
+  p.tok_scale = f8 ? f8->tok : nullptr;
+  p.w_scale = f8 ? f8->w : nullptr;
   // one k-block per stage: with the logits written this launch is bound by
   // HBM, and deeper single-block stages measured marginally faster
-  DG_CUDA(launch_cluster(ue::unembed_pair_kernel<1>, dim3(2 * p.n_pairs),
+  DG_CUDA(launch_cluster(f8 ? ue::unembed_pair_kernel<1, true> : ue::unembed_pair_kernel<1, false>,
+                         dim3(2 * p.n_pairs),
                          dim3(ue::threads_for(ue::STORE_EPI_WARPS)),
                          ue::SMEM_BYTES, s, dim3(2, 1, 1), tw, tx, p));
   count_launch();
@@ -501,14 +540,18 @@ int launch_unembed_sample(const void* h, const void* w_u, int d, const float* ss
                           int n_ssq_in, float inv_k, float eps, int32_t* tok,
                           uint8_t* committed, int32_t* prev_argmax, int32_t* seq_status,
                           const dg::SampleParams& sp, const dg_step_out* out, void* ws,
-                          cudaStream_t s) {
+                          cudaStream_t s, const Fp8Scales* f8 = nullptr) {
   namespace ue = dg::unembed;
   const int M = sp.B * sp.C, V = sp.V;
   const FusedPlan f = plan_fused(M, V);
   if (!fused_attr_done) {
-    DG_CUDA(cudaFuncSetAttribute(ue::unembed_sample_kernel<1>,
+    DG_CUDA(cudaFuncSetAttribute(ue::unembed_sample_kernel<1, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, ue::SMEM_BYTES));
-    DG_CUDA(cudaFuncSetAttribute(ue::unembed_sample_kernel<2>,
+    DG_CUDA(cudaFuncSetAttribute(ue::unembed_sample_kernel<2, false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, ue::SMEM_BYTES));
+    DG_CUDA(cudaFuncSetAttribute(ue::unembed_sample_kernel<1, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, ue::SMEM_BYTES));
+    DG_CUDA(cudaFuncSetAttribute(ue::unembed_sample_kernel<2, true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, ue::SMEM_BYTES));
     fused_attr_done = true;
   }
@@ -516,22 +559,32 @@ int launch_unembed_sample(const void* h, const void* w_u, int d, const float* ss
   dg::RowStats* stats = (dg::RowStats*)((char*)ws + align_up((size_t)M * f.nparts *
                                                              sizeof(dg::FusedPartial), 256));
   CUtensorMap tx, tw;
-  DG_TRY(make_tmap(&tx, h, d, M, (uint64_t)d * 2, ue::HALF));
-  DG_TRY(make_tmap(&tw, w_u, d, V, (uint64_t)d * 2, ue::HALF));
+  if (f8) {
+    DG_TRY(make_tmap_u8(&tx, h, d, M, (uint64_t)d, ue::HALF));
+    DG_TRY(make_tmap_u8(&tw, w_u, d, V, (uint64_t)d, ue::HALF));
+  } else {
+    DG_TRY(make_tmap(&tx, h, d, M, (uint64_t)d * 2, ue::HALF));
+    DG_TRY(make_tmap(&tw, w_u, d, V, (uint64_t)d * 2, ue::HALF));
+  }
   ue::SampleFusedParams p;
   p.M = M; p.N = V; p.K = d;
   p.n_vtiles = V / ue::TILE;
   p.segs = f.segs;
   p.n_pairs = f.n_pairs;
   p.ssq_in = ssq_in; p.n_ssq_in = n_ssq_in; p.inv_k = inv_k; p.eps = eps;
+  p.tok_scale = f8 ? f8->tok : nullptr;
+  p.w_scale = f8 ? f8->w : nullptr;
   p.sp = sp;
   p.tok = tok;
   p.part = part;
   // two k-blocks per stage (256 contiguous bytes of each weight row per
   // request: 4% faster than one) when the width allows
-  DG_CUDA(launch_cluster((d / 64) % 2 == 0 ? ue::unembed_sample_kernel<2>
-                                            : ue::unembed_sample_kernel<1>,
-                         dim3(2 * f.n_pairs),
+  const int nkb = f8 ? d / 128 : d / 64;  // 128-byte k-blocks per row
+  auto* kern = f8 ? (nkb % 2 == 0 ? ue::unembed_sample_kernel<2, true>
+                                  : ue::unembed_sample_kernel<1, true>)
+                  : (nkb % 2 == 0 ? ue::unembed_sample_kernel<2, false>
+                                  : ue::unembed_sample_kernel<1, false>);
+  DG_CUDA(launch_cluster(kern, dim3(2 * f.n_pairs),
                          dim3(ue::threads_for(ue::SAMPLE_EPI_WARPS)), ue::SMEM_BYTES, s,
                          dim3(2, 1, 1), tx, tw, p));
   count_launch();
@@ -591,6 +644,11 @@ int check_model(const dg_model* m) {
                 "d, ffn, vocab, Hq*hd and (Hq+2Hkv)*hd must be multiples of 128");
   if (!aligned16(m->embed) || !aligned16(m->unembed))
     return fail(DG_ERR_ALIGNMENT, "model: embed/unembed not 16-byte aligned");
+  if ((m->unembed_e4m3 != nullptr) != (m->unembed_scale != nullptr))
+    return fail(DG_ERR_INVALID_ARG, "model: unembed_e4m3 and unembed_scale go together");
+  if (m->unembed_e4m3 && (!aligned16(m->unembed_e4m3) || c.vocab % dg::unembed::TILE))
+    return fail(DG_ERR_UNSUPPORTED_SHAPE,
+                "model: the e4m3 unembedding needs vocab %% 256 == 0 and 16-byte alignment");
   for (int l = 0; l < c.n_layers; ++l) {
     const dg_layer_weights& w = m->layers[l];
     if (!w.w_qkv || !w.w_o || !w.w_up || !w.w_down)
@@ -620,7 +678,7 @@ int check_state(const dg_state* st, const dg_model_cfg& c, bool need_canvas) {
 
 // Workspace carve-up for a forward over M = B * Lq rows.
 struct FwdLayout {
-  size_t x, xn, qkv, ao, up, ssq_x, ssq_h, attn, logits, spart, flag, total;
+  size_t x, xn, qkv, ao, up, ssq_x, ssq_h, attn, logits, spart, flag, hq, hs, total;
 };
 
 FwdLayout fwd_layout(const dg_model_cfg& c, int B, int Lq, int max_prefix, bool logits) {
@@ -648,6 +706,8 @@ FwdLayout fwd_layout(const dg_model_cfg& c, int B, int Lq, int max_prefix, bool 
                                         ? fused_ws_bytes(B, Lq, c.vocab) : (size_t)0)
                          : 0);
   L.flag = take(logits ? 16 : 0);
+  L.hq = take(logits ? (size_t)M * c.d : 0);        // e4m3 hidden states (FP8 unembedding)
+  L.hs = take(logits ? (size_t)M * sizeof(float) : 0);
   L.total = off;
   return L;
 }
@@ -664,6 +724,16 @@ struct Fwd {
   FwdLayout L;
   bool unembed_elsewhere = false;  // the caller fuses the unembedding into its sampler step
 };
+
+// The last layer's bf16 residual stream quantised per token to e4m3 codes
+// (L.hq) and scales (L.hs); the final RMSNorm stays a row scale of the logits.
+int quantize_hidden(const Fwd& f, cudaStream_t s) {
+  DG_CUDA(launch_ex(dg::quant::quantize_rows_kernel, dim3(f.B * f.Lq), dim3(dg::quant::THREADS),
+                    0, s, 1, (const __nv_bfloat16*)(f.ws + f.L.xn), f.m->cfg.d,
+                    (uint8_t*)(f.ws + f.L.hq), (float*)(f.ws + f.L.hs)));
+  count_launch();
+  return DG_OK;
+}
 
 int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s) {
   const dg_model_cfg& c = f.m->cfg;
@@ -718,9 +788,16 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
     DG_TRY(linear(up, w.w_down, M, c.d, c.ffn, ed, s));
   }
   if (f.want_logits && !f.unembed_elsewhere) {
-    // logits of RMSNorm(x)
-    DG_TRY(launch_unembed(xb, f.m->unembed, logits, M, c.d, c.vocab, ssq_x, nt, 1.f / c.d, c.eps,
-                          s));
+    // logits of RMSNorm(x), on e4m3 operands when the model carries them
+    if (f.m->unembed_e4m3) {
+      DG_TRY(quantize_hidden(f, s));
+      const Fp8Scales f8{(const float*)(f.ws + f.L.hs), f.m->unembed_scale};
+      DG_TRY(launch_unembed(f.ws + f.L.hq, f.m->unembed_e4m3, logits, M, c.d, c.vocab, ssq_x, nt,
+                            1.f / c.d, c.eps, s, &f8));
+    } else {
+      DG_TRY(launch_unembed(xb, f.m->unembed, logits, M, c.d, c.vocab, ssq_x, nt, 1.f / c.d,
+                            c.eps, s));
+    }
   }
   return DG_OK;
 }
@@ -951,6 +1028,75 @@ int dg_unembed_sample_commit(const void* h, const void* w_u, int d, int32_t* tok
                                seq_status, p, out, workspace, (cudaStream_t)stream);
 }
 
+int dg_quantize_e4m3(const void* in, int rows, int cols, int per_row, uint8_t* out,
+                     float* scales, void* stream) {
+  if (!in || !out || !scales) return fail(DG_ERR_INVALID_ARG, "dg_quantize_e4m3: null pointer");
+  if (rows <= 0 || cols <= 0 || cols % 8)
+    return fail(DG_ERR_UNSUPPORTED_SHAPE, "dg_quantize_e4m3: need cols %% 8 == 0");
+  if (!aligned16(in) || !aligned16(out))
+    return fail(DG_ERR_ALIGNMENT, "dg_quantize_e4m3: pointers must be 16-byte aligned");
+  cudaStream_t s = (cudaStream_t)stream;
+  namespace qt = dg::quant;
+  if (per_row) {
+    DG_CUDA(launch_ex(qt::quantize_rows_kernel, dim3(rows), dim3(qt::THREADS), 0, s, 1,
+                      (const __nv_bfloat16*)in, cols, out, scales));
+    count_launch();
+    return DG_OK;
+  }
+  const size_t n = (size_t)rows * cols;
+  const int blocks = (int)std::min<size_t>(4 * kNumSMs, (n / 8 + qt::THREADS - 1) / qt::THREADS);
+  DG_CUDA(cudaMemsetAsync(scales, 0, sizeof(float), s));
+  qt::absmax_kernel<<<blocks, qt::THREADS, 0, s>>>((const __nv_bfloat16*)in, n,
+                                                   (unsigned int*)scales);
+  qt::quantize_tensor_kernel<<<blocks, qt::THREADS, 0, s>>>(
+      (const __nv_bfloat16*)in, n, out, (const unsigned int*)scales);
+  qt::amax_to_scale_kernel<<<1, 1, 0, s>>>((unsigned int*)scales);
+  count_launch(3);
+  DG_CUDA(cudaGetLastError());
+  return DG_OK;
+}
+
+int dg_unembed_e4m3(const uint8_t* h_q, const float* h_scale, const uint8_t* w_q,
+                    const float* w_scale, float* logits, int M, int d, int V, void* stream) {
+  if (!h_q || !h_scale || !w_q || !w_scale || !logits)
+    return fail(DG_ERR_INVALID_ARG, "dg_unembed_e4m3: null pointer");
+  if (M <= 0 || d <= 0 || V <= 0 || V % dg::unembed::TILE || d % 128)
+    return fail(DG_ERR_UNSUPPORTED_SHAPE, "dg_unembed_e4m3: need V %% 256 == 0, d %% 128 == 0");
+  if (!aligned16(h_q) || !aligned16(w_q) || !aligned16(logits))
+    return fail(DG_ERR_ALIGNMENT, "dg_unembed_e4m3: pointers must be 16-byte aligned");
+  const Fp8Scales f8{h_scale, w_scale};
+  return launch_unembed(h_q, w_q, logits, M, d, V, nullptr, 0, 0.f, 0.f, (cudaStream_t)stream,
+                        &f8);
+}
+
+int dg_unembed_sample_commit_e4m3(const uint8_t* h_q, const float* h_scale, const uint8_t* w_q,
+                                  const float* w_scale, int d, int32_t* tok, uint8_t* committed,
+                                  int32_t* prev_argmax, int32_t* seq_status,
+                                  const dg_sampler_cfg* cfg, uint32_t seed, int block, int step,
+                                  int B, int C, int V, const dg_step_out* out, void* workspace,
+                                  size_t workspace_bytes, void* stream) {
+  if (!h_q || !h_scale || !w_q || !w_scale || !tok || !committed || !prev_argmax ||
+      !seq_status || !cfg)
+    return fail(DG_ERR_INVALID_ARG, "dg_unembed_sample_commit_e4m3: null pointer");
+  if (B <= 0 || C <= 0 || C > 1024 || V <= 0 || V % dg::unembed::TILE || d <= 0 || d % 128 ||
+      step < 0 || block < 0)
+    return fail(DG_ERR_UNSUPPORTED_SHAPE,
+                "dg_unembed_sample_commit_e4m3: need C <= 1024, V %% 256 == 0, d %% 128 == 0");
+  if (!sampler_cfg_ok(*cfg))
+    return fail(DG_ERR_INVALID_ARG, "dg_unembed_sample_commit_e4m3: bad sampler settings");
+  if (!aligned16(h_q) || !aligned16(w_q))
+    return fail(DG_ERR_ALIGNMENT,
+                "dg_unembed_sample_commit_e4m3: pointers must be 16-byte aligned");
+  const size_t need = fused_ws_bytes(B, C, V);
+  if (!workspace || workspace_bytes < need || !aligned16(workspace))
+    return fail(DG_ERR_WORKSPACE_TOO_SMALL,
+                "dg_unembed_sample_commit_e4m3: workspace needs %zu bytes", need);
+  const dg::SampleParams p = make_sample_params(*cfg, seed, block, nullptr, step, B, C, V);
+  const Fp8Scales f8{h_scale, w_scale};
+  return launch_unembed_sample(h_q, w_q, d, nullptr, 0, 0.f, 0.f, tok, committed, prev_argmax,
+                               seq_status, p, out, workspace, (cudaStream_t)stream, &f8);
+}
+
 int dg_sample_commit_noalloc(const float* logits, int32_t* tok, uint8_t* committed,
                              int32_t* prev_argmax, int32_t* seq_status, const dg_sampler_cfg* cfg,
                              uint32_t seed, int block, int step, int B, int C, int V,
@@ -1082,11 +1228,20 @@ int dg_denoise_block(const dg_model* m, dg_state* st, const dg_sampler_cfg* cfg,
   // with a vocabulary of 256-entry tiles the sampler's row pass runs inside
   // the unembedding and the logits never reach memory
   const bool fused = V % dg::unembed::TILE == 0;
+  const bool fp8 = m->unembed_e4m3 != nullptr;  // check_model: vocab % 256 == 0 then
   Fwd fl = f;
   fl.unembed_elsewhere = fused;
   for (int it = 0; it < cfg->max_steps; ++it) {
     DG_TRY(run_forward(fl, st->tok, logits, s));
-    if (fused)
+    if (fused && fp8) {
+      // the hidden states quantised per token, then the e4m3 unembedding + sampler
+      DG_TRY(quantize_hidden(fl, s));
+      const Fp8Scales f8{(const float*)(ws + L.hs), m->unembed_scale};
+      DG_TRY(launch_unembed_sample(ws + L.hq, m->unembed_e4m3, m->cfg.d,
+                                   (const float*)(ws + L.ssq_x), m->cfg.d / 128, 1.f / m->cfg.d,
+                                   m->cfg.eps, st->tok, st->committed, st->prev_argmax,
+                                   st->seq_status, sp, nullptr, ws + L.spart, s, &f8));
+    } else if (fused)
       DG_TRY(launch_unembed_sample(ws + L.xn, m->unembed, m->cfg.d, (const float*)(ws + L.ssq_x),
                                    m->cfg.d / 128, 1.f / m->cfg.d, m->cfg.eps, st->tok,
                                    st->committed, st->prev_argmax, st->seq_status, sp, nullptr,

@@ -338,6 +338,17 @@ __device__ __forceinline__ void umma_ss_pair(uint32_t d_tmem, uint64_t a_desc, u
       : "memory");
 }
 
+// Pair MMA on 8-bit operands (kind::f8f6f4, K = 32 per instruction).
+__device__ __forceinline__ void umma_ss_pair_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive on the mbarrier at `bar`'s offset in every CTA of `cta_mask` once the
 // pair MMAs issued so far by this thread have completed.
 __device__ __forceinline__ void umma_commit_pair(uint64_t* bar, uint16_t cta_mask) {
@@ -401,6 +412,14 @@ __device__ __forceinline__ bool mbar_wait_pair(uint64_t* bar, uint32_t parity,
       }
     }
   }
+}
+
+// Instruction descriptor, kind::f8f6f4 with e4m3 A/B (format code 0), fp32 D,
+// both operands K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4)                                  // D format: f32
+         | (static_cast<uint32_t>(N >> 3) << 17)    // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);   // M / 16
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

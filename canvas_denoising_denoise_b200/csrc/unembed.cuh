@@ -69,15 +69,19 @@ __host__ __device__ constexpr int threads_for(int epi_warps) { return 64 + 32 * 
 // prepare(li) before the tile's accumulator is ready, consume(li, taddr, col0,
 // ncols) once it is, finish() after the last tile.
 // ---------------------------------------------------------------------------
-template <int EPI_WARPS, int KPS, class Sched, class Epi>
+template <int EPI_WARPS, int KPS, bool F8, class Sched, class Epi>
 __device__ __forceinline__ void pair_pipeline(const CUtensorMap* tm_a, const CUtensorMap* tm_b,
                                               uint64_t pol_a, uint64_t pol_b, const Sched& sc,
                                               Epi& epi) {
   // A stage holds KPS consecutive k-blocks (their A tiles, then their B
   // tiles), so each row of a weight tile is requested KPS * 128 contiguous
-  // bytes at a time.  sc.nkb is a multiple of KPS.
+  // bytes at a time.  sc.nkb is a multiple of KPS.  A k-block is one 128-byte
+  // swizzle row per operand row: 64 bf16 or, with F8, 128 e4m3 elements
+  // (kind::f8f6f4, 32 K per MMA instead of 16: the same 32-byte step).
   constexpr int STAGE_BYTES = KPS * (A_BYTES + B_BYTES);
   constexpr int STAGES = RING_BYTES / STAGE_BYTES;
+  constexpr int KB_ELEMS = F8 ? 128 : BK;
+  constexpr uint32_t MMA_IDESC = F8 ? idesc_e4m3_f32(TILE, TILE) : IDESC;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -125,13 +129,13 @@ __device__ __forceinline__ void pair_pipeline(const CUtensorMap* tm_a, const CUt
     const int st = g % STAGES;
     for (int j = 0; j < KPS; ++j)
       tma_load_2d_pair(smem + st * STAGE_BYTES + j * A_BYTES, tm_a, full_even + st * 8,
-                       (KPS * (g % nstg) + j) * BK, sc.a_row(g / nstg) + roff, pol_a);
+                       (KPS * (g % nstg) + j) * KB_ELEMS, sc.a_row(g / nstg) + roff, pol_a);
   };
   auto issue_b = [&](int g) {
     const int st = g % STAGES;
     for (int j = 0; j < KPS; ++j)
       tma_load_2d_pair(smem + st * STAGE_BYTES + KPS * A_BYTES + j * B_BYTES, tm_b,
-                       full_even + st * 8, (KPS * (g % nstg) + j) * BK,
+                       full_even + st * 8, (KPS * (g % nstg) + j) * KB_ELEMS,
                        sc.b_row(g / nstg) + roff, pol_b);
   };
 
@@ -202,10 +206,14 @@ __device__ __forceinline__ void pair_pipeline(const CUtensorMap* tm_a, const CUt
 #pragma unroll
           for (int j = 0; j < KPS; ++j)
 #pragma unroll
-            for (int kk = 0; kk < BK / 16; ++kk)
-              umma_ss_pair(d, sdesc_sw128(a_base + j * A_BYTES + kk * 32, 16, 1024),
-                           sdesc_sw128(b_base + j * B_BYTES + kk * 32, 16, 1024), IDESC,
-                           (q | j | kk) != 0 ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk) {  // four 32-byte K steps per 128-byte row
+              const uint64_t ad = sdesc_sw128(a_base + j * A_BYTES + kk * 32, 16, 1024);
+              const uint64_t bd = sdesc_sw128(b_base + j * B_BYTES + kk * 32, 16, 1024);
+              if constexpr (F8)
+                umma_ss_pair_f8(d, ad, bd, MMA_IDESC, (q | j | kk) != 0 ? 1u : 0u);
+              else
+                umma_ss_pair(d, ad, bd, MMA_IDESC, (q | j | kk) != 0 ? 1u : 0u);
+            }
           umma_commit_pair(&empty[st], 0x3);
         }
         if (ok) umma_commit_pair(&acc_full[b], 0x3);
@@ -265,6 +273,17 @@ __device__ __forceinline__ float row_scale(const float* ssq_in, int n_ssq_in, in
   return rsqrtf(acc * inv_k + eps);
 }
 
+// The dequantisation scales of an e4m3 launch folded into the row scale:
+// per-token scale of the activations (or null) times the weights' tensor scale
+// (device scalar, or null).
+__device__ __forceinline__ float fp8_scale(const float* tok_scale, const float* w_scale, int M,
+                                           int t) {
+  float s = 1.f;
+  if (tok_scale != nullptr && t < M) s = tok_scale[t];
+  if (w_scale != nullptr) s *= *w_scale;
+  return s;
+}
+
 // ---------------------------------------------------------------------------
 // Logits to memory.
 // ---------------------------------------------------------------------------
@@ -277,6 +296,8 @@ struct Params {
   const float* ssq_in;   // [n_ssq_in, M] or null (rs = 1)
   int n_ssq_in;
   float inv_k, eps;
+  const float* tok_scale;  // e4m3 operands: per-token scale [M], else null
+  const float* w_scale;    // e4m3 operands: the weights' scale (device scalar), else null
 };
 
 struct StoreSched {
@@ -299,7 +320,8 @@ struct StoreEpi {
     const int tb = sc->b_row(li);
 #pragma unroll
     for (int c = 0; c < TILE / 32; ++c)
-      rs[c] = row_scale(p->ssq_in, p->n_ssq_in, p->M, tb + c * 32 + lane, p->inv_k, p->eps);
+      rs[c] = row_scale(p->ssq_in, p->n_ssq_in, p->M, tb + c * 32 + lane, p->inv_k, p->eps) *
+              fp8_scale(p->tok_scale, p->w_scale, p->M, tb + c * 32 + lane);
   }
   __device__ void consume(int li, uint32_t taddr, int col0, int ncols) {
     (void)col0;
@@ -323,13 +345,13 @@ struct StoreEpi {
   __device__ void finish() {}
 };
 
-template <int KPS>
+template <int KPS, bool F8>
 __global__ void __launch_bounds__(threads_for(STORE_EPI_WARPS), 1)
     unembed_pair_kernel(const __grid_constant__ CUtensorMap tm_w,
                         const __grid_constant__ CUtensorMap tm_x, Params p) {
   const int pair = static_cast<int>(blockIdx.x >> 1);
   StoreSched sc;
-  sc.nkb = p.K / BK;
+  sc.nkb = p.K / (F8 ? 128 : BK);
   sc.pair = pair;
   sc.n_pairs = p.n_pairs;
   sc.n_ttiles = p.n_ttiles;
@@ -340,7 +362,7 @@ __global__ void __launch_bounds__(threads_for(STORE_EPI_WARPS), 1)
   epi.rank = cluster_ctarank();
   epi.quarter = warp_id() & 3;
   epi.lane = lane_id();
-  pair_pipeline<STORE_EPI_WARPS, KPS>(&tm_w, &tm_x, l2_policy_evict_first(), l2_policy_evict_last(),
+  pair_pipeline<STORE_EPI_WARPS, KPS, F8>(&tm_w, &tm_x, l2_policy_evict_first(), l2_policy_evict_last(),
                                  sc, epi);
 }
 
@@ -361,6 +383,8 @@ struct SampleFusedParams {
   const float* ssq_in;
   int n_ssq_in;
   float inv_k, eps;
+  const float* tok_scale; // e4m3 operands: per-token scale [M], else null
+  const float* w_scale;   // e4m3 operands: the weights' scale (device scalar), else null
   SampleParams sp;        // sampler settings (B, C, V = N, seed, block, step, temperature)
   const int32_t* tok;     // [M] current canvas tokens
   FusedPartial* part;     // [M, SAMPLE_SLOTS * segs]
@@ -400,7 +424,8 @@ struct SampleEpi {
     step = static_cast<uint32_t>(s);
     block = static_cast<uint32_t>(p->sp.block);
     k2 = 1.4426950408889634f / step_temperature(s, p->sp.max_steps, p->sp.t_start, p->sp.t_end);
-    rs = row_scale(p->ssq_in, p->n_ssq_in, p->M, t, p->inv_k, p->eps);
+    rs = row_scale(p->ssq_in, p->n_ssq_in, p->M, t, p->inv_k, p->eps) *
+         fp8_scale(p->tok_scale, p->w_scale, p->M, t);
     c1 = (static_cast<uint32_t>(pos) & 0xFFFFFFu) | (kTagGumbel << 24);
     key = make_uint2(p->sp.seed, static_cast<uint32_t>(b));
     st.reset();
@@ -423,14 +448,14 @@ struct SampleEpi {
   }
 };
 
-template <int KPS>
+template <int KPS, bool F8>
 __global__ void __launch_bounds__(threads_for(SAMPLE_EPI_WARPS), 1)
     unembed_sample_kernel(const __grid_constant__ CUtensorMap tm_x,
                           const __grid_constant__ CUtensorMap tm_w, SampleFusedParams p) {
   const int pair = static_cast<int>(blockIdx.x >> 1);
   const int seg = pair % p.segs;
   SampleSched sc;
-  sc.nkb = p.K / BK;
+  sc.nkb = p.K / (F8 ? 128 : BK);
   sc.tt = pair / p.segs;
   sc.vt0 = static_cast<int>((static_cast<long long>(seg) * p.n_vtiles) / p.segs);
   sc.count = static_cast<int>((static_cast<long long>(seg + 1) * p.n_vtiles) / p.segs) - sc.vt0;
@@ -438,7 +463,7 @@ __global__ void __launch_bounds__(threads_for(SAMPLE_EPI_WARPS), 1)
   epi.p = &p;
   epi.sc = &sc;
   epi.seg = seg;
-  pair_pipeline<SAMPLE_EPI_WARPS, KPS>(&tm_x, &tm_w, l2_policy_evict_last(), l2_policy_evict_first(),
+  pair_pipeline<SAMPLE_EPI_WARPS, KPS, F8>(&tm_x, &tm_w, l2_policy_evict_last(), l2_policy_evict_first(),
                                   sc, epi);
 }
 

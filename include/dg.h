@@ -104,6 +104,12 @@ typedef struct dg_model {
   const void* embed;                /* bf16 [V, d] */
   const void* unembed;              /* bf16 [V, d] (untied) */
   const dg_layer_weights* layers;   /* host array of cfg.n_layers entries */
+  /* Optional e4m3 copy of the unembedding (dg_quantize_e4m3, one tensor
+   * scale): when set (V % 256 == 0, d % 128 == 0), the denoising loop's
+   * unembedding + sampler step runs on FP8 operands, the hidden states
+   * quantised per token each step.  NULL: bf16. */
+  const uint8_t* unembed_e4m3;      /* e4m3 [V, d] */
+  const float* unembed_scale;       /* device scalar */
 } dg_model;
 
 /* Which uncommitted positions a step commits.
@@ -268,6 +274,32 @@ int dg_unembed_sample_commit(const void* h, const void* w_u, int d, int32_t* tok
 size_t dg_unembed_sample_commit_workspace_bytes(int B, int C, int V);
 
 /*
+ * FP8 (e4m3) unembedding.  The pages quote FP8 checkpoints without fixing a
+ * recipe; this library's: e4m3 (1 sign, 4 exponent bits with bias 7,
+ * 3 mantissa bits, largest finite value 448), nearest value with ties to
+ * even, saturating; scale = max |x| / 448 in fp32 (1 for an all-zero block).
+ *
+ * dg_quantize_e4m3 - in bf16 [rows, cols] -> out e4m3 [rows, cols] and
+ *   scales: per_row != 0: one per row (scales[rows]); per_row == 0: one for
+ *   the tensor (scales[0]).  x ~= scale * e4m3_value.  cols % 8 == 0.
+ * dg_unembed_e4m3 - logits[m, v] = hs[m] * ws * sum_k dec(h_q[m, k]) dec(w_q[v, k])
+ *   (fp32 accumulate of exact products); h_scale device [M], w_scale device
+ *   scalar.  V % 256 == 0, d % 128 == 0.
+ * dg_unembed_sample_commit_e4m3 - dg_unembed_sample_commit with the logits of
+ *   dg_unembed_e4m3.  Workspace: dg_unembed_sample_commit_workspace_bytes().
+ */
+int dg_quantize_e4m3(const void* in, int rows, int cols, int per_row, uint8_t* out,
+                     float* scales, void* stream);
+int dg_unembed_e4m3(const uint8_t* h_q, const float* h_scale, const uint8_t* w_q,
+                    const float* w_scale, float* logits, int M, int d, int V, void* stream);
+int dg_unembed_sample_commit_e4m3(const uint8_t* h_q, const float* h_scale, const uint8_t* w_q,
+                                  const float* w_scale, int d, int32_t* tok, uint8_t* committed,
+                                  int32_t* prev_argmax, int32_t* seq_status,
+                                  const dg_sampler_cfg* cfg, uint32_t seed, int block, int step,
+                                  int B, int C, int V, const dg_step_out* out, void* workspace,
+                                  size_t workspace_bytes, void* stream);
+
+/*
  * dg_sample_commit_noalloc - dg_sample_commit without a workspace argument.
  * The paper has no counterpart: this is a library convenience.  It serves
  * callers that cannot allocate device memory - a plugin whose host owns every
@@ -318,7 +350,9 @@ size_t dg_prefill_workspace_bytes(const dg_model_cfg* cfg, int B, int P);
  * dg_denoise_logits - one bidirectional forward of the current canvas
  * (embedding, layers, final norm, unembedding) over the cached prefix, into
  * logits fp32 [B, C, V].  The building block of dg_denoise_block, exposed for
- * parity tests.  Workspace: dg_denoise_block_workspace_bytes().
+ * parity tests; with the model's e4m3 unembedding set, the logits are those of
+ * the FP8 path (hidden states quantised per token).  Workspace:
+ * dg_denoise_block_workspace_bytes().
  */
 int dg_denoise_logits(const dg_model* m, const dg_state* st, float* logits,
                       void* workspace, size_t workspace_bytes, void* stream);

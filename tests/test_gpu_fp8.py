@@ -1,0 +1,246 @@
+"""The FP8 (e4m3) unembedding against the oracle.
+
+Quantisation is integer work once the fp32 scale is fixed: codes and scales
+must equal the oracle's bit for bit.  The e4m3 unembedding sums exact products
+of e4m3 values in fp32 on the tensor cores, so its logits meet the oracle's
+fp64 sum to fp32 accumulation rounding.  The fused FP8 sampler step is held to
+the sampler's bar (exact decisions outside near-tie margins).  At model level,
+the FP8 logits of a denoising pass follow the oracle's FP8 forward (closer to
+it than to the oracle's bf16 logits), and the block driver on an FP8 model
+equals the same steps driven one call at a time.
+"""
+import numpy as np
+import pytest
+import torch
+
+from helpers import assert_close, gpu_weights, to64
+from oracle import fp8
+from oracle import model as M
+from oracle import sampler as S
+from canvas_denoising_denoise_b200 import synth
+from test_gpu_sampler import compare
+
+pytestmark = pytest.mark.gpu
+
+
+def rand_bf16(shape, scale, seed):
+    g = torch.Generator().manual_seed(seed)
+    return (torch.randn(shape, generator=g) * scale).to(torch.bfloat16)
+
+
+def gpu_quant(x, per_row):
+    import canvas_denoising_denoise_b200 as dg
+    xd = x.cuda()
+    q = torch.empty(x.shape, dtype=torch.uint8, device="cuda")
+    s = torch.empty(x.shape[0] if per_row else 1, dtype=torch.float32, device="cuda")
+    dg.quantize_e4m3(xd, q, s, per_row=per_row)
+    torch.cuda.synchronize()
+    dg.check_device_errors()
+    return q, s
+
+
+def spread_rows(R, C, seed):
+    """Rows at scales from 1e-4 to 3e4, one all-zero row, one row with a lone spike."""
+    g = torch.Generator().manual_seed(seed)
+    scale = 10.0 ** torch.empty(R, 1).uniform_(-4, 4.5, generator=g)
+    x = torch.randn((R, C), generator=g) * scale
+    x[R // 3] = 0
+    x[R // 2] = 0
+    x[R // 2, C // 2] = -7.0
+    return x.to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("R,C", [(300, 2048), (7, 8), (1, 4096), (256, 256)])
+def test_quantize_rows_bit_exact(R, C):
+    x = spread_rows(R, C, seed=R + C)
+    q, s = gpu_quant(x, per_row=True)
+    wq, ws = fp8.quantize_rows(x.float().numpy())
+    assert np.array_equal(s.cpu().numpy().view(np.uint32), ws.view(np.uint32))
+    assert np.array_equal(q.cpu().numpy(), wq)
+
+
+@pytest.mark.parametrize("R,C,scale", [(4096, 512, 0.02), (333, 8, 5.0), (64, 64, 0.0)])
+def test_quantize_tensor_bit_exact(R, C, scale):
+    x = rand_bf16((R, C), scale, seed=R)
+    q, s = gpu_quant(x, per_row=False)
+    wq, ws = fp8.quantize_tensor(x.float().numpy())
+    assert s.cpu().numpy().view(np.uint32)[0] == np.float32(ws).view(np.uint32)
+    assert np.array_equal(q.cpu().numpy(), wq)
+
+
+def quant_pair(Mr, d, V, seed):
+    h = rand_bf16((Mr, d), 1.0, seed)
+    w = rand_bf16((V, d), 0.02, seed + 1)
+    hq, hs = gpu_quant(h, per_row=True)
+    wq, ws = gpu_quant(w, per_row=False)
+    return h, w, hq, hs, wq, ws
+
+
+# V % 256 == 0 and d % 128 == 0; 600 rows leave a ragged token tile; V = 65536
+# gives each pair several tiles (both accumulator buffers reused); d = 128 is a
+# single k-block.
+@pytest.mark.parametrize("Mr,d,V", [(256, 256, 512), (256, 2048, 4096), (600, 512, 2048),
+                                    (1, 128, 256), (256, 512, 65536), (131, 384, 1024)])
+def test_unembed_e4m3_against_oracle(Mr, d, V):
+    import canvas_denoising_denoise_b200 as dg
+    h, w, hq, hs, wq, ws = quant_pair(Mr, d, V, seed=Mr + V)
+    logits = torch.empty((Mr, V), dtype=torch.float32, device="cuda")
+    dg.unembed_e4m3(hq, hs, wq, ws, logits)
+    torch.cuda.synchronize()
+    dg.check_device_errors()
+    want = fp8.unembed_logits(hq.cpu().numpy(), hs.cpu().numpy(), wq.cpu().numpy(),
+                              ws.cpu().numpy()[0])
+    # fp32 sums of exact products: rounding of order K 2^-24 of sum |products|
+    assert_close(logits, want, rel_l2=1e-5, max_abs=1e-4, what=f"e4m3 unembed {Mr}x{d}x{V}")
+    # and the FP8 rounding itself is visible against the bf16 product
+    exact = to64(h) @ to64(w).T
+    rel_q = np.linalg.norm(want - exact) / np.linalg.norm(exact)
+    assert 1e-3 < rel_q < 0.1
+
+
+def test_unembed_e4m3_full_vocab_sampled_rows():
+    """M = 256, d = 2048, V = 262144 on sampled outputs."""
+    import canvas_denoising_denoise_b200 as dg
+    Mr, d, V = 256, 2048, 262144
+    h, w, hq, hs, wq, ws = quant_pair(Mr, d, V, seed=11)
+    logits = torch.empty((Mr, V), dtype=torch.float32, device="cuda")
+    dg.unembed_e4m3(hq, hs, wq, ws, logits)
+    torch.cuda.synchronize()
+    rng = np.random.default_rng(1)
+    rows = rng.integers(0, Mr, size=16)
+    cols = rng.integers(0, V, size=512)
+    want = fp8.unembed_logits(hq[rows].cpu().numpy(), hs[rows].cpu().numpy(),
+                              wq[cols].cpu().numpy(), ws.cpu().numpy()[0])
+    assert_close(logits[rows][:, cols].cpu(), want, rel_l2=1e-5, max_abs=1e-4,
+                 what="e4m3 unembed full")
+
+
+def run_fused_e4m3(hq, hs, wq, ws, tok, committed, prev, settings, seed, block, step):
+    import canvas_denoising_denoise_b200 as dg
+    B, C = tok.shape
+    dev = "cuda"
+    t_tok = torch.as_tensor(tok, dtype=torch.int32).to(dev).contiguous()
+    t_com = torch.as_tensor(committed, dtype=torch.uint8).to(dev).contiguous()
+    t_prev = torch.as_tensor(prev, dtype=torch.int32).to(dev).contiguous()
+    t_stat = torch.zeros(B, dtype=torch.int32, device=dev)
+    out = {"x_hat": torch.empty((B, C), dtype=torch.int32, device=dev),
+           "argmax": torch.empty((B, C), dtype=torch.int32, device=dev),
+           "logconf": torch.empty((B, C), dtype=torch.float32, device=dev),
+           "entropy": torch.empty((B, C), dtype=torch.float32, device=dev),
+           "flags": torch.empty((B, C), dtype=torch.uint8, device=dev)}
+    dg.unembed_sample_commit_e4m3(hq, hs, wq, ws, t_tok, t_com, t_prev, t_stat, settings, seed,
+                                  block, step, out=out)
+    torch.cuda.synchronize()
+    dg.check_device_errors()
+    res = {k: v.cpu().numpy() for k, v in out.items()}
+    res.update(tok=t_tok.cpu().numpy(), committed=t_com.cpu().numpy().astype(bool),
+               prev=t_prev.cpu().numpy(), status=t_stat.cpu().numpy())
+    return res
+
+
+# w ~ N(0, 3/sqrt(d)) gives the logits the spread of the sampler workload.
+@pytest.mark.parametrize("B,C,V,d,step", [(1, 256, 512, 256, 0), (2, 256, 4096, 512, 9),
+                                          (1, 200, 8192, 256, 17), (1, 256, 1024, 2048, 47)])
+def test_fused_e4m3_step_against_oracle(B, C, V, d, step):
+    import canvas_denoising_denoise_b200 as dg
+    seed = B * 100 + V + step
+    h = rand_bf16((B * C, d), 1.0, seed)
+    w = rand_bf16((V, d), 3.0 / d ** 0.5, seed + 1)
+    hq, hs = gpu_quant(h, per_row=True)
+    wq, ws = gpu_quant(w, per_row=False)
+    rng = np.random.default_rng(seed)
+    tok = rng.integers(0, V, size=(B, C))
+    committed = rng.random((B, C)) < 0.3
+    prev = rng.integers(0, V, size=(B, C))
+    g = run_fused_e4m3(hq, hs, wq, ws, tok, committed, prev, dg.SamplerSettings(), 13, 3, step)
+    logits = fp8.unembed_logits(hq.cpu().numpy(), hs.cpu().numpy(), wq.cpu().numpy(),
+                                ws.cpu().numpy()[0]).reshape(B, C, V)
+    counters = {"near_gumbel": 0, "near_renoise": 0, "skipped_sequences": 0}
+    for b in range(B):
+        r = S.sampler_step(S.SamplerCfg(), logits[b], tok[b], committed[b], prev[b], step, 13, b,
+                           3)
+        compare(g, r, b, committed[b], counters)
+    print("near-tie counts", counters)
+
+
+SHAPE = synth.TINY
+OCFG = M.ModelCfg(SHAPE.d, SHAPE.n_layers, SHAPE.n_q_heads, SHAPE.n_kv_heads, SHAPE.head_dim,
+                  SHAPE.ffn, SHAPE.vocab, SHAPE.eps)
+P, C = 64, 256
+
+
+@pytest.fixture(scope="module")
+def fp8_model():
+    import canvas_denoising_denoise_b200 as dg
+    w_cpu = synth.make_weights(SHAPE, seed=0)
+    model = dg.DgModel(SHAPE, gpu_weights(w_cpu), fp8_unembed=True)
+    prompt = synth.make_prompt(1, P, SHAPE.vocab, seed=1)
+    return dg, model, M.weights_to_f64(w_cpu), prompt
+
+
+def test_model_keeps_the_oracle_quantised_unembedding(fp8_model):
+    dg, model, w64, _ = fp8_model
+    wq, ws = fp8.quantize_tensor(w64["unembed"])
+    assert np.array_equal(model.unembed_q.cpu().numpy(), wq)
+    assert model.unembed_scale.cpu().numpy()[0] == np.float32(ws)
+
+
+def test_denoise_logits_e4m3_follow_the_oracle(fp8_model):
+    """GPU FP8 logits vs the oracle's FP8 forward.
+
+    The GPU quantises the bf16 copy of the final residual (the RMSNorm a factor
+    of the logits), the oracle the bf16-rounded normalised state: the two bf16
+    roundings are independent, and one e4m3 step spans 32 bf16 steps, so about
+    one code in 32 differs by one e4m3 step (1/8 of its value).  That puts the
+    logits about sqrt(1/32) * 2^-3 / sqrt(3) ~ 1.3e-2 (rel L2) apart per unit of
+    FP8 rounding noise: bar 3e-2.  And the GPU logits must sit closer to the
+    oracle's FP8 logits than to its bf16 ones (a bf16 unembedding would not)."""
+    dg, model, w64, prompt = fp8_model
+    st = dg.DgState(SHAPE, 1, P + 2 * C, C)
+    dg.prefill(model, st, prompt.cuda())
+    canvas = torch.randint(0, SHAPE.vocab, (1, C), generator=torch.Generator().manual_seed(2))
+    st.tok.copy_(canvas.to(torch.int32))
+    logits = torch.empty((1, C, SHAPE.vocab), dtype=torch.float32, device="cuda")
+    dg.denoise_logits(model, st, logits)
+    torch.cuda.synchronize()
+    dg.check_device_errors()
+    kc, vc = M.empty_cache(OCFG, P + 2 * C)
+    L = M.prefill(OCFG, w64, prompt[0].numpy(), kc, vc)
+    want = M.denoise_logits(OCFG, w64, canvas[0].numpy(), kc, vc, L, e4m3_unembed=True)
+    bf16 = M.denoise_logits(OCFG, w64, canvas[0].numpy(), kc, vc, L)
+    got = to64(logits[0])
+    rel = np.linalg.norm(got - want) / np.linalg.norm(want)
+    rel_b = np.linalg.norm(got - bf16) / np.linalg.norm(bf16)
+    rel_q = np.linalg.norm(want - bf16) / np.linalg.norm(bf16)
+    print(f"gpu vs oracle fp8 {rel:.3e}; gpu vs oracle bf16 {rel_b:.3e}; "
+          f"oracle fp8 vs bf16 {rel_q:.3e}")
+    assert rel <= 3e-2 and rel < 0.6 * rel_b
+
+
+def test_block_driver_e4m3_matches_stepwise_calls(fp8_model):
+    """dg_denoise_block on an FP8 model (fused e4m3 unembedding + sampler) equals
+    dg_denoise_logits (FP8 logits stored) followed by dg_sample_commit."""
+    dg, model, _, prompt = fp8_model
+    seed, block = 3, 0
+    st = dg.DgState(SHAPE, 1, P + 2 * C, C)
+    dg.prefill(model, st, prompt.cuda())
+    steps = dg.denoise_block(model, st, dg.SamplerSettings(), seed, block)
+    torch.cuda.synchronize()
+    dg.check_device_errors()
+    tok_a = st.tok.clone()
+    st2 = dg.DgState(SHAPE, 1, P + 2 * C, C)
+    dg.prefill(model, st2, prompt.cuda())
+    st2.tok.copy_(torch.from_numpy(S.init_canvas(seed, 0, block, C, SHAPE.vocab)).view(1, C))
+    st2.committed.zero_(); st2.prev_argmax.fill_(-1); st2.seq_status.zero_()
+    logits = torch.empty((1, C, SHAPE.vocab), dtype=torch.float32, device="cuda")
+    settings = dg.SamplerSettings()
+    n = 0
+    for s in range(48):
+        dg.denoise_logits(model, st2, logits)
+        dg.sample_commit(logits, st2.tok, st2.committed, st2.prev_argmax, st2.seq_status,
+                         settings, seed, block, s)
+        n = s + 1
+        if int(st2.seq_status.item()) != 0:
+            break
+    assert n == steps
+    assert torch.equal(st2.tok, tok_a), "FP8 block driver and step-wise calls must agree"
