@@ -31,10 +31,12 @@ Weight layout (nn.Linear convention, [out_features, in_features]):
     w_o     [d, Hq hd]
     w_up    [F, d]          w_down  [d, F]
 
-FP8 unembedding (optional, ``e4m3_unembed=True``; a reading: the pages quote
-FP8 checkpoints but fix no recipe): the final normalised hidden state, stored
-as bfloat16, is quantised to e4m3 per token and the unembedding per tensor
-(oracle.fp8), and the logits are the scaled products of the codes.
+FP8 (a reading: the pages quote FP8 checkpoints but fix no recipe).  With
+``e4m3_unembed=True`` the final normalised hidden state, stored as bfloat16,
+is quantised to e4m3 per token and the unembedding per tensor (oracle.fp8),
+and the logits are the scaled products of the codes.  With
+``e4m3_layers=True`` every projection of the stack (QKV, output, MLP up and
+down) does the same with its input as stored (bf16) and its weight.
 
 Storage rounding: with ``bf16_storage=True`` (default) the oracle rounds to
 bfloat16 at the points where the product stores bfloat16 tensors - the
@@ -138,17 +140,33 @@ def _r(x, on):
     return round_bf16(x) if on else x
 
 
-def layer_forward(cfg, w, x, k_pre, v_pre, causal, bf16_storage=True, skip_tail=False):
+def linear_e4m3(a, w):
+    """a [R, K] @ w [N, K]^T on e4m3 operands: per-row codes and scales of a, one
+    scale for w, products of the decoded codes summed in fp64 and scaled
+    (the same arithmetic as the FP8 unembedding, whose pins cover it)."""
+    aq, as_ = fp8.quantize_rows(a)
+    wq, ws = fp8.quantize_tensor(w)
+    acc = fp8.decode(aq) @ fp8.decode(wq).T
+    return acc * (np.asarray(as_, dtype=np.float64) * np.float64(ws))[:, None]
+
+
+def layer_forward(cfg, w, x, k_pre, v_pre, causal, bf16_storage=True, skip_tail=False,
+                  e4m3=False):
     """One pre-norm transformer layer over one sequence's new rows.
 
     x [Lq, d] (residual stream, fp64); k_pre/v_pre [Hkv, L, hd] cached prefix.
     Returns (x_out, k_new, v_new) with k_new/v_new [Lq, Hkv, hd] as stored.
     With skip_tail the attention/MLP half is skipped (only K/V are wanted).
+    With e4m3 the four projections run on e4m3 operands (linear_e4m3).
     """
     hq, hkv, hd = cfg.n_q_heads, cfg.n_kv_heads, cfg.head_dim
     lq = x.shape[0]
+
+    def lin(a, name):
+        return linear_e4m3(a, w[name]) if e4m3 else a @ w[name].T
+
     xn = _r(rmsnorm(x, cfg.eps), bf16_storage)
-    qkv = _r(xn @ w["w_qkv"].T, bf16_storage)
+    qkv = _r(lin(xn, "w_qkv"), bf16_storage)
     q = qkv[:, : hq * hd].reshape(lq, hq, hd)
     k_new = qkv[:, hq * hd: (hq + hkv) * hd].reshape(lq, hkv, hd)
     v_new = qkv[:, (hq + hkv) * hd:].reshape(lq, hkv, hd)
@@ -156,10 +174,10 @@ def layer_forward(cfg, w, x, k_pre, v_pre, causal, bf16_storage=True, skip_tail=
         return x, k_new, v_new
     o = gqa_attention(q, k_new, v_new, k_pre, v_pre, causal, 1.0 / np.sqrt(hd))
     o = _r(o.reshape(lq, hq * hd), bf16_storage)
-    h = x + o @ w["w_o"].T
+    h = x + lin(o, "w_o")
     hn = _r(rmsnorm(h, cfg.eps), bf16_storage)
-    u = _r(gelu(hn @ w["w_up"].T), bf16_storage)
-    x_out = h + u @ w["w_down"].T
+    u = _r(gelu(lin(hn, "w_up")), bf16_storage)
+    x_out = h + lin(u, "w_down")
     return x_out, k_new, v_new
 
 
@@ -173,7 +191,7 @@ def unembed_e4m3(hn, w_unembed):
 
 
 def forward(cfg, weights, tokens, k_cache, v_cache, prefix_len, causal,
-            bf16_storage=True, want_logits=True, e4m3_unembed=False):
+            bf16_storage=True, want_logits=True, e4m3_unembed=False, e4m3_layers=False):
     """Run the stack over new rows of one sequence.
 
     tokens [Lq] int; k_cache/v_cache: per layer [Hkv, >=prefix_len, hd] arrays.
@@ -187,7 +205,8 @@ def forward(cfg, weights, tokens, k_cache, v_cache, prefix_len, causal,
         v_pre = v_cache[l][:, :prefix_len, :]
         last = (l == cfg.n_layers - 1)
         x, k_new, v_new = layer_forward(cfg, weights["layers"][l], x, k_pre, v_pre, causal,
-                                        bf16_storage, skip_tail=(last and not want_logits))
+                                        bf16_storage, skip_tail=(last and not want_logits),
+                                        e4m3=e4m3_layers)
         kv.append((k_new, v_new))
     if not want_logits:
         return None, kv
@@ -214,18 +233,19 @@ def commit_kv(k_cache, v_cache, kv, at):
     return at + kv[0][0].shape[0]
 
 
-def prefill(cfg, weights, prompt, k_cache, v_cache, bf16_storage=True):
+def prefill(cfg, weights, prompt, k_cache, v_cache, bf16_storage=True, e4m3_layers=False):
     """Causal pass over the prompt; writes its K/V at rows [0, P).  Returns P."""
     _, kv = forward(cfg, weights, prompt, k_cache, v_cache, 0, causal=True,
-                    bf16_storage=bf16_storage, want_logits=False)
+                    bf16_storage=bf16_storage, want_logits=False, e4m3_layers=e4m3_layers)
     return commit_kv(k_cache, v_cache, kv, 0)
 
 
 def denoise_logits(cfg, weights, canvas, k_cache, v_cache, prefix_len, bf16_storage=True,
-                   e4m3_unembed=False):
+                   e4m3_unembed=False, e4m3_layers=False):
     """Bidirectional pass of the canvas over the cached prefix -> logits [C, V]."""
     logits, _ = forward(cfg, weights, canvas, k_cache, v_cache, prefix_len, causal=False,
-                        bf16_storage=bf16_storage, want_logits=True, e4m3_unembed=e4m3_unembed)
+                        bf16_storage=bf16_storage, want_logits=True, e4m3_unembed=e4m3_unembed,
+                        e4m3_layers=e4m3_layers)
     return logits
 
 

@@ -210,3 +210,59 @@ def test_bf16_storage_close_to_fp64():
         out.append(M.denoise_logits(TINY, w, canvas, kc, vc, L, bf16))
     rel = np.linalg.norm(out[0] - out[1]) / np.linalg.norm(out[0])
     assert 0 < rel < 2e-2
+
+
+def test_e4m3_linear_exact_on_representable_operands():
+    """Rows of a that are e4m3 values times 2^j with one entry at +-448 * 2^j, and a
+    weight of e4m3 values times 2^-5 with one entry at 448 * 2^-5, quantise exactly
+    (scale = amax / 448 is the power of two), so the FP8 product is the exact product."""
+    from oracle import fp8
+    rng = np.random.default_rng(12)
+    finite = np.concatenate([np.arange(0, 127), np.arange(128, 255)]).astype(np.uint8)
+    a = fp8.decode(rng.choice(finite, size=(7, 48)))
+    a[:, 5] = 448.0 * np.where(rng.random(7) < 0.5, 1, -1)
+    a = a * (2.0 ** rng.integers(-6, 6, size=(7, 1)))
+    w = fp8.decode(rng.choice(finite, size=(24, 48)))
+    w[3, 9] = 448.0
+    w = w * 2.0 ** -5
+    got = M.linear_e4m3(a, w)
+    assert np.array_equal(got, a @ w.T)
+    assert not np.allclose(got, a @ w[::-1].T)
+
+
+def test_e4m3_layers_zero_projections_identity_and_equivariance():
+    w = rand_weights(TINY, seed=13)
+    lw = dict(w["layers"][0])
+    lw["w_o"] = np.zeros_like(lw["w_o"])
+    lw["w_down"] = np.zeros_like(lw["w_down"])
+    rng = np.random.default_rng(14)
+    x = rng.normal(size=(5, TINY.d))
+    empty = np.zeros((TINY.n_kv_heads, 0, TINY.head_dim))
+    out, _, _ = M.layer_forward(TINY, lw, x, empty, empty, False, bf16_storage=True, e4m3=True)
+    assert np.array_equal(out, x)
+    # per-token activation scales and one weight scale keep the canvas pass
+    # permutation-equivariant
+    kc, vc = M.empty_cache(TINY, 40)
+    prompt = rng.integers(0, TINY.vocab, size=8)
+    L = M.prefill(TINY, w, prompt, kc, vc, e4m3_layers=True)
+    canvas = rng.integers(0, TINY.vocab, size=16)
+    perm = rng.permutation(16)
+    lg = M.denoise_logits(TINY, w, canvas, kc, vc, L, e4m3_layers=True)
+    lgp = M.denoise_logits(TINY, w, canvas[perm], kc, vc, L, e4m3_layers=True)
+    assert np.allclose(lgp, lg[perm], atol=1e-9)
+
+
+def test_e4m3_layers_close_to_bf16_forward():
+    """FP8 projections move the logits by the format's rounding (a few percent),
+    not more, and not zero."""
+    w = rand_weights(TINY, seed=15)
+    rng = np.random.default_rng(16)
+    prompt = rng.integers(0, TINY.vocab, size=8)
+    canvas = rng.integers(0, TINY.vocab, size=16)
+    out = []
+    for e4m3 in (False, True):
+        kc, vc = M.empty_cache(TINY, 24)
+        L = M.prefill(TINY, w, prompt, kc, vc, e4m3_layers=e4m3)
+        out.append(M.denoise_logits(TINY, w, canvas, kc, vc, L, e4m3_layers=e4m3))
+    rel = np.linalg.norm(out[0] - out[1]) / np.linalg.norm(out[0])
+    assert 1e-3 < rel < 0.1
