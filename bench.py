@@ -33,6 +33,12 @@ sys.path.insert(0, ROOT)
 METRIC = "committed tokens/s (B=1, 256-tok canvas); canvas-attn % of BF16 tensor peak"
 
 
+def dtype_name(args):
+    """The arithmetic of the path: bf16, with e4m3 parts where asked."""
+    parts = [p for p, on in (("projections", args.fp8_layers), ("unembed", args.fp8_unembed)) if on]
+    return "bf16" if not parts else "bf16+e4m3-" + "+".join(parts)
+
+
 def metric_name(batch):
     return METRIC.replace("B=1", f"B={batch}")
 UNIT = "tokens/s"
@@ -535,6 +541,25 @@ def run_kernel_bench(args):
                     "us": round(t * 1e6, 2),
                     "tflops": round(fl / t / 1e12, 1),
                     "weight_gbs": round(N * K * 2 / t / 1e9, 1)})
+        if K % 128 == 0:
+            # the same projection on e4m3 codes (the activation quantised per
+            # token first, as the forward pass does), and the GEMM alone
+            xq = torch.empty((M, K), dtype=torch.uint8, device="cuda")
+            xs = torch.empty(M, dtype=torch.float32, device="cuda")
+            wq = torch.empty((N, K), dtype=torch.uint8, device="cuda")
+            wsc = torch.empty(1, dtype=torch.float32, device="cuda")
+            dg.quantize_e4m3(w, wq, wsc, per_row=False)
+
+            def q_and_gemm():
+                dg.quantize_e4m3(x, xq, xs, per_row=True)
+                dg.linear_e4m3(xq, xs, wq, wsc, y, epi)
+            for name, fn in (("quantize_e4m3 + linear_e4m3", q_and_gemm),
+                             ("linear_e4m3", lambda: dg.linear_e4m3(xq, xs, wq, wsc, y, epi))):
+                t = timed(fn, args.steps)
+                out.append({"kernel": name, "epilogue": args.epi, "shape": [M, N, K],
+                            "us": round(t * 1e6, 2), "tflops": round(fl / t / 1e12, 1),
+                            "frac_fp8_peak": round(fl / t / 1e12 / (2 * peaks["bf16_tflops"]), 4),
+                            "weight_gbs": round(N * K / t / 1e9, 1)})
     for o in out:
         o["peaks"] = peaks["source"]
         print(json.dumps(o), flush=True)
@@ -562,6 +587,8 @@ def main():
     ap.add_argument("--heads", default="32,8", help="query,kv heads for --kernel attn")
     ap.add_argument("--fp8-unembed", action="store_true",
                     help="run the unembedding + sampler step on e4m3 operands")
+    ap.add_argument("--fp8-layers", action="store_true",
+                    help="run every projection of the stack on e4m3 operands")
     args = ap.parse_args()
     if args.kernel:
         return run_kernel_bench(args)
@@ -592,7 +619,7 @@ def main():
                    "layers": [{k: v.cuda() for k, v in lw.items()} for lw in w_cpu["layers"]]}
     else:
         weights = synth.make_weights_fast(shape, seed=0, device="cuda")
-    model = dg.DgModel(shape, weights, fp8_unembed=args.fp8_unembed)
+    model = dg.DgModel(shape, weights, fp8_unembed=args.fp8_unembed, fp8_layers=args.fp8_layers)
     blocks = workload_blocks(args.workload)
     lmax = prompt_len + CANVAS * blocks
     st = dg.DgState(shape, batch, lmax, CANVAS)
@@ -673,10 +700,11 @@ def main():
             "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(elapsed / args.steps * 1e3, 3), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None,
-            "dtype": "bf16+e4m3-unembed" if args.fp8_unembed else "bf16", "data": "synthetic",
+            "dtype": dtype_name(args), "data": "synthetic",
             "config": dict(workload_config(args.workload, world,
                                            steps_seen[-1] if steps_seen else None),
-                           unembed="e4m3" if args.fp8_unembed else "bf16"),
+                           unembed="e4m3" if args.fp8_unembed else "bf16",
+                           projections="e4m3" if args.fp8_layers else "bf16"),
             "roofline": roof,
             "canvas_attn": attn,
             "unembed_sample": samp,

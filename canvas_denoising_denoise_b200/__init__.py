@@ -7,7 +7,7 @@ CUDA device, and raises otherwise.
 
 Functions take torch tensors and pass their device pointers:
     canvas_attn, unembed, linear, sample_commit, unembed_sample_commit, kv_block_commit,
-    quantize_e4m3, unembed_e4m3, unembed_sample_commit_e4m3,
+    quantize_e4m3, linear_e4m3, unembed_e4m3, unembed_sample_commit_e4m3,
     philox
 Objects:
     DgModel   weights + configuration (dg_model)
@@ -23,7 +23,7 @@ from ._lib import (EPI_BF16, EPI_F32, EPI_GELU_BF16, EPI_RESID_F32, MASK_BIDIR, 
                    UNSELECTED_KEEP, UNSELECTED_RENOISE, DgError)
 
 __all__ = ["canvas_attn", "unembed", "linear", "sample_commit", "unembed_sample_commit",
-           "quantize_e4m3", "unembed_e4m3", "unembed_sample_commit_e4m3",
+           "quantize_e4m3", "linear_e4m3", "unembed_e4m3", "unembed_sample_commit_e4m3",
            "kv_block_commit", "philox",
            "DgModel", "DgState", "SamplerSettings", "prefill", "denoise_logits", "denoise_block",
            "check_device_errors", "Workspace", "DgError", "MASK_BIDIR", "MASK_CAUSAL",
@@ -206,6 +206,15 @@ def quantize_e4m3(x, out, scales, per_row=True, stream=None):
                                             _ptr(scales), _stream(stream)))
 
 
+def linear_e4m3(x_q, x_scale, w_q, w_scale, out, epilogue=EPI_BF16, stream=None):
+    """linear on e4m3 codes: acc = x_scale[m] w_scale (x_q[M, K] . w_q[N, K]), then the epilogue."""
+    _need_contig(x_q, x_scale, w_q, w_scale, out)
+    M, K = x_q.shape
+    N = w_q.shape[0]
+    _lib.check(_lib.load().dg_linear_e4m3(_ptr(x_q), _ptr(x_scale), _ptr(w_q), _ptr(w_scale),
+                                          _ptr(out), M, N, K, epilogue, _stream(stream)))
+
+
 def unembed_e4m3(h_q, h_scale, w_q, w_scale, logits, stream=None):
     """logits[M, V] = h_scale[m] w_scale (h_q[M, d] . w_q[V, d]) on e4m3 codes."""
     _need_contig(h_q, h_scale, w_q, w_scale, logits)
@@ -261,10 +270,12 @@ class DgModel:
     """Model weights (bf16 device tensors, [out, in]) and their dg_model view.
 
     fp8_unembed=True also keeps an e4m3 copy of the unembedding (one tensor
-    scale), which the denoising loop's unembedding + sampler step then uses.
+    scale), which the denoising loop's unembedding + sampler step then uses;
+    fp8_layers=True keeps e4m3 copies of every projection weight (one scale
+    each), and every forward pass then runs its projections in FP8.
     """
 
-    def __init__(self, shape, weights, fp8_unembed=False):
+    def __init__(self, shape, weights, fp8_unembed=False, fp8_layers=False):
         self.shape = shape
         self.w = weights
         n = shape.n_layers
@@ -280,10 +291,29 @@ class DgModel:
             self.unembed_q = torch.empty(wu.shape, dtype=torch.uint8, device=wu.device)
             self.unembed_scale = torch.empty(1, dtype=torch.float32, device=wu.device)
             quantize_e4m3(wu, self.unembed_q, self.unembed_scale, per_row=False)
+        self.layers_q = None
+        self._layers_q = None
+        if fp8_layers:
+            self.layers_q = []
+            self._layers_q = (_lib.LayerWeightsE4M3 * n)()
+            for i, lw in enumerate(weights["layers"]):
+                q = {}
+                sc = torch.empty(4, dtype=torch.float32, device=lw["w_qkv"].device)
+                for j, name in enumerate(("w_qkv", "w_o", "w_up", "w_down")):
+                    q[name] = torch.empty(lw[name].shape, dtype=torch.uint8,
+                                          device=lw[name].device)
+                    quantize_e4m3(lw[name], q[name], sc[j:j + 1], per_row=False)
+                q["scales"] = sc
+                self.layers_q.append(q)
+                self._layers_q[i] = _lib.LayerWeightsE4M3(
+                    q["w_qkv"].data_ptr(), q["w_o"].data_ptr(), q["w_up"].data_ptr(),
+                    q["w_down"].data_ptr(), sc.data_ptr())
         self.c = _lib.Model(self.cfg, weights["embed"].data_ptr(), weights["unembed"].data_ptr(),
                             ctypes.cast(self._layers, ctypes.POINTER(_lib.LayerWeights)),
                             self.unembed_q.data_ptr() if fp8_unembed else None,
-                            self.unembed_scale.data_ptr() if fp8_unembed else None)
+                            self.unembed_scale.data_ptr() if fp8_unembed else None,
+                            ctypes.cast(self._layers_q, ctypes.POINTER(_lib.LayerWeightsE4M3))
+                            if fp8_layers else None)
 
 
 class DgState:

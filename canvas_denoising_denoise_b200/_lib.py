@@ -38,10 +38,15 @@ class LayerWeights(ctypes.Structure):
     _fields_ = [("w_qkv", c_void_p), ("w_o", c_void_p), ("w_up", c_void_p), ("w_down", c_void_p)]
 
 
+class LayerWeightsE4M3(ctypes.Structure):
+    _fields_ = [("w_qkv", c_void_p), ("w_o", c_void_p), ("w_up", c_void_p), ("w_down", c_void_p),
+                ("scales", c_void_p)]
+
+
 class Model(ctypes.Structure):
     _fields_ = [("cfg", ModelCfg), ("embed", c_void_p), ("unembed", c_void_p),
                 ("layers", P(LayerWeights)), ("unembed_e4m3", c_void_p),
-                ("unembed_scale", c_void_p)]
+                ("unembed_scale", c_void_p), ("layers_e4m3", P(LayerWeightsE4M3))]
 
 
 class SamplerCfg(ctypes.Structure):
@@ -90,6 +95,8 @@ SIGNATURES = {
                                          c_void_p]),
     "dg_unembed_sample_commit_workspace_bytes": (c_size_t, [c_int, c_int, c_int]),
     "dg_quantize_e4m3": (c_int, [c_void_p, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p]),
+    "dg_linear_e4m3": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int,
+                               c_int, c_int, c_void_p]),
     "dg_unembed_e4m3": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_int,
                                 c_int, c_void_p]),
     "dg_unembed_sample_commit_e4m3": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_int,

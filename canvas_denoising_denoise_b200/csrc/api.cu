@@ -188,8 +188,8 @@ struct GemmPlan {
 // that puts the most CTAs on the SMs in a single wave, preferring fewer splits
 // and then wider tiles; each split keeps >= 4 k-blocks.  Shapes with more
 // tiles than SMs use 256-token tiles without splitting.
-GemmPlan plan_gemm(int M, int N, int K) {
-  const int kb = K / dg::gemm::BK;
+GemmPlan plan_gemm(int M, int N, int K, int kb_elems = dg::gemm::BK) {
+  const int kb = K / kb_elems;
   const int ft = N / dg::gemm::BM;
   GemmPlan best{1, kb, 256};
   int best_ctas = -1;
@@ -223,33 +223,65 @@ struct GemmEpi {
   unsigned long long* trace = nullptr;
 };
 
-template <int S, int BN>
+template <int S, int BN, bool F8>
 cudaError_t launch_gemm_t(dim3 grid, cudaStream_t s, const CUtensorMap& tw, const CUtensorMap& tx,
                           const dg::gemm::Params& p) {
-  return launch_ex(dg::gemm::gemm_kernel<S, BN>, grid, dim3(dg::gemm::THREADS),
+  return launch_ex(dg::gemm::gemm_kernel<S, BN, F8>, grid, dim3(dg::gemm::THREADS),
                    dg::gemm::SMEM_BYTES, s, S, tw, tx, p);
 }
 
-template <int S, int BN>
+template <int S, int BN, bool F8>
 cudaError_t gemm_set_attr() {
-  return cudaFuncSetAttribute(dg::gemm::gemm_kernel<S, BN>,
+  return cudaFuncSetAttribute(dg::gemm::gemm_kernel<S, BN, F8>,
                               cudaFuncAttributeMaxDynamicSharedMemorySize, dg::gemm::SMEM_BYTES);
 }
 
+template <bool F8>
+cudaError_t gemm_set_attrs() {
+  cudaError_t e;
+  if ((e = gemm_set_attr<1, 256, F8>()) != cudaSuccess) return e;
+  if ((e = gemm_set_attr<2, 256, F8>()) != cudaSuccess) return e;
+  if ((e = gemm_set_attr<4, 256, F8>()) != cudaSuccess) return e;
+  if ((e = gemm_set_attr<1, 128, F8>()) != cudaSuccess) return e;
+  if ((e = gemm_set_attr<2, 128, F8>()) != cudaSuccess) return e;
+  return gemm_set_attr<4, 128, F8>();
+}
+
+template <bool F8>
+cudaError_t launch_gemm_plan(const GemmPlan& pl, dim3 grid, cudaStream_t s, const CUtensorMap& tw,
+                             const CUtensorMap& tx, const dg::gemm::Params& p) {
+  if (pl.bn == 256) {
+    switch (pl.splits) {
+      case 1: return launch_gemm_t<1, 256, F8>(grid, s, tw, tx, p);
+      case 2: return launch_gemm_t<2, 256, F8>(grid, s, tw, tx, p);
+      case 4: return launch_gemm_t<4, 256, F8>(grid, s, tw, tx, p);
+    }
+  } else if (pl.bn == 128) {
+    switch (pl.splits) {
+      case 1: return launch_gemm_t<1, 128, F8>(grid, s, tw, tx, p);
+      case 2: return launch_gemm_t<2, 128, F8>(grid, s, tw, tx, p);
+      case 4: return launch_gemm_t<4, 128, F8>(grid, s, tw, tx, p);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+// x [M, K] and w [N, K]: bf16, or e4m3 codes with their scales when f8 is set.
 int launch_gemm(const void* x, const void* w, int M, int N, int K, const GemmPlan& pl,
-                const GemmEpi& e, cudaStream_t s) {
+                const GemmEpi& e, cudaStream_t s, const Fp8Scales* f8 = nullptr) {
   if (!gemm_attr_done) {
-    DG_CUDA((gemm_set_attr<1, 256>()));
-    DG_CUDA((gemm_set_attr<2, 256>()));
-    DG_CUDA((gemm_set_attr<4, 256>()));
-    DG_CUDA((gemm_set_attr<1, 128>()));
-    DG_CUDA((gemm_set_attr<2, 128>()));
-    DG_CUDA((gemm_set_attr<4, 128>()));
+    DG_CUDA(gemm_set_attrs<false>());
+    DG_CUDA(gemm_set_attrs<true>());
     gemm_attr_done = true;
   }
   CUtensorMap tw, tx;
-  DG_TRY(make_tmap(&tw, w, K, N, (uint64_t)K * 2, dg::gemm::BM));
-  DG_TRY(make_tmap(&tx, x, K, M, (uint64_t)K * 2, pl.bn));
+  if (f8) {
+    DG_TRY(make_tmap_u8(&tw, w, K, N, (uint64_t)K, dg::gemm::BM));
+    DG_TRY(make_tmap_u8(&tx, x, K, M, (uint64_t)K, pl.bn));
+  } else {
+    DG_TRY(make_tmap(&tw, w, K, N, (uint64_t)K * 2, dg::gemm::BM));
+    DG_TRY(make_tmap(&tx, x, K, M, (uint64_t)K * 2, pl.bn));
+  }
   dg::gemm::Params p;
   p.M = M; p.N = N; p.K = K;
   p.kb_per_split = pl.kb_per_split;
@@ -264,21 +296,11 @@ int launch_gemm(const void* x, const void* w, int M, int N, int K, const GemmPla
   p.eps = e.eps;
   p.ssq_out = e.ssq_out;
   p.trace = e.trace;
+  p.tok_scale = f8 ? f8->tok : nullptr;
+  p.w_scale = f8 ? f8->w : nullptr;
   const dim3 grid(cdiv(M, pl.bn), N / dg::gemm::BM, pl.splits);
-  cudaError_t err = cudaErrorInvalidValue;
-  if (pl.bn == 256) {
-    switch (pl.splits) {
-      case 1: err = launch_gemm_t<1, 256>(grid, s, tw, tx, p); break;
-      case 2: err = launch_gemm_t<2, 256>(grid, s, tw, tx, p); break;
-      case 4: err = launch_gemm_t<4, 256>(grid, s, tw, tx, p); break;
-    }
-  } else if (pl.bn == 128) {
-    switch (pl.splits) {
-      case 1: err = launch_gemm_t<1, 128>(grid, s, tw, tx, p); break;
-      case 2: err = launch_gemm_t<2, 128>(grid, s, tw, tx, p); break;
-      case 4: err = launch_gemm_t<4, 128>(grid, s, tw, tx, p); break;
-    }
-  }
+  const cudaError_t err = f8 ? launch_gemm_plan<true>(pl, grid, s, tw, tx, p)
+                             : launch_gemm_plan<false>(pl, grid, s, tw, tx, p);
   if (err != cudaSuccess)
     return fail(DG_ERR_CUDA, "gemm launch (S=%d, BN=%d) failed: %s", pl.splits, pl.bn,
                 cudaGetErrorString(err));
@@ -286,10 +308,11 @@ int launch_gemm(const void* x, const void* w, int M, int N, int K, const GemmPla
   return DG_OK;
 }
 
-// y = epilogue(x w^T) with the split plan chosen for this shape.
+// y = epilogue(x w^T) with the split plan chosen for this shape (e4m3
+// operands with their scales when f8 is set: 128-element k-blocks).
 int linear(const void* x, const void* w, int M, int N, int K, const GemmEpi& e,
-           cudaStream_t s) {
-  return launch_gemm(x, w, M, N, K, plan_gemm(M, N, K), e, s);
+           cudaStream_t s, const Fp8Scales* f8 = nullptr) {
+  return launch_gemm(x, w, M, N, K, plan_gemm(M, N, K, f8 ? 128 : dg::gemm::BK), e, s, f8);
 }
 
 // logits = rs * (h w_u^T).  Vocabularies that are a multiple of 256 run on
@@ -649,6 +672,15 @@ int check_model(const dg_model* m) {
   if (m->unembed_e4m3 && (!aligned16(m->unembed_e4m3) || c.vocab % dg::unembed::TILE))
     return fail(DG_ERR_UNSUPPORTED_SHAPE,
                 "model: the e4m3 unembedding needs vocab %% 256 == 0 and 16-byte alignment");
+  if (m->layers_e4m3) {
+    for (int l = 0; l < c.n_layers; ++l) {
+      const dg_layer_weights_e4m3& q = m->layers_e4m3[l];
+      if (!q.w_qkv || !q.w_o || !q.w_up || !q.w_down || !q.scales)
+        return fail(DG_ERR_INVALID_ARG, "model: e4m3 layer %d has a null pointer", l);
+      if (!aligned16(q.w_qkv) || !aligned16(q.w_o) || !aligned16(q.w_up) || !aligned16(q.w_down))
+        return fail(DG_ERR_ALIGNMENT, "model: e4m3 layer %d weight not 16-byte aligned", l);
+    }
+  }
   for (int l = 0; l < c.n_layers; ++l) {
     const dg_layer_weights& w = m->layers[l];
     if (!w.w_qkv || !w.w_o || !w.w_up || !w.w_down)
@@ -678,7 +710,7 @@ int check_state(const dg_state* st, const dg_model_cfg& c, bool need_canvas) {
 
 // Workspace carve-up for a forward over M = B * Lq rows.
 struct FwdLayout {
-  size_t x, xn, qkv, ao, up, ssq_x, ssq_h, attn, logits, spart, flag, hq, hs, total;
+  size_t x, xn, qkv, ao, up, ssq_x, ssq_h, attn, logits, spart, flag, aq, as, total;
 };
 
 FwdLayout fwd_layout(const dg_model_cfg& c, int B, int Lq, int max_prefix, bool logits) {
@@ -706,8 +738,10 @@ FwdLayout fwd_layout(const dg_model_cfg& c, int B, int Lq, int max_prefix, bool 
                                         ? fused_ws_bytes(B, Lq, c.vocab) : (size_t)0)
                          : 0);
   L.flag = take(logits ? 16 : 0);
-  L.hq = take(logits ? (size_t)M * c.d : 0);        // e4m3 hidden states (FP8 unembedding)
-  L.hs = take(logits ? (size_t)M * sizeof(float) : 0);
+  // e4m3 codes and per-token scales of the input of the next FP8 projection
+  // (or of the final hidden states for the FP8 unembedding)
+  L.aq = take((size_t)M * std::max(std::max(c.d, hqd), c.ffn));
+  L.as = take((size_t)M * sizeof(float));
   L.total = off;
   return L;
 }
@@ -725,14 +759,20 @@ struct Fwd {
   bool unembed_elsewhere = false;  // the caller fuses the unembedding into its sampler step
 };
 
-// The last layer's bf16 residual stream quantised per token to e4m3 codes
-// (L.hq) and scales (L.hs); the final RMSNorm stays a row scale of the logits.
-int quantize_hidden(const Fwd& f, cudaStream_t s) {
+// A bf16 activation [B*Lq, cols] quantised per token to e4m3 codes (L.aq)
+// and scales (L.as).  A normalised input is quantised before its RMSNorm,
+// which stays a row scale of the product (per-row scaling commutes with it).
+int quantize_act(const Fwd& f, const void* in, int cols, cudaStream_t s) {
   DG_CUDA(launch_ex(dg::quant::quantize_rows_kernel, dim3(f.B * f.Lq), dim3(dg::quant::THREADS),
-                    0, s, 1, (const __nv_bfloat16*)(f.ws + f.L.xn), f.m->cfg.d,
-                    (uint8_t*)(f.ws + f.L.hq), (float*)(f.ws + f.L.hs)));
+                    0, s, 1, (const __nv_bfloat16*)in, f.B * f.Lq, cols,
+                    (uint8_t*)(f.ws + f.L.aq), (float*)(f.ws + f.L.as)));
   count_launch();
   return DG_OK;
+}
+
+// The last layer's bf16 residual stream, quantised for the FP8 unembedding.
+int quantize_hidden(const Fwd& f, cudaStream_t s) {
+  return quantize_act(f, f.ws + f.L.xn, f.m->cfg.d, s);
 }
 
 int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s) {
@@ -758,11 +798,20 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
   for (int l = 0; l < c.n_layers; ++l) {
     const dg_layer_weights& w = f.m->layers[l];
     const bool last = l == c.n_layers - 1;
+    const dg_layer_weights_e4m3* q8 = f.m->layers_e4m3 ? &f.m->layers_e4m3[l] : nullptr;
+    // y = epilogue(in w^T): bf16, or e4m3 with the input quantised per token
+    auto proj = [&](const void* in, const void* wb, const uint8_t* wq, int widx, int N, int K,
+                    const GemmEpi& e) -> int {
+      if (!q8) return linear(in, wb, M, N, K, e, s);
+      DG_TRY(quantize_act(f, in, K, s));
+      const Fp8Scales f8{(const float*)(f.ws + f.L.as), q8->scales + widx};
+      return linear(f.ws + f.L.aq, wq, M, N, K, e, s, &f8);
+    };
     GemmEpi eq;  // QKV of RMSNorm(x)
     eq.epi = dg::gemm::EPI_BF16;
     eq.out_bf16 = qkv;
     eq.ssq_in = ssq_x; eq.n_ssq_in = nt; eq.inv_k = 1.f / c.d; eq.eps = c.eps;
-    DG_TRY(linear(xb, w.w_qkv, M, nqkv, c.d, eq, s));
+    DG_TRY(proj(xb, w.w_qkv, q8 ? q8->w_qkv : nullptr, 0, nqkv, c.d, eq));
     if (f.commit_kv) {
       const void* kb = qkv + hq * hd;
       const void* vb = qkv + (hq + hkv) * hd;
@@ -776,23 +825,23 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
     GemmEpi eo;  // h = x + O w_o^T
     eo.epi = dg::gemm::EPI_RESID;
     eo.x = x; eo.out_bf16 = xb; eo.ssq_out = ssq_h;
-    DG_TRY(linear(ao, w.w_o, M, c.d, hq * hd, eo, s));
+    DG_TRY(proj(ao, w.w_o, q8 ? q8->w_o : nullptr, 1, c.d, hq * hd, eo));
     GemmEpi eu;  // gelu(RMSNorm(h) w_up^T)
     eu.epi = dg::gemm::EPI_GELU;
     eu.out_bf16 = up;
     eu.ssq_in = ssq_h; eu.n_ssq_in = nt; eu.inv_k = 1.f / c.d; eu.eps = c.eps;
-    DG_TRY(linear(xb, w.w_up, M, c.ffn, c.d, eu, s));
+    DG_TRY(proj(xb, w.w_up, q8 ? q8->w_up : nullptr, 2, c.ffn, c.d, eu));
     GemmEpi ed;  // x = h + u w_down^T
     ed.epi = dg::gemm::EPI_RESID;
     ed.x = x; ed.out_bf16 = xb; ed.ssq_out = ssq_x;
-    DG_TRY(linear(up, w.w_down, M, c.d, c.ffn, ed, s));
+    DG_TRY(proj(up, w.w_down, q8 ? q8->w_down : nullptr, 3, c.d, c.ffn, ed));
   }
   if (f.want_logits && !f.unembed_elsewhere) {
     // logits of RMSNorm(x), on e4m3 operands when the model carries them
     if (f.m->unembed_e4m3) {
       DG_TRY(quantize_hidden(f, s));
-      const Fp8Scales f8{(const float*)(f.ws + f.L.hs), f.m->unembed_scale};
-      DG_TRY(launch_unembed(f.ws + f.L.hq, f.m->unembed_e4m3, logits, M, c.d, c.vocab, ssq_x, nt,
+      const Fp8Scales f8{(const float*)(f.ws + f.L.as), f.m->unembed_scale};
+      DG_TRY(launch_unembed(f.ws + f.L.aq, f.m->unembed_e4m3, logits, M, c.d, c.vocab, ssq_x, nt,
                             1.f / c.d, c.eps, s, &f8));
     } else {
       DG_TRY(launch_unembed(xb, f.m->unembed, logits, M, c.d, c.vocab, ssq_x, nt, 1.f / c.d,
@@ -974,6 +1023,35 @@ int dg_linear(const void* x, const void* w, void* out, int M, int N, int K, int 
   return linear(x, w, M, N, K, e, (cudaStream_t)stream);
 }
 
+int dg_linear_e4m3(const uint8_t* x_q, const float* x_scale, const uint8_t* w_q,
+                   const float* w_scale, void* out, int M, int N, int K, int epilogue,
+                   void* stream) {
+  if (!x_q || !x_scale || !w_q || !w_scale || !out)
+    return fail(DG_ERR_INVALID_ARG, "dg_linear_e4m3: null pointer");
+  if (M <= 0 || N <= 0 || K <= 0 || epilogue < 0 || epilogue > DG_EPI_RESID_F32)
+    return fail(DG_ERR_INVALID_ARG, "dg_linear_e4m3: bad sizes or epilogue");
+  if (N % 128 || K % 128)
+    return fail(DG_ERR_UNSUPPORTED_SHAPE, "dg_linear_e4m3: N %% 128 and K %% 128 must be 0");
+  if (!aligned16(x_q) || !aligned16(w_q) || !aligned16(out))
+    return fail(DG_ERR_ALIGNMENT, "dg_linear_e4m3: pointers must be 16-byte aligned");
+  GemmEpi e;
+  if (epilogue == DG_EPI_F32) {
+    e.epi = dg::gemm::EPI_F32;
+    e.out_f32 = (float*)out;
+  } else if (epilogue == DG_EPI_BF16) {
+    e.epi = dg::gemm::EPI_BF16;
+    e.out_bf16 = (__nv_bfloat16*)out;
+  } else if (epilogue == DG_EPI_GELU_BF16) {
+    e.epi = dg::gemm::EPI_GELU;
+    e.out_bf16 = (__nv_bfloat16*)out;
+  } else {
+    e.epi = dg::gemm::EPI_RESID;
+    e.x = (float*)out;
+  }
+  const Fp8Scales f8{x_scale, w_scale};
+  return linear(x_q, w_q, M, N, K, e, (cudaStream_t)stream, &f8);
+}
+
 size_t dg_sample_commit_workspace_bytes(int B, int C, int V) {
   if (B <= 0 || C <= 0 || V <= 0) return 0;
   return sample_ws_bytes(B, C, V);
@@ -1039,7 +1117,7 @@ int dg_quantize_e4m3(const void* in, int rows, int cols, int per_row, uint8_t* o
   namespace qt = dg::quant;
   if (per_row) {
     DG_CUDA(launch_ex(qt::quantize_rows_kernel, dim3(rows), dim3(qt::THREADS), 0, s, 1,
-                      (const __nv_bfloat16*)in, cols, out, scales));
+                      (const __nv_bfloat16*)in, rows, cols, out, scales));
     count_launch();
     return DG_OK;
   }
@@ -1236,8 +1314,8 @@ int dg_denoise_block(const dg_model* m, dg_state* st, const dg_sampler_cfg* cfg,
     if (fused && fp8) {
       // the hidden states quantised per token, then the e4m3 unembedding + sampler
       DG_TRY(quantize_hidden(fl, s));
-      const Fp8Scales f8{(const float*)(ws + L.hs), m->unembed_scale};
-      DG_TRY(launch_unembed_sample(ws + L.hq, m->unembed_e4m3, m->cfg.d,
+      const Fp8Scales f8{(const float*)(ws + L.as), m->unembed_scale};
+      DG_TRY(launch_unembed_sample(ws + L.aq, m->unembed_e4m3, m->cfg.d,
                                    (const float*)(ws + L.ssq_x), m->cfg.d / 128, 1.f / m->cfg.d,
                                    m->cfg.eps, st->tok, st->committed, st->prev_argmax,
                                    st->seq_status, sp, nullptr, ws + L.spart, s, &f8));

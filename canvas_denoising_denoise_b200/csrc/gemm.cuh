@@ -19,6 +19,11 @@
 // input applies rs in its epilogue, computed from per-(128-column tile, token)
 // sums of squares that the producer of x wrote (summed in a fixed order).
 //
+// With e4m3 operands (F8: x and w as codes, x scaled per token by sx[t], w
+// per tensor by sw) the MMA is kind::f8f6f4 and every epilogue takes acc as
+// sx[t] * sw * (sum of code products): a k-block is 128 codes, still one
+// 128-byte swizzle row.
+//
 // Epilogues:
 //   EPI_F32    out_f32[t, f]  = rs * acc
 //   EPI_BF16   out_bf16[t, f] = bf16(rs * acc)
@@ -65,7 +70,7 @@ enum Epi : int { EPI_F32 = 0, EPI_BF16 = 1, EPI_GELU = 2, EPI_RESID = 3 };
 
 struct Params {
   int M, N, K;
-  int kb_per_split;        // k-blocks (of 64) per split
+  int kb_per_split;        // k-blocks (128-byte rows: 64 bf16 or 128 e4m3) per split
   int splits;              // cluster size along z (1 = no cluster)
   int epi;
   float* out_f32;          // EPI_F32
@@ -76,6 +81,8 @@ struct Params {
   float inv_k;             // 1 / (input width) for the mean
   float eps;
   float* ssq_out;          // [N / 128, M] (EPI_RESID), or null
+  const float* tok_scale;  // F8: [M] per-token scale of x
+  const float* w_scale;    // F8: per-tensor scale of w (device scalar)
   unsigned long long* trace;  // optional [grid, 8] %globaltimer stamps of the phases
 };
 
@@ -141,7 +148,18 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t addr) {
   return v;
 }
 
-template <int S, int BN>
+// Single-CTA MMA on 8-bit operands (kind::f8f6f4, K = 32 per instruction).
+__device__ __forceinline__ void umma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+template <int S, int BN, bool F8 = false>
 __global__ void __launch_bounds__(THREADS, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                 Params p) {
@@ -170,7 +188,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int f0 = blockIdx.y * BM;
   const int split = blockIdx.z;
   const int kb_begin = split * p.kb_per_split;
-  const int nkb = min(p.kb_per_split, p.K / BK - kb_begin);
+  constexpr int KB_ELEMS = F8 ? 128 : BK;  // elements per 128-byte k-block row
+  const int nkb = min(p.kb_per_split, p.K / KB_ELEMS - kb_begin);
 
   if (threadIdx.x == 0) {
     trace_stamp(p, 0);
@@ -211,12 +230,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         uint8_t* a = smem + (q % STAGES) * STAGE_BYTES;
         for (int j = 0; j < stage_kbs(q); ++j)
           tma_load_2d_hint(a + j * A_BYTES, &tm_w, &full[q % STAGES],
-                           (kb_begin + q * KPS + j) * BK, f0, pol_w);
+                           (kb_begin + q * KPS + j) * KB_ELEMS, f0, pol_w);
       };
       auto load_x = [&](int q) {
         uint8_t* b = smem + (q % STAGES) * STAGE_BYTES + KPS * A_BYTES;
         for (int j = 0; j < stage_kbs(q); ++j)
-          tma_load_2d(b + j * TC::B_BYTES, &tm_x, &full[q % STAGES], (kb_begin + q * KPS + j) * BK,
+          tma_load_2d(b + j * TC::B_BYTES, &tm_x, &full[q % STAGES],
+                      (kb_begin + q * KPS + j) * KB_ELEMS,
                       t0);
       };
       // the weights are never written by another kernel: the first stages'
@@ -256,10 +276,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t b_base = a_base + KPS * A_BYTES;
         for (int j = 0; j < stage_kbs(q); ++j) {
 #pragma unroll
-          for (int kk = 0; kk < BK / 16; ++kk) {
-            umma_ss(tmem_acc, sdesc_sw128(a_base + j * A_BYTES + kk * 32, 16, 1024),
-                    sdesc_sw128(b_base + j * TC::B_BYTES + kk * 32, 16, 1024), TC::IDESC,
-                    (q | j | kk) != 0 ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {  // four 32-byte K steps per 128-byte row
+            const uint64_t ad = sdesc_sw128(a_base + j * A_BYTES + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b_base + j * TC::B_BYTES + kk * 32, 16, 1024);
+            if constexpr (F8)
+              umma_ss_f8(tmem_acc, ad, bd, idesc_e4m3_f32(BM, BN), (q | j | kk) != 0 ? 1u : 0u);
+            else
+              umma_ss(tmem_acc, ad, bd, TC::IDESC, (q | j | kk) != 0 ? 1u : 0u);
           }
         }
         umma_commit(&empty[st]);
@@ -279,6 +302,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         float acc = 0.f;
         for (int j = 0; j < p.n_ssq_in; ++j) acc += p.ssq_in[static_cast<size_t>(j) * p.M + tg];
         rs = rsqrtf(acc * p.inv_k + p.eps);
+      }
+      if constexpr (F8) {
+        if (tg < p.M) rs *= p.tok_scale[tg] * *p.w_scale;
       }
       rowscale[t] = rs;
     }
@@ -354,6 +380,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int f = f0 + lane * 4;
       const size_t o = static_cast<size_t>(tg) * p.N + f;
       if (p.epi == EPI_RESID) {
+        if constexpr (F8) {
+          const float sc = rowscale[t];
+          a.x *= sc; a.y *= sc; a.z *= sc; a.w *= sc;
+        }
         float4* xp = reinterpret_cast<float4*>(p.x + o);
         float4 xv = *xp;
         xv.x += a.x; xv.y += a.y; xv.z += a.z; xv.w += a.w;

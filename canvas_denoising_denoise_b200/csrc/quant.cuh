@@ -25,17 +25,25 @@ __device__ __forceinline__ float scale_of(float amax) {
   return amax == 0.f ? 1.f : __fdiv_rn(amax, 448.f);
 }
 
-// One CTA per row; cols a multiple of 8.
+// One CTA per row; cols a multiple of 8.  A thread holds up to REG_CHUNKS
+// 8-element chunks of its row in registers (rows of up to 8192 bf16 are read
+// once); longer rows are read again for the codes.
+constexpr int REG_CHUNKS = 4;
+
 __global__ void __launch_bounds__(THREADS) quantize_rows_kernel(
-    const __nv_bfloat16* __restrict__ in, int cols, uint8_t* __restrict__ out,
+    const __nv_bfloat16* __restrict__ in, int rows, int cols, uint8_t* __restrict__ out,
     float* __restrict__ scales) {
   griddep_wait();
   griddep_launch();
   __shared__ float red[THREADS / 32];
-  const size_t base = static_cast<size_t>(blockIdx.x) * cols;
+  const int row = blockIdx.x;
+  if (row >= rows) return;
+  const size_t base = static_cast<size_t>(row) * cols;
+  uint4 keep[REG_CHUNKS];
   float amax = 0.f;
-  for (int c = threadIdx.x * 8; c < cols; c += THREADS * 8) {
+  for (int i = 0, c = threadIdx.x * 8; c < cols; ++i, c += THREADS * 8) {
     const uint4 raw = *reinterpret_cast<const uint4*>(in + base + c);
+    if (i < REG_CHUNKS) keep[i] = raw;
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
 #pragma unroll
     for (int e = 0; e < 4; ++e) {
@@ -47,17 +55,13 @@ __global__ void __launch_bounds__(THREADS) quantize_rows_kernel(
   for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = amax;
   __syncthreads();
-  if (threadIdx.x < 32) {
-    float a = threadIdx.x < THREADS / 32 ? red[threadIdx.x] : 0.f;
+  float a = red[0];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) a = fmaxf(a, __shfl_xor_sync(0xffffffffu, a, o));
-    if (threadIdx.x == 0) red[0] = a;
-  }
-  __syncthreads();
-  const float s = scale_of(red[0]);
-  if (threadIdx.x == 0) scales[blockIdx.x] = s;
-  for (int c = threadIdx.x * 8; c < cols; c += THREADS * 8) {
-    const uint4 raw = *reinterpret_cast<const uint4*>(in + base + c);
+  for (int w = 1; w < THREADS / 32; ++w) a = fmaxf(a, red[w]);
+  const float s = scale_of(a);
+  if (threadIdx.x == 0) scales[row] = s;
+  for (int i = 0, c = threadIdx.x * 8; c < cols; ++i, c += THREADS * 8) {
+    const uint4 raw = i < REG_CHUNKS ? keep[i] : *reinterpret_cast<const uint4*>(in + base + c);
     const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&raw);
     uint32_t w[2] = {0u, 0u};
 #pragma unroll

@@ -99,6 +99,15 @@ typedef struct dg_layer_weights {
   const void* w_down;  /* [d, F] */
 } dg_layer_weights;
 
+/* e4m3 copies of a layer's projection weights (dg_quantize_e4m3 per tensor). */
+typedef struct dg_layer_weights_e4m3 {
+  const uint8_t* w_qkv;
+  const uint8_t* w_o;
+  const uint8_t* w_up;
+  const uint8_t* w_down;
+  const float* scales;  /* device [4]: the scales of w_qkv, w_o, w_up, w_down */
+} dg_layer_weights_e4m3;
+
 typedef struct dg_model {
   dg_model_cfg cfg;
   const void* embed;                /* bf16 [V, d] */
@@ -110,6 +119,11 @@ typedef struct dg_model {
    * quantised per token each step.  NULL: bf16. */
   const uint8_t* unembed_e4m3;      /* e4m3 [V, d] */
   const float* unembed_scale;       /* device scalar */
+  /* Optional e4m3 projections: when set, every projection of every forward
+   * pass (prefill, denoising, block re-encode) runs on FP8 operands, its bf16
+   * input quantised per token just before it.  Host array of cfg.n_layers
+   * entries, or NULL (bf16). */
+  const dg_layer_weights_e4m3* layers_e4m3;
 } dg_model;
 
 /* Which uncommitted positions a step commits.
@@ -287,9 +301,17 @@ size_t dg_unembed_sample_commit_workspace_bytes(int B, int C, int V);
  *   scalar.  V % 256 == 0, d % 128 == 0.
  * dg_unembed_sample_commit_e4m3 - dg_unembed_sample_commit with the logits of
  *   dg_unembed_e4m3.  Workspace: dg_unembed_sample_commit_workspace_bytes().
+ * dg_linear_e4m3 - dg_linear on e4m3 operands: x_q [M, K] codes with per-row
+ *   scales x_scale (device [M]), w_q [N, K] codes with one scale w_scale
+ *   (device scalar); acc[m, n] = x_scale[m] w_scale sum_k dec(x_q[m, k])
+ *   dec(w_q[n, k]) (fp32 accumulation of exact products), then the epilogue
+ *   of dg_linear.  N % 128 == 0, K % 128 == 0.  No workspace.
  */
 int dg_quantize_e4m3(const void* in, int rows, int cols, int per_row, uint8_t* out,
                      float* scales, void* stream);
+int dg_linear_e4m3(const uint8_t* x_q, const float* x_scale, const uint8_t* w_q,
+                   const float* w_scale, void* out, int M, int N, int K, int epilogue,
+                   void* stream);
 int dg_unembed_e4m3(const uint8_t* h_q, const float* h_scale, const uint8_t* w_q,
                     const float* w_scale, float* logits, int M, int d, int V, void* stream);
 int dg_unembed_sample_commit_e4m3(const uint8_t* h_q, const float* h_scale, const uint8_t* w_q,

@@ -244,3 +244,96 @@ def test_block_driver_e4m3_matches_stepwise_calls(fp8_model):
             break
     assert n == steps
     assert torch.equal(st2.tok, tok_a), "FP8 block driver and step-wise calls must agree"
+
+
+@pytest.fixture(scope="module")
+def fp8_full_model():
+    """Every projection and the unembedding on e4m3 operands."""
+    import canvas_denoising_denoise_b200 as dg
+    w_cpu = synth.make_weights(SHAPE, seed=0)
+    model = dg.DgModel(SHAPE, gpu_weights(w_cpu), fp8_unembed=True, fp8_layers=True)
+    prompt = synth.make_prompt(1, P, SHAPE.vocab, seed=1)
+    return dg, model, M.weights_to_f64(w_cpu), prompt
+
+
+def test_model_keeps_the_oracle_quantised_projections(fp8_full_model):
+    dg, model, w64, _ = fp8_full_model
+    for l, q in enumerate(model.layers_q):
+        for j, name in enumerate(("w_qkv", "w_o", "w_up", "w_down")):
+            wq, ws = fp8.quantize_tensor(w64["layers"][l][name])
+            assert np.array_equal(q[name].cpu().numpy(), wq), (l, name)
+            assert q["scales"].cpu().numpy()[j] == np.float32(ws), (l, name)
+
+
+def test_denoise_logits_e4m3_layers_follow_the_oracle(fp8_full_model):
+    """Prefill and denoising pass with every projection and the unembedding in
+    FP8, against the oracle's FP8 forward.
+
+    Nine quantised products in a row make the FP8 logits of this small random
+    model as sensitive to rounding as to quantisation itself: the oracle's own
+    FP8 logits move by about as much when its bf16 storage rounding is switched
+    off as FP8 moves them from bf16.  So the model-level bar is that
+    sensitivity (the exact pins are the kernel tests above: codes bit for bit,
+    products to fp32 rounding): the GPU must sit within 1.5x of it from the
+    oracle's FP8 logits, and its FP8 logits must differ from its own bf16 ones
+    (the FP8 path runs)."""
+    dg, model, w64, prompt = fp8_full_model
+    canvas = torch.randint(0, SHAPE.vocab, (1, C), generator=torch.Generator().manual_seed(2))
+
+    def gpu_logits(m):
+        st = dg.DgState(SHAPE, 1, P + 2 * C, C)
+        dg.prefill(m, st, prompt.cuda())
+        st.tok.copy_(canvas.to(torch.int32))
+        out = torch.empty((1, C, SHAPE.vocab), dtype=torch.float32, device="cuda")
+        dg.denoise_logits(m, st, out)
+        torch.cuda.synchronize()
+        dg.check_device_errors()
+        return to64(out[0])
+
+    got = gpu_logits(model)
+    bf16_model = dg.DgModel(SHAPE, model.w)
+    got_bf16 = gpu_logits(bf16_model)
+
+    def oracle(bf16_storage):
+        kc, vc = M.empty_cache(OCFG, P + 2 * C)
+        L = M.prefill(OCFG, w64, prompt[0].numpy(), kc, vc, bf16_storage=bf16_storage,
+                      e4m3_layers=True)
+        return M.denoise_logits(OCFG, w64, canvas[0].numpy(), kc, vc, L, bf16_storage=bf16_storage,
+                                e4m3_unembed=True, e4m3_layers=True)
+
+    want = oracle(True)
+    sens = np.linalg.norm(oracle(False) - want) / np.linalg.norm(want)
+    rel = np.linalg.norm(got - want) / np.linalg.norm(want)
+    moved = np.linalg.norm(got - got_bf16) / np.linalg.norm(got_bf16)
+    print(f"gpu vs oracle fp8 {rel:.3e}; oracle rounding sensitivity {sens:.3e}; "
+          f"gpu fp8 vs gpu bf16 {moved:.3e}")
+    assert rel <= 1.5 * sens and rel < 0.1
+    assert moved > 1e-2
+
+
+def test_block_driver_e4m3_layers_matches_stepwise_calls(fp8_full_model):
+    """The FP8 model's block driver equals dg_denoise_logits + dg_sample_commit."""
+    dg, model, _, prompt = fp8_full_model
+    seed, block = 5, 1
+    st = dg.DgState(SHAPE, 1, P + 2 * C, C)
+    dg.prefill(model, st, prompt.cuda())
+    steps = dg.denoise_block(model, st, dg.SamplerSettings(), seed, block)
+    torch.cuda.synchronize()
+    dg.check_device_errors()
+    tok_a = st.tok.clone()
+    st2 = dg.DgState(SHAPE, 1, P + 2 * C, C)
+    dg.prefill(model, st2, prompt.cuda())
+    st2.tok.copy_(torch.from_numpy(S.init_canvas(seed, 0, block, C, SHAPE.vocab)).view(1, C))
+    st2.committed.zero_(); st2.prev_argmax.fill_(-1); st2.seq_status.zero_()
+    logits = torch.empty((1, C, SHAPE.vocab), dtype=torch.float32, device="cuda")
+    settings = dg.SamplerSettings()
+    n = 0
+    for s in range(48):
+        dg.denoise_logits(model, st2, logits)
+        dg.sample_commit(logits, st2.tok, st2.committed, st2.prev_argmax, st2.seq_status,
+                         settings, seed, block, s)
+        n = s + 1
+        if int(st2.seq_status.item()) != 0:
+            break
+    assert n == steps
+    assert torch.equal(st2.tok, tok_a), "FP8 block driver and step-wise calls must agree"

@@ -117,3 +117,51 @@ def test_gelu_epilogue_matches_exact_gelu_to_the_bf16_step():
     # of the bf16 step, so mismatches (midpoint cases) must be rare
     big = ex.abs() >= 1e-2
     assert int((diff & big).sum()) <= 0.01 * int(big.sum())
+
+
+def quant_gpu(t, per_row):
+    import canvas_denoising_denoise_b200 as dg
+    q = torch.empty(t.shape, dtype=torch.uint8, device="cuda")
+    s = torch.empty(t.shape[0] if per_row else 1, dtype=torch.float32, device="cuda")
+    dg.quantize_e4m3(t.cuda(), q, s, per_row=per_row)
+    return q, s
+
+
+# e4m3 operands (128-element k-blocks): K = 128 is one k-block; 8192 splits
+# over a cluster of four; 200 and 1000 rows leave ragged token tiles.
+@pytest.mark.parametrize("Mr,N,K", [(256, 128, 128), (256, 384, 384), (200, 256, 2048),
+                                    (64, 512, 256), (1000, 128, 128), (256, 2048, 2048),
+                                    (256, 2048, 8192)])
+@pytest.mark.parametrize("epi", ["f32", "bf16", "gelu", "resid"])
+def test_linear_e4m3_epilogues(Mr, N, K, epi):
+    """Against the oracle's product of the same codes (exact e4m3 products in fp64)."""
+    import canvas_denoising_denoise_b200 as dg
+    from oracle import fp8
+    x = rand_bf16(Mr, K, seed=1)
+    w = rand_bf16(N, K, scale=K ** -0.5, seed=2)
+    xq, xs = quant_gpu(x, True)
+    wq, ws = quant_gpu(w, False)
+    torch.cuda.synchronize()
+    acc = (fp8.decode(xq.cpu().numpy()) @ fp8.decode(wq.cpu().numpy()).T) * (
+        xs.cpu().numpy().astype(np.float64)[:, None] * np.float64(ws.cpu().numpy()[0]))
+    tight = dict(rel_l2=1e-5, max_abs=1e-4)
+    if epi == "f32":
+        out = torch.empty((Mr, N), dtype=torch.float32, device="cuda")
+        dg.linear_e4m3(xq, xs, wq, ws, out, dg.EPI_F32)
+        want, tol = acc, tight
+    elif epi == "bf16":
+        out = torch.empty((Mr, N), dtype=torch.bfloat16, device="cuda")
+        dg.linear_e4m3(xq, xs, wq, ws, out, dg.EPI_BF16)
+        want, tol = acc, {}
+    elif epi == "gelu":
+        out = torch.empty((Mr, N), dtype=torch.bfloat16, device="cuda")
+        dg.linear_e4m3(xq, xs, wq, ws, out, dg.EPI_GELU_BF16)
+        want, tol = M.gelu(acc), {}
+    else:
+        base = torch.randn((Mr, N), generator=torch.Generator().manual_seed(3))
+        out = base.clone().cuda()
+        dg.linear_e4m3(xq, xs, wq, ws, out, dg.EPI_RESID_F32)
+        want, tol = to64(base) + acc, tight
+    torch.cuda.synchronize()
+    dg.check_device_errors()
+    assert_close(out, want, what=f"e4m3 {epi} {Mr}x{N}x{K}", **tol)
