@@ -311,6 +311,53 @@ def attn_roofline(dg, shape, batch, prefix, peaks, stream):
             "prefix": prefix}
 
 
+def kv_commit_roofline(dg, shape, batch, st, prefix, peaks, stream):
+    """The block K/V commit of every layer (one launch): 2 x its bytes (read +
+    write) over the CUDA-event time, against the measured HBM rate."""
+    import torch
+    nl, hq, hkv, hd = shape.n_layers, shape.n_q_heads, shape.n_kv_heads, shape.head_dim
+    nqkv = (hq + 2 * hkv) * hd
+    qkv = torch.randn((batch, CANVAS, nqkv), device="cuda").to(torch.bfloat16)
+    k_blk = [qkv[:, :, hq * hd:(hq + hkv) * hd]] * nl
+    v_blk = [qkv[:, :, (hq + hkv) * hd:]] * nl
+    flush = L2Flush()
+    times = []
+    for i in range(10):
+        flush()
+        st.cache_len.fill_(prefix)
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        dg.kv_block_commit(k_blk, v_blk, st.k_cache, st.v_cache, st.cache_len, n_kv_heads=hkv,
+                           head_dim=hd, stream=stream)
+        e.record(stream)
+        torch.cuda.synchronize()
+        if i >= 3:
+            times.append(s.elapsed_time(e) / 1000.0)
+    t = statistics.median(times)
+    moved = 2.0 * (2 * nl * batch * hkv * CANVAS * hd * 2)
+    return {"kernel": "kv_commit_kernel", "achieved": round(moved / t / 1e9, 1),
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": round(moved / t / 1e9 / peaks["hbm_gbs"], 4),
+            "bytes": int(moved), "us": round(t * 1e6, 1)}
+
+
+def step_upper_bound(shape, batch, prefix, steps, peaks):
+    """tokens/s <= B*256 / ((steps + 1) * max(F_step / P_bf16, Bytes_step / BW_hbm)) for
+    one block at the workload's prefix (the fused path moves no logits)."""
+    d, nl, hq, hkv, hd, ffn, V = (shape.d, shape.n_layers, shape.n_q_heads, shape.n_kv_heads,
+                                  shape.head_dim, shape.ffn, shape.vocab)
+    M = batch * CANVAS
+    params = nl * ((hq + 2 * hkv) * hd * d + d * hq * hd + 2 * ffn * d)
+    flops = 2.0 * M * params + 4.0 * batch * hq * CANVAS * (prefix + CANVAS) * hd * nl \
+        + 2.0 * M * V * d
+    nbytes = 2.0 * (params + V * d) + 2 * nl * batch * hkv * prefix * hd * 2.0
+    t = max(flops / (peaks["bf16_tflops"] * 1e12), nbytes / (peaks["hbm_gbs"] * 1e9))
+    return {"value": round(M / ((steps + 1) * t), 1), "unit": UNIT,
+            "per_step_tflop": round(flops / 1e12, 3), "per_step_gb": round(nbytes / 1e9, 3),
+            "bound": "tensor" if flops / (peaks["bf16_tflops"] * 1e12) > nbytes / (peaks["hbm_gbs"] * 1e9)
+            else "hbm"}
+
+
 def cpu_baseline_sample(w_cpu, shape, prefix, budget_s=30.0):
     """The CPU oracle on one denoising step of the workload (bounded sample).
 
@@ -686,6 +733,8 @@ def main():
     attn = attn_roofline(dg, shape, batch, prompt_len, peaks, stream)
     samp = (sampler_step_roofline(dg, model, shape, batch, peaks, stream)
             if shape.vocab % 256 == 0 else None)
+    kvc = kv_commit_roofline(dg, shape, batch, st, prompt_len, peaks, stream)
+    ub = step_upper_bound(shape, batch, prompt_len, steps_seen[-1] if steps_seen else 48, peaks)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -708,6 +757,8 @@ def main():
             "roofline": roof,
             "canvas_attn": attn,
             "unembed_sample": samp,
+            "kv_commit": kvc,
+            "upper_bound": ub,
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_val, 2), "unit": UNIT,
                     "h2d_bytes_per_step": int(host_prompt.numel() * 4),

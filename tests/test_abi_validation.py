@@ -1,0 +1,155 @@
+"""Argument checking of the C ABI, on the host: every entry point rejects bad
+arguments with its documented status before it touches device memory, so
+these run without a GPU (the pointers below are never dereferenced).  Also
+the workspace-size queries and the sampler defaults against the pages'
+settings."""
+import ctypes
+import os
+
+import pytest
+
+from conftest import ROOT
+
+OK, INVALID, SHAPE, ALIGN, WS = 0, 1, 2, 3, 4
+P = ctypes.c_void_p(0x100000)       # a 16-byte aligned stand-in for a device pointer
+MIS = ctypes.c_void_p(0x100008)     # 8-byte aligned only
+NULL = None
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from canvas_denoising_denoise_b200 import _lib
+    return _lib.load()
+
+
+@pytest.fixture(scope="module")
+def L():
+    from canvas_denoising_denoise_b200 import _lib
+    return _lib
+
+
+def settings():
+    out = {}
+    with open(os.path.join(ROOT, "tests", "golden", "sampler_settings.txt")) as f:
+        for line in f:
+            if line.strip() and not line.startswith("#"):
+                k, v = line.split()[:2]
+                out[k] = float(v)
+    return out
+
+
+def defaults(lib, L):
+    c = L.SamplerCfg()
+    lib.dg_sampler_defaults(ctypes.byref(c))
+    return c
+
+
+def test_sampler_defaults_are_the_pages_settings(lib, L):
+    c, g = defaults(lib, L), settings()
+    assert c.max_steps == g["max_steps"]
+    assert c.t_start == pytest.approx(g["t_start"]) and c.t_end == pytest.approx(g["t_end"])
+    assert c.stop_entropy == pytest.approx(g["stop_entropy"])
+    assert c.entropy_bound == pytest.approx(g["select_entropy"])
+    assert g["commit_min"] <= c.commit_k <= g["commit_max"]
+    assert c.selection == 0 and c.unselected_policy == 0
+
+
+def test_unembed_rejects_bad_arguments(lib):
+    assert lib.dg_unembed(NULL, P, P, 256, 2048, 262144, None, 0, None) == INVALID
+    assert lib.dg_unembed(P, P, P, 256, 2048, 1000, None, 0, None) == SHAPE       # V % 128
+    assert lib.dg_unembed(P, P, P, 256, 100, 262144, None, 0, None) == SHAPE      # d % 64
+    assert lib.dg_unembed(MIS, P, P, 256, 2048, 262144, None, 0, None) == ALIGN
+    assert lib.dg_unembed(P, P, P, 0, 2048, 262144, None, 0, None) != OK
+
+
+def test_linear_rejects_bad_arguments(lib):
+    assert lib.dg_linear(P, P, P, 256, 2048, 2048, 7, None, 0, None) == INVALID   # epilogue
+    assert lib.dg_linear(P, P, P, 256, 200, 2048, 1, None, 0, None) == SHAPE      # N % 128
+    assert lib.dg_linear(P, P, P, 256, 256, 100, 1, None, 0, None) == SHAPE       # K % 64
+    assert lib.dg_linear(P, MIS, P, 256, 256, 256, 1, None, 0, None) == ALIGN
+    assert lib.dg_linear_e4m3(P, P, P, P, P, 256, 256, 192, 1, None) == SHAPE     # K % 128
+    assert lib.dg_linear_e4m3(P, NULL, P, P, P, 256, 256, 256, 1, None) == INVALID
+
+
+def test_quantize_and_fp8_unembedding_reject_bad_arguments(lib):
+    assert lib.dg_quantize_e4m3(P, 4, 12, 1, P, P, None) == SHAPE                  # cols % 8
+    assert lib.dg_quantize_e4m3(NULL, 4, 16, 1, P, P, None) == INVALID
+    assert lib.dg_quantize_e4m3(P, 4, 16, 1, MIS, P, None) == ALIGN
+    assert lib.dg_unembed_e4m3(P, P, P, P, P, 256, 2048, 1024 + 128, None) == SHAPE  # V % 256
+    assert lib.dg_unembed_e4m3(P, P, P, P, P, 256, 2048 + 64, 1024, None) == SHAPE   # d % 128
+
+
+def test_sample_commit_rejects_bad_arguments(lib, L):
+    c = defaults(lib, L)
+    ws = lib.dg_sample_commit_workspace_bytes(1, 256, 262144)
+    args = lambda C, V, cfg, w, wn: lib.dg_sample_commit(  # noqa: E731
+        P, P, P, P, P, ctypes.byref(cfg), 0, 0, 0, 1, C, V, None, w, wn, None)
+    assert args(1025, 262144, c, P, ws) == SHAPE                                   # C > 1024
+    assert args(256, 262146, c, P, ws) == SHAPE                                    # V % 4
+    assert args(256, 262144, c, P, ws - 16) == WS
+    assert args(256, 262144, c, NULL, ws) == WS
+    bad = defaults(lib, L)
+    bad.max_steps = 0
+    assert args(256, 262144, bad, P, ws) == INVALID
+    bad = defaults(lib, L)
+    bad.selection = 2
+    assert args(256, 262144, bad, P, ws) == INVALID
+    bad = defaults(lib, L)
+    bad.t_end = 0.0
+    assert args(256, 262144, bad, P, ws) == INVALID
+
+
+def test_canvas_attn_rejects_bad_arguments(lib):
+    def call(hd=128, Hq=16, Hkv=8, mask=0, ld=16 * 128, ldkv=8 * 128, q=P, maxp=4096, lmax=4352):
+        return lib.dg_canvas_attn(q, ld, P, P, ldkv, P, P, P, maxp, lmax, P, ld, None, 1, Hq,
+                                  Hkv, 256, hd, 0.088, mask, P, 1 << 30, None)
+    assert call(hd=96, ld=16 * 96, ldkv=8 * 96) == SHAPE
+    assert call(Hq=12, Hkv=8) == INVALID          # Hq % Hkv
+    assert call(mask=5) == INVALID
+    assert call(maxp=5000) == INVALID             # prefix beyond the cache
+    assert call(ld=16 * 128 - 8) == ALIGN         # leading dimension below Hq * hd
+    assert call(q=MIS) == ALIGN
+    assert call(q=NULL) == INVALID
+
+
+def test_workspace_queries(lib, L):
+    assert lib.dg_sample_commit_workspace_bytes(0, 256, 512) == 0
+    assert lib.dg_unembed_sample_commit_workspace_bytes(1, 256, 1000) == 0         # V % 256
+    # the fused path's partials: tokens x 3 x (vocabulary segments per token
+    # tile), and a wider batch spreads the pairs over more token tiles
+    a = lib.dg_unembed_sample_commit_workspace_bytes(1, 256, 262144)
+    b = lib.dg_unembed_sample_commit_workspace_bytes(8, 256, 262144)
+    assert a > 0 and b > 0
+    assert lib.dg_canvas_attn_workspace_bytes(1, 16, 8, 256, 128, 4096) > 0
+    cfg = L.ModelCfg(2048, 24, 16, 8, 128, 8192, 262144, 1e-6)
+    w1 = lib.dg_denoise_block_workspace_bytes(ctypes.byref(cfg), 1, 256, 4352)
+    w8 = lib.dg_denoise_block_workspace_bytes(ctypes.byref(cfg), 8, 256, 4352)
+    assert 0 < w1 < w8
+    assert lib.dg_denoise_block_workspace_bytes(ctypes.byref(cfg), 0, 256, 4352) == 0
+
+
+def test_model_checks_reject_bad_configurations(lib, L):
+    layers = (L.LayerWeights * 2)(*[L.LayerWeights(P.value, P.value, P.value, P.value)] * 2)
+    st = L.State()
+
+    def model(**kw):
+        c = dict(d=256, n_layers=2, n_q_heads=4, n_kv_heads=2, head_dim=64, ffn=1024, vocab=512,
+                 eps=1e-6)
+        c.update(kw)
+        cfg = L.ModelCfg(c["d"], c["n_layers"], c["n_q_heads"], c["n_kv_heads"], c["head_dim"],
+                         c["ffn"], c["vocab"], c["eps"])
+        return L.Model(cfg, P.value, P.value, ctypes.cast(layers, ctypes.POINTER(L.LayerWeights)),
+                       None, None, None)
+
+    scfg = defaults(lib, L)
+    steps = ctypes.c_int(0)
+
+    def run(m):
+        return lib.dg_denoise_block(ctypes.byref(m), ctypes.byref(st), ctypes.byref(scfg), 0, 0,
+                                    ctypes.byref(steps), P, 1 << 30, None)
+    assert run(model(head_dim=96)) == SHAPE
+    assert run(model(n_q_heads=3)) == INVALID      # Hq % Hkv
+    assert run(model(ffn=1000)) == SHAPE           # not a multiple of 128
+    m = model()
+    m.unembed_e4m3 = P.value                       # an e4m3 unembedding without its scale
+    assert run(m) == INVALID
