@@ -43,6 +43,15 @@ bool pdl_enabled() {
   return on;
 }
 
+// The denoising loop replays each step as a CUDA graph unless DG_GRAPHS=0.
+bool graphs_enabled() {
+  static const bool on = [] {
+    const char* e = getenv("DG_GRAPHS");
+    return !(e && e[0] == '0');
+  }();
+  return on;
+}
+
 // Launch with programmatic stream serialization (the kernel must call
 // griddep_wait before touching its predecessors' data) and an optional
 // cluster shape along z.
@@ -892,6 +901,45 @@ int noalloc_scratch(void** out) {
 // ===========================================================================
 // C ABI
 // ===========================================================================
+// A captured denoising step: the launches are recorded on a private stream
+// (launch counts included) and replayed with cudaGraphLaunch on the caller's
+// stream.  A failed capture leaves exec null and the caller launches directly.
+struct StepGraph {
+  cudaGraph_t graph = nullptr;
+  cudaGraphExec_t exec = nullptr;
+  unsigned long long launches = 0;  // kernels per replay
+  ~StepGraph() {
+    if (exec) cudaGraphExecDestroy(exec);
+    if (graph) cudaGraphDestroy(graph);
+  }
+  template <class F>
+  int capture(F&& enqueue) {
+    static cudaStream_t streams[64] = {};  // one private capture stream per device
+    int dev = 0;
+    DG_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= 64) return DG_OK;  // no capture: launch the steps directly
+    if (!streams[dev]) DG_CUDA(cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking));
+    cudaStream_t cs = streams[dev];
+    const unsigned long long c0 = g_launches.load(std::memory_order_relaxed);
+    DG_CUDA(cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal));
+    const int rc = enqueue(cs);
+    const cudaError_t end = cudaStreamEndCapture(cs, &graph);
+    launches = g_launches.load(std::memory_order_relaxed) - c0;
+    g_launches.fetch_sub(launches, std::memory_order_relaxed);  // recorded, not run
+    if (rc != DG_OK) return rc;
+    if (end != cudaSuccess || cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess) {
+      (void)cudaGetLastError();
+      exec = nullptr;  // launch the steps directly instead
+    }
+    return DG_OK;
+  }
+  int launch(cudaStream_t s) {
+    DG_CUDA(cudaGraphLaunch(exec, s));
+    count_launch(launches);
+    return DG_OK;
+  }
+};
+
 extern "C" {
 
 const char* dg_status_string(int status) {
@@ -1309,28 +1357,48 @@ int dg_denoise_block(const dg_model* m, dg_state* st, const dg_sampler_cfg* cfg,
   const bool fp8 = m->unembed_e4m3 != nullptr;  // check_model: vocab % 256 == 0 then
   Fwd fl = f;
   fl.unembed_elsewhere = fused;
-  for (int it = 0; it < cfg->max_steps; ++it) {
-    DG_TRY(run_forward(fl, st->tok, logits, s));
+  // one denoising step: forward pass, unembedding + sampler, step advance
+  auto enqueue_step = [&](cudaStream_t q) -> int {
+    DG_TRY(run_forward(fl, st->tok, logits, q));
     if (fused && fp8) {
       // the hidden states quantised per token, then the e4m3 unembedding + sampler
-      DG_TRY(quantize_hidden(fl, s));
+      DG_TRY(quantize_hidden(fl, q));
       const Fp8Scales f8{(const float*)(ws + L.as), m->unembed_scale};
       DG_TRY(launch_unembed_sample(ws + L.aq, m->unembed_e4m3, m->cfg.d,
                                    (const float*)(ws + L.ssq_x), m->cfg.d / 128, 1.f / m->cfg.d,
                                    m->cfg.eps, st->tok, st->committed, st->prev_argmax,
-                                   st->seq_status, sp, nullptr, ws + L.spart, s, &f8));
-    } else if (fused)
+                                   st->seq_status, sp, nullptr, ws + L.spart, q, &f8));
+    } else if (fused) {
       DG_TRY(launch_unembed_sample(ws + L.xn, m->unembed, m->cfg.d, (const float*)(ws + L.ssq_x),
                                    m->cfg.d / 128, 1.f / m->cfg.d, m->cfg.eps, st->tok,
                                    st->committed, st->prev_argmax, st->seq_status, sp, nullptr,
-                                   ws + L.spart, s));
-    else
+                                   ws + L.spart, q));
+    } else {
       DG_TRY(launch_sample(logits, st->tok, st->committed, st->prev_argmax, st->seq_status, sp,
-                           nullptr, ws + L.spart, s));
-    dg::step_advance_kernel<<<1, 256, 0, s>>>(B, cfg->max_steps, st->seq_status, st->step,
+                           nullptr, ws + L.spart, q));
+    }
+    dg::step_advance_kernel<<<1, 256, 0, q>>>(B, cfg->max_steps, st->seq_status, st->step,
                                               running);
     count_launch();
     DG_CUDA(cudaGetLastError());
+    return DG_OK;
+  };
+  // Steps after the first replay one captured graph of the step's launches
+  // (the step index lives on the device, so every replay is the next step):
+  // the GPU dispatches a graph's kernels with less overhead than stream
+  // launches.  Not when the caller's stream is itself being captured.
+  StepGraph g;
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  DG_CUDA(cudaStreamIsCapturing(s, &cap));
+  const bool use_graph = graphs_enabled() && cap == cudaStreamCaptureStatusNone &&
+                         cfg->max_steps > 2;
+  for (int it = 0; it < cfg->max_steps; ++it) {
+    if (use_graph && it == 1) DG_TRY(g.capture(enqueue_step));
+    if (g.exec) {
+      DG_TRY(g.launch(s));
+    } else {
+      DG_TRY(enqueue_step(s));
+    }
     int32_t host_running = 0;
     DG_CUDA(cudaMemcpyAsync(&host_running, running, sizeof(int32_t), cudaMemcpyDeviceToHost, s));
     DG_CUDA(cudaStreamSynchronize(s));
