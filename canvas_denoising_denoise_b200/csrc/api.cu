@@ -479,9 +479,10 @@ int launch_attn(const void* q, int ldq, const void* k_new, const void* v_new, in
 // Sampler
 // ---------------------------------------------------------------------------
 int sample_chunking(int V, int* chunk) {
-  // chunks of >= 16384 elements (>= 64 per thread), at most 64 per row, in
+  // chunks of >= 65536 elements (>= 256 per thread: the CTA's closing
+  // reduction is then a small share of its work), at most 64 per row, in
   // multiples of 4 elements
-  int nchunk = std::max(1, std::min(64, V / 16384));
+  int nchunk = std::max(1, std::min(64, V / 65536));
   int c = cdiv(V, nchunk);
   c = (c + 3) / 4 * 4;
   nchunk = cdiv(V, c);
