@@ -317,9 +317,11 @@ def kv_commit_roofline(dg, shape, batch, st, prefix, peaks, stream):
     import torch
     nl, hq, hkv, hd = shape.n_layers, shape.n_q_heads, shape.n_kv_heads, shape.head_dim
     nqkv = (hq + 2 * hkv) * hd
-    qkv = torch.randn((batch, CANVAS, nqkv), device="cuda").to(torch.bfloat16)
-    k_blk = [qkv[:, :, hq * hd:(hq + hkv) * hd]] * nl
-    v_blk = [qkv[:, :, (hq + hkv) * hd:]] * nl
+    # each layer its own QKV output, as in the re-encode (no source re-read from L2)
+    qkv = [torch.randn((batch, CANVAS, nqkv), device="cuda").to(torch.bfloat16)
+           for _ in range(nl)]
+    k_blk = [t[:, :, hq * hd:(hq + hkv) * hd] for t in qkv]
+    v_blk = [t[:, :, (hq + hkv) * hd:] for t in qkv]
     flush = L2Flush()
     times = []
     for i in range(10):
@@ -446,6 +448,8 @@ def run_kernel_bench(args):
     --kernel gemm     one projection y = x w^T for --shape M,N,K (bf16 out).
     --kernel unembed  the unembedding alone, logits to memory.
     --kernel fused    the unembedding fused with a sampler step, and unfused.
+    --kernel kvcommit the block K/V commit of the full model (24 layers) at
+                      prefix --prefix (default 4096), B = --batch.
     """
     import torch
     import canvas_denoising_denoise_b200 as dg
@@ -508,6 +512,13 @@ def run_kernel_bench(args):
                     "gbs": round(byts / t / 1e9, 1),
                     "frac_hbm_peak": round(byts / t / 1e9 / peaks["hbm_gbs"], 4),
                     "committed_tokens_per_s": round(16 * B / t, 1)})
+    elif args.kernel == "kvcommit":
+        # the block K/V commit of the full model (24 layers) at the given prefix
+        shape = synth.FULL
+        prefix = args.prefix or 4096
+        st = dg.DgState(shape, args.batch, prefix + CANVAS, CANVAS)
+        out.append(kv_commit_roofline(dg, shape, args.batch, st, prefix, peaks,
+                                      torch.cuda.current_stream()))
     elif args.kernel == "unembed":
         # the unembedding launch of the full workload: logits [256, 262144] fp32
         M, d, V = 256 * args.batch, 2048, 262144
@@ -626,7 +637,8 @@ def main():
                          "8 canvases after a 2048-token prompt at B = 1 / 8")
     ap.add_argument("--impl", default="dg", choices=["dg", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--kernel", choices=["attn", "sampler", "gemm", "unembed", "fused"],
+    ap.add_argument("--kernel", choices=["attn", "sampler", "gemm", "unembed", "fused",
+                                         "kvcommit"],
                     default=None,
                     help="time one kernel alone instead of the denoising step")
     ap.add_argument("--prefix", type=int, default=0)

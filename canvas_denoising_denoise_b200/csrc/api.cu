@@ -651,9 +651,13 @@ int launch_kv_commit(const void* const* k_blk, const void* const* v_blk, int ld_
     tab.v_cache[l] = (__nv_bfloat16*)v_cache[l];
   }
   dg::KVParams p{n_layers, B, Hkv, C, hd, lmax, ld_blk, cache_len};
-  const size_t total = (size_t)n_layers * 2 * B * Hkv * C * (hd / 8);
-  const int blocks = (int)std::min<size_t>((total + 255) / 256, (size_t)kNumSMs * 16);
-  dg::kv_commit_kernel<<<std::max(1, blocks), 256, 0, s>>>(tab, p);
+  // one grid row per (layer, K or V, sequence, kv head); x covers its vectors
+  const int groups = n_layers * 2 * B * Hkv;
+  const int nvec = C * (hd / 8);
+  const int bx = std::max(1, std::min(cdiv(nvec, dg::KV_THREADS * dg::KV_UNROLL),
+                                      cdiv(8 * kNumSMs, std::max(1, groups))));
+  if (groups > 65535) return fail(DG_ERR_UNSUPPORTED_SHAPE, "kv commit: too many row groups");
+  dg::kv_commit_kernel<<<dim3(bx, groups), dg::KV_THREADS, 0, s>>>(tab, p);
   count_launch();
   DG_CUDA(cudaGetLastError());
   return DG_OK;
@@ -1258,8 +1262,10 @@ int dg_kv_block_commit(const void* const* k_blk, const void* const* v_blk, int l
   if (n_layers <= 0 || n_layers > dg::KV_MAX_LAYERS || B <= 0 || Hkv <= 0 || C <= 0 || lmax <= 0)
     return fail(DG_ERR_INVALID_ARG, "dg_kv_block_commit: bad sizes (n_layers <= %d)",
                 dg::KV_MAX_LAYERS);
-  if (hd % 8 || ld_blk % 8 || ld_blk < Hkv * hd)
-    return fail(DG_ERR_ALIGNMENT, "dg_kv_block_commit: hd and ld_blk must be multiples of 8");
+  if (hd != 64 && hd != 128)
+    return fail(DG_ERR_UNSUPPORTED_SHAPE, "dg_kv_block_commit: head_dim %d not in {64,128}", hd);
+  if (ld_blk % 8 || ld_blk < Hkv * hd)
+    return fail(DG_ERR_ALIGNMENT, "dg_kv_block_commit: ld_blk must be a multiple of 8, >= Hkv hd");
   for (int l = 0; l < n_layers; ++l)
     if (!aligned16(k_blk[l]) || !aligned16(v_blk[l]) || !aligned16(k_cache[l]) ||
         !aligned16(v_cache[l]) || !k_blk[l] || !v_blk[l] || !k_cache[l] || !v_cache[l])

@@ -5,10 +5,10 @@
 // block starts (aiexpert.news architecture paragraph: each fully denoised
 // block is committed and a new canvas is conditioned on the history).
 //
-// Pure data movement: each thread moves one 16-byte vector (8 bf16) from the
-// token-major block K/V [B, C, ld] into the head-major cache [B, Hkv, lmax, hd]
-// at row cache_len[b] + t.  A second one-CTA kernel then bumps cache_len, so
-// every copy reads the same base row.
+// Pure data movement: 16-byte vectors (8 bf16) from the token-major block K/V
+// [B, C, ld] into the head-major cache [B, Hkv, lmax, hd] at rows
+// cache_len[b] + t.  A second one-CTA kernel then bumps cache_len, so every
+// copy reads the same base row.
 #pragma once
 
 #include "dg_common.cuh"
@@ -29,33 +29,53 @@ struct KVParams {
   const int32_t* cache_len;
 };
 
-// Grid-stride over n_layers * 2 (K, V) * B * Hkv * C * (hd / 8) vectors.
-__global__ void kv_commit_kernel(const __grid_constant__ KVTables tab, KVParams p) {
-  const int vec_per_row = p.hd / 8;
-  const size_t per_kv = static_cast<size_t>(p.B) * p.Hkv * p.C * vec_per_row;
-  const size_t total = per_kv * 2 * p.n_layers;
-  for (size_t idx = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; idx < total;
-       idx += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    size_t r = idx;
-    const int v8 = static_cast<int>(r % vec_per_row); r /= vec_per_row;
-    const int t = static_cast<int>(r % p.C); r /= p.C;
-    const int g = static_cast<int>(r % p.Hkv); r /= p.Hkv;
-    const int b = static_cast<int>(r % p.B); r /= p.B;
-    const int which = static_cast<int>(r % 2); r /= 2;
-    const int l = static_cast<int>(r);
-    const int base = p.cache_len[b];
-    if (base < 0 || base + p.C > p.lmax) {
-      if (v8 == 0 && t == 0 && g == 0 && which == 0 && l == 0)
-        raise_error(ERR_CHECK | 0x401, static_cast<uint32_t>(b));
-      continue;
+constexpr int KV_THREADS = 256;
+constexpr int KV_UNROLL = 4;
+
+// Grid: y = one row group (layer, K or V, sequence, kv head), x strides over
+// its C * hd / 8 vectors.  Within a row group the destination rows
+// [cache_len, cache_len + C) are one contiguous run of the head-major cache
+// and each source token row is hd contiguous elements, so consecutive threads
+// move consecutive 16-byte vectors; the index arithmetic is one shift and one
+// mask per vector (hd is 64 or 128).
+__global__ void __launch_bounds__(KV_THREADS) kv_commit_kernel(const __grid_constant__ KVTables tab,
+                                                               KVParams p) {
+  int y = blockIdx.y;
+  const int g = y % p.Hkv;
+  y /= p.Hkv;
+  const int b = y % p.B;
+  y /= p.B;
+  const int which = y & 1;
+  const int l = y >> 1;
+  const int base = p.cache_len[b];
+  if (base < 0 || base + p.C > p.lmax) {
+    if (blockIdx.x == 0 && threadIdx.x == 0 && g == 0 && which == 0 && l == 0)
+      raise_error(ERR_CHECK | 0x401, static_cast<uint32_t>(b));
+    return;
+  }
+  const int shift = p.hd == 128 ? 4 : 3;  // log2(hd / 8)
+  const int nvec = p.C << shift;
+  const __nv_bfloat16* src = (which == 0 ? tab.k_blk[l] : tab.v_blk[l]) +
+                             static_cast<size_t>(b) * p.C * p.ld_blk +
+                             static_cast<size_t>(g) * p.hd;
+  __nv_bfloat16* dst = (which == 0 ? tab.k_cache[l] : tab.v_cache[l]) +
+                       ((static_cast<size_t>(b) * p.Hkv + g) * p.lmax + base) * p.hd;
+  // KV_UNROLL loads in flight per thread before their stores
+  const int stride = gridDim.x * KV_THREADS;
+  for (int i0 = blockIdx.x * KV_THREADS + threadIdx.x; i0 < nvec; i0 += KV_UNROLL * stride) {
+    uint4 val[KV_UNROLL];
+#pragma unroll
+    for (int u = 0; u < KV_UNROLL; ++u) {
+      const int i = i0 + u * stride;
+      if (i < nvec)
+        val[u] = __ldg(reinterpret_cast<const uint4*>(
+            src + static_cast<size_t>(i >> shift) * p.ld_blk + (i & ((1 << shift) - 1)) * 8));
     }
-    const __nv_bfloat16* src = (which == 0 ? tab.k_blk[l] : tab.v_blk[l]) +
-                               (static_cast<size_t>(b) * p.C + t) * p.ld_blk +
-                               static_cast<size_t>(g) * p.hd + v8 * 8;
-    __nv_bfloat16* dst = (which == 0 ? tab.k_cache[l] : tab.v_cache[l]) +
-                         ((static_cast<size_t>(b) * p.Hkv + g) * p.lmax + base + t) * p.hd +
-                         v8 * 8;
-    *reinterpret_cast<uint4*>(dst) = __ldg(reinterpret_cast<const uint4*>(src));
+#pragma unroll
+    for (int u = 0; u < KV_UNROLL; ++u) {
+      const int i = i0 + u * stride;
+      if (i < nvec) *reinterpret_cast<uint4*>(dst + static_cast<size_t>(i) * 8) = val[u];
+    }
   }
 }
 

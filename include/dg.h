@@ -351,9 +351,10 @@ int dg_sample_commit_noalloc(const float* logits, int32_t* tok, uint8_t* committ
  * For each layer l, sequence b, kv head g, row t < C:
  *   k_cache[l][b, g, cache_len[b] + t, :] = k_blk[l][(b*C + t)*ld_blk + g*hd ...]
  * (same for v), then cache_len[b] += C.  Tables k_blk, v_blk, k_cache,
- * v_cache are host arrays of n_layers device pointers (n_layers <= 128).
- * A sequence with cache_len[b] + C > lmax is skipped and the device error
- * word records DG_ERR_DEVICE_CHECK.
+ * v_cache are host arrays of n_layers device pointers (n_layers <= 64);
+ * hd is 64 or 128 (DG_ERR_UNSUPPORTED_SHAPE otherwise).  A sequence with
+ * cache_len[b] + C > lmax is skipped and the device error word records
+ * DG_ERR_DEVICE_CHECK.
  */
 int dg_kv_block_commit(const void* const* k_blk, const void* const* v_blk, int ld_blk,
                        void* const* k_cache, void* const* v_cache, int32_t* cache_len,

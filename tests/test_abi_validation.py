@@ -153,3 +153,15 @@ def test_model_checks_reject_bad_configurations(lib, L):
     m = model()
     m.unembed_e4m3 = P.value                       # an e4m3 unembedding without its scale
     assert run(m) == INVALID
+
+
+def test_kv_block_commit_rejects_bad_arguments(lib):
+    arr = ctypes.c_void_p * 2
+    tab = arr(P.value, P.value)
+    call = lambda hd, ld=8 * 128, nl=2: lib.dg_kv_block_commit(  # noqa: E731
+        tab, tab, ld, tab, tab, P, nl, 1, 8, 256, hd, 4352, None)
+    assert call(96, ld=8 * 96) == SHAPE            # head_dim not 64 or 128
+    assert call(128, ld=8 * 128 - 8) == ALIGN      # leading dimension below Hkv * hd
+    assert call(128, nl=65) == INVALID             # more layers than the tables hold
+    assert lib.dg_kv_block_commit(tab, tab, 1024, tab, tab, NULL, 2, 1, 8, 256, 128, 4352,
+                                  None) == INVALID
