@@ -22,10 +22,13 @@
  *     thread-local detail message for the last failure in this thread.
  *   - No C++ exception crosses this boundary.
  *   - Ownership: the caller allocates and owns every device buffer.  The
- *     library never allocates device memory.  Scratch space comes from a
- *     caller-supplied workspace whose size the *_workspace_bytes() queries
- *     return.  Host arrays passed in (pointer tables, structs) are read during
- *     the call only.
+ *     library never allocates device memory (the driver-side resources of
+ *     the CUDA graph that dg_denoise_block instantiates aside; see there).
+ *     Scratch space comes from a caller-supplied workspace whose size the
+ *     *_workspace_bytes() queries return.  Host arrays passed in (pointer
+ *     tables, structs) are read during the call only.
+ *   - One host thread at a time: the library keeps a little process-wide
+ *     state (kernel attributes set once, a capture stream per device).
  *   - All device work is enqueued on the caller's stream (a cudaStream_t passed
  *     as void*; NULL is the legacy default stream) and is asynchronous, except
  *     where a function says it synchronises.  Results are deterministic: the
@@ -387,6 +390,10 @@ int dg_denoise_logits(const dg_model* m, const dg_state* st, float* logits,
  * (0, pos | 2 << 24, 0, block)), runs sampler steps until every sequence has
  * stopped (dg_sample_commit semantics), then the causal re-encode and the
  * block commit.  Synchronises `stream` once per step to read the stop state.
+ * Steps after the first replay a CUDA graph of one step's launches, captured
+ * on a private stream of the library (set DG_GRAPHS=0 in the environment to
+ * launch every step directly; a stream that is itself being captured always
+ * gets direct launches).
  * steps_taken (host, may be NULL) receives the largest step count over the batch.
  * Workspace: dg_denoise_block_workspace_bytes().
  */
