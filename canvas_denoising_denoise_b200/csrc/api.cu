@@ -317,11 +317,97 @@ int launch_gemm(const void* x, const void* w, int M, int N, int K, const GemmPla
   return DG_OK;
 }
 
-// y = epilogue(x w^T) with the split plan chosen for this shape (e4m3
-// operands with their scales when f8 is set: 128-element k-blocks).
+// Projections with many tokens run on the persistent CTA-pair pipeline
+// (unembed.cuh, 256 x 256 tiles, double-buffered accumulators) when its tiles
+// fill the pairs at least once; fewer tokens take the split-K GEMM.
+bool proj_use_pair(int M, int N, int K, bool f8) {
+  const int kbe = f8 ? 128 : dg::gemm::BK;
+  if (N % dg::unembed::TILE || K % kbe || K / kbe < 4) return false;
+  return (N / dg::unembed::TILE) * cdiv(M, dg::unembed::TILE) >= kNumSMs / 2;
+}
+
+bool proj_attr_done = false;
+
+template <int KPS, bool F8>
+cudaError_t proj_set_attrs() {
+  namespace ue = dg::unembed;
+  namespace gm = dg::gemm;
+  cudaError_t e;
+  const int smem = ue::SMEM_BYTES;
+  const auto a = cudaFuncAttributeMaxDynamicSharedMemorySize;
+  if ((e = cudaFuncSetAttribute(ue::proj_pair_kernel<KPS, F8, gm::EPI_F32>, a, smem))) return e;
+  if ((e = cudaFuncSetAttribute(ue::proj_pair_kernel<KPS, F8, gm::EPI_BF16>, a, smem))) return e;
+  if ((e = cudaFuncSetAttribute(ue::proj_pair_kernel<KPS, F8, gm::EPI_GELU>, a, smem))) return e;
+  return cudaFuncSetAttribute(ue::proj_pair_kernel<KPS, F8, gm::EPI_RESID>, a, smem);
+}
+
+template <int KPS, bool F8>
+decltype(&dg::unembed::proj_pair_kernel<1, false, 0>) proj_kernel(int epi) {
+  namespace ue = dg::unembed;
+  namespace gm = dg::gemm;
+  switch (epi) {
+    case gm::EPI_F32: return ue::proj_pair_kernel<KPS, F8, gm::EPI_F32>;
+    case gm::EPI_GELU: return ue::proj_pair_kernel<KPS, F8, gm::EPI_GELU>;
+    case gm::EPI_RESID: return ue::proj_pair_kernel<KPS, F8, gm::EPI_RESID>;
+    default: return ue::proj_pair_kernel<KPS, F8, gm::EPI_BF16>;
+  }
+}
+
+int launch_proj_pair(const void* x, const void* w, int M, int N, int K, const GemmEpi& e,
+                     cudaStream_t s, const Fp8Scales* f8) {
+  namespace ue = dg::unembed;
+  if (!proj_attr_done) {
+    DG_CUDA((proj_set_attrs<1, false>()));
+    DG_CUDA((proj_set_attrs<2, false>()));
+    DG_CUDA((proj_set_attrs<1, true>()));
+    DG_CUDA((proj_set_attrs<2, true>()));
+    proj_attr_done = true;
+  }
+  CUtensorMap tw, tx;
+  if (f8) {
+    DG_TRY(make_tmap_u8(&tw, w, K, N, (uint64_t)K, ue::HALF));
+    DG_TRY(make_tmap_u8(&tx, x, K, M, (uint64_t)K, ue::HALF));
+  } else {
+    DG_TRY(make_tmap(&tw, w, K, N, (uint64_t)K * 2, ue::HALF));
+    DG_TRY(make_tmap(&tx, x, K, M, (uint64_t)K * 2, ue::HALF));
+  }
+  ue::ProjParams p;
+  p.M = M; p.N = N; p.K = K;
+  p.n_ttiles = cdiv(M, ue::TILE);
+  p.n_tiles = (N / ue::TILE) * p.n_ttiles;
+  p.n_pairs = std::min(kNumSMs / 2, p.n_tiles);
+  p.epi = e.epi;
+  p.out_f32 = e.out_f32;
+  p.out_bf16 = e.out_bf16;
+  p.x = e.x;
+  p.ssq_in = e.ssq_in; p.n_ssq_in = e.n_ssq_in; p.inv_k = e.inv_k; p.eps = e.eps;
+  p.ssq_out = e.ssq_out;
+  p.tok_scale = f8 ? f8->tok : nullptr;
+  p.w_scale = f8 ? f8->w : nullptr;
+  const int nkb = K / (f8 ? 128 : dg::gemm::BK);
+  (void)nkb;
+  auto* kern = f8 ? proj_kernel<1, true>(e.epi) : proj_kernel<1, false>(e.epi);
+  DG_CUDA(launch_cluster(kern, dim3(2 * p.n_pairs), dim3(ue::threads_for(ue::STORE_EPI_WARPS)),
+                         ue::SMEM_BYTES, s, dim3(2, 1, 1), tw, tx, p));
+  count_launch();
+  return DG_OK;
+}
+
+// y = epilogue(x w^T) with the plan chosen for this shape (e4m3 operands with
+// their scales when f8 is set: 128-element k-blocks).  EPI_RESID writes its
+// sums of squares per 128 features on the split-K GEMM and per 32 on the
+// pair pipeline (see ssq_group).
 int linear(const void* x, const void* w, int M, int N, int K, const GemmEpi& e,
            cudaStream_t s, const Fp8Scales* f8 = nullptr) {
+  if (proj_use_pair(M, N, K, f8 != nullptr)) return launch_proj_pair(x, w, M, N, K, e, s, f8);
   return launch_gemm(x, w, M, N, K, plan_gemm(M, N, K, f8 ? 128 : dg::gemm::BK), e, s, f8);
+}
+
+// Features per sum-of-squares partial of the residual stream in a forward
+// pass over M tokens: 32 when its residual projections (N = d) run on the
+// pair pipeline, else 128.
+int ssq_group(const dg_model_cfg& c, int M, bool f8) {
+  return proj_use_pair(M, c.d, c.n_q_heads * c.head_dim, f8) ? 32 : 128;
 }
 
 // logits = rs * (h w_u^T).  Vocabularies that are a multiple of 256 run on
@@ -743,8 +829,8 @@ FwdLayout fwd_layout(const dg_model_cfg& c, int B, int Lq, int max_prefix, bool 
   L.qkv = take((size_t)M * nqkv * 2);
   L.ao = take((size_t)M * hqd * 2);
   L.up = take((size_t)M * c.ffn * 2);
-  L.ssq_x = take((size_t)(c.d / 128) * M * 4);
-  L.ssq_h = take((size_t)(c.d / 128) * M * 4);
+  L.ssq_x = take((size_t)(c.d / 32) * M * 4);  // per 32 or 128 features (ssq_group)
+  L.ssq_h = take((size_t)(c.d / 32) * M * 4);
   L.attn = take(attn_ws_bytes(B, c.n_q_heads, c.n_kv_heads, Lq, c.head_dim, max_prefix));
   L.logits = take(logits ? (size_t)M * c.vocab * 4 : 0);
   L.spart = take(logits ? std::max(sample_ws_bytes(B, Lq, c.vocab),
@@ -803,10 +889,11 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
   float* ssq_h = (float*)(f.ws + f.L.ssq_h);
   void* aws = f.ws + f.L.attn;
   const float scale = 1.0f / std::sqrt((float)hd);
-  const int nt = c.d / 128;
+  const int group = ssq_group(c, M, f.m->layers_e4m3 != nullptr);
+  const int nt = c.d / group;  // sum-of-squares partials per token
 
   DG_CUDA(launch_ex(dg::gemm::embed_kernel, dim3(M), dim3(dg::gemm::EMBED_THREADS), 0, s, 1, tok,
-                    (const __nv_bfloat16*)f.m->embed, c.vocab, c.d, M, x, xb, ssq_x));
+                    (const __nv_bfloat16*)f.m->embed, c.vocab, c.d, M, x, xb, ssq_x, group));
   count_launch();
   DG_CUDA(cudaGetLastError());
   for (int l = 0; l < c.n_layers; ++l) {
@@ -1364,6 +1451,7 @@ int dg_denoise_block(const dg_model* m, dg_state* st, const dg_sampler_cfg* cfg,
   const bool fp8 = m->unembed_e4m3 != nullptr;  // check_model: vocab % 256 == 0 then
   Fwd fl = f;
   fl.unembed_elsewhere = fused;
+  const int nt = m->cfg.d / ssq_group(m->cfg, B * C, m->layers_e4m3 != nullptr);
   // one denoising step: forward pass, unembedding + sampler, step advance
   auto enqueue_step = [&](cudaStream_t q) -> int {
     DG_TRY(run_forward(fl, st->tok, logits, q));
@@ -1372,12 +1460,12 @@ int dg_denoise_block(const dg_model* m, dg_state* st, const dg_sampler_cfg* cfg,
       DG_TRY(quantize_hidden(fl, q));
       const Fp8Scales f8{(const float*)(ws + L.as), m->unembed_scale};
       DG_TRY(launch_unembed_sample(ws + L.aq, m->unembed_e4m3, m->cfg.d,
-                                   (const float*)(ws + L.ssq_x), m->cfg.d / 128, 1.f / m->cfg.d,
+                                   (const float*)(ws + L.ssq_x), nt, 1.f / m->cfg.d,
                                    m->cfg.eps, st->tok, st->committed, st->prev_argmax,
                                    st->seq_status, sp, nullptr, ws + L.spart, q, &f8));
     } else if (fused) {
       DG_TRY(launch_unembed_sample(ws + L.xn, m->unembed, m->cfg.d, (const float*)(ws + L.ssq_x),
-                                   m->cfg.d / 128, 1.f / m->cfg.d, m->cfg.eps, st->tok,
+                                   nt, 1.f / m->cfg.d, m->cfg.eps, st->tok,
                                    st->committed, st->prev_argmax, st->seq_status, sp, nullptr,
                                    ws + L.spart, q));
     } else {

@@ -427,12 +427,14 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // One CTA per token row: x[t] = embed[tok[t]] (fp32), xb[t] = bf16(x[t]),
-// ssq[j, t] = sum of x[t, 128 j .. 128 j + 127]^2.
+// ssq[j, t] = sum of x[t, G j .. G j + G - 1]^2 for groups of G = 128 or 32
+// columns (the granularity the forward pass's residual producers use).
 constexpr int EMBED_THREADS = 256;
 
 __global__ void __launch_bounds__(EMBED_THREADS) embed_kernel(
     const int32_t* __restrict__ tok, const __nv_bfloat16* __restrict__ embed, int V, int d, int M,
-    float* __restrict__ x, __nv_bfloat16* __restrict__ xb, float* __restrict__ ssq) {
+    float* __restrict__ x, __nv_bfloat16* __restrict__ xb, float* __restrict__ ssq,
+    int ssq_group) {
   griddep_wait();
   griddep_launch();
   const int t = blockIdx.x;
@@ -455,8 +457,17 @@ __global__ void __launch_bounds__(EMBED_THREADS) embed_kernel(
     const float4 a = make_float4(__low2float(lo), __high2float(lo), __low2float(hi),
                                  __high2float(hi));
     *reinterpret_cast<float4*>(xr + c) = a;
-    const float sq = warp_sum(a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w);
-    if (lane == 0) ssq[static_cast<size_t>(j) * M + t] = sq;
+    if (ssq_group == 128) {
+      const float sq = warp_sum(a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w);
+      if (lane == 0) ssq[static_cast<size_t>(j) * M + t] = sq;
+    } else {
+      // eight lanes per 32-column group
+      float sq = a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
+      sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+      sq += __shfl_xor_sync(0xffffffffu, sq, 2);
+      sq += __shfl_xor_sync(0xffffffffu, sq, 4);
+      if ((lane & 7) == 0) ssq[static_cast<size_t>(j * 4 + (lane >> 3)) * M + t] = sq;
+    }
   }
 }
 

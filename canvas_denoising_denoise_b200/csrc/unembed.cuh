@@ -31,6 +31,10 @@
 //                          memory; each (token, pair segment) leaves one
 //                          partial for the merge.
 //
+// The projections of the stack use the same pipeline when there are enough
+// 256 x 256 tiles (many tokens: prefill, wide batches): proj_pair_kernel,
+// A = weights, B = activations, with the projection epilogues of gemm.cuh.
+//
 // Roles: warp 0 issues the TMA loads (both CTAs, each into its own ring,
 // completion counted on the even CTA's barrier); warp 1 owns TMEM and, in the
 // even CTA, one lane issues the MMAs; the epilogue warps (2 ..) read this
@@ -38,6 +42,7 @@
 #pragma once
 
 #include "dg_common.cuh"
+#include "gemm.cuh"
 #include "sampler.cuh"
 
 namespace dg {
@@ -364,6 +369,165 @@ __global__ void __launch_bounds__(threads_for(STORE_EPI_WARPS), 1)
   epi.lane = lane_id();
   pair_pipeline<STORE_EPI_WARPS, KPS, F8>(&tm_w, &tm_x, l2_policy_evict_first(), l2_policy_evict_last(),
                                  sc, epi);
+}
+
+// ---------------------------------------------------------------------------
+// Projections of the stack on CTA pairs (many tokens).  The epilogues of
+// gemm.cuh: EPI_F32 / EPI_BF16 / EPI_GELU take rs[t] * acc; EPI_RESID adds
+// acc (times the e4m3 scales) to the fp32 residual stream, writes its bf16
+// copy and the sums of squares of each 32-feature group (one warp's lanes),
+// ssq_out [N / 32, M], so that no warp waits on another.
+// ---------------------------------------------------------------------------
+struct ProjParams {
+  int M, N, K;
+  int n_ttiles, n_tiles, n_pairs;
+  int epi;                   // dg::gemm::Epi
+  float* out_f32;            // EPI_F32
+  __nv_bfloat16* out_bf16;   // EPI_BF16 / EPI_GELU / EPI_RESID (optional there)
+  float* x;                  // EPI_RESID residual stream [M, N]
+  const float* ssq_in;       // [n_ssq_in, M] or null (rs = 1)
+  int n_ssq_in;
+  float inv_k, eps;
+  float* ssq_out;            // EPI_RESID: [N / 32, M], or null
+  const float* tok_scale;    // e4m3 operands: per-token scale [M], else null
+  const float* w_scale;      // e4m3 operands: the weights' scale (device scalar), else null
+};
+
+template <int EPI>
+struct ProjEpi {
+  ProjParams p;  // a copy: read in a rolled loop, a pointer to the launch's
+                 // parameters would put them on the stack
+  const StoreSched* sc;
+  uint32_t rank;
+  int quarter, lane;
+  float rs[TILE / 32];  // scale of token (tile base + 32 c + lane)
+
+  __device__ void start() {}
+  __device__ void prepare(int li) {
+    const int tb = sc->b_row(li);
+#pragma unroll
+    for (int c = 0; c < TILE / 32; ++c)
+      rs[c] = row_scale(p.ssq_in, p.n_ssq_in, p.M, tb + c * 32 + lane, p.inv_k, p.eps) *
+              fp8_scale(p.tok_scale, p.w_scale, p.M, tb + c * 32 + lane);
+  }
+  // A rolled loop over 32-token chunks with a small unrolled body (the whole
+  // tile unrolled is thousands of instructions per warp and measured slower
+  // than the mainloop it should hide behind).  Per 16 tokens: the residual
+  // rows are all loaded before the first store; bf16 outputs go out two rows
+  // per store with every lane active (even lanes row k, odd lanes row k + 1,
+  // after one exchange of neighbours); the sums of squares of the 16 rows are
+  // one transposed reduction (16 shuffles instead of 5 per row).
+  __device__ void consume(int li, uint32_t taddr, int col0, int ncols) {
+    (void)col0;
+    (void)ncols;
+    constexpr bool kBf16 = EPI != gemm::EPI_F32;
+    const unsigned full = 0xffffffffu;
+    const int M = p.M;
+    const size_t N = static_cast<size_t>(p.N);
+    const int tb = sc->b_row(li);
+    const int fq = sc->a_row(li) + static_cast<int>(rank) * HALF + quarter * 32;  // this warp's features
+    const bool odd = (lane & 1) != 0;
+    const int fpair = fq + (lane & ~1);  // first feature of this lane's bf16 pair
+    const int nch = min(TILE, M - tb + 31) / 32;
+    // rs is rotated so that rs[0] is the current chunk's (static indices only)
+    float rsr[TILE / 32];
+#pragma unroll
+    for (int c = 0; c < TILE / 32; ++c) rsr[c] = rs[c];
+#pragma unroll 1
+    for (int c = 0; c < nch; ++c) {
+      const float rsc = rsr[0];
+#pragma unroll
+      for (int c2 = 0; c2 + 1 < TILE / 32; ++c2) rsr[c2] = rsr[c2 + 1];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int t0 = tb + c * 32 + h * 16;
+        const size_t o0 = static_cast<size_t>(t0) * N + fq + lane;
+        uint32_t r[16];
+        tmem_ld16(taddr + c * 32 + h * 16, r);
+        float y[16];
+        if constexpr (EPI == gemm::EPI_RESID) {
+#pragma unroll
+          for (int k = 0; k < 16; ++k) y[k] = t0 + k < M ? p.x[o0 + k * N] : 0.f;
+        }
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const float v = __uint_as_float(r[k]) * __shfl_sync(full, rsc, h * 16 + k);
+          if constexpr (EPI == gemm::EPI_RESID) {
+            y[k] += v;
+            if (t0 + k < M) p.x[o0 + k * N] = y[k];
+          } else if constexpr (EPI == gemm::EPI_F32) {
+            if (t0 + k < M) p.out_f32[o0 + k * N] = v;
+          } else if constexpr (EPI == gemm::EPI_GELU) {
+            y[k] = gemm::gelu_erf(v);
+          } else {
+            y[k] = v;
+          }
+        }
+        if (kBf16 && p.out_bf16 != nullptr) {
+#pragma unroll
+          for (int k = 0; k < 16; k += 2) {
+            const float got = __shfl_xor_sync(full, odd ? y[k] : y[k + 1], 1);
+            const uint32_t w = odd ? pack_bf16x2(got, y[k + 1]) : pack_bf16x2(y[k], got);
+            const int row = t0 + k + (odd ? 1 : 0);
+            if (row < M)
+              *reinterpret_cast<uint32_t*>(p.out_bf16 + static_cast<size_t>(row) * N + fpair) = w;
+          }
+        }
+        if constexpr (EPI == gemm::EPI_RESID) {
+          if (p.ssq_out != nullptr) {
+            // halving exchange: after the step on lane bit b a lane keeps the
+            // upper half of its rows if that bit is set; 16 rows end as one
+            // per lane, row = bit-reverse of lane % 16
+            float a[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) a[k] = y[k] * y[k];
+#pragma unroll
+            for (int b = 0; b < 4; ++b) {
+              const int n = 16 >> b;
+              const bool up = ((lane >> b) & 1) != 0;
+#pragma unroll
+              for (int i = 0; i < n / 2; ++i) {
+                const float send = up ? a[i] : a[i + n / 2];
+                const float keep = up ? a[i + n / 2] : a[i];
+                a[i] = keep + __shfl_xor_sync(full, send, 1 << b);
+              }
+            }
+            const float sq = a[0] + __shfl_xor_sync(full, a[0], 16);
+            const int row = ((lane & 1) << 3) | ((lane & 2) << 1) | ((lane & 4) >> 1) |
+                            ((lane & 8) >> 3);
+            if (lane < 16 && t0 + row < M)
+              p.ssq_out[static_cast<size_t>(fq / 32) * M + t0 + row] = sq;
+          }
+        }
+      }
+    }
+  }
+  __device__ void finish() {}
+};
+
+// One kernel per epilogue: each carries a single unrolled store path.
+template <int KPS, bool F8, int EPI>
+__global__ void __launch_bounds__(threads_for(STORE_EPI_WARPS), 1)
+    proj_pair_kernel(const __grid_constant__ CUtensorMap tm_w,
+                     const __grid_constant__ CUtensorMap tm_x, ProjParams p) {
+  const int pair = static_cast<int>(blockIdx.x >> 1);
+  StoreSched sc;
+  sc.nkb = p.K / (F8 ? 128 : BK);
+  sc.pair = pair;
+  sc.n_pairs = p.n_pairs;
+  sc.n_ttiles = p.n_ttiles;
+  sc.count = pair < p.n_tiles ? (p.n_tiles - 1 - pair) / p.n_pairs + 1 : 0;
+  ProjEpi<EPI> epi;
+  epi.p = p;
+  epi.sc = &sc;
+  epi.rank = cluster_ctarank();
+  epi.quarter = warp_id() & 3;
+  epi.lane = lane_id();
+  // a weight tile is read by every token tile (consecutive tiles): keep it
+  // in L2 as long as the activations
+  pair_pipeline<STORE_EPI_WARPS, KPS, F8>(&tm_w, &tm_x, l2_policy_evict_first(),
+                                          l2_policy_evict_last(), sc, epi);
 }
 
 // ---------------------------------------------------------------------------

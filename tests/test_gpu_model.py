@@ -174,3 +174,25 @@ def test_two_blocks_batch_two(setup):
     # each sequence's cache equals its own one-shot prefill of the final tokens is covered
     # above; here the two sequences must differ (per-sequence Philox keys)
     assert not torch.equal(st.tok[0], st.tok[1])
+
+
+def test_denoise_logits_many_sequences_pair_path(setup):
+    """75 sequences (19200 canvas tokens): every projection of the tiny model
+    runs on the CTA-pair pipeline, and the residual stream's sums of squares
+    come per 32 features.  Sampled sequences against the oracle."""
+    dg, model, w64, _ = setup
+    Bn = 75
+    st = dg.DgState(SHAPE, Bn, P + 2 * C, C)
+    prompts = synth.make_prompt(Bn, P, SHAPE.vocab, seed=21)
+    dg.prefill(model, st, prompts.cuda())
+    canvas = torch.randint(0, SHAPE.vocab, (Bn, C), generator=torch.Generator().manual_seed(22))
+    st.tok.copy_(canvas.to(torch.int32))
+    logits = torch.empty((Bn, C, SHAPE.vocab), dtype=torch.float32, device="cuda")
+    dg.denoise_logits(model, st, logits)
+    torch.cuda.synchronize()
+    dg.check_device_errors()
+    for b in (0, 37, 74):
+        kc, vc = M.empty_cache(OCFG, P + 2 * C)
+        L = M.prefill(OCFG, w64, prompts[b].numpy(), kc, vc)
+        want = M.denoise_logits(OCFG, w64, canvas[b].numpy(), kc, vc, L)
+        assert_close(logits[b].cpu(), want, what=f"logits of sequence {b}")
