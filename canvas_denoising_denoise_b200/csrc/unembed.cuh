@@ -453,16 +453,18 @@ struct ProjEpi {
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
           const float v = __uint_as_float(r[k]) * __shfl_sync(full, rsc, h * 16 + k);
-          if constexpr (EPI == gemm::EPI_RESID) {
+          if constexpr (EPI == gemm::EPI_RESID)
             y[k] += v;
-            if (t0 + k < M) p.x[o0 + k * N] = y[k];
-          } else if constexpr (EPI == gemm::EPI_F32) {
-            if (t0 + k < M) p.out_f32[o0 + k * N] = v;
-          } else if constexpr (EPI == gemm::EPI_GELU) {
+          else if constexpr (EPI == gemm::EPI_GELU)
             y[k] = gemm::gelu_erf(v);
-          } else {
+          else
             y[k] = v;
-          }
+        }
+        if constexpr (EPI == gemm::EPI_RESID || EPI == gemm::EPI_F32) {
+          float* const dst = EPI == gemm::EPI_RESID ? p.x : p.out_f32;
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            if (t0 + k < M) dst[o0 + k * N] = y[k];
         }
         if (kBf16 && p.out_bf16 != nullptr) {
 #pragma unroll
