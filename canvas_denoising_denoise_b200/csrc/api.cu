@@ -387,7 +387,7 @@ int launch_proj_pair(const void* x, const void* w, int M, int N, int K, const Ge
   const int nkb = K / (f8 ? 128 : dg::gemm::BK);
   (void)nkb;
   auto* kern = f8 ? proj_kernel<1, true>(e.epi) : proj_kernel<1, false>(e.epi);
-  DG_CUDA(launch_cluster(kern, dim3(2 * p.n_pairs), dim3(ue::threads_for(ue::STORE_EPI_WARPS)),
+  DG_CUDA(launch_cluster(kern, dim3(2 * p.n_pairs), dim3(ue::threads_for(ue::PROJ_EPI_WARPS)),
                          ue::SMEM_BYTES, s, dim3(2, 1, 1), tw, tx, p));
   count_launch();
   return DG_OK;

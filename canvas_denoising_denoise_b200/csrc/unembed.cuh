@@ -63,6 +63,10 @@ constexpr uint32_t IDESC = idesc_bf16_f32(TILE, TILE, false, false);
 // warps per TMEM lane quarter, each taking a third of a tile's columns: the
 // row pass is a long dependent chain per element, and more warps hide it).
 constexpr int STORE_EPI_WARPS = 4;
+// The projections' epilogues: two warps per lane quarter, each taking half of
+// a tile's token columns, so that twice the residual loads are in flight and a
+// launch's last tile (whose epilogue nothing hides) drains in half the time.
+constexpr int PROJ_EPI_WARPS = 8;
 constexpr int SAMPLE_EPI_WARPS = 12;
 constexpr int SAMPLE_SLOTS = SAMPLE_EPI_WARPS / 4;  // partials per (token, segment)
 __host__ __device__ constexpr int threads_for(int epi_warps) { return 64 + 32 * epi_warps; }
@@ -418,8 +422,6 @@ struct ProjEpi {
   // after one exchange of neighbours); the sums of squares of the 16 rows are
   // one transposed reduction (16 shuffles instead of 5 per row).
   __device__ void consume(int li, uint32_t taddr, int col0, int ncols) {
-    (void)col0;
-    (void)ncols;
     constexpr bool kBf16 = EPI != gemm::EPI_F32;
     const unsigned full = 0xffffffffu;
     const int M = p.M;
@@ -428,11 +430,19 @@ struct ProjEpi {
     const int fq = sc->a_row(li) + static_cast<int>(rank) * HALF + quarter * 32;  // this warp's features
     const bool odd = (lane & 1) != 0;
     const int fpair = fq + (lane & ~1);  // first feature of this lane's bf16 pair
-    const int nch = min(TILE, M - tb + 31) / 32;
+    // this warp's token columns [col0, col0 + ncols) of the tile (taddr
+    // already points at col0)
+    const int tc0 = tb + col0;
+    const int nch = M - tc0 <= 0 ? 0 : min(ncols, M - tc0 + 31) / 32;
     // rs is rotated so that rs[0] is the current chunk's (static indices only)
     float rsr[TILE / 32];
 #pragma unroll
     for (int c = 0; c < TILE / 32; ++c) rsr[c] = rs[c];
+#pragma unroll 1
+    for (int c = 0; c < col0 / 32; ++c) {
+#pragma unroll
+      for (int c2 = 0; c2 + 1 < TILE / 32; ++c2) rsr[c2] = rsr[c2 + 1];
+    }
 #pragma unroll 1
     for (int c = 0; c < nch; ++c) {
       const float rsc = rsr[0];
@@ -440,7 +450,7 @@ struct ProjEpi {
       for (int c2 = 0; c2 + 1 < TILE / 32; ++c2) rsr[c2] = rsr[c2 + 1];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int t0 = tb + c * 32 + h * 16;
+        const int t0 = tc0 + c * 32 + h * 16;
         const size_t o0 = static_cast<size_t>(t0) * N + fq + lane;
         uint32_t r[16];
         tmem_ld16(taddr + c * 32 + h * 16, r);
@@ -510,7 +520,7 @@ struct ProjEpi {
 
 // One kernel per epilogue: each carries a single unrolled store path.
 template <int KPS, bool F8, int EPI>
-__global__ void __launch_bounds__(threads_for(STORE_EPI_WARPS), 1)
+__global__ void __launch_bounds__(threads_for(PROJ_EPI_WARPS), 1)
     proj_pair_kernel(const __grid_constant__ CUtensorMap tm_w,
                      const __grid_constant__ CUtensorMap tm_x, ProjParams p) {
   const int pair = static_cast<int>(blockIdx.x >> 1);
@@ -528,8 +538,8 @@ __global__ void __launch_bounds__(threads_for(STORE_EPI_WARPS), 1)
   epi.lane = lane_id();
   // a weight tile is read by every token tile (consecutive tiles): keep it
   // in L2 as long as the activations
-  pair_pipeline<STORE_EPI_WARPS, KPS, F8>(&tm_w, &tm_x, l2_policy_evict_first(),
-                                          l2_policy_evict_last(), sc, epi);
+  pair_pipeline<PROJ_EPI_WARPS, KPS, F8>(&tm_w, &tm_x, l2_policy_evict_first(),
+                                         l2_policy_evict_last(), sc, epi);
 }
 
 // ---------------------------------------------------------------------------
