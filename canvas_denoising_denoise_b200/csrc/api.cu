@@ -216,7 +216,20 @@ GemmPlan plan_gemm(int M, int N, int K, int kb_elems = dg::gemm::BK) {
   return best;
 }
 
-bool gemm_attr_done = false;
+// "Kernel attributes are set" flags.  A kernel's attributes belong to one
+// device's context, so the flag is kept per device (a device beyond the
+// table re-sets them on every call).
+struct PerDeviceFlag {
+  bool done[64] = {};
+  bool spare = false;
+  bool& operator()() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return spare = false;
+    return done[dev];
+  }
+};
+
+PerDeviceFlag gemm_attr_done;
 
 // Epilogue operands of one GEMM launch (see gemm.cuh).
 struct GemmEpi {
@@ -278,10 +291,10 @@ cudaError_t launch_gemm_plan(const GemmPlan& pl, dim3 grid, cudaStream_t s, cons
 // x [M, K] and w [N, K]: bf16, or e4m3 codes with their scales when f8 is set.
 int launch_gemm(const void* x, const void* w, int M, int N, int K, const GemmPlan& pl,
                 const GemmEpi& e, cudaStream_t s, const Fp8Scales* f8 = nullptr) {
-  if (!gemm_attr_done) {
+  if (!gemm_attr_done()) {
     DG_CUDA(gemm_set_attrs<false>());
     DG_CUDA(gemm_set_attrs<true>());
-    gemm_attr_done = true;
+    gemm_attr_done() = true;
   }
   CUtensorMap tw, tx;
   if (f8) {
@@ -326,7 +339,7 @@ bool proj_use_pair(int M, int N, int K, bool f8) {
   return (N / dg::unembed::TILE) * cdiv(M, dg::unembed::TILE) >= kNumSMs / 2;
 }
 
-bool proj_attr_done = false;
+PerDeviceFlag proj_attr_done;
 
 template <int KPS, bool F8>
 cudaError_t proj_set_attrs() {
@@ -356,12 +369,12 @@ decltype(&dg::unembed::proj_pair_kernel<1, false, 0>) proj_kernel(int epi) {
 int launch_proj_pair(const void* x, const void* w, int M, int N, int K, const GemmEpi& e,
                      cudaStream_t s, const Fp8Scales* f8) {
   namespace ue = dg::unembed;
-  if (!proj_attr_done) {
+  if (!proj_attr_done()) {
     DG_CUDA((proj_set_attrs<1, false>()));
     DG_CUDA((proj_set_attrs<2, false>()));
     DG_CUDA((proj_set_attrs<1, true>()));
     DG_CUDA((proj_set_attrs<2, true>()));
-    proj_attr_done = true;
+    proj_attr_done() = true;
   }
   CUtensorMap tw, tx;
   if (f8) {
@@ -412,7 +425,7 @@ int ssq_group(const dg_model_cfg& c, int M, bool f8) {
 
 // logits = rs * (h w_u^T).  Vocabularies that are a multiple of 256 run on
 // the persistent CTA-pair kernel (unembed.cuh); others on the single-CTA GEMM.
-bool unembed_attr_done = false;
+PerDeviceFlag unembed_attr_done;
 
 int launch_unembed(const void* h, const void* w_u, float* logits, int M, int d, int V,
                    const float* ssq_in, int n_ssq_in, float inv_k, float eps, cudaStream_t s,
@@ -425,12 +438,12 @@ int launch_unembed(const void* h, const void* w_u, float* logits, int M, int d, 
     e.ssq_in = ssq_in; e.n_ssq_in = n_ssq_in; e.inv_k = inv_k; e.eps = eps;
     return launch_gemm(h, w_u, M, V, d, GemmPlan{1, d / dg::gemm::BK, 256}, e, s);
   }
-  if (!unembed_attr_done) {
+  if (!unembed_attr_done()) {
     DG_CUDA(cudaFuncSetAttribute(ue::unembed_pair_kernel<1, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, ue::SMEM_BYTES));
     DG_CUDA(cudaFuncSetAttribute(ue::unembed_pair_kernel<1, true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, ue::SMEM_BYTES));
-    unembed_attr_done = true;
+    unembed_attr_done() = true;
   }
   CUtensorMap tw, tx;
   if (f8) {
@@ -489,7 +502,7 @@ size_t attn_ws_bytes(int B, int Hq, int Hkv, int Lq, int hd, int max_prefix) {
   return align_up(rows * hd * 2, 256) + align_up(rows * sizeof(float), 256);
 }
 
-bool attn_attr_done[2] = {false, false};
+PerDeviceFlag attn_attr_done[2];
 
 int launch_attn(const void* q, int ldq, const void* k_new, const void* v_new, int ldkv,
                 const void* k_cache, const void* v_cache, const int32_t* cache_len,
@@ -522,21 +535,21 @@ int launch_attn(const void* q, int ldq, const void* k_new, const void* v_new, in
   }
   dim3 grid(B * Hkv * p.n_pairs, S);
   if (hd == 128) {
-    if (!attn_attr_done[1]) {
+    if (!attn_attr_done[1]()) {
       DG_CUDA(cudaFuncSetAttribute(dg::attn::attn_kernel<128>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    dg::attn::Cfg<128>::SMEM_BYTES));
-      attn_attr_done[1] = true;
+      attn_attr_done[1]() = true;
     }
     DG_CUDA(launch_ex(dg::attn::attn_kernel<128>, grid, dim3(dg::attn::THREADS),
                       dg::attn::Cfg<128>::SMEM_BYTES, s, 1, tq, tkn, tvn, tkc, tvc, p));
     count_launch();
   } else {
-    if (!attn_attr_done[0]) {
+    if (!attn_attr_done[0]()) {
       DG_CUDA(cudaFuncSetAttribute(dg::attn::attn_kernel<64>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
                                    dg::attn::Cfg<64>::SMEM_BYTES));
-      attn_attr_done[0] = true;
+      attn_attr_done[0]() = true;
     }
     DG_CUDA(launch_ex(dg::attn::attn_kernel<64>, grid, dim3(dg::attn::THREADS),
                       dg::attn::Cfg<64>::SMEM_BYTES, s, 1, tq, tkn, tvn, tkc, tvc, p));
@@ -653,7 +666,7 @@ size_t fused_ws_bytes(int B, int C, int V) {
          align_up((size_t)M * sizeof(dg::RowStats), 256);
 }
 
-bool fused_attr_done = false;
+PerDeviceFlag fused_attr_done;
 
 int launch_unembed_sample(const void* h, const void* w_u, int d, const float* ssq_in,
                           int n_ssq_in, float inv_k, float eps, int32_t* tok,
@@ -663,7 +676,7 @@ int launch_unembed_sample(const void* h, const void* w_u, int d, const float* ss
   namespace ue = dg::unembed;
   const int M = sp.B * sp.C, V = sp.V;
   const FusedPlan f = plan_fused(M, V);
-  if (!fused_attr_done) {
+  if (!fused_attr_done()) {
     DG_CUDA(cudaFuncSetAttribute(ue::unembed_sample_kernel<1, false>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, ue::SMEM_BYTES));
     DG_CUDA(cudaFuncSetAttribute(ue::unembed_sample_kernel<2, false>,
@@ -672,7 +685,7 @@ int launch_unembed_sample(const void* h, const void* w_u, int d, const float* ss
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, ue::SMEM_BYTES));
     DG_CUDA(cudaFuncSetAttribute(ue::unembed_sample_kernel<2, true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, ue::SMEM_BYTES));
-    fused_attr_done = true;
+    fused_attr_done() = true;
   }
   dg::FusedPartial* part = (dg::FusedPartial*)ws;
   dg::RowStats* stats = (dg::RowStats*)((char*)ws + align_up((size_t)M * f.nparts *

@@ -28,7 +28,9 @@
  *     *_workspace_bytes() queries return.  Host arrays passed in (pointer
  *     tables, structs) are read during the call only.
  *   - One host thread at a time: the library keeps a little process-wide
- *     state (kernel attributes set once, a capture stream per device).
+ *     state (kernel attributes set once per device, a capture stream per
+ *     device).  Calls may target any device: the current CUDA device is the
+ *     one whose memory the pointers refer to.
  *   - All device work is enqueued on the caller's stream (a cudaStream_t passed
  *     as void*; NULL is the legacy default stream) and is asynchronous, except
  *     where a function says it synchronises.  Results are deterministic: the
