@@ -232,10 +232,17 @@ int dg_unembed(const void* h, const void* w_u, float* logits, int M, int d, int 
                void* workspace, size_t workspace_bytes, void* stream);
 
 /*
- * dg_linear - the layer projections of the stack (QKV, output, MLP up/down):
+ * dg_linear - the layer projections of the stack (QKV, output, MLP up/down;
+ * aiexpert.news architecture paragraph, with the dense GELU MLP standing in
+ * for the expert FFN):
  *   y[m, n] = sum_k x[m, k] w[n, k], then the epilogue (enum dg_epilogue).
  * x bf16 [M, K]; w bf16 [N, K]; out per epilogue.  N % 128 == 0, K % 64 == 0.
- * Workspace: dg_linear_workspace_bytes() (split-K partial sums).
+ * Few tokens run on a GEMM whose K is split over a thread-block cluster; many
+ * tokens (N % 256 == 0 and at least 74 output tiles of 256 x 256) on a
+ * persistent grid of CTA pairs.  The path depends on the shape only, so a
+ * shape always gives the same bits; the two paths sum K in different orders.
+ * Needs no workspace: dg_linear_workspace_bytes() returns 0 (the split-K
+ * partial sums stay in the cluster's shared memory); pass NULL, 0.
  */
 int dg_linear(const void* x, const void* w, void* out, int M, int N, int K, int epilogue,
               void* workspace, size_t workspace_bytes, void* stream);
@@ -310,7 +317,8 @@ size_t dg_unembed_sample_commit_workspace_bytes(int B, int C, int V);
  *   scales x_scale (device [M]), w_q [N, K] codes with one scale w_scale
  *   (device scalar); acc[m, n] = x_scale[m] w_scale sum_k dec(x_q[m, k])
  *   dec(w_q[n, k]) (fp32 accumulation of exact products), then the epilogue
- *   of dg_linear.  N % 128 == 0, K % 128 == 0.  No workspace.
+ *   of dg_linear, on the same two paths (kind::f8f6f4 MMAs).  N % 128 == 0,
+ *   K % 128 == 0.  No workspace.
  */
 int dg_quantize_e4m3(const void* in, int rows, int cols, int per_row, uint8_t* out,
                      float* scales, void* stream);
