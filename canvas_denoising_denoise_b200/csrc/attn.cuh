@@ -107,9 +107,16 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int warp = warp_id();
   const int lane = lane_id();
-  const int pi = blockIdx.x % p.n_pairs;
-  const int g = (blockIdx.x / p.n_pairs) % p.Hkv;
-  const int b = blockIdx.x / (p.n_pairs * p.Hkv);
+  // Causal launches take their heaviest query tiles (the last rows, which see
+  // the most keys) first, so that the light ones fill the tail of the grid;
+  // the canvas mask gives every pair the same work.
+  const int nbg = p.Hkv * p.B;
+  const int pi = p.causal ? p.n_pairs - 1 - static_cast<int>(blockIdx.x) / nbg
+                          : static_cast<int>(blockIdx.x) % p.n_pairs;
+  const int gb = p.causal ? static_cast<int>(blockIdx.x) % nbg
+                          : static_cast<int>(blockIdx.x) / p.n_pairs;
+  const int g = gb % p.Hkv;
+  const int b = gb / p.Hkv;
   const int split = blockIdx.y;
   const int nq = p.group * p.n_rt;  // query tiles of this kv head
   int hX[2], i0X[2];
