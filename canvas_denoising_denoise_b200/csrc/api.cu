@@ -409,18 +409,28 @@ int launch_proj_pair(const void* x, const void* w, int M, int N, int K, const Ge
 // y = epilogue(x w^T) with the plan chosen for this shape (e4m3 operands with
 // their scales when f8 is set: 128-element k-blocks).  EPI_RESID writes its
 // sums of squares per 128 features on the split-K GEMM and per 32 on the
-// pair pipeline (see ssq_group).
+// pair pipeline (see ssq_group); pair_ok = false keeps a shape on the former.
 int linear(const void* x, const void* w, int M, int N, int K, const GemmEpi& e,
-           cudaStream_t s, const Fp8Scales* f8 = nullptr) {
-  if (proj_use_pair(M, N, K, f8 != nullptr)) return launch_proj_pair(x, w, M, N, K, e, s, f8);
+           cudaStream_t s, const Fp8Scales* f8 = nullptr, bool pair_ok = true) {
+  if (pair_ok && proj_use_pair(M, N, K, f8 != nullptr))
+    return launch_proj_pair(x, w, M, N, K, e, s, f8);
   return launch_gemm(x, w, M, N, K, plan_gemm(M, N, K, f8 ? 128 : dg::gemm::BK), e, s, f8);
 }
 
+// Both residual projections of a forward pass over M tokens (the output
+// projection, K = Hq hd, and the MLP down projection, K = F) write the sums of
+// squares their consumers read, so they take one path together: the pair
+// pipeline only when both shapes qualify for it.
+bool resid_on_pair(const dg_model_cfg& c, int M, bool f8) {
+  return proj_use_pair(M, c.d, c.n_q_heads * c.head_dim, f8) &&
+         proj_use_pair(M, c.d, c.ffn, f8);
+}
+
 // Features per sum-of-squares partial of the residual stream in a forward
-// pass over M tokens: 32 when its residual projections (N = d) run on the
-// pair pipeline, else 128.
+// pass over M tokens: 32 when its residual projections run on the pair
+// pipeline, else 128.
 int ssq_group(const dg_model_cfg& c, int M, bool f8) {
-  return proj_use_pair(M, c.d, c.n_q_heads * c.head_dim, f8) ? 32 : 128;
+  return resid_on_pair(c, M, f8) ? 32 : 128;
 }
 
 // logits = rs * (h w_u^T).  Vocabularies that are a multiple of 256 run on
@@ -904,6 +914,7 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
   const float scale = 1.0f / std::sqrt((float)hd);
   const int group = ssq_group(c, M, f.m->layers_e4m3 != nullptr);
   const int nt = c.d / group;  // sum-of-squares partials per token
+  const bool resid_pair = group == 32;
 
   DG_CUDA(launch_ex(dg::gemm::embed_kernel, dim3(M), dim3(dg::gemm::EMBED_THREADS), 0, s, 1, tok,
                     (const __nv_bfloat16*)f.m->embed, c.vocab, c.d, M, x, xb, ssq_x, group));
@@ -915,17 +926,17 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
     const dg_layer_weights_e4m3* q8 = f.m->layers_e4m3 ? &f.m->layers_e4m3[l] : nullptr;
     // y = epilogue(in w^T): bf16, or e4m3 with the input quantised per token
     auto proj = [&](const void* in, const void* wb, const uint8_t* wq, int widx, int N, int K,
-                    const GemmEpi& e) -> int {
-      if (!q8) return linear(in, wb, M, N, K, e, s);
+                    const GemmEpi& e, bool pair_ok) -> int {
+      if (!q8) return linear(in, wb, M, N, K, e, s, nullptr, pair_ok);
       DG_TRY(quantize_act(f, in, K, s));
       const Fp8Scales f8{(const float*)(f.ws + f.L.as), q8->scales + widx};
-      return linear(f.ws + f.L.aq, wq, M, N, K, e, s, &f8);
+      return linear(f.ws + f.L.aq, wq, M, N, K, e, s, &f8, pair_ok);
     };
     GemmEpi eq;  // QKV of RMSNorm(x)
     eq.epi = dg::gemm::EPI_BF16;
     eq.out_bf16 = qkv;
     eq.ssq_in = ssq_x; eq.n_ssq_in = nt; eq.inv_k = 1.f / c.d; eq.eps = c.eps;
-    DG_TRY(proj(xb, w.w_qkv, q8 ? q8->w_qkv : nullptr, 0, nqkv, c.d, eq));
+    DG_TRY(proj(xb, w.w_qkv, q8 ? q8->w_qkv : nullptr, 0, nqkv, c.d, eq, true));
     if (f.commit_kv) {
       const void* kb = qkv + hq * hd;
       const void* vb = qkv + (hq + hkv) * hd;
@@ -939,16 +950,16 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
     GemmEpi eo;  // h = x + O w_o^T
     eo.epi = dg::gemm::EPI_RESID;
     eo.x = x; eo.out_bf16 = xb; eo.ssq_out = ssq_h;
-    DG_TRY(proj(ao, w.w_o, q8 ? q8->w_o : nullptr, 1, c.d, hq * hd, eo));
+    DG_TRY(proj(ao, w.w_o, q8 ? q8->w_o : nullptr, 1, c.d, hq * hd, eo, resid_pair));
     GemmEpi eu;  // gelu(RMSNorm(h) w_up^T)
     eu.epi = dg::gemm::EPI_GELU;
     eu.out_bf16 = up;
     eu.ssq_in = ssq_h; eu.n_ssq_in = nt; eu.inv_k = 1.f / c.d; eu.eps = c.eps;
-    DG_TRY(proj(xb, w.w_up, q8 ? q8->w_up : nullptr, 2, c.ffn, c.d, eu));
+    DG_TRY(proj(xb, w.w_up, q8 ? q8->w_up : nullptr, 2, c.ffn, c.d, eu, true));
     GemmEpi ed;  // x = h + u w_down^T
     ed.epi = dg::gemm::EPI_RESID;
     ed.x = x; ed.out_bf16 = xb; ed.ssq_out = ssq_x;
-    DG_TRY(proj(up, w.w_down, q8 ? q8->w_down : nullptr, 3, c.d, c.ffn, ed));
+    DG_TRY(proj(up, w.w_down, q8 ? q8->w_down : nullptr, 3, c.d, c.ffn, ed, resid_pair));
   }
   if (f.want_logits && !f.unembed_elsewhere) {
     // logits of RMSNorm(x), on e4m3 operands when the model carries them

@@ -337,3 +337,37 @@ def test_block_driver_e4m3_layers_matches_stepwise_calls(fp8_full_model):
             break
     assert n == steps
     assert torch.equal(st2.tok, tok_a), "FP8 block driver and step-wise calls must agree"
+
+
+def test_denoise_logits_e4m3_layers_many_sequences(fp8_full_model):
+    """75 sequences (19200 canvas tokens) on the FP8 model.  The MLP down
+    projection (K = F, eight e4m3 k-blocks) would qualify for the CTA-pair
+    pipeline while the output projection (K = Hq hd, two k-blocks) does not;
+    both write the residual's sums of squares that the next norm reads, so
+    they must take one path together.  Sampled sequences against the oracle's
+    FP8 forward at the bar of the one-sequence test."""
+    dg, model, w64, _ = fp8_full_model
+    Bn = 75
+    st = dg.DgState(SHAPE, Bn, P + 2 * C, C)
+    prompts = synth.make_prompt(Bn, P, SHAPE.vocab, seed=21)
+    dg.prefill(model, st, prompts.cuda())
+    canvas = torch.randint(0, SHAPE.vocab, (Bn, C), generator=torch.Generator().manual_seed(22))
+    st.tok.copy_(canvas.to(torch.int32))
+    logits = torch.empty((Bn, C, SHAPE.vocab), dtype=torch.float32, device="cuda")
+    dg.denoise_logits(model, st, logits)
+    torch.cuda.synchronize()
+    dg.check_device_errors()
+
+    def oracle(b, bf16_storage):
+        kc, vc = M.empty_cache(OCFG, P + 2 * C)
+        L = M.prefill(OCFG, w64, prompts[b].numpy(), kc, vc, bf16_storage=bf16_storage,
+                      e4m3_layers=True)
+        return M.denoise_logits(OCFG, w64, canvas[b].numpy(), kc, vc, L,
+                                bf16_storage=bf16_storage, e4m3_unembed=True, e4m3_layers=True)
+
+    for b in (0, 74):
+        want = oracle(b, True)
+        sens = np.linalg.norm(oracle(b, False) - want) / np.linalg.norm(want)
+        rel = np.linalg.norm(to64(logits[b]) - want) / np.linalg.norm(want)
+        print(f"sequence {b}: gpu vs oracle fp8 {rel:.3e}; oracle rounding sensitivity {sens:.3e}")
+        assert rel <= 1.5 * sens and rel < 0.1, f"sequence {b}"
