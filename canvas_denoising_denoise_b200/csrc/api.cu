@@ -331,12 +331,15 @@ int launch_gemm(const void* x, const void* w, int M, int N, int K, const GemmPla
 }
 
 // Projections with many tokens run on the persistent CTA-pair pipeline
-// (unembed.cuh, 256 x 256 tiles, double-buffered accumulators) when its tiles
-// fill the pairs at least once; fewer tokens take the split-K GEMM.
+// (unembed.cuh, 256 x 256 tiles, double-buffered accumulators); fewer tokens
+// take the split-K GEMM.
 bool proj_use_pair(int M, int N, int K, bool f8) {
   const int kbe = f8 ? 128 : dg::gemm::BK;
   if (N % dg::unembed::TILE || K % kbe || K / kbe < 4) return false;
-  return (N / dg::unembed::TILE) * cdiv(M, dg::unembed::TILE) >= kNumSMs / 2;
+  // a full wave of pairs, or 48..73 tiles where the many-token shapes
+  // measured faster than the split-K plans (M >= 1536)
+  const int tiles = (N / dg::unembed::TILE) * cdiv(M, dg::unembed::TILE);
+  return tiles >= kNumSMs / 2 || (tiles >= 48 && M >= 1536);
 }
 
 PerDeviceFlag proj_attr_done;

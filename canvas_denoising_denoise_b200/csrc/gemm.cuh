@@ -299,8 +299,16 @@ __global__ void __launch_bounds__(THREADS, 1)
       float rs = 1.f;
       const int tg = t0 + t;
       if (p.ssq_in != nullptr && tg < p.M) {
+        // index order, sixteen loads in flight (as the pair pipelines)
         float acc = 0.f;
-        for (int j = 0; j < p.n_ssq_in; ++j) acc += p.ssq_in[static_cast<size_t>(j) * p.M + tg];
+        for (int j0 = 0; j0 < p.n_ssq_in; j0 += 16) {
+          float v[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            v[j] = j0 + j < p.n_ssq_in ? p.ssq_in[static_cast<size_t>(j0 + j) * p.M + tg] : 0.f;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) acc += v[j];
+        }
         rs = rsqrtf(acc * p.inv_k + p.eps);
       }
       if constexpr (F8) {

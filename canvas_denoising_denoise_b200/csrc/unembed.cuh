@@ -273,12 +273,22 @@ __device__ __forceinline__ void pair_pipeline(const CUtensorMap* tm_a, const CUt
   }
 }
 
-// Row scale of token t (1 without sums of squares).
+// Row scale of token t (1 without sums of squares).  The partials are summed
+// in index order; they are loaded sixteen at a time so that one round trip to
+// L2 serves sixteen of them (adding the zeros past the end changes nothing:
+// the sum is non-negative).
 __device__ __forceinline__ float row_scale(const float* ssq_in, int n_ssq_in, int M, int t,
                                            float inv_k, float eps) {
   if (ssq_in == nullptr || t >= M) return 1.f;
   float acc = 0.f;
-  for (int q = 0; q < n_ssq_in; ++q) acc += ssq_in[static_cast<size_t>(q) * M + t];
+  for (int q0 = 0; q0 < n_ssq_in; q0 += 16) {
+    float v[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      v[j] = q0 + j < n_ssq_in ? ssq_in[static_cast<size_t>(q0 + j) * M + t] : 0.f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) acc += v[j];
+  }
   return rsqrtf(acc * inv_k + eps);
 }
 
@@ -407,12 +417,21 @@ struct ProjEpi {
   float rs[TILE / 32];  // scale of token (tile base + 32 c + lane)
 
   __device__ void start() {}
+  // the scales of this warp's own token chunks only (the pipeline gives warp
+  // set (warp - 2) / 4 the chunks [4 k, 4 k + 4) of a tile)
   __device__ void prepare(int li) {
+    static_assert(PROJ_EPI_WARPS == 8, "two warps per lane quarter, four chunks each");
     const int tb = sc->b_row(li);
+    const int mine = (warp_id() - 2) >> 2;
 #pragma unroll
-    for (int c = 0; c < TILE / 32; ++c)
+    for (int c = 0; c < TILE / 32; ++c) {
+      if (c / (TILE / 64) != mine) {
+        rs[c] = 1.f;  // another warp's chunk
+        continue;
+      }
       rs[c] = row_scale(p.ssq_in, p.n_ssq_in, p.M, tb + c * 32 + lane, p.inv_k, p.eps) *
               fp8_scale(p.tok_scale, p.w_scale, p.M, tb + c * 32 + lane);
+    }
   }
   // A rolled loop over 32-token chunks with a small unrolled body (the whole
   // tile unrolled is thousands of instructions per warp and measured slower

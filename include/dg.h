@@ -238,8 +238,9 @@ int dg_unembed(const void* h, const void* w_u, float* logits, int M, int d, int 
  *   y[m, n] = sum_k x[m, k] w[n, k], then the epilogue (enum dg_epilogue).
  * x bf16 [M, K]; w bf16 [N, K]; out per epilogue.  N % 128 == 0, K % 64 == 0.
  * Few tokens run on a GEMM whose K is split over a thread-block cluster; many
- * tokens (N % 256 == 0 and at least 74 output tiles of 256 x 256) on a
- * persistent grid of CTA pairs.  The path depends on the shape only, so a
+ * tokens (N % 256 == 0 and at least 74 output tiles of 256 x 256, or 48 with
+ * M >= 1536; K at least four 128-byte k-blocks) on a persistent grid of CTA
+ * pairs.  The path depends on the shape only, so a
  * shape always gives the same bits; the two paths sum K in different orders.
  * Needs no workspace: dg_linear_workspace_bytes() returns 0 (the split-K
  * partial sums stay in the cluster's shared memory); pass NULL, 0.

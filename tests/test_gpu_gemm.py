@@ -168,16 +168,19 @@ def test_linear_e4m3_epilogues(Mr, N, K, epi):
 
 
 # Many tokens: the projections run on the persistent CTA-pair pipeline
-# (256 x 256 tiles, at least one full wave of pairs); 1300 rows leave a ragged
-# token tile; K = 128 / 256 are one or two e4m3 k-blocks per stage.
+# (256 x 256 tiles: at least one full wave of pairs, or 48 and more tiles with
+# 1536 and more tokens, as 1600 x 2048 has: 56 tiles, some pairs idle); 1300
+# and 1600 rows leave a ragged token tile; K = 128 / 256 are one or two e4m3
+# k-blocks per stage.
 @pytest.mark.parametrize("Mr,N,K", [(1024, 8192, 2048), (4096, 2048, 2048), (1300, 8192, 512),
-                                    (2048, 4096, 768)])
+                                    (2048, 4096, 768), (1600, 2048, 512)])
 @pytest.mark.parametrize("epi", ["f32", "bf16", "gelu", "resid"])
 def test_linear_many_tokens_pair_path(Mr, N, K, epi):
     test_linear_epilogues(Mr, N, K, epi)
 
 
-@pytest.mark.parametrize("Mr,N,K", [(1024, 8192, 2048), (1300, 8192, 512), (4096, 2048, 384)])
+@pytest.mark.parametrize("Mr,N,K", [(1024, 8192, 2048), (1300, 8192, 512), (4096, 2048, 384),
+                                    (1600, 2048, 512)])
 @pytest.mark.parametrize("epi", ["f32", "bf16", "resid"])
 def test_linear_e4m3_many_tokens_pair_path(Mr, N, K, epi):
     test_linear_e4m3_epilogues(Mr, N, K, epi)
