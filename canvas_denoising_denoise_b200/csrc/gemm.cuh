@@ -17,7 +17,8 @@
 // RMSNorm with unit gain is a per-token scale, so norm(x) w^T = rs * (x w^T)
 // with rs[t] = 1/sqrt(mean_k x[t,k]^2 + eps): the consumer of a normalised
 // input applies rs in its epilogue, computed from per-(128-column tile, token)
-// sums of squares that the producer of x wrote (summed in a fixed order).
+// sums of squares that the producer of x wrote (per 32 columns when the
+// producers run on the CTA-pair pipeline; summed in index order).
 //
 // With e4m3 operands (F8: x and w as codes, x scaled per token by sx[t], w
 // per tensor by sw) the MMA is kind::f8f6f4 and every epilogue takes acc as
