@@ -21,6 +21,7 @@
 #include "dg_common.cuh"
 #include "gemm.cuh"
 #include "kvcommit.cuh"
+#include "norm.cuh"
 #include "quant.cuh"
 #include "unembed.cuh"
 #include "sampler.cuh"
@@ -434,6 +435,13 @@ bool resid_on_pair(const dg_model_cfg& c, int M, bool f8) {
 // pipeline, else 128.
 int ssq_group(const dg_model_cfg& c, int M, bool f8) {
   return resid_on_pair(c, M, f8) ? 32 : 128;
+}
+
+// Partial sums of squares per token that a consumer of the norm reads: the
+// 32-feature partials of the pair path are collapsed into one after each
+// producer (norm.cuh); the split-K GEMM's d / 128 are read as they are.
+int ssq_partials_read(const dg_model_cfg& c, int M, bool f8) {
+  return ssq_group(c, M, f8) == 32 ? 1 : c.d / 128;
 }
 
 // logits = rs * (h w_u^T).  Vocabularies that are a multiple of 256 run on
@@ -918,11 +926,21 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
   const int group = ssq_group(c, M, f.m->layers_e4m3 != nullptr);
   const int nt = c.d / group;  // sum-of-squares partials per token
   const bool resid_pair = group == 32;
+  // partials a consumer of the norm reads: one once they are collapsed
+  const int n_use = ssq_partials_read(c, M, f.m->layers_e4m3 != nullptr);
+  auto collapse = [&](float* ssq) -> int {
+    if (!resid_pair) return DG_OK;
+    DG_CUDA(launch_ex(dg::norm::ssq_collapse_kernel, dim3(cdiv(M, dg::norm::COLLAPSE_THREADS)),
+                      dim3(dg::norm::COLLAPSE_THREADS), 0, s, 1, ssq, nt, M));
+    count_launch();
+    return DG_OK;
+  };
 
   DG_CUDA(launch_ex(dg::gemm::embed_kernel, dim3(M), dim3(dg::gemm::EMBED_THREADS), 0, s, 1, tok,
                     (const __nv_bfloat16*)f.m->embed, c.vocab, c.d, M, x, xb, ssq_x, group));
   count_launch();
   DG_CUDA(cudaGetLastError());
+  DG_TRY(collapse(ssq_x));
   for (int l = 0; l < c.n_layers; ++l) {
     const dg_layer_weights& w = f.m->layers[l];
     const bool last = l == c.n_layers - 1;
@@ -938,7 +956,7 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
     GemmEpi eq;  // QKV of RMSNorm(x)
     eq.epi = dg::gemm::EPI_BF16;
     eq.out_bf16 = qkv;
-    eq.ssq_in = ssq_x; eq.n_ssq_in = nt; eq.inv_k = 1.f / c.d; eq.eps = c.eps;
+    eq.ssq_in = ssq_x; eq.n_ssq_in = n_use; eq.inv_k = 1.f / c.d; eq.eps = c.eps;
     DG_TRY(proj(xb, w.w_qkv, q8 ? q8->w_qkv : nullptr, 0, nqkv, c.d, eq, true));
     if (f.commit_kv) {
       const void* kb = qkv + hq * hd;
@@ -954,25 +972,27 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
     eo.epi = dg::gemm::EPI_RESID;
     eo.x = x; eo.out_bf16 = xb; eo.ssq_out = ssq_h;
     DG_TRY(proj(ao, w.w_o, q8 ? q8->w_o : nullptr, 1, c.d, hq * hd, eo, resid_pair));
+    DG_TRY(collapse(ssq_h));
     GemmEpi eu;  // gelu(RMSNorm(h) w_up^T)
     eu.epi = dg::gemm::EPI_GELU;
     eu.out_bf16 = up;
-    eu.ssq_in = ssq_h; eu.n_ssq_in = nt; eu.inv_k = 1.f / c.d; eu.eps = c.eps;
+    eu.ssq_in = ssq_h; eu.n_ssq_in = n_use; eu.inv_k = 1.f / c.d; eu.eps = c.eps;
     DG_TRY(proj(xb, w.w_up, q8 ? q8->w_up : nullptr, 2, c.ffn, c.d, eu, true));
     GemmEpi ed;  // x = h + u w_down^T
     ed.epi = dg::gemm::EPI_RESID;
     ed.x = x; ed.out_bf16 = xb; ed.ssq_out = ssq_x;
     DG_TRY(proj(up, w.w_down, q8 ? q8->w_down : nullptr, 3, c.d, c.ffn, ed, resid_pair));
+    DG_TRY(collapse(ssq_x));
   }
   if (f.want_logits && !f.unembed_elsewhere) {
     // logits of RMSNorm(x), on e4m3 operands when the model carries them
     if (f.m->unembed_e4m3) {
       DG_TRY(quantize_hidden(f, s));
       const Fp8Scales f8{(const float*)(f.ws + f.L.as), f.m->unembed_scale};
-      DG_TRY(launch_unembed(f.ws + f.L.aq, f.m->unembed_e4m3, logits, M, c.d, c.vocab, ssq_x, nt,
+      DG_TRY(launch_unembed(f.ws + f.L.aq, f.m->unembed_e4m3, logits, M, c.d, c.vocab, ssq_x, n_use,
                             1.f / c.d, c.eps, s, &f8));
     } else {
-      DG_TRY(launch_unembed(xb, f.m->unembed, logits, M, c.d, c.vocab, ssq_x, nt, 1.f / c.d,
+      DG_TRY(launch_unembed(xb, f.m->unembed, logits, M, c.d, c.vocab, ssq_x, n_use, 1.f / c.d,
                             c.eps, s));
     }
   }
@@ -1478,7 +1498,7 @@ int dg_denoise_block(const dg_model* m, dg_state* st, const dg_sampler_cfg* cfg,
   const bool fp8 = m->unembed_e4m3 != nullptr;  // check_model: vocab % 256 == 0 then
   Fwd fl = f;
   fl.unembed_elsewhere = fused;
-  const int nt = m->cfg.d / ssq_group(m->cfg, B * C, m->layers_e4m3 != nullptr);
+  const int nt = ssq_partials_read(m->cfg, B * C, m->layers_e4m3 != nullptr);
   // one denoising step: forward pass, unembedding + sampler, step advance
   auto enqueue_step = [&](cudaStream_t q) -> int {
     DG_TRY(run_forward(fl, st->tok, logits, q));
