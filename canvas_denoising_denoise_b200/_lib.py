@@ -85,6 +85,8 @@ SIGNATURES = {
     "dg_linear": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_void_p,
                           c_size_t, c_void_p]),
     "dg_linear_workspace_bytes": (c_size_t, [c_int, c_int, c_int]),
+    "dg_linear_plan_of": (c_int, [c_int, c_int, c_int, c_int]),
+    "dg_model_residual_on_pairs": (c_int, [P(ModelCfg), c_int, c_int]),
     "dg_sample_commit": (c_int, [c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, P(SamplerCfg),
                                  c_uint32, c_int, c_int, c_int, c_int, c_int, P(StepOut),
                                  c_void_p, c_size_t, c_void_p]),

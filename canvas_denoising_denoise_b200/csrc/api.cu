@@ -1175,6 +1175,17 @@ int dg_unembed(const void* h, const void* w_u, float* logits, int M, int d, int 
   return launch_unembed(h, w_u, logits, M, d, V, nullptr, 0, 0.f, 0.f, (cudaStream_t)stream);
 }
 
+int dg_linear_plan_of(int M, int N, int K, int e4m3) {
+  const int kbe = e4m3 ? 128 : dg::gemm::BK;
+  if (M <= 0 || N <= 0 || K <= 0 || N % 128 || K % kbe) return -1;
+  return proj_use_pair(M, N, K, e4m3 != 0) ? DG_PLAN_PAIRS : DG_PLAN_SPLIT_K;
+}
+
+int dg_model_residual_on_pairs(const dg_model_cfg* cfg, int M, int e4m3) {
+  if (!cfg || M < 1) return -1;
+  return resid_on_pair(*cfg, M, e4m3 != 0) ? 1 : 0;
+}
+
 size_t dg_linear_workspace_bytes(int M, int N, int K) {
   (void)M;
   (void)N;

@@ -249,6 +249,25 @@ int dg_linear(const void* x, const void* w, void* out, int M, int N, int K, int 
               void* workspace, size_t workspace_bytes, void* stream);
 size_t dg_linear_workspace_bytes(int M, int N, int K);
 
+/* Execution plans of the projections (host-side queries; no device work). */
+enum dg_linear_plan {
+  DG_PLAN_SPLIT_K = 0,  /* tcgen05 GEMM, K split over a thread-block cluster */
+  DG_PLAN_PAIRS = 1     /* persistent grid of CTA pairs, 256 x 256 tiles */
+};
+
+/*
+ * dg_linear_plan_of - the plan dg_linear (e4m3 = 0) or dg_linear_e4m3
+ * (e4m3 != 0) uses for this shape; -1 for a shape they reject.
+ * dg_model_residual_on_pairs - 1 when a forward pass of the model over M
+ * tokens runs both residual projections (output, K = Hq hd; MLP down, K = F)
+ * on CTA pairs, which then write the residual's sums of squares per 32
+ * features and collapse them once per token; 0 otherwise (per 128 features,
+ * read as written); -1 for a null cfg or M < 1.  The two projections always
+ * take one plan together.
+ */
+int dg_linear_plan_of(int M, int N, int K, int e4m3);
+int dg_model_residual_on_pairs(const dg_model_cfg* cfg, int M, int e4m3);
+
 /*
  * dg_sample_commit - one sampler step over logits [B, C, V] fp32.
  * Source: Google docs table "Configuracao de exibicao recomendada" (step cap,

@@ -165,3 +165,49 @@ def test_kv_block_commit_rejects_bad_arguments(lib):
     assert call(128, nl=65) == INVALID             # more layers than the tables hold
     assert lib.dg_kv_block_commit(tab, tab, 1024, tab, tab, NULL, 2, 1, 8, 256, 128, 4352,
                                   None) == INVALID
+
+
+def test_projection_plans(lib):
+    """One canvas takes the split-K GEMM; many tokens the CTA pairs (a full
+    wave of 74 pairs of 256 x 256 tiles, or 48 tiles and more with 1536 tokens
+    and more), when N is a multiple of 256 and K holds four 128-byte k-blocks."""
+    SK, PR = 0, 1
+    plan = lib.dg_linear_plan_of
+    assert plan(256, 2048, 8192, 0) == SK          # one canvas, MLP down: 8 tiles
+    assert plan(256, 262144, 2048, 0) == PR        # 1024 tiles
+    assert plan(4096, 2048, 2048, 0) == PR         # 128 tiles
+    assert plan(1024, 4096, 2048, 0) == SK         # 64 tiles, 1024 tokens
+    assert plan(1536, 2048, 2048, 0) == PR         # 48 tiles, 1536 tokens
+    assert plan(1535, 2048, 2048, 0) == SK         # 48 tiles, 1535 tokens
+    assert plan(1600, 2048, 512, 0) == PR          # 56 tiles, ragged token tile
+    assert plan(4096, 2048 + 128, 2048, 0) == SK   # N not a multiple of 256
+    assert plan(4096, 2048, 192, 0) == SK          # three bf16 k-blocks
+    assert plan(4096, 2048, 384, 1) == SK          # three e4m3 k-blocks
+    assert plan(4096, 2048, 512, 1) == PR
+    assert plan(4096, 2048, 100, 0) == -1          # K % 64
+    assert plan(4096, 2048, 192, 1) == -1          # K % 128 on e4m3 codes
+    assert plan(0, 2048, 2048, 0) == -1
+
+
+def test_residual_projections_share_one_plan(lib, L):
+    """The output and MLP-down projections write the sums of squares the next
+    norm reads: they take the pairs together or not at all."""
+    tiny = L.ModelCfg(256, 2, 4, 2, 64, 1024, 512, 1e-6)
+    full = L.ModelCfg(2048, 24, 16, 8, 128, 8192, 262144, 1e-6)
+
+    def on_pairs(cfg, M, e4m3):
+        return lib.dg_model_residual_on_pairs(ctypes.byref(cfg), M, e4m3)
+    assert on_pairs(full, 256, 0) == 0             # one canvas
+    assert on_pairs(full, 2048, 0) == 1            # eight canvases: 64 tiles
+    assert on_pairs(full, 4096, 0) == 1            # a 4096-token prefill
+    assert on_pairs(full, 2048, 1) == 1
+    assert on_pairs(tiny, 48 * 256, 0) == 1        # d = 256: one tile per 256 tokens
+    assert on_pairs(tiny, 47 * 256, 0) == 0
+    # e4m3: Hq hd = 256 is two 128-wide k-blocks, so the output projection
+    # stays on the split-K GEMM, and the MLP down projection, which alone
+    # would qualify, stays with it
+    assert lib.dg_linear_plan_of(75 * 256, 256, 1024, 1) == 1
+    assert lib.dg_linear_plan_of(75 * 256, 256, 256, 1) == 0
+    assert on_pairs(tiny, 75 * 256, 1) == 0
+    assert lib.dg_model_residual_on_pairs(None, 256, 0) == -1
+    assert on_pairs(full, 0, 0) == -1
