@@ -555,8 +555,9 @@ __global__ void __launch_bounds__(threads_for(PROJ_EPI_WARPS), 1)
   epi.rank = cluster_ctarank();
   epi.quarter = warp_id() & 3;
   epi.lane = lane_id();
-  // a weight tile is read by every token tile (consecutive tiles): keep it
-  // in L2 as long as the activations
+  // the pairs that share a weight tile run at the same time (token tile
+  // fastest), so the weights can go first from L2 while the activations,
+  // read by every weight tile, stay (evict-normal weights measured the same)
   pair_pipeline<PROJ_EPI_WARPS, KPS, F8>(&tm_w, &tm_x, l2_policy_evict_first(),
                                          l2_policy_evict_last(), sc, epi);
 }
