@@ -375,9 +375,7 @@ int launch_proj_pair(const void* x, const void* w, int M, int N, int K, const Ge
   namespace ue = dg::unembed;
   if (!proj_attr_done()) {
     DG_CUDA((proj_set_attrs<1, false>()));
-    DG_CUDA((proj_set_attrs<2, false>()));
     DG_CUDA((proj_set_attrs<1, true>()));
-    DG_CUDA((proj_set_attrs<2, true>()));
     proj_attr_done() = true;
   }
   CUtensorMap tw, tx;
@@ -401,8 +399,8 @@ int launch_proj_pair(const void* x, const void* w, int M, int N, int K, const Ge
   p.ssq_out = e.ssq_out;
   p.tok_scale = f8 ? f8->tok : nullptr;
   p.w_scale = f8 ? f8->w : nullptr;
-  const int nkb = K / (f8 ? 128 : dg::gemm::BK);
-  (void)nkb;
+  // one k-block per stage (two, 256 bytes per row request, measured the same
+  // here, unlike the unembedding's weight stream)
   auto* kern = f8 ? proj_kernel<1, true>(e.epi) : proj_kernel<1, false>(e.epi);
   DG_CUDA(launch_cluster(kern, dim3(2 * p.n_pairs), dim3(ue::threads_for(ue::PROJ_EPI_WARPS)),
                          ue::SMEM_BYTES, s, dim3(2, 1, 1), tw, tx, p));
