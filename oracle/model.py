@@ -191,12 +191,15 @@ def unembed_e4m3(hn, w_unembed):
 
 
 def forward(cfg, weights, tokens, k_cache, v_cache, prefix_len, causal,
-            bf16_storage=True, want_logits=True, e4m3_unembed=False, e4m3_layers=False):
+            bf16_storage=True, want_logits=True, e4m3_unembed=False, e4m3_layers=False,
+            logit_rows=None):
     """Run the stack over new rows of one sequence.
 
     tokens [Lq] int; k_cache/v_cache: per layer [Hkv, >=prefix_len, hd] arrays.
     Returns (logits [Lq, V] or None, list of per-layer (k_new, v_new)).
-    The embedding lookup has no scaling.
+    The embedding lookup has no scaling.  With logit_rows (indices into the
+    Lq rows) only those rows are unembedded, in that order: every row of the
+    stack is still computed, since attention mixes them.
     """
     x = weights["embed"][np.asarray(tokens)].astype(np.float64)
     kv = []
@@ -211,6 +214,8 @@ def forward(cfg, weights, tokens, k_cache, v_cache, prefix_len, causal,
     if not want_logits:
         return None, kv
     hn = _r(rmsnorm(x, cfg.eps), bf16_storage)
+    if logit_rows is not None:
+        hn = hn[np.asarray(logit_rows)]
     if e4m3_unembed:
         return unembed_e4m3(hn, weights["unembed"]), kv
     logits = hn @ weights["unembed"].T
@@ -241,11 +246,12 @@ def prefill(cfg, weights, prompt, k_cache, v_cache, bf16_storage=True, e4m3_laye
 
 
 def denoise_logits(cfg, weights, canvas, k_cache, v_cache, prefix_len, bf16_storage=True,
-                   e4m3_unembed=False, e4m3_layers=False):
-    """Bidirectional pass of the canvas over the cached prefix -> logits [C, V]."""
+                   e4m3_unembed=False, e4m3_layers=False, rows=None):
+    """Bidirectional pass of the canvas over the cached prefix -> logits [C, V]
+    (or [len(rows), V] for the canvas rows listed in `rows`)."""
     logits, _ = forward(cfg, weights, canvas, k_cache, v_cache, prefix_len, causal=False,
                         bf16_storage=bf16_storage, want_logits=True, e4m3_unembed=e4m3_unembed,
-                        e4m3_layers=e4m3_layers)
+                        e4m3_layers=e4m3_layers, logit_rows=rows)
     return logits
 
 
@@ -258,9 +264,9 @@ def block_commit(cfg, weights, block_tokens, k_cache, v_cache, prefix_len, bf16_
 
 def weights_to_f64(w_torch):
     """Convert a weight dict of bf16 torch tensors to fp64 NumPy arrays (exact)."""
-    out = {"embed": w_torch["embed"].float().numpy().astype(np.float64),
-           "unembed": w_torch["unembed"].float().numpy().astype(np.float64),
+    out = {"embed": w_torch["embed"].double().numpy(),
+           "unembed": w_torch["unembed"].double().numpy(),
            "layers": []}
     for lw in w_torch["layers"]:
-        out["layers"].append({k: v.float().numpy().astype(np.float64) for k, v in lw.items()})
+        out["layers"].append({k: v.double().numpy() for k, v in lw.items()})
     return out

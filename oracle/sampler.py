@@ -232,6 +232,10 @@ def sampler_step(cfg, logits, tok, committed, prev_argmax, step, seed, b, block,
                         (e_out - e_in) < tie_margin)
             if near_cut:
                 boundary[np.array(order[k - 1:k + 1], dtype=np.int64)] = True
+        elif 1 < k == uncommitted.size and abs(csum[k - 1] - cfg.entropy_bound) < tie_margin:
+            # everything selected with the sum just under the bound: a slightly
+            # larger sum would leave the last-ranked position out
+            boundary[order[k - 1]] = True
     else:
         lam_u = np.sort(lam[uncommitted])[::-1]
         if 0 < k < uncommitted.size and (lam_u[k - 1] - lam_u[k]) < tie_margin:

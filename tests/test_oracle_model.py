@@ -266,3 +266,21 @@ def test_e4m3_layers_close_to_bf16_forward():
         out.append(M.denoise_logits(TINY, w, canvas, kc, vc, L, e4m3_layers=e4m3))
     rel = np.linalg.norm(out[0] - out[1]) / np.linalg.norm(out[0])
     assert 1e-3 < rel < 0.1
+
+
+@pytest.mark.parametrize("e4m3", [False, True])
+def test_logit_rows_select_rows_of_the_full_unembedding(e4m3):
+    """denoise_logits(rows=r) is the r-th rows of the full result, bit for bit
+    (the selection happens after every row of the stack is computed)."""
+    w = rand_weights(TINY, seed=4)
+    kc, vc = M.empty_cache(TINY, 40)
+    L = M.prefill(TINY, w, np.arange(8) % TINY.vocab, kc, vc)
+    canvas = np.random.default_rng(2).integers(0, TINY.vocab, size=24)
+    full = M.denoise_logits(TINY, w, canvas, kc, vc, L, e4m3_unembed=e4m3)
+    rows = [17, 0, 5, 23]
+    part = M.denoise_logits(TINY, w, canvas, kc, vc, L, e4m3_unembed=e4m3, rows=rows)
+    if e4m3:
+        # per-token scales: each row's codes and scale depend on that row only
+        assert np.array_equal(part, full[rows])
+    else:
+        np.testing.assert_allclose(part, full[rows], rtol=1e-13, atol=1e-15)
