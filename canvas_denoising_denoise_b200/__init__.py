@@ -26,9 +26,15 @@ __all__ = ["canvas_attn", "unembed", "linear", "sample_commit", "unembed_sample_
            "quantize_e4m3", "linear_e4m3", "unembed_e4m3", "unembed_sample_commit_e4m3",
            "kv_block_commit", "philox",
            "DgModel", "DgState", "SamplerSettings", "prefill", "denoise_logits", "denoise_block",
+           "linear_plan_of", "model_residual_on_pairs", "set_wait_limit_ns", "self_test_wait",
            "check_device_errors", "Workspace", "DgError", "MASK_BIDIR", "MASK_CAUSAL",
            "EPI_F32", "EPI_BF16", "EPI_GELU_BF16", "EPI_RESID_F32", "UNSELECTED_KEEP",
            "UNSELECTED_RENOISE"]
+
+
+# dg_step_out fields, in order: x_hat, argmax (int32 [B, C]), logconf,
+# entropy (fp32 [B, C]), flags (uint8 [B, C]), near_ties (int32 [B, 3])
+_OUT_KEYS = ("x_hat", "argmax", "logconf", "entropy", "flags", "near_ties")
 
 
 def _stream(stream=None):
@@ -160,7 +166,7 @@ def sample_commit(logits, tok, committed, prev_argmax, seq_status, settings, see
     """One sampler step over logits [B, C, V] fp32; updates the canvas in place.
 
     out: optional dict of device tensors [B, C]: x_hat, argmax (int32),
-    logconf, entropy (fp32), flags (uint8).
+    logconf, entropy (fp32), flags (uint8); and near_ties (int32 [B, 3]).
     """
     _need_contig(logits, tok, committed, prev_argmax, seq_status)
     lib = _lib.load()
@@ -168,7 +174,7 @@ def sample_commit(logits, tok, committed, prev_argmax, seq_status, settings, see
     so = None
     if out is not None:
         so = _lib.StepOut(*[(out[k].data_ptr() if out.get(k) is not None else None)
-                            for k in ("x_hat", "argmax", "logconf", "entropy", "flags")])
+                            for k in _OUT_KEYS])
     wp, wn = _ws(ws).args(lib.dg_sample_commit_workspace_bytes(B, C, V))
     _lib.check(lib.dg_sample_commit(_ptr(logits), _ptr(tok), _ptr(committed), _ptr(prev_argmax),
                                     _ptr(seq_status), ctypes.byref(settings.c), seed, block, step,
@@ -190,7 +196,7 @@ def unembed_sample_commit(h, w_u, tok, committed, prev_argmax, seq_status, setti
     so = None
     if out is not None:
         so = _lib.StepOut(*[(out[k].data_ptr() if out.get(k) is not None else None)
-                            for k in ("x_hat", "argmax", "logconf", "entropy", "flags")])
+                            for k in _OUT_KEYS])
     wp, wn = _ws(ws).args(lib.dg_unembed_sample_commit_workspace_bytes(B, C, V))
     _lib.check(lib.dg_unembed_sample_commit(
         _ptr(h), _ptr(w_u), d, _ptr(tok), _ptr(committed), _ptr(prev_argmax), _ptr(seq_status),
@@ -235,7 +241,7 @@ def unembed_sample_commit_e4m3(h_q, h_scale, w_q, w_scale, tok, committed, prev_
     so = None
     if out is not None:
         so = _lib.StepOut(*[(out[k].data_ptr() if out.get(k) is not None else None)
-                            for k in ("x_hat", "argmax", "logconf", "entropy", "flags")])
+                            for k in _OUT_KEYS])
     wp, wn = _ws(ws).args(lib.dg_unembed_sample_commit_workspace_bytes(B, C, V))
     _lib.check(lib.dg_unembed_sample_commit_e4m3(
         _ptr(h_q), _ptr(h_scale), _ptr(w_q), _ptr(w_scale), d, _ptr(tok), _ptr(committed),
@@ -264,6 +270,17 @@ def philox(inp, out, stream=None):
     _need_contig(inp, out)
     _lib.check(_lib.load().dg_philox4x32_10(_ptr(inp), _ptr(out), inp.shape[0], _stream(stream)))
     return out
+
+
+def set_wait_limit_ns(ns, stream=None):
+    """Wait limit of the kernels' bounded waits on the current device (0: the 2 s default)."""
+    _lib.check(_lib.load().dg_set_wait_limit_ns(int(ns), _stream(stream)))
+
+
+def self_test_wait(kind=0, stream=None):
+    """Launch a kernel whose wait can never complete (0: one CTA, 1: a CTA pair);
+    check_device_errors() then reports DG_ERR_TIMEOUT."""
+    _lib.check(_lib.load().dg_self_test_wait(int(kind), _stream(stream)))
 
 
 class DgModel:
@@ -359,6 +376,16 @@ def prefill(model, state, prompt, ws=None, stream=None):
     wp, wn = _ws(ws).args(need)
     _lib.check(lib.dg_prefill(ctypes.byref(model.c), ctypes.byref(state.c), _ptr(prompt), P, wp, wn,
                               _stream(stream)))
+
+
+def linear_plan_of(M, N, K, e4m3=False):
+    """The plan dg_linear (or dg_linear_e4m3) uses for this shape: 0 split-K, 1 CTA pairs, -1 rejected."""
+    return _lib.load().dg_linear_plan_of(M, N, K, 1 if e4m3 else 0)
+
+
+def model_residual_on_pairs(model, M, e4m3=False):
+    """1 when a forward pass of `model` over M tokens runs its residual projections on CTA pairs."""
+    return _lib.load().dg_model_residual_on_pairs(ctypes.byref(model.cfg), M, 1 if e4m3 else 0)
 
 
 def denoise_workspace_bytes(model, state):

@@ -57,7 +57,7 @@ class SamplerCfg(ctypes.Structure):
 
 class StepOut(ctypes.Structure):
     _fields_ = [("x_hat", c_void_p), ("argmax", c_void_p), ("logconf", c_void_p),
-                ("entropy", c_void_p), ("flags", c_void_p)]
+                ("entropy", c_void_p), ("flags", c_void_p), ("near_ties", c_void_p)]
 
 
 class State(ctypes.Structure):
@@ -118,6 +118,8 @@ SIGNATURES = {
                                  c_void_p, c_size_t, c_void_p]),
     "dg_denoise_block_workspace_bytes": (c_size_t, [P(ModelCfg), c_int, c_int, c_int]),
     "dg_philox4x32_10": (c_int, [c_void_p, c_void_p, c_int, c_void_p]),
+    "dg_set_wait_limit_ns": (c_int, [ctypes.c_uint64, c_void_p]),
+    "dg_self_test_wait": (c_int, [c_int, c_void_p]),
 }
 
 _LIB = None

@@ -25,6 +25,7 @@
 #include "quant.cuh"
 #include "unembed.cuh"
 #include "sampler.cuh"
+#include "selftest.cuh"
 
 namespace {
 
@@ -499,15 +500,10 @@ int attn_pairs(int Hq, int Hkv, int Lq) {
   return cdiv((Hq / Hkv) * cdiv(Lq, dg::attn::BQ), 2);
 }
 
+// The split count depends on the shape only (it sets the summation order,
+// so a shape always gives the same bits).
 int attn_splits(int B, int Hq, int Hkv, int Lq, int max_prefix) {
-  static const int forced = [] {
-    const char* e = getenv("DG_ATTN_SPLITS");  // tuning override
-    return e ? atoi(e) : 0;
-  }();
   const int units = B * Hkv * attn_pairs(Hq, Hkv, Lq);
-  if (forced > 0)
-    return std::min({forced, dg::attn::MAX_SPLITS,
-                     std::max(1, cdiv(max_prefix, dg::attn::BKV) + cdiv(Lq, dg::attn::BKV))});
   const int tmax = cdiv(max_prefix, dg::attn::BKV) + cdiv(Lq, dg::attn::BKV);
   int s = std::max(1, kNumSMs / std::max(1, units));
   s = std::min(s, std::max(1, tmax / 2));
@@ -640,6 +636,7 @@ dg::SampleParams make_sample_params(const dg_sampler_cfg& cfg, uint32_t seed, in
   p.policy = cfg.unselected_policy;
   p.selection = cfg.selection;
   p.entropy_bound = cfg.entropy_bound;
+  p.near_ties = nullptr;
   return p;
 }
 
@@ -651,8 +648,11 @@ int launch_sample(const float* logits, int32_t* tok, uint8_t* committed, int32_t
                     0, s, 1, logits, (const int32_t*)seq_status, p, part));
   count_launch();
   const int threads = (p.C + 31) / 32 * 32;
+  dg::SampleParams pc = p;
+  pc.near_ties = out ? out->near_ties : nullptr;
   DG_CUDA(launch_ex(dg::sample_commit_kernel, dim3(p.B), dim3(threads), 0, s, 1, logits,
-                    (const dg::RowPartial*)part, (const dg::RowStats*)nullptr, p, tok, committed, prev_argmax, seq_status,
+                    (const dg::RowPartial*)part, (const dg::RowStats*)nullptr, pc, tok, committed,
+                    prev_argmax, seq_status,
                     out ? out->x_hat : (int32_t*)nullptr, out ? out->argmax : (int32_t*)nullptr,
                     out ? out->logconf : (float*)nullptr, out ? out->entropy : (float*)nullptr,
                     out ? out->flags : (uint8_t*)nullptr));
@@ -744,9 +744,11 @@ int launch_unembed_sample(const void* h, const void* w_u, int d, const float* ss
                     (const uint8_t*)committed, sp, stats));
   count_launch();
   const int threads = (sp.C + 31) / 32 * 32;
+  dg::SampleParams pc = sp;
+  pc.near_ties = out ? out->near_ties : nullptr;
   DG_CUDA(launch_ex(dg::sample_commit_kernel, dim3(sp.B), dim3(threads), 0, s, 1,
                     (const float*)nullptr, (const dg::RowPartial*)nullptr,
-                    (const dg::RowStats*)stats, sp, tok, committed, prev_argmax, seq_status,
+                    (const dg::RowStats*)stats, pc, tok, committed, prev_argmax, seq_status,
                     out ? out->x_hat : (int32_t*)nullptr, out ? out->argmax : (int32_t*)nullptr,
                     out ? out->logconf : (float*)nullptr, out ? out->entropy : (float*)nullptr,
                     out ? out->flags : (uint8_t*)nullptr));
@@ -1573,6 +1575,43 @@ int dg_philox4x32_10(const uint32_t* in, uint32_t* out, int n, void* stream) {
   if (!in || !out || n < 0) return fail(DG_ERR_INVALID_ARG, "dg_philox4x32_10: bad arguments");
   if (n == 0) return DG_OK;
   dg::philox_kernel<<<cdiv(n, 256), 256, 0, (cudaStream_t)stream>>>(in, out, n);
+  count_launch();
+  DG_CUDA(cudaGetLastError());
+  return DG_OK;
+}
+
+int dg_set_wait_limit_ns(uint64_t ns, void* stream) {
+  if (ns != 0 && (ns < 1000ull || ns > 600000000000ull))
+    return fail(DG_ERR_INVALID_ARG, "dg_set_wait_limit_ns: %llu ns is outside [1 us, 600 s]",
+                (unsigned long long)ns);
+  const uint64_t v = ns ? ns : dg::kWaitLimitDefaultNs;
+  cudaStream_t s = (cudaStream_t)stream;
+  DG_CUDA(cudaMemcpyToSymbolAsync(dg::g_wait_limit_ns, &v, sizeof(v), 0, cudaMemcpyHostToDevice,
+                                  s));
+  DG_CUDA(cudaStreamSynchronize(s));
+  return DG_OK;
+}
+
+int dg_self_test_wait(int kind, void* stream) {
+  cudaStream_t s = (cudaStream_t)stream;
+  if (kind == 0) {
+    dg::wait_selftest_kernel<<<1, 32, 0, s>>>();
+  } else if (kind == 1) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(2);
+    cfg.blockDim = dim3(32);
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    DG_CUDA(cudaLaunchKernelEx(&cfg, dg::wait_pair_selftest_kernel));
+  } else {
+    return fail(DG_ERR_INVALID_ARG, "dg_self_test_wait: kind %d is not 0 or 1", kind);
+  }
   count_launch();
   DG_CUDA(cudaGetLastError());
   return DG_OK;

@@ -33,9 +33,12 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
-// Waits give up after this long (ns).  Healthy waits in these kernels last
-// microseconds; two seconds means something upstream never arrived.
-constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Waits give up after g_wait_limit_ns (per device; dg_set_wait_limit_ns sets
+// it, default two seconds).  Healthy waits in these kernels last microseconds;
+// a wait that reaches the limit means something upstream never arrived.  The
+// limit is read only on a wait's slow path, after its first poll failed.
+constexpr uint64_t kWaitLimitDefaultNs = 2000000000ull;
+__constant__ uint64_t g_wait_limit_ns = kWaitLimitDefaultNs;
 
 // Programmatic dependent launch.  A kernel launched with programmatic stream
 // serialization may start before its predecessor finishes; it must call
@@ -94,11 +97,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
                                           uint32_t site) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = g_wait_limit_ns;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 15u) == 0) {
       if (abort != nullptr && *abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit) {
         raise_error(ERR_TIMEOUT | site, blockIdx.x);
         if (abort != nullptr) *abort = 1;
         return false;
@@ -411,11 +415,12 @@ __device__ __forceinline__ bool mbar_wait_pair(uint64_t* bar, uint32_t parity,
                                                uint32_t site) {
   if (mbar_try_wait_cluster(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
+  const uint64_t limit = g_wait_limit_ns;
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait_cluster(bar, parity)) return true;
     if ((it & 15u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit) {
         raise_error(ERR_TIMEOUT | site, blockIdx.x);
         *abort = 1;
         st_cluster_u32(abort_peer, 1u);

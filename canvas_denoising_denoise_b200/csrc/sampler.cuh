@@ -234,7 +234,12 @@ struct SampleParams {
   int policy;
   int selection;             // 0: top commit_k by confidence, 1: entropy-bounded
   float entropy_bound;
+  int32_t* near_ties;        // optional [B, 3] decision counters (sample_commit_kernel)
 };
+
+// A decision whose deciding quantity lies within this distance (log space,
+// nats) of flipping is counted as a near-tie.
+constexpr float kNearTieMargin = 1e-4f;
 
 __device__ __forceinline__ int read_step(const SampleParams& p) {
   return p.step_ptr ? *p.step_ptr : p.step_val;
@@ -422,6 +427,9 @@ __global__ void __launch_bounds__(1024) sample_commit_kernel(
   __shared__ uint8_t s_unc[1024];
   __shared__ float s_red[32];
   __shared__ int s_flag;
+  __shared__ float s_mean_h;
+  __shared__ float s_cut[2];    // selection key (confidence, or entropy) at ranks k - 1 and k
+  __shared__ double s_csum[2];  // entropy-bounded: entropies summed through those ranks
 
   griddep_wait();
   griddep_launch();
@@ -484,6 +492,9 @@ __global__ void __launch_bounds__(1024) sample_commit_kernel(
     const bool crit = (mean_h < p.stop_entropy) && step >= 1 && all_same;
     const bool cap = step >= p.max_steps - 1;
     s_flag = (crit || cap) ? 1 : 0;
+    s_mean_h = mean_h;
+    s_cut[0] = s_cut[1] = 0.f;
+    s_csum[0] = s_csum[1] = 0.0;
   }
   if (live) {
     s_lam[i] = lam;
@@ -494,12 +505,14 @@ __global__ void __launch_bounds__(1024) sample_commit_kernel(
   const bool final_step = s_flag != 0;
 
   bool selected = false;
+  int rank = -1;       // rank among the uncommitted positions, in selection order
+  double csum = 0.0;   // entropy-bounded: the entropies summed through this rank
   if (live && !was_committed && p.selection == 1) {
     // entropy-bounded: rank by (entropy, position) among the uncommitted; the
     // selection is the ranked prefix whose entropies sum to <= the bound, and
     // at least rank 0 (the sum is taken in fp64: order-independent)
-    int rank = 0;
-    double csum = static_cast<double>(ent);
+    rank = 0;
+    csum = static_cast<double>(ent);
     for (int j = 0; j < p.C; ++j) {
       if (s_unc[j] && j != i) {
         const float ej = s_ent[j];
@@ -513,7 +526,7 @@ __global__ void __launch_bounds__(1024) sample_commit_kernel(
   } else if (live && !was_committed) {
     // top-k among uncommitted: rank = number of uncommitted positions that beat this one
     const int k = min(p.commit_k, n_unc);
-    int rank = 0;
+    rank = 0;
     for (int j = 0; j < p.C; ++j) {
       if (s_unc[j]) {
         const float lj = s_lam[j];
@@ -521,6 +534,47 @@ __global__ void __launch_bounds__(1024) sample_commit_kernel(
       }
     }
     selected = rank < k;
+  }
+
+  if (p.near_ties != nullptr) {
+    // Decisions within kNearTieMargin of flipping, per sequence:
+    // [0] positions at the commit cut: the keys on either side of the cut
+    //     nearly tie (then the uncommitted positions near the cut count), or,
+    //     entropy-bounded, a sum through the cut nearly meets the bound;
+    // [1] committed positions whose confidence is near the re-noise threshold;
+    // [2] 1 when the mean entropy is near the stop threshold.
+    const float m = kNearTieMargin;
+    const int n_sel = __syncthreads_count(selected);
+    const float key = p.selection == 1 ? ent : lam;
+    if (rank >= 0 && rank == n_sel - 1) { s_cut[0] = key; s_csum[0] = csum; }
+    if (rank >= 0 && rank == n_sel) { s_cut[1] = key; s_csum[1] = csum; }
+    __syncthreads();
+    const double bound = static_cast<double>(p.entropy_bound);
+    bool cut = false;
+    float edge = 0.f;
+    if (n_sel > 0 && n_sel < n_unc) {
+      if (p.selection == 1) {
+        cut = fabs(s_csum[1] - bound) < m || fabs(s_csum[0] - bound) < m ||
+              (s_cut[1] - s_cut[0]) < m;
+      } else {
+        cut = (s_cut[0] - s_cut[1]) < m;
+        edge = 0.5f * (s_cut[0] + s_cut[1]);
+      }
+    } else if (p.selection == 1 && n_sel > 1 && n_sel == n_unc) {
+      cut = fabs(s_csum[0] - bound) < m;  // all selected, the sum just under the bound
+    }
+    bool at_cut = false;
+    if (cut && rank >= 0) {
+      at_cut = p.selection == 1 ? (rank == n_sel - 1 || (n_sel < n_unc && rank == n_sel))
+                                : fabsf(lam - edge) < m;
+    }
+    const int n_cut = __syncthreads_count(at_cut);
+    const int n_ren = __syncthreads_count(live && was_committed && fabsf(lam - p.log_tau) < m);
+    if (i == 0) {
+      p.near_ties[b * 3 + 0] = n_cut;
+      p.near_ties[b * 3 + 1] = n_ren;
+      p.near_ties[b * 3 + 2] = fabsf(s_mean_h - p.stop_entropy) < m ? 1 : 0;
+    }
   }
 
   int new_tok = cur;

@@ -43,6 +43,11 @@
  *     dg_check_device_errors() synchronises the stream, reads and clears it.
  *   - Device pointers must be 16-byte aligned; matrices are row-major with the
  *     last dimension contiguous.  bf16 means IEEE bfloat16.
+ *   - Two environment variables change how work is scheduled, never what it
+ *     computes: DG_PDL=0 launches kernels without programmatic dependent
+ *     launch (each starts once its predecessor has finished), DG_GRAPHS=0
+ *     makes dg_denoise_block launch every step directly instead of replaying
+ *     a CUDA graph.  Both are read once per process.
  */
 #ifndef DG_H_
 #define DG_H_
@@ -153,13 +158,30 @@ typedef struct dg_sampler_cfg {
   float entropy_bound;  /* DG_SELECT_ENTROPY: summed-entropy limit, nats (0.1) */
 } dg_sampler_cfg;
 
-/* Per-step sampler diagnostics: caller-owned device arrays [B, C]; any may be NULL. */
+/* Per-step sampler diagnostics: caller-owned device arrays; any may be NULL.
+ * near_ties counts, per sequence, the step's decisions that lie within 1e-4
+ * (nats) of flipping, so that a caller comparing two implementations can
+ * tell a rounding-level disagreement from a real one:
+ *   [b*3 + 0] positions at the commit cut: with top-k, when the k-th and
+ *             (k+1)-th largest log confidences of the uncommitted positions
+ *             differ by less than 1e-4, the uncommitted positions within 1e-4
+ *             of their midpoint; with DG_SELECT_ENTROPY, the last selected and
+ *             first unselected positions when a sum of entropies through
+ *             either lies within 1e-4 of entropy_bound or their entropies
+ *             differ by less than 1e-4 (the last selected alone when every
+ *             uncommitted position was selected with a sum within 1e-4 of it);
+ *   [b*3 + 1] committed positions whose log confidence is within 1e-4 of
+ *             ln(renoise_conf);
+ *   [b*3 + 2] 1 when the mean entropy is within 1e-4 of stop_entropy.
+ * The top-2 margins of the raw logits and of the Gumbel-perturbed scores are
+ * not counted: the row pass keeps only each position's leader. */
 typedef struct dg_step_out {
-  int32_t* x_hat;     /* the Gumbel-max sample of each position */
-  int32_t* argmax;    /* argmax of the raw logits (the step's "prediction") */
-  float* logconf;     /* log softmax confidence (tempered) of the token at stake */
-  float* entropy;     /* tempered entropy, nats */
-  uint8_t* flags;     /* bit0: committed this step, bit1: re-noised this step */
+  int32_t* x_hat;     /* [B, C] the Gumbel-max sample of each position */
+  int32_t* argmax;    /* [B, C] argmax of the raw logits (the step's "prediction") */
+  float* logconf;     /* [B, C] log softmax confidence (tempered) of the token at stake */
+  float* entropy;     /* [B, C] tempered entropy, nats */
+  uint8_t* flags;     /* [B, C] bit0: committed this step, bit1: re-noised this step */
+  int32_t* near_ties; /* [B, 3] near-tie counters (above); untouched for stopped sequences */
 } dg_step_out;
 
 /*
@@ -363,10 +385,13 @@ int dg_unembed_sample_commit_e4m3(const uint8_t* h_q, const float* h_scale, cons
  * device array that every GPU loading the library keeps until process exit;
  * nothing is allocated per call (no cudaMalloc, cudaFree or allocating library
  * routine).  Sizes whose scratch exceeds 4 MiB (dg_sample_commit_workspace_bytes
- * of B, C, V; e.g. B > 32 at C = 256, V = 262144) return
- * DG_ERR_UNSUPPORTED_SHAPE.  The first call on a device looks up the array's
- * device address (cudaGetSymbolAddress) with that device current; make that
- * first call before any stream capture.  All calls share the one array and it
+ * of B, C, V: 32 bytes per position and 65536-entry vocabulary chunk, so at
+ * C = 256, V = 262144 up to B = 128) return DG_ERR_UNSUPPORTED_SHAPE.  The
+ * first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current and keeps it for the life
+ * of the process; make that first call before any stream capture.  A device
+ * reset (cudaDeviceReset) between calls is not supported: the module may be
+ * reloaded elsewhere and the kept address would be stale.  All calls share the one array and it
  * keeps the last call's contents (every slot read is written earlier in the
  * same call, so nothing needs clearing); calls that overlap on the GPU - on
  * different streams, or from different threads - race on it and must be
@@ -396,7 +421,14 @@ int dg_kv_block_commit(const void* const* k_blk, const void* const* v_blk, int l
 /*
  * dg_prefill - causal pass of prompts [B, P] (device int32) through the
  * model; writes their K/V to cache rows [0, P) and sets cache_len to P
- * (and st->cache_len_host).  Workspace: dg_prefill_workspace_bytes().
+ * (and st->cache_len_host).
+ * Source: "DiffusionGemma Guia do Desenvolvedor ...", section "Block
+ * Autoregressive Diffusion para Sequencias Longas", the Prefill bullet (the
+ * prompt is processed with ordinary causal attention and its keys and values
+ * go to the KV cache); aiexpert.news architecture paragraph (the same prefill
+ * machinery as an autoregressive model); Google docs page "DiffusionGemma",
+ * bullet "Arquitetura de codificador-decodificador" (an autoregressive
+ * encoder caches the context).  Workspace: dg_prefill_workspace_bytes().
  */
 int dg_prefill(const dg_model* m, dg_state* st, const int32_t* prompt, int P,
                void* workspace, size_t workspace_bytes, void* stream);
@@ -416,6 +448,17 @@ int dg_denoise_logits(const dg_model* m, const dg_state* st, float* logits,
 /*
  * dg_denoise_block - denoise one canvas per sequence to its adaptive stop,
  * re-encode it causally and commit its K/V (cache_len += C).
+ * Source: "DiffusionGemma Guia do Desenvolvedor ...", section "Block
+ * Autoregressive Diffusion para Sequencias Longas", the Denoising bullet (a
+ * 256-token block is refined in parallel by bidirectional attention over the
+ * cached prefix and, once finished, committed to the KV cache before the next
+ * block starts) and section "Difusao de Estado Uniforme" (the block starts
+ * as random placeholder tokens); Google docs page "DiffusionGemma", table
+ * "Configuracao de exibicao recomendada" (48-step cap, linear 0.8 -> 0.4
+ * temperature, adaptive stop on mean entropy below 0.005 with two identical
+ * consecutive predictions).  The committed K/V are those of a causal pass
+ * over the finished block, so a block-committed cache equals a one-shot
+ * causal prefill of the same tokens.
  * Initialises the canvas with uniform tokens (Philox tag 2, counter
  * (0, pos | 2 << 24, 0, block)), runs sampler steps until every sequence has
  * stopped (dg_sample_commit semantics), then the causal re-encode and the
@@ -439,6 +482,27 @@ size_t dg_denoise_block_workspace_bytes(const dg_model_cfg* cfg, int B, int C, i
  * out: device uint32 [n, 4].
  */
 int dg_philox4x32_10(const uint32_t* in, uint32_t* out, int n, void* stream);
+
+/*
+ * Failure detection.  The pages have no counterpart: these serve the
+ * library's own fault handling.  Every wait inside the kernels (on an
+ * mbarrier, a CTA-pair barrier or a counter) polls a clock and gives up once
+ * it has waited longer than the device's wait limit; it then records
+ * DG_ERR_TIMEOUT in the device error word, releases the kernel's other roles
+ * and returns, so a lost arrival never hangs the GPU.
+ *
+ * dg_set_wait_limit_ns - set the wait limit of the current device, in ns
+ *   (1 us .. 600 s; 0 restores the default of 2 s).  Enqueued on `stream`,
+ *   which it then synchronises; kernels launched afterwards use the new limit.
+ * dg_self_test_wait - launch a tiny kernel that waits on an mbarrier nothing
+ *   arrives at: kind 0 one CTA (the single-CTA pipeline wait), kind 1 a
+ *   cluster of two CTAs (the CTA-pair wait, which also raises the peer's abort
+ *   flag).  After it, dg_check_device_errors() returns DG_ERR_TIMEOUT; with a
+ *   short limit set first that takes about the limit.  Nothing traps and the
+ *   context stays usable.
+ */
+int dg_set_wait_limit_ns(uint64_t ns, void* stream);
+int dg_self_test_wait(int kind, void* stream);
 
 #ifdef __cplusplus
 }

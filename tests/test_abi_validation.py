@@ -211,3 +211,13 @@ def test_residual_projections_share_one_plan(lib, L):
     assert on_pairs(tiny, 75 * 256, 1) == 0
     assert lib.dg_model_residual_on_pairs(None, 256, 0) == -1
     assert on_pairs(full, 0, 0) == -1
+
+
+def test_wait_limit_and_self_test_arguments(lib):
+    """The wait limit must lie in [1 us, 600 s] (0: the default), and the
+    self-test kind must be 0 or 1; both are checked before any device work."""
+    for bad in (1, 999, 600_000_000_001):
+        assert lib.dg_set_wait_limit_ns(bad, None) == 1
+        assert b"outside" in lib.dg_last_error()
+    assert lib.dg_self_test_wait(2, None) == 1
+    assert lib.dg_self_test_wait(-1, None) == 1

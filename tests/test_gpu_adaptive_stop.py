@@ -1,0 +1,205 @@
+"""The adaptive stop on the device, against the oracle.
+
+Google docs page "DiffusionGemma", table "Configuracao de exibicao
+recomendada", row "Parada antecipada adaptativa": denoising of a canvas stops
+once (A) the mean entropy over the canvas falls below 0.005 and (B) two
+consecutive denoiser predictions are identical.  Random weights never get
+there (their confidences are ~1/V), so these cases plant the sharp
+distributions a trained model would produce:
+
+* the sampler alone on planted logits (+50 on one token per position): a
+  sequence whose planted tokens stay put stops after step 1 with the final
+  fill, one whose planted tokens move does not, one with flat logits does not;
+* the fused unembedding + sampler on hidden states and an unembedding built
+  so that each position's logits are one-hot;
+* the block driver on a model built to be an identity on the residual stream
+  (zero output and MLP-down projections) with one-hot embeddings and a
+  diagonal unembedding: every canvas stops after two steps, and the step
+  advance, final fill, re-encode and commit follow.
+Decisions are bit-exact against the oracle (no near-ties exist here: every
+gap is tens of nats).
+"""
+import numpy as np
+import pytest
+import torch
+
+from helpers import gpu_weights
+from oracle import model as M
+from oracle import sampler as S
+from canvas_denoising_denoise_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+
+def device_state(tok, committed, prev, status):
+    dev = "cuda"
+    return (torch.as_tensor(tok, dtype=torch.int32).to(dev).contiguous(),
+            torch.as_tensor(committed, dtype=torch.uint8).to(dev).contiguous(),
+            torch.as_tensor(prev, dtype=torch.int32).to(dev).contiguous(),
+            torch.as_tensor(status, dtype=torch.int32).to(dev).contiguous())
+
+
+def planted_logits(B, C, V, planted, height, seed):
+    g = torch.Generator().manual_seed(seed)
+    x = torch.randn((B, C, V), generator=g, dtype=torch.float32)
+    if height:
+        x.scatter_add_(2, torch.as_tensor(planted).view(B, C, 1),
+                       torch.full((B, C, 1), float(height)))
+    return x
+
+
+def oracle_two_steps(logits_by_step, tok, committed, seed, block):
+    """The oracle's sampler over consecutive steps of one batch; returns the
+    per-step results and each sequence's stop status (0 or s + 1)."""
+    B = tok.shape[0]
+    cfg = S.SamplerCfg()
+    tok = tok.copy()
+    committed = committed.copy()
+    prev = [None] * B
+    status = np.zeros(B, dtype=np.int64)
+    for s, lg in enumerate(logits_by_step):
+        for b in range(B):
+            if status[b]:
+                continue
+            r = S.sampler_step(cfg, lg[b], tok[b], committed[b], prev[b], s, seed, b, block)
+            tok[b], committed[b], prev[b] = r.tok, r.committed, r.argmax
+            if r.stopped:
+                status[b] = s + 1
+    return tok, committed, status
+
+
+def test_sampler_stops_on_entropy_and_identical_predictions():
+    import canvas_denoising_denoise_b200 as dg
+    B, C, V, seed, block = 3, 256, 512, 4, 1
+    rng = np.random.default_rng(0)
+    planted0 = rng.integers(0, V, size=(B, C))
+    planted1 = planted0.copy()
+    moved = rng.random(C) < 0.1
+    planted1[1, moved] = (planted1[1, moved] + 7) % V      # sequence 1: predictions move
+    steps = [planted_logits(B, C, V, planted0, 50.0, seed=1),
+             planted_logits(B, C, V, planted1, 50.0, seed=2)]
+    for st in steps:
+        st[2] = 3.0 * torch.randn((C, V), generator=torch.Generator().manual_seed(3))  # flat
+    tok0 = rng.integers(0, V, size=(B, C))
+    com0 = np.zeros((B, C), bool)
+    t_tok, t_com, t_prev, t_stat = device_state(tok0, com0, np.full((B, C), -1), np.zeros(B))
+    settings = dg.SamplerSettings()
+    for s, lg in enumerate(steps):
+        dg.sample_commit(lg.cuda(), t_tok, t_com, t_prev, t_stat, settings, seed, block, s)
+    torch.cuda.synchronize()
+    dg.check_device_errors()
+    want_tok, want_com, want_stat = oracle_two_steps([x.numpy() for x in steps], tok0, com0,
+                                                     seed, block)
+    assert want_stat.tolist() == [2, 0, 0]
+    assert t_stat.cpu().tolist() == want_stat.tolist()
+    assert np.array_equal(t_tok.cpu().numpy(), want_tok)
+    assert np.array_equal(t_com.cpu().numpy().astype(bool), want_com)
+    # the stopped canvas is complete: every position took its sample
+    assert bool(t_com[0].all()) and np.array_equal(t_tok[0].cpu().numpy(), planted0[0])
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_fused_unembed_sampler_stops_on_entropy(fp8):
+    """h[i] = 8 e_{t_i} and w_u[v] = 8 e_v (v < d), 0 beyond: logit 64 at t_i,
+    0 elsewhere (exact in bf16 and in e4m3).  Sequence 1 keeps random hidden
+    states and runs on."""
+    import canvas_denoising_denoise_b200 as dg
+    B, C, V, d, seed, block = 2, 256, 512, 256, 9, 0
+    rng = np.random.default_rng(1)
+    targets = rng.integers(0, d, size=C)
+    h = torch.zeros((B * C, d), dtype=torch.float32)
+    h[torch.arange(C), torch.as_tensor(targets)] = 8.0
+    h[C:] = torch.randn((C, d), generator=torch.Generator().manual_seed(2))
+    w = torch.zeros((V, d), dtype=torch.float32)
+    w[torch.arange(d), torch.arange(d)] = 8.0
+    w[d:] = torch.randn((V - d, d), generator=torch.Generator().manual_seed(3)) * 0.05
+    h, w = h.to(torch.bfloat16), w.to(torch.bfloat16)
+    tok0 = rng.integers(0, V, size=(B, C))
+    com0 = np.zeros((B, C), bool)
+    t_tok, t_com, t_prev, t_stat = device_state(tok0, com0, np.full((B, C), -1), np.zeros(B))
+    settings = dg.SamplerSettings()
+    hd, wd = h.cuda(), w.cuda()
+    if fp8:
+        hq = torch.empty((B * C, d), dtype=torch.uint8, device="cuda")
+        hs = torch.empty(B * C, dtype=torch.float32, device="cuda")
+        wq = torch.empty((V, d), dtype=torch.uint8, device="cuda")
+        ws = torch.empty(1, dtype=torch.float32, device="cuda")
+        dg.quantize_e4m3(hd, hq, hs, per_row=True)
+        dg.quantize_e4m3(wd, wq, ws, per_row=False)
+    for s in range(2):
+        if fp8:
+            dg.unembed_sample_commit_e4m3(hq, hs, wq, ws, t_tok, t_com, t_prev, t_stat,
+                                          settings, seed, block, s)
+        else:
+            dg.unembed_sample_commit(hd, wd, t_tok, t_com, t_prev, t_stat, settings, seed,
+                                     block, s)
+    torch.cuda.synchronize()
+    dg.check_device_errors()
+    if fp8:
+        from oracle import fp8 as F8
+        q, qs = F8.quantize_rows(h.double().numpy())
+        wq8, ws8 = F8.quantize_tensor(w.double().numpy())
+        logits = F8.unembed_logits(q, qs, wq8, ws8).astype(np.float64).reshape(B, C, V)
+    else:
+        logits = (h.double() @ w.double().T).float().numpy().astype(np.float64).reshape(B, C, V)
+    want_tok, want_com, want_stat = oracle_two_steps([logits, logits], tok0, com0, seed, block)
+    assert want_stat.tolist() == [2, 0]
+    assert t_stat.cpu().tolist() == want_stat.tolist()
+    assert np.array_equal(t_tok.cpu().numpy(), want_tok)
+    assert np.array_equal(t_com.cpu().numpy().astype(bool), want_com)
+    assert np.array_equal(want_tok[0], targets)
+
+
+def identity_stack_weights(shape, seed=0):
+    """Tiny-model weights whose layers leave the residual stream unchanged
+    (w_o = w_down = 0) and whose logits are one-hot: embed[v] = e_{v mod d},
+    unembed[v] = 4 e_v for v < d and 0 beyond, so position i's logits are
+    ~64 at tok_i mod d and 0 elsewhere."""
+    w = synth.make_weights(shape, seed=seed)
+    d, V = shape.d, shape.vocab
+    e = torch.zeros((V, d))
+    e[torch.arange(V), torch.arange(V) % d] = 1.0
+    u = torch.zeros((V, d))
+    u[torch.arange(d), torch.arange(d)] = 4.0
+    w["embed"], w["unembed"] = e.to(torch.bfloat16), u.to(torch.bfloat16)
+    for lw in w["layers"]:
+        lw["w_o"].zero_()
+        lw["w_down"].zero_()
+    return w
+
+
+@pytest.mark.parametrize("fp8", [False, True])
+def test_block_driver_stops_on_entropy(fp8):
+    import canvas_denoising_denoise_b200 as dg
+    shape = synth.TINY
+    ocfg = M.ModelCfg(shape.d, shape.n_layers, shape.n_q_heads, shape.n_kv_heads,
+                      shape.head_dim, shape.ffn, shape.vocab, shape.eps)
+    P, C, B, seed, block = 64, 256, 2, 6, 0
+    w_cpu = identity_stack_weights(shape)
+    model = dg.DgModel(shape, gpu_weights(w_cpu), fp8_unembed=fp8)
+    prompts = synth.make_prompt(B, P, shape.vocab, seed=5)
+    st = dg.DgState(shape, B, P + C, C)
+    dg.prefill(model, st, prompts.cuda())
+    steps = dg.denoise_block(model, st, dg.SamplerSettings(), seed, block)
+    torch.cuda.synchronize()
+    dg.check_device_errors()
+    assert steps == 2
+    assert st.seq_status.cpu().tolist() == [2] * B
+    assert st.cache_len.cpu().tolist() == [P + C] * B and st.cache_len_host == P + C
+    assert bool(st.committed.all())
+    # the oracle's loop over the same model: its own forward, its own sampler
+    w64 = M.weights_to_f64(w_cpu)
+    for b in range(B):
+        kc, vc = M.empty_cache(ocfg, P + C)
+        L = M.prefill(ocfg, w64, prompts[b].numpy(), kc, vc)
+        tok = S.init_canvas(seed, b, block, C, shape.vocab)
+        committed = np.zeros(C, bool)
+        prev = None
+        for s in range(48):
+            lg = M.denoise_logits(ocfg, w64, tok, kc, vc, L, e4m3_unembed=fp8)
+            r = S.sampler_step(S.SamplerCfg(), lg, tok, committed, prev, s, seed, b, block)
+            tok, committed, prev = r.tok, r.committed, r.argmax
+            if r.stopped:
+                break
+        assert (s, r.reason) == (1, "entropy")
+        assert np.array_equal(st.tok[b].cpu().numpy(), tok)

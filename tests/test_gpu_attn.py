@@ -59,26 +59,31 @@ def test_attention_batch_ragged_prefix_and_gqa(hd):
     run_case(2, 4, 4, hd, 256, [257, 5], lmax=300, causal=True, seed=4)
 
 
-def test_attention_microbench_shape_sampled():
-    """Microbench shape at L = 4096: Q [32, 256, 128], KV [8, L, 128], checked on sampled rows."""
+@pytest.mark.parametrize("L", [4096, 16384, 32768])
+def test_attention_microbench_shape_sampled(L):
+    """The attention microbench shape, Q [32, 256, 128] over KV [8, L, 128]
+    plus the canvas's own 256 keys: rows sampled from every 128-row query
+    tile of every head (so from every CTA and every key split) against the
+    oracle's attention."""
     import canvas_denoising_denoise_b200 as dg
-    B, Hq, Hkv, hd, Lq, L = 1, 32, 8, 128, 256, 4096
+    B, Hq, Hkv, hd, Lq = 1, 32, 8, 128, 256
     q, kn, vn, kc, vc = synth.make_attn_inputs(B, Hq, Hkv, hd, Lq, L, seed=7)
     out = torch.zeros((B, Lq, Hq * hd), dtype=torch.bfloat16, device="cuda")
     dg.canvas_attn(q.cuda(), kn.cuda(), vn.cuda(), kc.cuda(), vc.cuda(),
                    torch.tensor([L], dtype=torch.int32, device="cuda"), L, out, n_q_heads=Hq,
                    n_kv_heads=Hkv, head_dim=hd)
     torch.cuda.synchronize()
-    rng = np.random.default_rng(1)
+    dg.check_device_errors()
+    rng = np.random.default_rng(L)
     got = to64(out.cpu())
-    for h in rng.integers(0, Hq, size=4):
-        g = h // (Hq // Hkv)
-        rows = rng.integers(0, Lq, size=32)
-        qh = to64(q[0, rows, h * hd:(h + 1) * hd])
+    for g in range(Hkv):
         k = np.concatenate([to64(kc[0, g]), to64(kn[0, :, g * hd:(g + 1) * hd])])
         v = np.concatenate([to64(vc[0, g]), to64(vn[0, :, g * hd:(g + 1) * hd])])
-        want = M.attention_head(qh, k, v, np.ones((len(rows), len(k)), bool), hd ** -0.5)
-        assert_close(got[0, rows, h * hd:(h + 1) * hd], want, what=f"head {h}")
+        for h in range(g * (Hq // Hkv), (g + 1) * (Hq // Hkv)):
+            rows = np.concatenate([rng.integers(0, 128, size=3), rng.integers(128, 256, size=3)])
+            qh = to64(q[0, rows, h * hd:(h + 1) * hd])
+            want = M.attention_head(qh, k, v, np.ones((len(rows), len(k)), bool), hd ** -0.5)
+            assert_close(got[0, rows, h * hd:(h + 1) * hd], want, what=f"L {L} head {h}")
 
 
 def test_permutation_equivariance_on_device():
@@ -95,6 +100,7 @@ def test_permutation_equivariance_on_device():
                        kc.cuda(), vc.cuda(), cl, L, o, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=hd)
         outs.append(o)
     torch.cuda.synchronize()
+    dg.check_device_errors()
     # only the fp32 summation order within the canvas tile changes
     assert_close(outs[1].cpu(), to64(outs[0].cpu())[:, perm.numpy()], rel_l2=1e-3, max_abs=1.6e-2,
                  what="equivariance")

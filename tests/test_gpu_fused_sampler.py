@@ -45,7 +45,8 @@ def run(path, h, w, tok, committed, prev, settings, seed, block, step):
            "argmax": torch.empty((B, C), dtype=torch.int32, device=dev),
            "logconf": torch.empty((B, C), dtype=torch.float32, device=dev),
            "entropy": torch.empty((B, C), dtype=torch.float32, device=dev),
-           "flags": torch.empty((B, C), dtype=torch.uint8, device=dev)}
+           "flags": torch.empty((B, C), dtype=torch.uint8, device=dev),
+           "near_ties": torch.full((B, 3), -1, dtype=torch.int32, device=dev)}
     hd, wd = h.to(dev), w.to(dev)
     if path == "fused":
         dg.unembed_sample_commit(hd, wd, t_tok, t_com, t_prev, t_stat, settings, seed, block,
@@ -85,7 +86,8 @@ def test_fused_step_against_oracle(B, C, V, d, step):
 
 
 def test_fused_matches_unfused_at_full_vocab():
-    """256 x 262144 x 2048, mid-schedule: fused vs dg_unembed + dg_sample_commit."""
+    """256 x 262144 x 2048, mid-schedule: fused vs dg_unembed + dg_sample_commit,
+    and both against the oracle on all 256 rows."""
     import canvas_denoising_denoise_b200 as dg
     B, C, V, d, step = 1, 256, 262144, 2048, 20
     h, w, tok, committed, prev = make_case(B, C, V, d, seed=77, commit_frac=0.25)
@@ -102,15 +104,17 @@ def test_fused_matches_unfused_at_full_vocab():
         assert np.array_equal(f["flags"], u["flags"])
         assert np.array_equal(f["tok"], u["tok"])
         assert np.array_equal(f["committed"], u["committed"])
-    # the oracle's per-position statistics on sampled rows
-    T = S.temperature(S.SamplerCfg(), step)
-    for pos in np.random.default_rng(5).choice(C, size=6, replace=False):
-        row = (h[pos].double() @ w.double().T).float().numpy()
-        ps = S.position_stats(row, T, 7, 0, 0, step, int(pos))
-        assert f["argmax"][0, pos] == ps.argmax or ps.argmax_gap < 1e-4
-        if ps.gumbel_gap >= 1e-4:
-            assert f["x_hat"][0, pos] == ps.x_hat
-        np.testing.assert_allclose(f["entropy"][0, pos], ps.entropy, rtol=1e-4, atol=2e-4)
+    # every row against the oracle's sampler on the fp64 logits (rounded to
+    # fp32): bit-exact decisions outside its near-ties; a sample on which the
+    # fused and unfused paths differ must be one of those near-ties
+    logits = (h.double() @ w.double().T).float().numpy()
+    r = S.sampler_step(S.SamplerCfg(), logits, tok[0], committed[0], prev[0], step, 7, 0, 0)
+    counters = {"near_gumbel": 0, "near_renoise": 0, "skipped_sequences": 0}
+    compare(f, r, 0, committed[0], counters)
+    compare(u, r, 0, committed[0], counters)
+    assert counters["skipped_sequences"] == 0
+    assert np.all(r.near_tie["gumbel"][~same])
+    print("near-tie counts", counters, "fused/unfused sample differences", int((~same).sum()))
 
 
 def test_fused_step_entropy_bounded_selection():

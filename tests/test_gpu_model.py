@@ -159,6 +159,7 @@ def test_block_driver_matches_stepwise_calls_and_prefill(setup):
     M.block_commit(OCFG, w64, tok_a[0].cpu().numpy(), kc, vc, L)
     for l in range(SHAPE.n_layers):
         assert_close(st.k_cache[l][0, :, P:P + C].cpu(), kc[l][:, P:P + C], what=f"oracle K {l}")
+        assert_close(st.v_cache[l][0, :, P:P + C].cpu(), vc[l][:, P:P + C], what=f"oracle V {l}")
 
 
 def test_two_blocks_batch_two(setup):

@@ -26,7 +26,8 @@ def gpu_step(logits, tok, committed, prev, status, settings, seed, block, step):
            "argmax": torch.empty((B, C), dtype=torch.int32, device=dev),
            "logconf": torch.empty((B, C), dtype=torch.float32, device=dev),
            "entropy": torch.empty((B, C), dtype=torch.float32, device=dev),
-           "flags": torch.empty((B, C), dtype=torch.uint8, device=dev)}
+           "flags": torch.empty((B, C), dtype=torch.uint8, device=dev),
+           "near_ties": torch.full((B, 3), -1, dtype=torch.int32, device=dev)}
     dg.sample_commit(logits, t_tok, t_com, t_prev, t_stat, settings, seed, block, step, out=out)
     torch.cuda.synchronize()
     dg.check_device_errors()
@@ -39,6 +40,10 @@ def gpu_step(logits, tok, committed, prev, status, settings, seed, block, step):
 def compare(g, r, b, committed_in, counters):
     """Compare GPU sequence b with oracle result r; returns nothing, asserts."""
     near = r.near_tie
+    if "near_ties" in g:
+        # the device's counters of the decisions it can see near a flip
+        assert g["near_ties"][b].tolist() == [int(near["commit_boundary"].sum()),
+                                              int(near["renoise"].sum()), int(near["stop"])]
     ok_pos = ~near["gumbel"]
     counters["near_gumbel"] += int(near["gumbel"].sum())
     assert np.array_equal(g["argmax"][b], r.argmax), "raw-logit argmax must be exact"
@@ -99,6 +104,32 @@ def test_sampler_parity_full_vocab():
     counters = {"near_gumbel": 0, "near_renoise": 0, "skipped_sequences": 0}
     compare(g, r, 0, committed[0], counters)
     print("near-tie counts", counters)
+    # the one sequence was compared in full, not skipped as a global tie
+    assert counters["skipped_sequences"] == 0
+    assert int((g["flags"][0] & 1).sum()) == 16
+
+
+@pytest.mark.parametrize("B,seqs", [(4, (0, 1, 2, 3)), (16, (0, 6, 15))])
+def test_sampler_parity_full_vocab_batched(B, seqs):
+    """The sampler sweep's batches (B = 4 and 16, V = 262144) in one call; the
+    oracle checks every sequence at B = 4 and three of them at B = 16
+    (sequences are independent: each has its own Philox key)."""
+    import canvas_denoising_denoise_b200 as dg
+    C, V, step = 256, 262144, 31
+    logits = synth.make_sampler_logits(B, C, V, seed=8, step=step, device="cuda")
+    rng = np.random.default_rng(B)
+    tok = rng.integers(0, V, size=(B, C))
+    committed = rng.random((B, C)) < 0.25
+    prev = rng.integers(0, V, size=(B, C))
+    prev[:, ::3] = -1
+    g = gpu_step(logits, tok, committed, prev, np.zeros(B), dg.SamplerSettings(), 21, 4, step)
+    counters = {"near_gumbel": 0, "near_renoise": 0, "skipped_sequences": 0}
+    for b in seqs:
+        r = S.sampler_step(S.SamplerCfg(), logits[b].cpu().numpy(), tok[b], committed[b], prev[b],
+                           step, 21, b, 4)
+        compare(g, r, b, committed[b], counters)
+    print("near-tie counts", counters)
+    assert counters["skipped_sequences"] == 0
 
 
 def test_frozen_sequences_are_untouched():
@@ -124,8 +155,15 @@ def test_unselected_policy_on_device(policy):
                  dg.SamplerSettings(unselected_policy=policy), 4, 1, step)
     r = S.sampler_step(S.SamplerCfg(unselected_policy=policy), logits[0].numpy(), tok[0],
                        committed[0], None, step, 4, 0, 1)
-    if not r.near_tie["gumbel"].any() and not r.near_tie["commit_boundary"].any():
-        assert np.array_equal(g["tok"][0], r.tok)
+    counters = {"near_gumbel": 0, "near_renoise": 0, "skipped_sequences": 0}
+    compare(g, r, 0, committed[0], counters)
+    assert counters["skipped_sequences"] == 0
+    assert np.array_equal(g["tok"][0], r.tok)
+    unsel = ~r.commit_mask
+    if policy == 0:  # unselected positions hold the step's sample
+        assert np.array_equal(g["tok"][0][unsel], g["x_hat"][0][unsel])
+    else:            # unselected positions hold a fresh uniform token
+        assert not np.array_equal(g["tok"][0][unsel], g["x_hat"][0][unsel])
 
 
 def test_sixteen_step_completion_on_device():
@@ -173,3 +211,64 @@ def test_entropy_bounded_selection_parity(step):
         n_commit.append(int(r.commit_mask.sum()))
     assert max(n_commit) > 1  # the bound admitted several positions
     assert counters["skipped_sequences"] < B
+
+
+def test_near_tie_counters_on_planted_margins():
+    """The device's near-tie counters against the oracle's classifier on rows
+    whose deciding quantity is planted 0.5e-4 inside or 2e-4 outside the
+    margin (two live outcomes, two far below: closed-form confidences and
+    entropies, as in the oracle's own pins)."""
+    import math
+    import canvas_denoising_denoise_b200 as dg
+    V, step, block = 4, 3, 0
+    T = S.temperature(S.SamplerCfg(), step)
+
+    def rows(deltas):
+        lg = np.full((1, len(deltas), V), -1e4 * T, dtype=np.float32)
+        lg[0, :, 0] = np.asarray(deltas) * T
+        lg[0, :, 1] = 0.0
+        return torch.from_numpy(lg)
+
+    def run_case(deltas, committed, settings, scfg, want):
+        lg = rows(deltas)
+        C = len(deltas)
+        tok = np.zeros((1, C), dtype=np.int64)
+        com = np.asarray(committed, bool).reshape(1, C)
+        for seed in range(100):  # a seed under which the uncommitted rows sample outcome 0
+            r = S.sampler_step(scfg, lg[0].numpy(), tok[0], com[0], None, step, seed, 0, block)
+            if np.all(r.x_hat[~com[0]] == 0):
+                break
+        g = gpu_step(lg.cuda(), tok, com, np.full((1, C), -1), np.zeros(1), settings, seed,
+                     block, step)
+        got = g["near_ties"][0].tolist()
+        assert got == [int(r.near_tie["commit_boundary"].sum()), int(r.near_tie["renoise"].sum()),
+                       int(r.near_tie["stop"])]
+        assert got == want
+        assert np.array_equal(g["x_hat"][0], r.x_hat)
+
+    softplus = lambda x: math.log1p(math.exp(x))
+    sp_inv = lambda y: math.log(math.expm1(y))
+
+    def h_delta(h):  # two-outcome delta > 0 with entropy h
+        lo, hi = 1e-9, 60.0
+        for _ in range(200):
+            mid = 0.5 * (lo + hi)
+            p = 1 / (1 + math.exp(-mid))
+            lo, hi = (mid, hi) if -(p * math.log(p) + (1 - p) * math.log(1 - p)) > h else (lo, mid)
+        return 0.5 * (lo + hi)
+
+    topk = (dg.SamplerSettings(commit_k=1), S.SamplerCfg(commit_k=1))
+    for gap, n in ((0.5e-4, 2), (2e-4, 0)):
+        run_case([3.0, -sp_inv(softplus(-3.0) + gap)], [False, False], *topk, want=[n, 0, 0])
+    ent = (dg.SamplerSettings(selection=1, entropy_bound=0.1),
+           S.SamplerCfg(selection=S.SELECT_ENTROPY, entropy_bound=0.1))
+    for e, n in ((0.5e-4, 2), (2e-4, 0)):
+        run_case([h_delta(x) for x in (0.05 + e, 0.02, 0.03)], [False] * 3, *ent, want=[n, 0, 0])
+    for e, n in ((0.5e-4, 1), (2e-4, 0)):
+        run_case([h_delta(x) for x in (0.05 - e, 0.02, 0.03)], [False] * 3, *ent, want=[n, 0, 0])
+    dflt = (dg.SamplerSettings(), S.SamplerCfg())
+    lt = math.log(0.05)
+    offs = [-0.5e-4, 0.5e-4, -2e-4, 2e-4]
+    run_case([-sp_inv(-(lt + o)) for o in offs], [True] * 4, *dflt, want=[0, 2, 0])
+    for off, n in ((0.5e-4, 1), (-2e-4, 0)):
+        run_case([h_delta(0.005 + off)] * 4, [True] * 4, *dflt, want=[0, 0, n])
