@@ -167,9 +167,10 @@ def time_region(fn, steps, stream):
     return start.elapsed_time(end) / 1000.0
 
 
-def captured_traffic(profile, sources):
+def captured_traffic(profile, sources, shape):
     """DRAM bytes per launch from a committed ncu summary, or None when the
-    kernel sources changed since the capture (hash recorded in the summary)."""
+    kernel sources changed since the capture (hash recorded in the summary) or
+    the launch is not the shape that was captured (`captured_shape`)."""
     import hashlib
     path = os.path.join(ROOT, "profiles", profile)
     if not os.path.exists(path):
@@ -185,6 +186,8 @@ def captured_traffic(profile, sources):
                 k, v = line.split(":", 1)
                 fields[k.strip()] = v.strip()
     if fields.get("kernel_sources_sha256_16") != h.hexdigest()[:16]:
+        return None
+    if fields.get("captured_shape") != ",".join(str(int(v)) for v in shape):
         return None
     try:
         return int(fields["traffic_bytes_per_launch"])
@@ -232,8 +235,8 @@ def gemm_roofline(dg, model, shape, batch, peaks, stream):
     return {"kernel": "gemm_kernel (MLP down projection launch)", "shape": [M, N, K],
             "bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
             "frac": round(achieved / peak, 4),
-            "traffic": (captured_traffic("gemm_mlp_down_full.md", ["gemm.cuh", "dg_common.cuh"])
-                        if batch == 1 else None),
+            "traffic": captured_traffic("gemm_mlp_down_full.md", ["gemm.cuh", "dg_common.cuh"],
+                                        (M, N, K)),
             "algorithmic_bytes": int(N * K * 2 + M * K * 2 + M * N * 4 * 2),
             "hbm_frac": round((N * K * 2 + M * K * 2 + M * N * 8) / t / 1e9 / peaks["hbm_gbs"], 4),
             "peak_source": f"{peaks['source']} burst bf16",

@@ -193,6 +193,7 @@ struct Fp8Scales {
 // ---------------------------------------------------------------------------
 struct GemmPlan {
   int splits, kb_per_split, bn;
+  int ring_kb = 192;  // 192: one CTA per SM; 96: two CTAs per SM
 };
 
 // Choose the token tile (128 or 256) and the K split (cluster of 1, 2 or 4)
@@ -247,46 +248,52 @@ struct GemmEpi {
   unsigned long long* trace = nullptr;
 };
 
-template <int S, int BN, bool F8>
+// The GEMM instantiations: (split count, token tile, ring KB).
+#define DG_GEMM_VARIANTS(X)                                                              \
+  X(1, 256, 192) X(2, 256, 192) X(4, 256, 192) X(1, 128, 192) X(2, 128, 192)           \
+  X(4, 128, 192) X(1, 128, 96) X(2, 128, 96) X(4, 128, 96) X(8, 128, 96) X(1, 64, 96)   \
+  X(2, 64, 96) X(4, 64, 96) X(8, 64, 96)
+
+template <int S, int BN, bool F8, int R>
 cudaError_t launch_gemm_t(dim3 grid, cudaStream_t s, const CUtensorMap& tw, const CUtensorMap& tx,
                           const dg::gemm::Params& p) {
-  return launch_ex(dg::gemm::gemm_kernel<S, BN, F8>, grid, dim3(dg::gemm::THREADS),
-                   dg::gemm::SMEM_BYTES, s, S, tw, tx, p);
+  return launch_ex(dg::gemm::gemm_kernel<S, BN, F8, R>, grid, dim3(dg::gemm::THREADS),
+                   dg::gemm::smem_bytes(R), s, S, tw, tx, p);
 }
 
-template <int S, int BN, bool F8>
+template <int S, int BN, bool F8, int R>
 cudaError_t gemm_set_attr() {
-  return cudaFuncSetAttribute(dg::gemm::gemm_kernel<S, BN, F8>,
-                              cudaFuncAttributeMaxDynamicSharedMemorySize, dg::gemm::SMEM_BYTES);
+  return cudaFuncSetAttribute(dg::gemm::gemm_kernel<S, BN, F8, R>,
+                              cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              dg::gemm::smem_bytes(R));
 }
 
 template <bool F8>
 cudaError_t gemm_set_attrs() {
   cudaError_t e;
-  if ((e = gemm_set_attr<1, 256, F8>()) != cudaSuccess) return e;
-  if ((e = gemm_set_attr<2, 256, F8>()) != cudaSuccess) return e;
-  if ((e = gemm_set_attr<4, 256, F8>()) != cudaSuccess) return e;
-  if ((e = gemm_set_attr<1, 128, F8>()) != cudaSuccess) return e;
-  if ((e = gemm_set_attr<2, 128, F8>()) != cudaSuccess) return e;
-  return gemm_set_attr<4, 128, F8>();
+#define DG_X(S_, BN_, R_) \
+  if ((e = gemm_set_attr<S_, BN_, F8, R_>()) != cudaSuccess) return e;
+  DG_GEMM_VARIANTS(DG_X)
+#undef DG_X
+  return cudaSuccess;
+}
+
+bool gemm_plan_known(const GemmPlan& pl) {
+#define DG_X(S_, BN_, R_) \
+  if (pl.splits == S_ && pl.bn == BN_ && pl.ring_kb == R_) return true;
+  DG_GEMM_VARIANTS(DG_X)
+#undef DG_X
+  return false;
 }
 
 template <bool F8>
 cudaError_t launch_gemm_plan(const GemmPlan& pl, dim3 grid, cudaStream_t s, const CUtensorMap& tw,
                              const CUtensorMap& tx, const dg::gemm::Params& p) {
-  if (pl.bn == 256) {
-    switch (pl.splits) {
-      case 1: return launch_gemm_t<1, 256, F8>(grid, s, tw, tx, p);
-      case 2: return launch_gemm_t<2, 256, F8>(grid, s, tw, tx, p);
-      case 4: return launch_gemm_t<4, 256, F8>(grid, s, tw, tx, p);
-    }
-  } else if (pl.bn == 128) {
-    switch (pl.splits) {
-      case 1: return launch_gemm_t<1, 128, F8>(grid, s, tw, tx, p);
-      case 2: return launch_gemm_t<2, 128, F8>(grid, s, tw, tx, p);
-      case 4: return launch_gemm_t<4, 128, F8>(grid, s, tw, tx, p);
-    }
-  }
+#define DG_X(S_, BN_, R_)                                    \
+  if (pl.splits == S_ && pl.bn == BN_ && pl.ring_kb == R_) \
+    return launch_gemm_t<S_, BN_, F8, R_>(grid, s, tw, tx, p);
+  DG_GEMM_VARIANTS(DG_X)
+#undef DG_X
   return cudaErrorInvalidValue;
 }
 
@@ -326,8 +333,8 @@ int launch_gemm(const void* x, const void* w, int M, int N, int K, const GemmPla
   const cudaError_t err = f8 ? launch_gemm_plan<true>(pl, grid, s, tw, tx, p)
                              : launch_gemm_plan<false>(pl, grid, s, tw, tx, p);
   if (err != cudaSuccess)
-    return fail(DG_ERR_CUDA, "gemm launch (S=%d, BN=%d) failed: %s", pl.splits, pl.bn,
-                cudaGetErrorString(err));
+    return fail(DG_ERR_CUDA, "gemm launch (S=%d, BN=%d, ring %d KB) failed: %s", pl.splits,
+                pl.bn, pl.ring_kb, cudaGetErrorString(err));
   count_launch();
   return DG_OK;
 }
@@ -410,37 +417,22 @@ int launch_proj_pair(const void* x, const void* w, int M, int N, int K, const Ge
 }
 
 // y = epilogue(x w^T) with the plan chosen for this shape (e4m3 operands with
-// their scales when f8 is set: 128-element k-blocks).  EPI_RESID writes its
-// sums of squares per 128 features on the split-K GEMM and per 32 on the
-// pair pipeline (see ssq_group); pair_ok = false keeps a shape on the former.
+// their scales when f8 is set: 128-element k-blocks).  An EPI_RESID with
+// ssq_out writes its sums of squares per 128 features on the split-K GEMM
+// and per 32 on the pair pipeline.
 int linear(const void* x, const void* w, int M, int N, int K, const GemmEpi& e,
-           cudaStream_t s, const Fp8Scales* f8 = nullptr, bool pair_ok = true) {
-  if (pair_ok && proj_use_pair(M, N, K, f8 != nullptr))
+           cudaStream_t s, const Fp8Scales* f8 = nullptr) {
+  if (proj_use_pair(M, N, K, f8 != nullptr))
     return launch_proj_pair(x, w, M, N, K, e, s, f8);
   return launch_gemm(x, w, M, N, K, plan_gemm(M, N, K, f8 ? 128 : dg::gemm::BK), e, s, f8);
 }
 
-// Both residual projections of a forward pass over M tokens (the output
-// projection, K = Hq hd, and the MLP down projection, K = F) write the sums of
-// squares their consumers read, so they take one path together: the pair
-// pipeline only when both shapes qualify for it.
+// Whether both residual projections of a forward pass over M tokens (the
+// output projection, K = Hq hd, and the MLP down projection, K = F) run on
+// the pair pipeline.  Each projection picks its plan from its own shape.
 bool resid_on_pair(const dg_model_cfg& c, int M, bool f8) {
   return proj_use_pair(M, c.d, c.n_q_heads * c.head_dim, f8) &&
          proj_use_pair(M, c.d, c.ffn, f8);
-}
-
-// Features per sum-of-squares partial of the residual stream in a forward
-// pass over M tokens: 32 when its residual projections run on the pair
-// pipeline, else 128.
-int ssq_group(const dg_model_cfg& c, int M, bool f8) {
-  return resid_on_pair(c, M, f8) ? 32 : 128;
-}
-
-// Partial sums of squares per token that a consumer of the norm reads: the
-// 32-feature partials of the pair path are collapsed into one after each
-// producer (norm.cuh); the split-K GEMM's d / 128 are read as they are.
-int ssq_partials_read(const dg_model_cfg& c, int M, bool f8) {
-  return ssq_group(c, M, f8) == 32 ? 1 : c.d / 128;
 }
 
 // logits = rs * (h w_u^T).  Vocabularies that are a multiple of 256 run on
@@ -573,8 +565,8 @@ int launch_attn(const void* q, int ldq, const void* k_new, const void* v_new, in
   DG_CUDA(cudaGetLastError());
   if (S > 1) {
     const int rows = B * Hq * Lq;
-    const int threads = 256;
-    const int blocks = cdiv(rows * 32, threads);
+    const int threads = dg::attn::COMBINE_THREADS;
+    const int blocks = cdiv(rows * (hd / 8), threads);  // hd / 8 threads per row
     if (hd == 128)
       DG_CUDA(launch_ex(dg::attn::attn_combine_kernel<128>, dim3(blocks), dim3(threads), 0, s, 1,
                         (const __nv_bfloat16*)p.part_o, (const float*)p.part_lse, S, B, Hq, Lq,
@@ -844,7 +836,7 @@ int check_state(const dg_state* st, const dg_model_cfg& c, bool need_canvas) {
 
 // Workspace carve-up for a forward over M = B * Lq rows.
 struct FwdLayout {
-  size_t x, xn, qkv, ao, up, ssq_x, ssq_h, attn, logits, spart, flag, aq, as, total;
+  size_t x, xn, qkv, ao, up, attn, logits, spart, flag, aq, as, total;
 };
 
 FwdLayout fwd_layout(const dg_model_cfg& c, int B, int Lq, int max_prefix, bool logits) {
@@ -863,8 +855,6 @@ FwdLayout fwd_layout(const dg_model_cfg& c, int B, int Lq, int max_prefix, bool 
   L.qkv = take((size_t)M * nqkv * 2);
   L.ao = take((size_t)M * hqd * 2);
   L.up = take((size_t)M * c.ffn * 2);
-  L.ssq_x = take((size_t)(c.d / 32) * M * 4);  // per 32 or 128 features (ssq_group)
-  L.ssq_h = take((size_t)(c.d / 32) * M * 4);
   L.attn = take(attn_ws_bytes(B, c.n_q_heads, c.n_kv_heads, Lq, c.head_dim, max_prefix));
   L.logits = take(logits ? (size_t)M * c.vocab * 4 : 0);
   L.spart = take(logits ? std::max(sample_ws_bytes(B, Lq, c.vocab),
@@ -894,8 +884,8 @@ struct Fwd {
 };
 
 // A bf16 activation [B*Lq, cols] quantised per token to e4m3 codes (L.aq)
-// and scales (L.as).  A normalised input is quantised before its RMSNorm,
-// which stays a row scale of the product (per-row scaling commutes with it).
+// and scales (L.as): the normalised residual stream, the attention output or
+// the GELU output, as stored in bf16.
 int quantize_act(const Fwd& f, const void* in, int cols, cudaStream_t s) {
   DG_CUDA(launch_ex(dg::quant::quantize_rows_kernel, dim3(f.B * f.Lq), dim3(dg::quant::THREADS),
                     0, s, 1, (const __nv_bfloat16*)in, f.B * f.Lq, cols,
@@ -904,7 +894,7 @@ int quantize_act(const Fwd& f, const void* in, int cols, cudaStream_t s) {
   return DG_OK;
 }
 
-// The last layer's bf16 residual stream, quantised for the FP8 unembedding.
+// The final normalised hidden states, quantised for the FP8 unembedding.
 int quantize_hidden(const Fwd& f, cudaStream_t s) {
   return quantize_act(f, f.ws + f.L.xn, f.m->cfg.d, s);
 }
@@ -914,50 +904,41 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
   const int M = f.B * f.Lq;
   const int hd = c.head_dim, hq = c.n_q_heads, hkv = c.n_kv_heads;
   const int nqkv = (hq + 2 * hkv) * hd;
-  float* x = (float*)(f.ws + f.L.x);
-  __nv_bfloat16* xb = (__nv_bfloat16*)(f.ws + f.L.xn);  // bf16 copy of the residual stream
+  float* x = (float*)(f.ws + f.L.x);                      // residual stream, fp32
+  __nv_bfloat16* xn = (__nv_bfloat16*)(f.ws + f.L.xn);    // bf16(RMSNorm(x)), the next input
   __nv_bfloat16* qkv = (__nv_bfloat16*)(f.ws + f.L.qkv);
   __nv_bfloat16* ao = (__nv_bfloat16*)(f.ws + f.L.ao);
   __nv_bfloat16* up = (__nv_bfloat16*)(f.ws + f.L.up);
-  float* ssq_x = (float*)(f.ws + f.L.ssq_x);
-  float* ssq_h = (float*)(f.ws + f.L.ssq_h);
   void* aws = f.ws + f.L.attn;
   const float scale = 1.0f / std::sqrt((float)hd);
-  const int group = ssq_group(c, M, f.m->layers_e4m3 != nullptr);
-  const int nt = c.d / group;  // sum-of-squares partials per token
-  const bool resid_pair = group == 32;
-  // partials a consumer of the norm reads: one once they are collapsed
-  const int n_use = ssq_partials_read(c, M, f.m->layers_e4m3 != nullptr);
-  auto collapse = [&](float* ssq) -> int {
-    if (!resid_pair) return DG_OK;
-    DG_CUDA(launch_ex(dg::norm::ssq_collapse_kernel, dim3(cdiv(M, dg::norm::COLLAPSE_THREADS)),
-                      dim3(dg::norm::COLLAPSE_THREADS), 0, s, 1, ssq, nt, M));
+  // xn = bf16(RMSNorm(x)) after each residual update
+  auto norm = [&]() -> int {
+    DG_CUDA(launch_ex(dg::norm::rmsnorm_kernel, dim3(M), dim3(dg::norm::NORM_THREADS), 0, s, 1,
+                      (const float*)x, c.d, 1.f / c.d, c.eps, xn));
     count_launch();
     return DG_OK;
   };
 
-  DG_CUDA(launch_ex(dg::gemm::embed_kernel, dim3(M), dim3(dg::gemm::EMBED_THREADS), 0, s, 1, tok,
-                    (const __nv_bfloat16*)f.m->embed, c.vocab, c.d, M, x, xb, ssq_x, group));
+  DG_CUDA(launch_ex(dg::norm::embed_norm_kernel, dim3(M), dim3(dg::norm::NORM_THREADS), 0, s, 1,
+                    tok, (const __nv_bfloat16*)f.m->embed, c.vocab, c.d, 1.f / c.d, c.eps, x,
+                    xn));
   count_launch();
-  DG_CUDA(cudaGetLastError());
-  DG_TRY(collapse(ssq_x));
   for (int l = 0; l < c.n_layers; ++l) {
     const dg_layer_weights& w = f.m->layers[l];
     const bool last = l == c.n_layers - 1;
     const dg_layer_weights_e4m3* q8 = f.m->layers_e4m3 ? &f.m->layers_e4m3[l] : nullptr;
     // y = epilogue(in w^T): bf16, or e4m3 with the input quantised per token
     auto proj = [&](const void* in, const void* wb, const uint8_t* wq, int widx, int N, int K,
-                    const GemmEpi& e, bool pair_ok) -> int {
-      if (!q8) return linear(in, wb, M, N, K, e, s, nullptr, pair_ok);
+                    const GemmEpi& e) -> int {
+      if (!q8) return linear(in, wb, M, N, K, e, s, nullptr);
       DG_TRY(quantize_act(f, in, K, s));
       const Fp8Scales f8{(const float*)(f.ws + f.L.as), q8->scales + widx};
-      return linear(f.ws + f.L.aq, wq, M, N, K, e, s, &f8, pair_ok);
+      return linear(f.ws + f.L.aq, wq, M, N, K, e, s, &f8);
     };
     GemmEpi eq;  // QKV of RMSNorm(x)
     eq.epi = dg::gemm::EPI_BF16;
     eq.out_bf16 = qkv;
-    eq.ssq_in = ssq_x; eq.n_ssq_in = n_use; eq.inv_k = 1.f / c.d; eq.eps = c.eps;
-    DG_TRY(proj(xb, w.w_qkv, q8 ? q8->w_qkv : nullptr, 0, nqkv, c.d, eq, true));
+    DG_TRY(proj(xn, w.w_qkv, q8 ? q8->w_qkv : nullptr, 0, nqkv, c.d, eq));
     if (f.commit_kv) {
       const void* kb = qkv + hq * hd;
       const void* vb = qkv + (hq + hkv) * hd;
@@ -970,29 +951,28 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
                        f.B, hq, hkv, f.Lq, hd, scale, f.mask, aws, s));
     GemmEpi eo;  // h = x + O w_o^T
     eo.epi = dg::gemm::EPI_RESID;
-    eo.x = x; eo.out_bf16 = xb; eo.ssq_out = ssq_h;
-    DG_TRY(proj(ao, w.w_o, q8 ? q8->w_o : nullptr, 1, c.d, hq * hd, eo, resid_pair));
-    DG_TRY(collapse(ssq_h));
+    eo.x = x;
+    DG_TRY(proj(ao, w.w_o, q8 ? q8->w_o : nullptr, 1, c.d, hq * hd, eo));
+    DG_TRY(norm());
     GemmEpi eu;  // gelu(RMSNorm(h) w_up^T)
     eu.epi = dg::gemm::EPI_GELU;
     eu.out_bf16 = up;
-    eu.ssq_in = ssq_h; eu.n_ssq_in = n_use; eu.inv_k = 1.f / c.d; eu.eps = c.eps;
-    DG_TRY(proj(xb, w.w_up, q8 ? q8->w_up : nullptr, 2, c.ffn, c.d, eu, true));
+    DG_TRY(proj(xn, w.w_up, q8 ? q8->w_up : nullptr, 2, c.ffn, c.d, eu));
     GemmEpi ed;  // x = h + u w_down^T
     ed.epi = dg::gemm::EPI_RESID;
-    ed.x = x; ed.out_bf16 = xb; ed.ssq_out = ssq_x;
-    DG_TRY(proj(up, w.w_down, q8 ? q8->w_down : nullptr, 3, c.d, c.ffn, ed, resid_pair));
-    DG_TRY(collapse(ssq_x));
+    ed.x = x;
+    DG_TRY(proj(up, w.w_down, q8 ? q8->w_down : nullptr, 3, c.d, c.ffn, ed));
+    DG_TRY(norm());  // the next layer's input, or the unembedding's after the last layer
   }
   if (f.want_logits && !f.unembed_elsewhere) {
     // logits of RMSNorm(x), on e4m3 operands when the model carries them
     if (f.m->unembed_e4m3) {
       DG_TRY(quantize_hidden(f, s));
       const Fp8Scales f8{(const float*)(f.ws + f.L.as), f.m->unembed_scale};
-      DG_TRY(launch_unembed(f.ws + f.L.aq, f.m->unembed_e4m3, logits, M, c.d, c.vocab, ssq_x, n_use,
-                            1.f / c.d, c.eps, s, &f8));
+      DG_TRY(launch_unembed(f.ws + f.L.aq, f.m->unembed_e4m3, logits, M, c.d, c.vocab, nullptr,
+                            0, 1.f / c.d, c.eps, s, &f8));
     } else {
-      DG_TRY(launch_unembed(xb, f.m->unembed, logits, M, c.d, c.vocab, ssq_x, n_use, 1.f / c.d,
+      DG_TRY(launch_unembed(xn, f.m->unembed, logits, M, c.d, c.vocab, nullptr, 0, 1.f / c.d,
                             c.eps, s));
     }
   }
@@ -1509,7 +1489,6 @@ int dg_denoise_block(const dg_model* m, dg_state* st, const dg_sampler_cfg* cfg,
   const bool fp8 = m->unembed_e4m3 != nullptr;  // check_model: vocab % 256 == 0 then
   Fwd fl = f;
   fl.unembed_elsewhere = fused;
-  const int nt = ssq_partials_read(m->cfg, B * C, m->layers_e4m3 != nullptr);
   // one denoising step: forward pass, unembedding + sampler, step advance
   auto enqueue_step = [&](cudaStream_t q) -> int {
     DG_TRY(run_forward(fl, st->tok, logits, q));
@@ -1517,13 +1496,13 @@ int dg_denoise_block(const dg_model* m, dg_state* st, const dg_sampler_cfg* cfg,
       // the hidden states quantised per token, then the e4m3 unembedding + sampler
       DG_TRY(quantize_hidden(fl, q));
       const Fp8Scales f8{(const float*)(ws + L.as), m->unembed_scale};
-      DG_TRY(launch_unembed_sample(ws + L.aq, m->unembed_e4m3, m->cfg.d,
-                                   (const float*)(ws + L.ssq_x), nt, 1.f / m->cfg.d,
-                                   m->cfg.eps, st->tok, st->committed, st->prev_argmax,
+      DG_TRY(launch_unembed_sample(ws + L.aq, m->unembed_e4m3, m->cfg.d, nullptr, 0,
+                                   1.f / m->cfg.d, m->cfg.eps, st->tok, st->committed,
+                                   st->prev_argmax,
                                    st->seq_status, sp, nullptr, ws + L.spart, q, &f8));
     } else if (fused) {
-      DG_TRY(launch_unembed_sample(ws + L.xn, m->unembed, m->cfg.d, (const float*)(ws + L.ssq_x),
-                                   nt, 1.f / m->cfg.d, m->cfg.eps, st->tok,
+      DG_TRY(launch_unembed_sample(ws + L.xn, m->unembed, m->cfg.d, nullptr, 0,
+                                   1.f / m->cfg.d, m->cfg.eps, st->tok,
                                    st->committed, st->prev_argmax, st->seq_status, sp, nullptr,
                                    ws + L.spart, q));
     } else {

@@ -130,7 +130,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     i0X[X] = (qq / p.group) * BQ;
   }
 
-  griddep_wait();
+  // The cache length and the cached prefix are written only by launches that
+  // are fully ordered before this one (prefill's length set, the block commit
+  // and its length bump), so they are read before griddepcontrol.wait; the
+  // query tiles and the new rows' keys come from the preceding projection and
+  // are read after it, as is every write.
   griddep_launch();
   int L = p.cache_len[b];
   if (L < 0 || L > p.lmax) {
@@ -148,6 +152,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (n <= 0) {
     // empty key range: this split contributes nothing to the merge
+    griddep_wait();
     for (int X = 0; X < 2; ++X) {
       if (!vX[X] || threadIdx.x >= BQ) continue;
       const int qrow = i0X[X] + threadIdx.x;
@@ -197,15 +202,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      mbar_expect_tx(q_full, CF::Q_BYTES * (vB ? 2 : 1));
-      for (int X = 0; X < (vB ? 2 : 1); ++X)
-        for (int hf = 0; hf < CF::HALVES; ++hf)
-          tma_load_2d(sQ + X * CF::Q_BYTES + hf * (BQ * 128), &tm_q, q_full,
-                      hX[X] * HD + hf * 64, b * p.Lq + i0X[X]);
-      int issued = 0;
-      for (int i = 0; i < n; ++i) {
+      auto load_kv = [&](int i) {
         const int st = i % ST;
-        if (i >= ST && !mbar_wait(&kv_empty[st], ((i / ST) - 1) & 1, abort_flag, 0x311)) break;
         const int t = t_beg + i;
         const CUtensorMap* mk;
         const CUtensorMap* mv;
@@ -229,6 +227,20 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_expect_tx(&v_full[st], CF::T_BYTES);
         for (int hf = 0; hf < CF::HALVES; ++hf)
           tma_load_2d(vd + hf * (BKV * 128), mv, &v_full[st], x0 + hf * 64, y0);
+      };
+      // the first stages' cached-prefix tiles need no wait on the predecessor
+      int issued = 0;
+      while (issued < min(ST, n) && t_beg + issued < nP) load_kv(issued++);
+      griddep_wait();
+      mbar_expect_tx(q_full, CF::Q_BYTES * (vB ? 2 : 1));
+      for (int X = 0; X < (vB ? 2 : 1); ++X)
+        for (int hf = 0; hf < CF::HALVES; ++hf)
+          tma_load_2d(sQ + X * CF::Q_BYTES + hf * (BQ * 128), &tm_q, q_full,
+                      hX[X] * HD + hf * 64, b * p.Lq + i0X[X]);
+      for (int i = issued; i < n; ++i) {
+        const int st = i % ST;
+        if (i >= ST && !mbar_wait(&kv_empty[st], ((i / ST) - 1) & 1, abort_flag, 0x311)) break;
+        load_kv(i);
         issued = i + 1;
       }
       if (*abort_flag) {
@@ -293,6 +305,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax (tile X)
+    griddep_wait();  // before this warpgroup's writes
     const int X = (warp - 2) >> 2;
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
@@ -476,76 +489,83 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // Merge key-range splits: O = sum_s w_s O_s / sum_s w_s, w_s = exp(lse_s - max).
-// One warp per (b, h, row): lane s holds split s's weight (S <= 32), and the
-// split rows are loaded in batches of 8 so that the loads overlap.
+// A row is HD / 8 threads, each owning 8 consecutive output values (one
+// 16-byte load per split).  Every split's log-sum-exp and partial row are
+// requested before any arithmetic, so a thread waits for memory once; the
+// sums run in split order (the bits do not depend on scheduling).
 constexpr int MAX_SPLITS = 32;
+constexpr int COMBINE_THREADS = 256;
+constexpr int COMBINE_BATCH = 16;  // splits in flight per thread
 
 template <int HD>
-__global__ void attn_combine_kernel(const __nv_bfloat16* __restrict__ part_o,
-                                    const float* __restrict__ part_lse, int S, int B, int Hq,
-                                    int Lq, __nv_bfloat16* __restrict__ out, int ldo,
-                                    float* __restrict__ lse) {
-  griddep_wait();
+__global__ void __launch_bounds__(COMBINE_THREADS)
+    attn_combine_kernel(const __nv_bfloat16* __restrict__ part_o,
+                        const float* __restrict__ part_lse, int S, int B, int Hq, int Lq,
+                        __nv_bfloat16* __restrict__ out, int ldo, float* __restrict__ lse) {
+  constexpr int TPR = HD / 8;  // threads per row
   griddep_launch();
-  const int warp_global = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
+  griddep_wait();
+  const int gt = static_cast<int>(blockIdx.x) * COMBINE_THREADS + static_cast<int>(threadIdx.x);
+  const int row = gt / TPR;
+  const int part = gt % TPR;
   const int rows = B * Hq * Lq;
-  if (warp_global >= rows) return;
+  if (row >= rows) return;
   const size_t stride = static_cast<size_t>(rows);
-  const float ls = lane < S ? part_lse[lane * stride + warp_global] : -INFINITY;
-  float mx = ls;
+  float mx = -INFINITY;
+  float ls[COMBINE_BATCH];
+  uint4 v[COMBINE_BATCH];
+  float acc[8];
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-  const float w = (ls == -INFINITY || mx == -INFINITY) ? 0.f : expf(ls - mx);
-  const float wsum = warp_sum(w);
-  constexpr int PER = HD / 32;
-  float acc[PER];
+  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+  float wsum = 0.f;
+  // pass over the splits in batches; the running max is the first batch's
+  // (the combine is exact for any reference, the max only keeps exp in range)
+  for (int s0 = 0; s0 < S; s0 += COMBINE_BATCH) {
 #pragma unroll
-  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
-  for (int s0 = 0; s0 < S; s0 += 8) {
-    float v[8][PER];
+    for (int k = 0; k < COMBINE_BATCH; ++k) {
+      const int sp = s0 + k;
+      ls[k] = sp < S ? part_lse[sp * stride + row] : -INFINITY;
+      v[k] = sp < S ? *reinterpret_cast<const uint4*>(part_o + (sp * stride + row) * HD + part * 8)
+                    : make_uint4(0u, 0u, 0u, 0u);
+    }
+    float bmx = -INFINITY;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      if (s0 + k < S) {
-        const __nv_bfloat16* src = part_o + ((s0 + k) * stride + warp_global) * HD + lane * PER;
-        if constexpr (PER == 4) {
-          const uint2 t = *reinterpret_cast<const uint2*>(src);
-          const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&t.x);
-          const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&t.y);
-          v[k][0] = __low2float(lo); v[k][1] = __high2float(lo);
-          v[k][2] = __low2float(hi); v[k][3] = __high2float(hi);
-        } else {
-          const uint32_t t = *reinterpret_cast<const uint32_t*>(src);
-          const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&t);
-          v[k][0] = __low2float(lo); v[k][1] = __high2float(lo);
-        }
-      }
+    for (int k = 0; k < COMBINE_BATCH; ++k) bmx = fmaxf(bmx, ls[k]);
+    if (bmx > mx) {
+      // rescale what the earlier batches accumulated
+      const float f = mx == -INFINITY ? 0.f : expf(mx - bmx);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] *= f;
+      wsum *= f;
+      mx = bmx;
     }
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const float wk = __shfl_sync(0xffffffffu, w, (s0 + k) & 31);
-      if (s0 + k < S && wk > 0.f) {
+    for (int k = 0; k < COMBINE_BATCH; ++k) {
+      if (ls[k] == -INFINITY) continue;  // an empty split
+      const float w = expf(ls[k] - mx);
+      wsum += w;
+      const uint32_t wd[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
 #pragma unroll
-        for (int e = 0; e < PER; ++e) acc[e] += wk * v[k][e];
+      for (int q = 0; q < 4; ++q) {
+        const __nv_bfloat162 p2 = *reinterpret_cast<const __nv_bfloat162*>(&wd[q]);
+        acc[2 * q] += w * __low2float(p2);
+        acc[2 * q + 1] += w * __high2float(p2);
       }
     }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
-  const int qrow = warp_global % Lq;
-  const int bh = warp_global / Lq;
+  const int qrow = row % Lq;
+  const int bh = row / Lq;
   const int h = bh % Hq;
   const int b = bh / Hq;
-  __nv_bfloat16* dst = out + (static_cast<size_t>(b) * Lq + qrow) * ldo +
-                       static_cast<size_t>(h) * HD + lane * PER;
-  if constexpr (PER == 4) {
-    uint2 wv;
-    wv.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-    wv.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-    *reinterpret_cast<uint2*>(dst) = wv;
-  } else {
-    *reinterpret_cast<uint32_t*>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-  }
-  if (lse && lane == 0) lse[warp_global] = (wsum > 0.f) ? mx + logf(wsum) : -INFINITY;
+  uint4 o;
+  o.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+  o.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+  o.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
+  o.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
+  *reinterpret_cast<uint4*>(out + (static_cast<size_t>(b) * Lq + qrow) * ldo +
+                            static_cast<size_t>(h) * HD + part * 8) = o;
+  if (lse && part == 0) lse[row] = (wsum > 0.f) ? mx + logf(wsum) : -INFINITY;
 }
 
 }  // namespace attn

@@ -14,12 +14,11 @@
 // of all S partials through distributed shared memory and applies the
 // epilogue.  Partial sums never leave the cluster.
 //
-// RMSNorm with unit gain is a per-token scale, so norm(x) w^T = rs * (x w^T)
-// with rs[t] = 1/sqrt(mean_k x[t,k]^2 + eps): the consumer of a normalised
-// input applies rs in its epilogue, computed from per-(128-column tile, token)
-// sums of squares that the producer of x wrote (per 32 columns when the
-// producers run on the CTA-pair pipeline; summed in index order).
-//
+// The epilogue can scale each token's row by rs[t] = 1/sqrt(mean_k x[t,k]^2 +
+// eps), computed from per-column-group sums of squares of the input (a
+// standalone use of dg_linear with row scales; the model's forward pass feeds
+// the projections rows that are already normalised, see norm.cuh).
+
 // With e4m3 operands (F8: x and w as codes, x scaled per token by sx[t], w
 // per tensor by sw) the MMA is kind::f8f6f4 and every epilogue takes acc as
 // sx[t] * sw * (sum of code products): a k-block is 128 codes, still one
@@ -47,23 +46,33 @@ constexpr int BK = 64;   // K per stage: one 128-byte swizzle row of bf16
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int THREADS = 192;
 constexpr int WARPS = THREADS / 32;
-constexpr int RING_BYTES = 192 * 1024;                    // TMA stage ring (also holds the fp32 tile)
 constexpr int TILE_ROW_FLOATS = BM;                       // staged tile: [BN][BM] fp32
-constexpr int SMEM_BYTES = 1024 + RING_BYTES + 256 * 4 + 256;
 constexpr int MAX_SPLITS = 8;
 
-// BN: tokens per tile (UMMA N), 128 or 256.  A stage holds KPS k-blocks (the
-// k-blocks' A tiles, then their B tiles): each stage costs a fixed share of
-// the pipeline's round trip whatever its size, so at BN = 128 two k-blocks per
-// stage (3 stages of 64 KB) stream faster than one (6 stages of 32 KB).
-template <int BN>
+// Shared memory of one CTA with a TMA stage ring of RING_KB kilobytes (the
+// ring also holds the fp32 tile after the mainloop), the row scales and the
+// barriers.  With a 96 KB ring two CTAs share an SM: each CTA's producer ->
+// MMA pipeline has a fixed round trip per stage, so two pipelines per SM move
+// more bytes than one pipeline with twice the stages.
+constexpr int smem_bytes(int ring_kb) { return 1024 + ring_kb * 1024 + 256 * 4 + 256; }
+
+// BN: tokens per tile (UMMA N), 64, 128 or 256.  A stage holds KPS k-blocks
+// (the k-blocks' A tiles, then their B tiles): each stage costs a fixed share
+// of the pipeline's round trip whatever its size, so with a 192 KB ring at
+// BN = 128 two k-blocks per stage (3 stages of 64 KB) stream faster than one
+// (6 stages of 32 KB).
+template <int BN, int RING_KB>
 struct TileCfg {
+  static constexpr int RING_BYTES = RING_KB * 1024;
   static constexpr int B_BYTES = BN * BK * 2;
-  static constexpr int KPS = BN == 128 ? 2 : 1;
+  static constexpr int KPS = (BN <= 128 && RING_KB >= 192) ? 2 : 1;
   static constexpr int STAGE_BYTES = KPS * (A_BYTES + B_BYTES);
-  static constexpr int STAGES = RING_BYTES / STAGE_BYTES;  // 4 (BN 256) or 3 (BN 128)
+  static constexpr int STAGES = RING_BYTES / STAGE_BYTES;
   static constexpr int TMEM_COLS = BN;
+  static constexpr int MIN_CTAS = RING_KB <= 96 ? 2 : 1;  // CTAs per SM
   static constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, false, false);
+  static_assert(BN == 64 || BN == 128 || BN == 256, "token tile");
+  static_assert(STAGES >= 2, "at least two stages");
   static_assert(BN * BM * 4 <= RING_BYTES, "staged tile must fit in the stage ring");
 };
 
@@ -160,12 +169,13 @@ __device__ __forceinline__ void umma_ss_f8(uint32_t d_tmem, uint64_t a_desc, uin
       : "memory");
 }
 
-template <int S, int BN, bool F8 = false>
-__global__ void __launch_bounds__(THREADS, 1)
+template <int S, int BN, bool F8 = false, int RING_KB = 192>
+__global__ void __launch_bounds__(THREADS, TileCfg<BN, RING_KB>::MIN_CTAS)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                 Params p) {
   static_assert(S == 1 || S == 2 || S == 4 || S == 8, "split count");
-  using TC = TileCfg<BN>;
+  using TC = TileCfg<BN, RING_KB>;
+  constexpr int RING_BYTES = TC::RING_BYTES;
   constexpr int STAGES = TC::STAGES;
   constexpr int STAGE_BYTES = TC::STAGE_BYTES;
   constexpr int TMEM_COLS = TC::TMEM_COLS;
@@ -432,51 +442,6 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_acc, TMEM_COLS);
-  }
-}
-
-// One CTA per token row: x[t] = embed[tok[t]] (fp32), xb[t] = bf16(x[t]),
-// ssq[j, t] = sum of x[t, G j .. G j + G - 1]^2 for groups of G = 128 or 32
-// columns (the granularity the forward pass's residual producers use).
-constexpr int EMBED_THREADS = 256;
-
-__global__ void __launch_bounds__(EMBED_THREADS) embed_kernel(
-    const int32_t* __restrict__ tok, const __nv_bfloat16* __restrict__ embed, int V, int d, int M,
-    float* __restrict__ x, __nv_bfloat16* __restrict__ xb, float* __restrict__ ssq,
-    int ssq_group) {
-  griddep_wait();
-  griddep_launch();
-  const int t = blockIdx.x;
-  int id = tok[t];
-  if (id < 0 || id >= V) {
-    if (threadIdx.x == 0) raise_error(ERR_CHECK | 0x201, static_cast<uint32_t>(t));
-    id = 0;
-  }
-  const __nv_bfloat16* e = embed + static_cast<size_t>(id) * d;
-  float* xr = x + static_cast<size_t>(t) * d;
-  __nv_bfloat16* br = xb + static_cast<size_t>(t) * d;
-  // a warp covers 128 columns (one ssq tile) per iteration: lane -> 4 columns
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int j = warp; j < d / 128; j += EMBED_THREADS / 32) {
-    const int c = j * 128 + lane * 4;
-    const uint2 raw = *reinterpret_cast<const uint2*>(e + c);
-    *reinterpret_cast<uint2*>(br + c) = raw;
-    const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
-    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
-    const float4 a = make_float4(__low2float(lo), __high2float(lo), __low2float(hi),
-                                 __high2float(hi));
-    *reinterpret_cast<float4*>(xr + c) = a;
-    if (ssq_group == 128) {
-      const float sq = warp_sum(a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w);
-      if (lane == 0) ssq[static_cast<size_t>(j) * M + t] = sq;
-    } else {
-      // eight lanes per 32-column group
-      float sq = a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
-      sq += __shfl_xor_sync(0xffffffffu, sq, 1);
-      sq += __shfl_xor_sync(0xffffffffu, sq, 2);
-      sq += __shfl_xor_sync(0xffffffffu, sq, 4);
-      if ((lane & 7) == 0) ssq[static_cast<size_t>(j * 4 + (lane >> 3)) * M + t] = sq;
-    }
   }
 }
 

@@ -1,12 +1,13 @@
-// norm.cuh - one sum of squares per token for the RMSNorm row scales.
+// norm.cuh - the RMSNorm of the residual stream, stored as the bf16 input of
+// the projection (or unembedding) that consumes it.
 //
-// When the residual projections run on the CTA-pair pipeline they leave one
-// partial sum of squares per 32 features and token ([d / 32, M]).  Every
-// consumer of the norm would otherwise add all of them up for each tile it
-// scales.  This kernel adds them once per token, in index order (the order
-// the consumers use, sixteen loads in flight), and stores the total in the
-// first partial's place: a consumer told to read one partial gets the same
-// bits as from all of them.
+//   xn[t, :] = bf16(x[t, :] * rs[t]),   rs[t] = 1 / sqrt(mean_k x[t, k]^2 + eps)
+//
+// with unit gain.  Rounding the normalised row (not the raw one) is what a
+// bf16 pipeline stores between the norm and the next product.  One CTA per
+// token row; the row's sum of squares is taken in a fixed order (each
+// thread's strided partial, the warp's butterfly, then the warps in index
+// order), so the bits do not depend on scheduling.
 #pragma once
 
 #include "dg_common.cuh"
@@ -14,26 +15,95 @@
 namespace dg {
 namespace norm {
 
-constexpr int COLLAPSE_THREADS = 256;
+constexpr int NORM_THREADS = 256;
 
-// ssq [n, M] in place: ssq[0, t] = sum_q ssq[q, t].  One thread per token
-// (a thread touches only its own column).
-__global__ void __launch_bounds__(COLLAPSE_THREADS)
-    ssq_collapse_kernel(float* __restrict__ ssq, int n, int M) {
-  griddep_wait();
-  griddep_launch();
-  const int t = static_cast<int>(blockIdx.x) * COLLAPSE_THREADS + static_cast<int>(threadIdx.x);
-  if (t >= M) return;
-  float acc = 0.f;
-  for (int q0 = 0; q0 < n; q0 += 16) {
-    float v[16];
+// Sum over the CTA of each thread's partial, in a fixed order (the warp's
+// butterfly, then the warps in index order); every thread returns the total.
+__device__ __forceinline__ float block_sum(float v, float* s_part) {
+  v = warp_sum(v);
+  if ((threadIdx.x & 31) == 0) s_part[threadIdx.x >> 5] = v;
+  __syncthreads();
+  float tot = 0.f;
 #pragma unroll
-    for (int j = 0; j < 16; ++j)
-      v[j] = q0 + j < n ? ssq[static_cast<size_t>(q0 + j) * M + t] : 0.f;
-#pragma unroll
-    for (int j = 0; j < 16; ++j) acc += v[j];
+  for (int w = 0; w < NORM_THREADS / 32; ++w) tot += s_part[w];
+  return tot;
+}
+
+__device__ __forceinline__ float4 bf16x4_to_float4(uint2 raw) {
+  const __nv_bfloat162 lo = *reinterpret_cast<const __nv_bfloat162*>(&raw.x);
+  const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&raw.y);
+  return make_float4(__low2float(lo), __high2float(lo), __low2float(hi), __high2float(hi));
+}
+
+__device__ __forceinline__ void store_scaled_row(const float4* __restrict__ xr, int n4, float rs,
+                                                 __nv_bfloat16* __restrict__ out) {
+  uint2* o = reinterpret_cast<uint2*>(out);
+  for (int i = threadIdx.x; i < n4; i += NORM_THREADS) {
+    const float4 a = xr[i];
+    uint2 w;
+    w.x = pack_bf16x2(a.x * rs, a.y * rs);
+    w.y = pack_bf16x2(a.z * rs, a.w * rs);
+    o[i] = w;
   }
-  ssq[t] = acc;
+}
+
+// x [M, d] fp32 -> xn [M, d] bf16; d % 4 == 0.  Grid: M CTAs.
+__global__ void __launch_bounds__(NORM_THREADS)
+    rmsnorm_kernel(const float* __restrict__ x, int d, float inv_d, float eps,
+                   __nv_bfloat16* __restrict__ xn) {
+  __shared__ float s_part[NORM_THREADS / 32];
+  // the successor (a projection) may launch and fetch its weights now; it
+  // reads xn only after its own wait, which covers this kernel's completion
+  griddep_launch();
+  griddep_wait();
+  const size_t row = blockIdx.x;
+  const float4* xr = reinterpret_cast<const float4*>(x + row * d);
+  const int n4 = d / 4;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < n4; i += NORM_THREADS) {
+    const float4 a = xr[i];
+    ss += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
+  }
+  const float rs = rsqrtf(block_sum(ss, s_part) * inv_d + eps);
+  store_scaled_row(xr, n4, rs, xn + row * d);
+}
+
+// The embedding lookup and the first norm: x[t] = embed[tok[t]] (fp32, no
+// scaling), xn[t] = bf16(RMSNorm(x[t])).  An out-of-range id is recorded in
+// the error word and read as id 0.  Grid: M CTAs; d % 4 == 0.
+__global__ void __launch_bounds__(NORM_THREADS)
+    embed_norm_kernel(const int32_t* __restrict__ tok, const __nv_bfloat16* __restrict__ embed,
+                      int V, int d, float inv_d, float eps, float* __restrict__ x,
+                      __nv_bfloat16* __restrict__ xn) {
+  __shared__ float s_part[NORM_THREADS / 32];
+  // the successor (a projection) may launch and fetch its weights now; it
+  // reads xn only after its own wait, which covers this kernel's completion
+  griddep_launch();
+  griddep_wait();
+  const int t = blockIdx.x;
+  int id = tok[t];
+  if (id < 0 || id >= V) {
+    if (threadIdx.x == 0) raise_error(ERR_CHECK | 0x201, static_cast<uint32_t>(t));
+    id = 0;
+  }
+  const uint2* e = reinterpret_cast<const uint2*>(embed + static_cast<size_t>(id) * d);
+  float4* xr = reinterpret_cast<float4*>(x + static_cast<size_t>(t) * d);
+  const int n4 = d / 4;
+  float ss = 0.f;
+  for (int i = threadIdx.x; i < n4; i += NORM_THREADS) {
+    const float4 a = bf16x4_to_float4(e[i]);
+    xr[i] = a;
+    ss += a.x * a.x + a.y * a.y + a.z * a.z + a.w * a.w;
+  }
+  const float rs = rsqrtf(block_sum(ss, s_part) * inv_d + eps);
+  uint2* o = reinterpret_cast<uint2*>(xn + static_cast<size_t>(t) * d);
+  for (int i = threadIdx.x; i < n4; i += NORM_THREADS) {
+    const float4 a = bf16x4_to_float4(e[i]);  // the embedding row again, not x
+    uint2 w;
+    w.x = pack_bf16x2(a.x * rs, a.y * rs);
+    w.y = pack_bf16x2(a.z * rs, a.w * rs);
+    o[i] = w;
+  }
 }
 
 }  // namespace norm

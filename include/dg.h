@@ -282,10 +282,8 @@ enum dg_linear_plan {
  * (e4m3 != 0) uses for this shape; -1 for a shape they reject.
  * dg_model_residual_on_pairs - 1 when a forward pass of the model over M
  * tokens runs both residual projections (output, K = Hq hd; MLP down, K = F)
- * on CTA pairs, which then write the residual's sums of squares per 32
- * features and collapse them once per token; 0 otherwise (per 128 features,
- * read as written); -1 for a null cfg or M < 1.  The two projections always
- * take one plan together.
+ * on CTA pairs, 0 otherwise; -1 for a null cfg or M < 1.  Each projection
+ * takes the plan of its own shape.
  */
 int dg_linear_plan_of(int M, int N, int K, int e4m3);
 int dg_model_residual_on_pairs(const dg_model_cfg* cfg, int M, int e4m3);

@@ -9,6 +9,22 @@ REL_L2 = 1e-2
 MAX_ABS = 3e-2
 
 
+def assert_close_bf16(got, want, rel_l2=REL_L2, max_abs=MAX_ABS, what=""):
+    """The bar for a tensor the product stores in bf16 (the KV cache): rel-L2
+    as for logits, and elementwise max-abs plus one bf16 step at the value's
+    magnitude (2^-7 relative), since a stored value may round to the
+    neighbouring bf16 number when its unrounded value sits within rounding of
+    the boundary."""
+    got = to64(got)
+    want = to64(want)
+    assert got.shape == want.shape, (got.shape, want.shape)
+    err = np.abs(got - want)
+    rel = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
+    excess = float(np.max(err - (max_abs + np.abs(want) * 2.0 ** -7))) if err.size else 0.0
+    assert rel <= rel_l2 and excess <= 0, f"{what}: rel_l2={rel:.3e} max excess={excess:.3e}"
+    return rel
+
+
 def cuda_ok():
     return torch.cuda.is_available()
 

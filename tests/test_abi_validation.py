@@ -190,8 +190,8 @@ def test_projection_plans(lib):
 
 
 def test_residual_projections_share_one_plan(lib, L):
-    """The output and MLP-down projections write the sums of squares the next
-    norm reads: they take the pairs together or not at all."""
+    """dg_model_residual_on_pairs: whether both residual projections (output
+    and MLP down) run on CTA pairs; each picks its plan from its own shape."""
     tiny = L.ModelCfg(256, 2, 4, 2, 64, 1024, 512, 1e-6)
     full = L.ModelCfg(2048, 24, 16, 8, 128, 8192, 262144, 1e-6)
 
@@ -204,8 +204,7 @@ def test_residual_projections_share_one_plan(lib, L):
     assert on_pairs(tiny, 48 * 256, 0) == 1        # d = 256: one tile per 256 tokens
     assert on_pairs(tiny, 47 * 256, 0) == 0
     # e4m3: Hq hd = 256 is two 128-wide k-blocks, so the output projection
-    # stays on the split-K GEMM, and the MLP down projection, which alone
-    # would qualify, stays with it
+    # stays on the split-K GEMM while the MLP down projection takes the pairs
     assert lib.dg_linear_plan_of(75 * 256, 256, 1024, 1) == 1
     assert lib.dg_linear_plan_of(75 * 256, 256, 256, 1) == 0
     assert on_pairs(tiny, 75 * 256, 1) == 0

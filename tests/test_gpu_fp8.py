@@ -188,13 +188,16 @@ def test_model_keeps_the_oracle_quantised_unembedding(fp8_model):
 def test_denoise_logits_e4m3_follow_the_oracle(fp8_model):
     """GPU FP8 logits vs the oracle's FP8 forward.
 
-    The GPU quantises the bf16 copy of the final residual (the RMSNorm a factor
-    of the logits), the oracle the bf16-rounded normalised state: the two bf16
-    roundings are independent, and one e4m3 step spans 32 bf16 steps, so about
-    one code in 32 differs by one e4m3 step (1/8 of its value).  That puts the
-    logits about sqrt(1/32) * 2^-3 / sqrt(3) ~ 1.3e-2 (rel L2) apart per unit of
-    FP8 rounding noise: bar 3e-2.  And the GPU logits must sit closer to the
-    oracle's FP8 logits than to its bf16 ones (a bf16 unembedding would not)."""
+    Both quantise the same tensor, the bf16-rounded normalised hidden states,
+    per token.  The bf16 layers before it agree with the oracle's to ~1e-3,
+    which is a few tenths of a bf16 step: a fraction of the hidden-state
+    elements round to the neighbouring bf16 value, and one in ~16 of those
+    then moves to the neighbouring e4m3 code (an e4m3 step spans 16-32 bf16
+    steps), a jump of 1/16-1/8 of its value.  That puts the FP8 logits
+    ~1.5e-2 (rel L2) apart although every product is exact (the kernel tests
+    above pin codes and products bit for bit): bar 3e-2.  And the GPU logits
+    must sit closer to the oracle's FP8 logits than to its bf16 ones (a bf16
+    unembedding would not)."""
     dg, model, w64, prompt = fp8_model
     st = dg.DgState(SHAPE, 1, P + 2 * C, C)
     dg.prefill(model, st, prompt.cuda())
@@ -267,16 +270,15 @@ def test_model_keeps_the_oracle_quantised_projections(fp8_full_model):
 
 def test_denoise_logits_e4m3_layers_follow_the_oracle(fp8_full_model):
     """Prefill and denoising pass with every projection and the unembedding in
-    FP8, against the oracle's FP8 forward.
-
-    Nine quantised products in a row make the FP8 logits of this small random
-    model as sensitive to rounding as to quantisation itself: the oracle's own
-    FP8 logits move by about as much when its bf16 storage rounding is switched
-    off as FP8 moves them from bf16.  So the model-level bar is that
-    sensitivity (the exact pins are the kernel tests above: codes bit for bit,
-    products to fp32 rounding): the GPU must sit within 1.5x of it from the
-    oracle's FP8 logits, and its FP8 logits must differ from its own bf16 ones
-    (the FP8 path runs)."""
+    FP8, against the oracle's FP8 forward.  Both sides quantise the same bf16
+    tensors (the normalised residual stream, the attention output, the GELU
+    output), but nine quantised products in a row amplify any rounding
+    difference upstream of a quantiser (see the unembedding-only test): the
+    oracle's own FP8 logits move by ~6e-2 when only its bf16 storage rounding
+    is switched off, as much as FP8 moves them from bf16.  So the model-level
+    bar is that measured sensitivity (the exact pins are the kernel tests
+    above): the GPU must sit within 1.5x of it from the oracle's FP8 logits,
+    and its FP8 logits must differ from its own bf16 ones (the FP8 path runs)."""
     dg, model, w64, prompt = fp8_full_model
     canvas = torch.randint(0, SHAPE.vocab, (1, C), generator=torch.Generator().manual_seed(2))
 
@@ -340,12 +342,11 @@ def test_block_driver_e4m3_layers_matches_stepwise_calls(fp8_full_model):
 
 
 def test_denoise_logits_e4m3_layers_many_sequences(fp8_full_model):
-    """75 sequences (19200 canvas tokens) on the FP8 model.  The MLP down
-    projection (K = F, eight e4m3 k-blocks) would qualify for the CTA-pair
-    pipeline while the output projection (K = Hq hd, two k-blocks) does not;
-    both write the residual's sums of squares that the next norm reads, so
-    they must take one path together.  Sampled sequences against the oracle's
-    FP8 forward at the bar of the one-sequence test."""
+    """75 sequences (19200 canvas tokens) on the FP8 model: the MLP down
+    projection (K = F, eight e4m3 k-blocks) runs on the CTA-pair pipeline
+    while the output projection (K = Hq hd, two k-blocks) stays on the split-K
+    GEMM.  Sampled sequences against the oracle's FP8 forward, at the bar of
+    the one-sequence test."""
     dg, model, w64, _ = fp8_full_model
     Bn = 75
     st = dg.DgState(SHAPE, Bn, P + 2 * C, C)
