@@ -566,7 +566,7 @@ int launch_attn(const void* q, int ldq, const void* k_new, const void* v_new, in
   if (S > 1) {
     const int rows = B * Hq * Lq;
     const int threads = dg::attn::COMBINE_THREADS;
-    const int blocks = cdiv(rows * (hd / 8), threads);  // hd / 8 threads per row
+    const int blocks = cdiv(rows * 32, threads);  // a warp per row
     if (hd == 128)
       DG_CUDA(launch_ex(dg::attn::attn_combine_kernel<128>, dim3(blocks), dim3(threads), 0, s, 1,
                         (const __nv_bfloat16*)p.part_o, (const float*)p.part_lse, S, B, Hq, Lq,
@@ -911,10 +911,30 @@ int run_forward(const Fwd& f, const int32_t* tok, float* logits, cudaStream_t s)
   __nv_bfloat16* up = (__nv_bfloat16*)(f.ws + f.L.up);
   void* aws = f.ws + f.L.attn;
   const float scale = 1.0f / std::sqrt((float)hd);
-  // xn = bf16(RMSNorm(x)) after each residual update
+  // xn = bf16(RMSNorm(x)) after each residual update: a warp per row while
+  // the row fits in its registers
   auto norm = [&]() -> int {
-    DG_CUDA(launch_ex(dg::norm::rmsnorm_kernel, dim3(M), dim3(dg::norm::NORM_THREADS), 0, s, 1,
-                      (const float*)x, c.d, 1.f / c.d, c.eps, xn));
+    namespace nm = dg::norm;
+    const dim3 rows_grid(cdiv(M, nm::ROW_WARPS)), rows_block(nm::ROW_WARPS * 32);
+    const float inv_d = 1.f / c.d;
+    cudaError_t e;
+    switch (c.d % 128 == 0 && c.d <= nm::ROW_MAX_D ? c.d / 128 : 0) {
+      case 1: e = launch_ex(nm::rmsnorm_rows_kernel<1>, rows_grid, rows_block, 0, s, 1,
+                            (const float*)x, M, c.d, inv_d, c.eps, xn); break;
+      case 2: e = launch_ex(nm::rmsnorm_rows_kernel<2>, rows_grid, rows_block, 0, s, 1,
+                            (const float*)x, M, c.d, inv_d, c.eps, xn); break;
+      case 4: e = launch_ex(nm::rmsnorm_rows_kernel<4>, rows_grid, rows_block, 0, s, 1,
+                            (const float*)x, M, c.d, inv_d, c.eps, xn); break;
+      case 8: e = launch_ex(nm::rmsnorm_rows_kernel<8>, rows_grid, rows_block, 0, s, 1,
+                            (const float*)x, M, c.d, inv_d, c.eps, xn); break;
+      case 16: e = launch_ex(nm::rmsnorm_rows_kernel<16>, rows_grid, rows_block, 0, s, 1,
+                             (const float*)x, M, c.d, inv_d, c.eps, xn); break;
+      case 32: e = launch_ex(nm::rmsnorm_rows_kernel<32>, rows_grid, rows_block, 0, s, 1,
+                             (const float*)x, M, c.d, inv_d, c.eps, xn); break;
+      default: e = launch_ex(nm::rmsnorm_kernel, dim3(M), dim3(nm::NORM_THREADS), 0, s, 1,
+                             (const float*)x, c.d, inv_d, c.eps, xn); break;
+    }
+    DG_CUDA(e);
     count_launch();
     return DG_OK;
   };

@@ -27,6 +27,8 @@
 // TMEM lanes 32*(w%4)..+31).
 #pragma once
 
+#include <type_traits>
+
 #include "dg_common.cuh"
 
 namespace dg {
@@ -489,53 +491,74 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // Merge key-range splits: O = sum_s w_s O_s / sum_s w_s, w_s = exp(lse_s - max).
-// A row is HD / 8 threads, each owning 8 consecutive output values (one
-// 16-byte load per split).  Every split's log-sum-exp and partial row are
-// requested before any arithmetic, so a thread waits for memory once; the
-// sums run in split order (the bits do not depend on scheduling).
+// One warp per (b, h, row), each lane owning HD / 32 consecutive values.
+// Every split's log-sum-exp and partial row are requested before any
+// arithmetic (a batch of COMBINE_BATCH splits in flight per lane), so a warp
+// waits for memory once per batch; the sums run in split order (the bits do
+// not depend on scheduling).  The register cap keeps three CTAs on an SM: the
+// kernel is bound by how many loads are in flight, not by arithmetic.
 constexpr int MAX_SPLITS = 32;
 constexpr int COMBINE_THREADS = 256;
-constexpr int COMBINE_BATCH = 16;  // splits in flight per thread
+
+// acc[0..] += w * (the bf16 values of a lane's slice of a row)
+__device__ __forceinline__ void add_weighted(float (&acc)[4], float w, uint2 v) {
+  const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&v.x);
+  const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&v.y);
+  acc[0] = fmaf(w, __low2float(a), acc[0]);
+  acc[1] = fmaf(w, __high2float(a), acc[1]);
+  acc[2] = fmaf(w, __low2float(b), acc[2]);
+  acc[3] = fmaf(w, __high2float(b), acc[3]);
+}
+__device__ __forceinline__ void add_weighted(float (&acc)[2], float w, uint32_t v) {
+  const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&v);
+  acc[0] = fmaf(w, __low2float(a), acc[0]);
+  acc[1] = fmaf(w, __high2float(a), acc[1]);
+}
+__device__ __forceinline__ uint2 pack_row(const float (&a)[4], float inv) {
+  return make_uint2(pack_bf16x2(a[0] * inv, a[1] * inv), pack_bf16x2(a[2] * inv, a[3] * inv));
+}
+__device__ __forceinline__ uint32_t pack_row(const float (&a)[2], float inv) {
+  return pack_bf16x2(a[0] * inv, a[1] * inv);
+}
+constexpr int COMBINE_BATCH = 12;
 
 template <int HD>
-__global__ void __launch_bounds__(COMBINE_THREADS)
+__global__ void __launch_bounds__(COMBINE_THREADS, 3)
     attn_combine_kernel(const __nv_bfloat16* __restrict__ part_o,
                         const float* __restrict__ part_lse, int S, int B, int Hq, int Lq,
                         __nv_bfloat16* __restrict__ out, int ldo, float* __restrict__ lse) {
-  constexpr int TPR = HD / 8;  // threads per row
+  constexpr int PER = HD / 32;  // values per lane: 4 (8 bytes) or 2 (4 bytes)
+  using Vec = typename std::conditional<PER == 4, uint2, uint32_t>::type;
   griddep_launch();
   griddep_wait();
-  const int gt = static_cast<int>(blockIdx.x) * COMBINE_THREADS + static_cast<int>(threadIdx.x);
-  const int row = gt / TPR;
-  const int part = gt % TPR;
+  const int row = (static_cast<int>(blockIdx.x) * COMBINE_THREADS +
+                   static_cast<int>(threadIdx.x)) >> 5;
+  const int lane = threadIdx.x & 31;
   const int rows = B * Hq * Lq;
-  if (row >= rows) return;
+  if (row >= rows) return;  // warp-uniform
   const size_t stride = static_cast<size_t>(rows);
-  float mx = -INFINITY;
-  float ls[COMBINE_BATCH];
-  uint4 v[COMBINE_BATCH];
-  float acc[8];
+  float mx = -INFINITY, wsum = 0.f;
+  float acc[PER];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) acc[e] = 0.f;
-  float wsum = 0.f;
-  // pass over the splits in batches; the running max is the first batch's
-  // (the combine is exact for any reference, the max only keeps exp in range)
+  for (int e = 0; e < PER; ++e) acc[e] = 0.f;
   for (int s0 = 0; s0 < S; s0 += COMBINE_BATCH) {
+    float ls[COMBINE_BATCH];
+    Vec v[COMBINE_BATCH];
 #pragma unroll
     for (int k = 0; k < COMBINE_BATCH; ++k) {
       const int sp = s0 + k;
       ls[k] = sp < S ? part_lse[sp * stride + row] : -INFINITY;
-      v[k] = sp < S ? *reinterpret_cast<const uint4*>(part_o + (sp * stride + row) * HD + part * 8)
-                    : make_uint4(0u, 0u, 0u, 0u);
+      v[k] = sp < S ? reinterpret_cast<const Vec*>(part_o + (sp * stride + row) * HD)[lane]
+                    : Vec{};
     }
     float bmx = -INFINITY;
 #pragma unroll
     for (int k = 0; k < COMBINE_BATCH; ++k) bmx = fmaxf(bmx, ls[k]);
     if (bmx > mx) {
-      // rescale what the earlier batches accumulated
+      // rescale what earlier batches accumulated (exact for any reference)
       const float f = mx == -INFINITY ? 0.f : expf(mx - bmx);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] *= f;
+      for (int e = 0; e < PER; ++e) acc[e] *= f;
       wsum *= f;
       mx = bmx;
     }
@@ -544,13 +567,7 @@ __global__ void __launch_bounds__(COMBINE_THREADS)
       if (ls[k] == -INFINITY) continue;  // an empty split
       const float w = expf(ls[k] - mx);
       wsum += w;
-      const uint32_t wd[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const __nv_bfloat162 p2 = *reinterpret_cast<const __nv_bfloat162*>(&wd[q]);
-        acc[2 * q] += w * __low2float(p2);
-        acc[2 * q + 1] += w * __high2float(p2);
-      }
+      add_weighted(acc, w, v[k]);
     }
   }
   const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
@@ -558,14 +575,10 @@ __global__ void __launch_bounds__(COMBINE_THREADS)
   const int bh = row / Lq;
   const int h = bh % Hq;
   const int b = bh / Hq;
-  uint4 o;
-  o.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
-  o.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
-  o.z = pack_bf16x2(acc[4] * inv, acc[5] * inv);
-  o.w = pack_bf16x2(acc[6] * inv, acc[7] * inv);
-  *reinterpret_cast<uint4*>(out + (static_cast<size_t>(b) * Lq + qrow) * ldo +
-                            static_cast<size_t>(h) * HD + part * 8) = o;
-  if (lse && part == 0) lse[row] = (wsum > 0.f) ? mx + logf(wsum) : -INFINITY;
+  const Vec o = pack_row(acc, inv);
+  reinterpret_cast<Vec*>(out + (static_cast<size_t>(b) * Lq + qrow) * ldo +
+                         static_cast<size_t>(h) * HD)[lane] = o;
+  if (lse && lane == 0) lse[row] = (wsum > 0.f) ? mx + logf(wsum) : -INFINITY;
 }
 
 }  // namespace attn

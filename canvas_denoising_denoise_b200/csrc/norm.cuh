@@ -47,13 +47,12 @@ __device__ __forceinline__ void store_scaled_row(const float4* __restrict__ xr, 
   }
 }
 
-// x [M, d] fp32 -> xn [M, d] bf16; d % 4 == 0.  Grid: M CTAs.
+// x [M, d] fp32 -> xn [M, d] bf16; d % 4 == 0.  Grid: M CTAs.  (Rows wider
+// than ROW_MAX_D; the warp-per-row kernel below takes the rest.)
 __global__ void __launch_bounds__(NORM_THREADS)
     rmsnorm_kernel(const float* __restrict__ x, int d, float inv_d, float eps,
                    __nv_bfloat16* __restrict__ xn) {
   __shared__ float s_part[NORM_THREADS / 32];
-  // the successor (a projection) may launch and fetch its weights now; it
-  // reads xn only after its own wait, which covers this kernel's completion
   griddep_launch();
   griddep_wait();
   const size_t row = blockIdx.x;
@@ -66,6 +65,37 @@ __global__ void __launch_bounds__(NORM_THREADS)
   }
   const float rs = rsqrtf(block_sum(ss, s_part) * inv_d + eps);
   store_scaled_row(xr, n4, rs, xn + row * d);
+}
+
+// One warp per row for rows of up to ROW_MAX_D values (d % 128 == 0): the
+// row sits in the warp's registers (lane k holds float4 groups k, k + 32, ...),
+// so it is read once and reduced with shuffles alone.  The sum of squares is
+// each lane's groups in order, then the butterfly: a fixed order.
+constexpr int ROW_MAX_D = 4096;
+constexpr int ROW_WARPS = 4;  // rows per CTA
+
+template <int G>  // float4 groups per lane: d / 128
+__global__ void __launch_bounds__(ROW_WARPS * 32)
+    rmsnorm_rows_kernel(const float* __restrict__ x, int M, int d, float inv_d, float eps,
+                        __nv_bfloat16* __restrict__ xn) {
+  griddep_launch();
+  griddep_wait();
+  const int row = static_cast<int>(blockIdx.x) * ROW_WARPS + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= M) return;  // warp-uniform
+  const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(row) * d);
+  float4 v[G];
+  float ss = 0.f;
+#pragma unroll
+  for (int g = 0; g < G; ++g) v[g] = xr[g * 32 + lane];
+#pragma unroll
+  for (int g = 0; g < G; ++g) ss += v[g].x * v[g].x + v[g].y * v[g].y + v[g].z * v[g].z + v[g].w * v[g].w;
+  const float rs = rsqrtf(warp_sum(ss) * inv_d + eps);
+  uint2* o = reinterpret_cast<uint2*>(xn + static_cast<size_t>(row) * d);
+#pragma unroll
+  for (int g = 0; g < G; ++g)
+    o[g * 32 + lane] = make_uint2(pack_bf16x2(v[g].x * rs, v[g].y * rs),
+                                  pack_bf16x2(v[g].z * rs, v[g].w * rs));
 }
 
 // The embedding lookup and the first norm: x[t] = embed[tok[t]] (fp32, no
