@@ -83,3 +83,55 @@ def unembed_logits(h_codes, h_scales, w_codes, w_scale, row_scale=None):
     if row_scale is not None:
         s = s * np.asarray(row_scale, dtype=np.float64)
     return (acc * s[:, None]).astype(np.float32)
+
+
+def attention_head_e4m3(q_codes, q_scales, k_codes, v_codes, k_scale, v_scale, mask, scale,
+                        shift=0.0):
+    """FP8 attention of one query head over its keys (a reading: the pages quote FP8
+    serving but fix no recipe for attention).
+
+    q_codes [Lq, hd] e4m3 codes with per-row (per-token) scales q_scales [Lq];
+    k_codes, v_codes [Lk, hd] codes with one scale each; mask [Lq, Lk] boolean.
+      s[i, j] = scale q_scales[i] k_scale sum_d dec(q)[i, d] dec(k)[j, d]
+      p[i, j] = exp(s[i, j] - max_j s[i, j])            (masked keys: p = 0)
+      out[i]  = v_scale sum_j e4m3(p[i, j]) dec(v)[j] / sum_j p[i, j]
+    The probabilities enter the value product as e4m3 values (the operand type of
+    an 8-bit product) and the normaliser as exact ones.  They are rounded relative
+    to the row maximum (p <= 1); `shift` rounds 2^shift p instead and divides the
+    result back, which is how a kernel whose running maximum lags the row's by a
+    factor 2^shift rounds them.  An integer shift changes nothing while p stays in
+    the normal range (e4m3 rounding commutes with powers of two there).
+    """
+    qd = decode(q_codes) * np.asarray(q_scales, dtype=np.float64)[:, None]
+    kd = decode(k_codes)
+    s = (qd @ kd.T) * (np.float64(k_scale) * scale)
+    s = np.where(mask, s, -np.inf)
+    m = np.max(s, axis=1, keepdims=True)
+    p = np.exp(s - m)
+    c = 2.0 ** shift
+    pq = decode(encode(p * c)) / c
+    return np.float64(v_scale) * (pq @ decode(v_codes)) / np.sum(p, axis=1, keepdims=True)
+
+
+def gqa_attention_e4m3(q_codes, q_scales, kn_codes, vn_codes, kp_codes, vp_codes, k_scale,
+                       v_scale, causal, scale, shift=0.0):
+    """Grouped-query FP8 attention of one sequence: q_codes [Lq, Hq, hd] with per-token
+    scales [Lq]; new rows' codes kn/vn [Lq, Hkv, hd]; cached prefix kp/vp [Hkv, L, hd];
+    one K scale and one V scale for prefix and new rows together.  The key set and the
+    mask are those of the bf16 attention (the prefix, then the new rows: full for a
+    canvas, lower-triangular for a causal pass).  Returns [Lq, Hq, hd] fp64."""
+    lq, hq, hd = q_codes.shape
+    hkv = kn_codes.shape[1]
+    group = hq // hkv
+    lp = kp_codes.shape[1]
+    pre = np.ones((lq, lp), dtype=bool)
+    own = np.tril(np.ones((lq, lq), dtype=bool)) if causal else np.ones((lq, lq), dtype=bool)
+    mask = np.concatenate([pre, own], axis=1)
+    out = np.empty((lq, hq, hd), dtype=np.float64)
+    for h in range(hq):
+        g = h // group
+        k = np.concatenate([kp_codes[g], kn_codes[:, g, :]], axis=0)
+        v = np.concatenate([vp_codes[g], vn_codes[:, g, :]], axis=0)
+        out[:, h, :] = attention_head_e4m3(q_codes[:, h, :], q_scales, k, v, k_scale, v_scale,
+                                           mask, scale, shift)
+    return out

@@ -103,3 +103,93 @@ def test_unembed_e4m3_within_the_format_error_bound():
     bound = rel * (np.abs(h) @ np.abs(w).T) + sub + 1e-6 * np.abs(exact)
     assert np.all(np.abs(got - exact) <= bound)
     assert np.abs(got - exact).max() > 0
+
+
+# ---------------------------------------------------------------- FP8 attention
+
+def _codes(vals):
+    return fp8.encode(np.asarray(vals, dtype=np.float64))
+
+
+def test_attention_e4m3_two_keys_closed_form():
+    # scores (ln(1/0.3), 0): p = (1, 0.3); e4m3(0.3) = 1.25 * 2^-2 = 0.3125 enters
+    # the value sum, the exact 0.3 the normaliser
+    q = _codes([[1.0]])
+    k = _codes([[1.0], [0.0]])
+    v = _codes([[2.0], [-4.0]])
+    mask = np.ones((1, 2), dtype=bool)
+    out = fp8.attention_head_e4m3(q, [1.0], k, v, 1.0, 0.5, mask, -np.log(0.3))
+    assert np.isclose(out[0, 0], 0.5 * (2.0 - 4.0 * 0.3125) / 1.3, rtol=1e-12, atol=0)
+
+
+def test_attention_e4m3_exact_probabilities_match_sdpa():
+    # integer dot products times ln 2: every probability is a power of two no
+    # smaller than 2^-6 (a normal e4m3 value), so only the dequantisation is left
+    # and the result is softmax attention of the decoded values (library routine)
+    rng = np.random.default_rng(3)
+    lq, lp, hq, hkv, hd = 6, 9, 4, 2, 16
+    qv = np.zeros((lq, hq, hd))
+    for i in range(lq):
+        for h in range(hq):
+            dims = rng.choice(hd, size=3, replace=False)
+            qv[i, h, dims] = rng.choice([-1.0, 1.0], size=3)
+    kn = rng.choice([-1.0, 1.0], size=(lq, hkv, hd))
+    kp = rng.choice([-1.0, 1.0], size=(hkv, lp, hd))
+    vn = rng.normal(size=(lq, hkv, hd))
+    vp = rng.normal(size=(hkv, lp, hd))
+    qc = _codes(qv)                                     # codes of +-1 and 0
+    vnc, vpc = _codes(vn * 16), _codes(vp * 16)
+    for causal in (False, True):
+        got = fp8.gqa_attention_e4m3(qc, np.ones(lq), _codes(kn), vnc, _codes(kp), vpc,
+                                     1.0, 1.0 / 16, causal, np.log(2.0))
+        mask = np.concatenate([np.ones((lq, lp), dtype=bool),
+                               np.tril(np.ones((lq, lq), dtype=bool)) if causal
+                               else np.ones((lq, lq), dtype=bool)], axis=1)
+        for h in range(hq):
+            g = h // (hq // hkv)
+            k = torch.from_numpy(np.concatenate([kp[g], kn[:, g]], axis=0))
+            v = torch.from_numpy(fp8.decode(np.concatenate([vpc[g], vnc[:, g]], axis=0)) / 16)
+            want = torch.nn.functional.scaled_dot_product_attention(
+                torch.from_numpy(qv[:, h])[None], k[None], v[None],
+                attn_mask=torch.from_numpy(mask)[None], scale=float(np.log(2.0)))[0].numpy()
+            assert np.allclose(got[:, h], want, rtol=1e-12, atol=1e-14), (causal, h)
+
+
+def test_attention_e4m3_integer_reference_shift_changes_nothing_in_the_normal_range():
+    rng = np.random.default_rng(4)
+    q = _codes(rng.normal(size=(8, 32)))
+    k = _codes(rng.normal(size=(40, 32)))
+    v = _codes(rng.normal(size=(40, 32)))
+    qs = np.full(8, 0.05)
+    mask = np.ones((8, 40), dtype=bool)
+    # small scores: every p lies in [2^-5, 1], well inside the normal range
+    base = fp8.attention_head_e4m3(q, qs, k, v, 1.0, 1.0, mask, 0.3)
+    s = (fp8.decode(q) * qs[:, None]) @ fp8.decode(k).T * 0.3
+    assert np.min(np.exp(s - s.max(axis=1, keepdims=True))) > 2.0 ** -5
+    for c in (1, 3, 8):
+        assert np.array_equal(fp8.attention_head_e4m3(q, qs, k, v, 1.0, 1.0, mask, 0.3, c), base)
+    moved = fp8.attention_head_e4m3(q, qs, k, v, 1.0, 1.0, mask, 0.3, 0.5)
+    assert not np.array_equal(moved, base)
+
+
+def test_attention_e4m3_within_the_rounding_bound_of_exact_attention():
+    # the only rounding after dequantisation is e4m3(p): relative 2^-4 for normal
+    # values, absolute 2^-10 below 2^-6
+    rng = np.random.default_rng(5)
+    lq, lk, hd = 16, 300, 64
+    q = _codes(rng.normal(size=(lq, hd)) * 20)
+    qs = rng.uniform(0.02, 0.06, lq)
+    k = _codes(rng.normal(size=(lk, hd)) * 20)
+    v = _codes(rng.normal(size=(lk, hd)) * 20)
+    mask = np.ones((lq, lk), dtype=bool)
+    mask[3, 100:] = False
+    got = fp8.attention_head_e4m3(q, qs, k, v, 0.05, 0.05, mask, 1 / np.sqrt(hd))
+    qd = fp8.decode(q) * qs[:, None]
+    s = (qd @ fp8.decode(k).T) * 0.05 / np.sqrt(hd)
+    s = np.where(mask, s, -np.inf)
+    p = np.exp(s - s.max(axis=1, keepdims=True))
+    vd = fp8.decode(v) * 0.05
+    exact = (p @ vd) / p.sum(axis=1, keepdims=True)
+    bound = ((np.maximum(p * 2.0 ** -4, 2.0 ** -10)) @ np.abs(vd)) / p.sum(axis=1, keepdims=True)
+    assert np.all(np.abs(got - exact) <= bound * (1 + 1e-9))
+    assert np.max(np.abs(got - exact)) > 0                # the rounding is there
