@@ -532,6 +532,36 @@ def run_kernel_bench(args):
                         "us": round(t * 1e6, 2),
                         "tflops": round(fl / t / 1e12, 1),
                         "frac_bf16_peak": round(fl / t / 1e12 / peaks["bf16_tflops"], 4)})
+            if args.fp8_attn:
+                # e4m3 codes made on the device (outside the timed region): per-token
+                # Q, one scale over the cached and new K (and V), V transposed
+                q8 = torch.empty((B * CANVAS, hq * hd), dtype=torch.uint8, device="cuda")
+                qs = torch.empty(B * CANVAS, dtype=torch.float32, device="cuda")
+                dg.quantize_e4m3(q.view(B * CANVAS, -1), q8, qs, per_row=True)
+                codes = {}
+                for name, cache, new in (("k", kc, kn), ("v", vc, vn)):
+                    both = torch.cat([cache.reshape(-1, hd), new.reshape(-1, hd)])
+                    c8 = torch.empty(both.shape, dtype=torch.uint8, device="cuda")
+                    sc = torch.empty(1, dtype=torch.float32, device="cuda")
+                    dg.quantize_e4m3(both, c8, sc, per_row=False)
+                    nc = cache.numel() // hd
+                    codes[name] = (c8[:nc].view(cache.shape), c8[nc:].view(new.shape), sc)
+                kc8, kn8, ks = codes["k"]
+                vc8, vn8, vs = codes["v"]
+                vt_c = vc8.transpose(-1, -2).contiguous()
+                vt_n = vn8.view(B, CANVAS, hkv, hd).permute(0, 2, 3, 1).contiguous()
+                kn8 = kn8.contiguous()
+                t8 = timed(lambda: dg.canvas_attn_e4m3(q8.view(B, CANVAS, -1), qs, kn8, vt_n,
+                                                       kc8, vt_c, ks, vs, cl, L, o,
+                                                       n_q_heads=hq, n_kv_heads=hkv, ws=ws),
+                           args.steps)
+                # e4m3 tensor peak: the measured bf16 peak times the nominal ratio 2
+                out.append({"kernel": "canvas_attn_e4m3", "heads": [hq, hkv], "prefix": L,
+                            "us": round(t8 * 1e6, 2), "tflops": round(fl / t8 / 1e12, 1),
+                            "frac_fp8_peak": round(fl / t8 / 1e12 / (2 * peaks["bf16_tflops"]), 4),
+                            "frac_bf16_peak": round(fl / t8 / 1e12 / peaks["bf16_tflops"], 4),
+                            "speedup_vs_bf16": round(t / t8, 3)})
+                del q8, codes, kc8, kn8, vc8, vn8, vt_c, vt_n
     elif args.kernel == "sampler":
         B, V = args.batch, 262144
         settings = dg.SamplerSettings()
@@ -689,6 +719,8 @@ def main():
     ap.add_argument("--epi", default="bf16", choices=["bf16", "gelu", "f32", "resid"],
                     help="epilogue for --kernel gemm")
     ap.add_argument("--heads", default="32,8", help="query,kv heads for --kernel attn")
+    ap.add_argument("--fp8-attn", action="store_true",
+                    help="--kernel attn: also time the e4m3 attention on the same inputs")
     ap.add_argument("--fp8-unembed", action="store_true",
                     help="run the unembedding + sampler step on e4m3 operands")
     ap.add_argument("--fp8-layers", action="store_true",

@@ -7,7 +7,7 @@ CUDA device, and raises otherwise.
 
 Functions take torch tensors and pass their device pointers:
     canvas_attn, unembed, linear, sample_commit, unembed_sample_commit, kv_block_commit,
-    quantize_e4m3, linear_e4m3, unembed_e4m3, unembed_sample_commit_e4m3,
+    canvas_attn_e4m3, quantize_e4m3, linear_e4m3, unembed_e4m3, unembed_sample_commit_e4m3,
     philox
 Objects:
     DgModel   weights + configuration (dg_model)
@@ -22,7 +22,7 @@ from . import _lib
 from ._lib import (EPI_BF16, EPI_F32, EPI_GELU_BF16, EPI_RESID_F32, MASK_BIDIR, MASK_CAUSAL,
                    UNSELECTED_KEEP, UNSELECTED_RENOISE, DgError)
 
-__all__ = ["canvas_attn", "unembed", "linear", "sample_commit", "unembed_sample_commit",
+__all__ = ["canvas_attn", "canvas_attn_e4m3", "unembed", "linear", "sample_commit", "unembed_sample_commit",
            "quantize_e4m3", "linear_e4m3", "unembed_e4m3", "unembed_sample_commit_e4m3",
            "kv_block_commit", "philox",
            "DgModel", "DgState", "SamplerSettings", "prefill", "denoise_logits", "denoise_block",
@@ -120,6 +120,36 @@ def canvas_attn(q, k_new, v_new, k_cache, v_cache, cache_len, max_prefix, out, *
                                   _ptr(k_cache), _ptr(v_cache), _ptr(cache_len), max_prefix,
                                   lmax, _ptr(out), out.stride(1), _ptr(lse), B, n_q_heads,
                                   n_kv_heads, Lq, head_dim, scale, mask, wp, wn, _stream(stream)))
+    return out
+
+
+def canvas_attn_e4m3(q, q_scale, k_new, vt_new, k_cache, vt_cache, k_scale, v_scale, cache_len,
+                     max_prefix, out, *, n_q_heads, n_kv_heads, lse=None, scale=None,
+                     mask=MASK_BIDIR, ws=None, stream=None):
+    """canvas_attn on e4m3 codes (uint8 tensors), head_dim 128.
+
+    q [B, Lq, >=Hq*128] with per-token scales q_scale [B*Lq] fp32; k_new [B, Lq, ld];
+    vt_new [B, Hkv, 128, ldvt] (V transposed, keys contiguous); k_cache [B, Hkv, lmax, 128];
+    vt_cache [B, Hkv, 128, lmax]; k_scale, v_scale one-element fp32 tensors; out bf16.
+    """
+    lib = _lib.load()
+    B, Lq = q.shape[0], q.shape[1]
+    lmax = k_cache.shape[2]
+    for t in (q, k_new, out):
+        if t.stride(-1) != 1 or t.stride(0) != t.shape[1] * t.stride(1):
+            raise ValueError("q/k_new/out must be [B, Lq, ld] with unit inner stride")
+    if vt_new.stride(-1) != 1 or vt_new.stride(2) * 128 != vt_new.stride(1) or \
+            vt_new.stride(1) * vt_new.shape[1] != vt_new.stride(0):
+        raise ValueError("vt_new must be [B, Hkv, 128, ldvt] with unit inner stride")
+    _need_contig(q_scale, k_cache, vt_cache, k_scale, v_scale, cache_len, lse)
+    scale = 128 ** -0.5 if scale is None else scale
+    need = lib.dg_canvas_attn_workspace_bytes(B, n_q_heads, n_kv_heads, Lq, 128, max_prefix)
+    wp, wn = _ws(ws).args(need)
+    _lib.check(lib.dg_canvas_attn_e4m3(
+        _ptr(q), q.stride(1), _ptr(q_scale), _ptr(k_new), k_new.stride(1), _ptr(vt_new),
+        vt_new.stride(2), _ptr(k_cache), _ptr(vt_cache), _ptr(k_scale), _ptr(v_scale),
+        _ptr(cache_len), max_prefix, lmax, _ptr(out), out.stride(1), _ptr(lse), B, n_q_heads,
+        n_kv_heads, Lq, 128, scale, mask, wp, wn, _stream(stream)))
     return out
 
 

@@ -80,6 +80,10 @@ SIGNATURES = {
                                c_int, c_int, c_int, c_float, c_int, c_void_p, c_size_t,
                                c_void_p]),
     "dg_canvas_attn_workspace_bytes": (c_size_t, [c_int, c_int, c_int, c_int, c_int, c_int]),
+    "dg_canvas_attn_e4m3": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_int, c_void_p, c_int,
+                                    c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_int,
+                                    c_int, c_void_p, c_int, c_void_p, c_int, c_int, c_int, c_int,
+                                    c_int, c_float, c_int, c_void_p, c_size_t, c_void_p]),
     "dg_unembed": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_size_t,
                            c_void_p]),
     "dg_linear": (c_int, [c_void_p, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_void_p,

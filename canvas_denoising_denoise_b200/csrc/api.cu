@@ -535,6 +535,7 @@ int launch_attn(const void* q, int ldq, const void* k_new, const void* v_new, in
   p.lse = lse;
   p.part_o = nullptr;
   p.part_lse = nullptr;
+  p.q_scale = p.k_scale = p.v_scale = nullptr;
   if (S > 1) {
     const size_t rows = (size_t)S * B * Hq * Lq;
     p.part_o = (__nv_bfloat16*)ws;
@@ -575,6 +576,68 @@ int launch_attn(const void* q, int ldq, const void* k_new, const void* v_new, in
       DG_CUDA(launch_ex(dg::attn::attn_combine_kernel<64>, dim3(blocks), dim3(threads), 0, s, 1,
                         (const __nv_bfloat16*)p.part_o, (const float*)p.part_lse, S, B, Hq, Lq,
                         (__nv_bfloat16*)out, ldo, lse));
+    count_launch();
+    DG_CUDA(cudaGetLastError());
+  }
+  return DG_OK;
+}
+
+PerDeviceFlag attn_f8_attr_done;
+
+// The e4m3 variant (hd = 128): the same plan, split count and merge; 8-bit
+// tensor maps (one 128-byte swizzle row per box row) over Q, K and V^T.
+int launch_attn_e4m3(const uint8_t* q, int ldq, const float* q_scale, const uint8_t* k_new,
+                     int ldkv, const uint8_t* vt_new, int ldvt, const uint8_t* k_cache,
+                     const uint8_t* vt_cache, const float* k_scale, const float* v_scale,
+                     const int32_t* cache_len, int max_prefix, int lmax, void* out, int ldo,
+                     float* lse, int B, int Hq, int Hkv, int Lq, float scale, int mask, void* ws,
+                     cudaStream_t s) {
+  constexpr int hd = 128;
+  const int S = attn_splits(B, Hq, Hkv, Lq, max_prefix);
+  CUtensorMap tq, tkn, tvn, tkc, tvc;
+  DG_TRY(make_tmap_u8(&tq, q, (uint64_t)Hq * hd, (uint64_t)B * Lq, (uint64_t)ldq, 128));
+  DG_TRY(make_tmap_u8(&tkn, k_new, (uint64_t)Hkv * hd, (uint64_t)B * Lq, (uint64_t)ldkv, 128));
+  DG_TRY(make_tmap_u8(&tvn, vt_new, (uint64_t)Lq, (uint64_t)B * Hkv * hd, (uint64_t)ldvt, 128));
+  DG_TRY(make_tmap_u8(&tkc, k_cache, hd, (uint64_t)B * Hkv * lmax, (uint64_t)hd, 128));
+  DG_TRY(make_tmap_u8(&tvc, vt_cache, (uint64_t)lmax, (uint64_t)B * Hkv * hd, (uint64_t)lmax,
+                      128));
+  dg::attn::Params p;
+  p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Lq = Lq; p.lmax = lmax; p.group = Hq / Hkv;
+  p.n_rt = cdiv(Lq, dg::attn::BQ);
+  p.n_pairs = attn_pairs(Hq, Hkv, Lq);
+  p.n_splits = S;
+  p.causal = mask == DG_MASK_CAUSAL ? 1 : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.cache_len = cache_len;
+  p.out = (__nv_bfloat16*)out;
+  p.ldo = ldo;
+  p.lse = lse;
+  p.part_o = nullptr;
+  p.part_lse = nullptr;
+  p.q_scale = q_scale;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  if (S > 1) {
+    const size_t rows = (size_t)S * B * Hq * Lq;
+    p.part_o = (__nv_bfloat16*)ws;
+    p.part_lse = (float*)((char*)ws + align_up(rows * hd * 2, 256));
+  }
+  using CF = dg::attn::Cfg<128, true>;
+  if (!attn_f8_attr_done()) {
+    DG_CUDA(cudaFuncSetAttribute(dg::attn::attn_kernel<128, true>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, CF::SMEM_BYTES));
+    attn_f8_attr_done() = true;
+  }
+  DG_CUDA(launch_ex(dg::attn::attn_kernel<128, true>, dim3(B * Hkv * p.n_pairs, S),
+                    dim3(dg::attn::THREADS), CF::SMEM_BYTES, s, 1, tq, tkn, tvn, tkc, tvc, p));
+  count_launch();
+  DG_CUDA(cudaGetLastError());
+  if (S > 1) {
+    const int rows = B * Hq * Lq;
+    const int threads = dg::attn::COMBINE_THREADS;
+    DG_CUDA(launch_ex(dg::attn::attn_combine_kernel<128>, dim3(cdiv(rows * 32, threads)),
+                      dim3(threads), 0, s, 1, (const __nv_bfloat16*)p.part_o,
+                      (const float*)p.part_lse, S, B, Hq, Lq, (__nv_bfloat16*)out, ldo, lse));
     count_launch();
     DG_CUDA(cudaGetLastError());
   }
@@ -1160,6 +1223,35 @@ int dg_canvas_attn(const void* q, int ldq, const void* k_new, const void* v_new,
   return launch_attn(q, ldq, k_new, v_new, ldkv, k_cache, v_cache, cache_len, max_prefix, lmax,
                      out, ldo, lse, B, Hq, Hkv, Lq, hd, scale, mask_mode, workspace,
                      (cudaStream_t)stream);
+}
+
+int dg_canvas_attn_e4m3(const uint8_t* q, int ldq, const float* q_scale, const uint8_t* k_new,
+                        int ldkv, const uint8_t* vt_new, int ldvt, const uint8_t* k_cache,
+                        const uint8_t* vt_cache, const float* k_scale, const float* v_scale,
+                        const int32_t* cache_len, int max_prefix, int lmax, void* out, int ldo,
+                        float* lse, int B, int Hq, int Hkv, int Lq, int hd, float scale,
+                        int mask_mode, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!q || !q_scale || !k_new || !vt_new || !k_cache || !vt_cache || !k_scale || !v_scale ||
+      !cache_len || !out)
+    return fail(DG_ERR_INVALID_ARG, "dg_canvas_attn_e4m3: null pointer");
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Lq <= 0 || Hq % Hkv || max_prefix < 0 || lmax < 1 ||
+      max_prefix > lmax || (mask_mode != DG_MASK_BIDIR && mask_mode != DG_MASK_CAUSAL))
+    return fail(DG_ERR_INVALID_ARG, "dg_canvas_attn_e4m3: bad sizes or mask");
+  if (hd != 128)
+    return fail(DG_ERR_UNSUPPORTED_SHAPE, "dg_canvas_attn_e4m3: head_dim %d is not 128", hd);
+  if (ldq % 16 || ldkv % 16 || ldvt % 16 || lmax % 16 || ldo % 8 || ldq < Hq * hd ||
+      ldkv < Hkv * hd || ldvt < Lq || ldo < Hq * hd)
+    return fail(DG_ERR_ALIGNMENT, "dg_canvas_attn_e4m3: leading dimensions");
+  if (!aligned16(q) || !aligned16(k_new) || !aligned16(vt_new) || !aligned16(k_cache) ||
+      !aligned16(vt_cache) || !aligned16(out))
+    return fail(DG_ERR_ALIGNMENT, "dg_canvas_attn_e4m3: pointers must be 16-byte aligned");
+  const size_t need = attn_ws_bytes(B, Hq, Hkv, Lq, hd, max_prefix);
+  if (need > 0 && (!workspace || workspace_bytes < need || !aligned16(workspace)))
+    return fail(DG_ERR_WORKSPACE_TOO_SMALL, "dg_canvas_attn_e4m3: workspace needs %zu bytes",
+                need);
+  return launch_attn_e4m3(q, ldq, q_scale, k_new, ldkv, vt_new, ldvt, k_cache, vt_cache, k_scale,
+                          v_scale, cache_len, max_prefix, lmax, out, ldo, lse, B, Hq, Hkv, Lq,
+                          scale, mask_mode, workspace, (cudaStream_t)stream);
 }
 
 int dg_unembed(const void* h, const void* w_u, float* logits, int M, int d, int V,

@@ -25,7 +25,16 @@
 // Warps: 0 = TMA producer, 1 = TMEM owner + MMA issuer, 2..5 = softmax of
 // tile A, 6..9 = softmax of tile B (one query row per thread; warp w owns
 // TMEM lanes 32*(w%4)..+31).
+//
+// The e4m3 variant (F8, hd = 128) runs both products as kind::f8f6f4 MMAs:
+// Q, K and V^T tiles are 8-bit codes, the scores are dequantised by the row's
+// query scale and the K scale inside the softmax's exponent, P is written to
+// TMEM as e4m3 (four per column), and the V scale joins 1/l.  The FP8 serving
+// figure this follows: aiexpert.news, "Google's DiffusionGemma Atinge 1.000
+// Tokens por Segundo", throughput paragraph (FP8 on one H200).
 #pragma once
+
+#include <cuda_fp8.h>
 
 #include <type_traits>
 
@@ -48,16 +57,36 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
-template <int HD>
+// F8: e4m3 operands (hd = 128).  Q, K and the probabilities are K-major as in
+// the bf16 kernel; V is stored transposed (keys contiguous), so that V^T tiles
+// are K-major B operands too.  Every MMA consumes 32 bytes of K either way.
+template <int HD, bool F8 = false>
 struct Cfg {
-  static constexpr int HALVES = HD / 64;
-  static constexpr int Q_BYTES = BQ * HD * 2;
-  static constexpr int T_BYTES = BKV * HD * 2;  // one K or V tile
-  static constexpr int STAGES = HD == 128 ? 2 : 3;
+  static constexpr int EB = F8 ? 1 : 2;              // bytes per element
+  static constexpr int ATOM = 128 / EB;              // elements per 128-byte swizzle row
+  static constexpr int HALVES = HD / ATOM;           // swizzle atoms across a row of hd
+  static constexpr int Q_BYTES = BQ * HD * EB;
+  static constexpr int T_BYTES = BKV * HD * EB;      // one K or V tile
+  static constexpr int STAGES = F8 ? 4 : (HD == 128 ? 2 : 3);
   static constexpr int SMEM_BYTES = 1024 + 2 * Q_BYTES + STAGES * 2 * T_BYTES + 256;
-  static constexpr uint32_t IDESC_QK = idesc_bf16_f32(BQ, BKV, false, false);
-  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(BQ, HD, false, true);
+  static constexpr int QK_MMAS = HD * EB / 32;
+  static constexpr int PV_MMAS = BKV * EB / 32;
+  static constexpr uint32_t IDESC_QK =
+      F8 ? idesc_e4m3_f32(BQ, BKV) : idesc_bf16_f32(BQ, BKV, false, false);
+  static constexpr uint32_t IDESC_PV =
+      F8 ? idesc_e4m3_f32(BQ, HD) : idesc_bf16_f32(BQ, HD, false, true);
+  // the epilogue stages both tiles' fp32 O in the K/V ring
+  static_assert(STAGES * 2 * T_BYTES >= 2 * BQ * HD * 4, "O staging does not fit the ring");
+  static_assert(!F8 || HD == 128, "e4m3 attention needs hd = 128");
 };
+
+// Four probabilities as e4m3 codes, the first in the lowest byte (the K order
+// of a TMEM A operand of an 8-bit MMA).
+__device__ __forceinline__ uint32_t pack_e4m3x4(float a, float b, float c, float d) {
+  const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
+  const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(c, d), __NV_SATFINITE, __NV_E4M3);
+  return lo | (hi << 16);
+}
 
 struct Params {
   int B, Hq, Hkv, Lq, lmax, group;
@@ -71,6 +100,10 @@ struct Params {
   float* lse;                // [B, Hq, Lq] natural log, or null
   __nv_bfloat16* part_o;     // [S, B, Hq, Lq, hd] bf16 (n_splits > 1)
   float* part_lse;           // [S, B, Hq, Lq]
+  // e4m3 operands: per-token query scales [B * Lq], K and V scales (scalars)
+  const float* q_scale;
+  const float* k_scale;
+  const float* v_scale;
 };
 
 
@@ -81,13 +114,13 @@ struct Params {
 // [PV_B(j), S_B(j+1)] so that one softmax warpgroup works while the other
 // tile's MMAs run.  S_X(j+1) is issued after PV_X(j), so once S_X(j+1) is
 // complete, O_X is stable and may be rescaled in TMEM.
-template <int HD>
+template <int HD, bool F8 = false>
 __global__ void __launch_bounds__(THREADS, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kn,
                 const __grid_constant__ CUtensorMap tm_vn,
                 const __grid_constant__ CUtensorMap tm_kc,
                 const __grid_constant__ CUtensorMap tm_vc, Params p) {
-  using CF = Cfg<HD>;
+  using CF = Cfg<HD, F8>;
   constexpr int ST = CF::STAGES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -209,26 +242,33 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int t = t_beg + i;
         const CUtensorMap* mk;
         const CUtensorMap* mv;
-        int x0, y0;
+        int x0, y0, key0;
         if (t < nP) {
           mk = &tm_kc;
           mv = &tm_vc;
           x0 = 0;
           y0 = (b * p.Hkv + g) * p.lmax + t * BKV;
+          key0 = t * BKV;
         } else {
           mk = &tm_kn;
           mv = &tm_vn;
           x0 = g * HD;
           y0 = b * p.Lq + (t - nP) * BKV;
+          key0 = (t - nP) * BKV;
         }
         uint8_t* kd = sK + st * CF::T_BYTES;
         uint8_t* vd = sV + st * CF::T_BYTES;
         mbar_expect_tx(&k_full[st], CF::T_BYTES);
         for (int hf = 0; hf < CF::HALVES; ++hf)
-          tma_load_2d(kd + hf * (BKV * 128), mk, &k_full[st], x0 + hf * 64, y0);
+          tma_load_2d(kd + hf * (BKV * 128), mk, &k_full[st], x0 + hf * CF::ATOM, y0);
         mbar_expect_tx(&v_full[st], CF::T_BYTES);
-        for (int hf = 0; hf < CF::HALVES; ++hf)
-          tma_load_2d(vd + hf * (BKV * 128), mv, &v_full[st], x0 + hf * 64, y0);
+        if constexpr (F8) {
+          // V^T tile: rows d of kv head (b, g), 128 keys from key0
+          tma_load_2d(vd, mv, &v_full[st], key0, (b * p.Hkv + g) * HD);
+        } else {
+          for (int hf = 0; hf < CF::HALVES; ++hf)
+            tma_load_2d(vd + hf * (BKV * 128), mv, &v_full[st], x0 + hf * CF::ATOM, y0);
+        }
       };
       // the first stages' cached-prefix tiles need no wait on the predecessor
       int issued = 0;
@@ -238,7 +278,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int X = 0; X < (vB ? 2 : 1); ++X)
         for (int hf = 0; hf < CF::HALVES; ++hf)
           tma_load_2d(sQ + X * CF::Q_BYTES + hf * (BQ * 128), &tm_q, q_full,
-                      hX[X] * HD + hf * 64, b * p.Lq + i0X[X]);
+                      hX[X] * HD + hf * CF::ATOM, b * p.Lq + i0X[X]);
       for (int i = issued; i < n; ++i) {
         const int st = i % ST;
         if (i >= ST && !mbar_wait(&kv_empty[st], ((i / ST) - 1) & 1, abort_flag, 0x311)) break;
@@ -262,10 +302,14 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t k_base = smem_u32(sK + (i % ST) * CF::T_BYTES);
         const uint32_t qb = q_base + X * CF::Q_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
+        for (int kk = 0; kk < CF::QK_MMAS; ++kk) {
           const uint32_t off = (kk >> 2) * (BQ * 128) + (kk & 3) * 32;
-          umma_ss(tmem + X * 128, sdesc_sw128(qb + off, 16, 1024),
-                  sdesc_sw128(k_base + off, 16, 1024), CF::IDESC_QK, kk > 0 ? 1u : 0u);
+          if constexpr (F8)
+            umma_ss_f8(tmem + X * 128, sdesc_sw128(qb + off, 16, 1024),
+                       sdesc_sw128(k_base + off, 16, 1024), CF::IDESC_QK, kk > 0 ? 1u : 0u);
+          else
+            umma_ss(tmem + X * 128, sdesc_sw128(qb + off, 16, 1024),
+                    sdesc_sw128(k_base + off, 16, 1024), CF::IDESC_QK, kk > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[X]);
       };
@@ -274,10 +318,17 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         const uint32_t v_base = smem_u32(sV + (j % ST) * CF::T_BYTES);
 #pragma unroll
-        for (int kk = 0; kk < BKV / 16; ++kk)
-          umma_ts(tmem + 256 + X * 128, tmem + X * 128 + kk * 8,
-                  sdesc_sw128(v_base + kk * 16 * 128, BKV * 128, 1024), CF::IDESC_PV,
-                  (j > 0 || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < CF::PV_MMAS; ++kk) {
+          // A = P (TMEM, 8 columns per MMA); B = V (MN-major bf16) or V^T (K-major e4m3)
+          if constexpr (F8)
+            umma_ts_f8(tmem + 256 + X * 128, tmem + X * 128 + kk * 8,
+                       sdesc_sw128(v_base + kk * 32, 16, 1024), CF::IDESC_PV,
+                       (j > 0 || kk > 0) ? 1u : 0u);
+          else
+            umma_ts(tmem + 256 + X * 128, tmem + X * 128 + kk * 8,
+                    sdesc_sw128(v_base + kk * 16 * 128, BKV * 128, 1024), CF::IDESC_PV,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+        }
         return true;
       };
       if (ok) ok = mbar_wait(&k_full[0], 0, abort_flag, 0x322);
@@ -318,6 +369,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     float m = -INFINITY;  // running max in scaled log2 units
     float l = 0.f;
     bool ok = vX[X];
+    // score -> log2 units: scale log2(e), times the dequantisation scales of
+    // the row's query and of K on e4m3 operands (all positive)
+    float sc = p.scale_log2;
+    if constexpr (F8)
+      sc *= (qrow < p.Lq ? p.q_scale[static_cast<size_t>(b) * p.Lq + qrow] : 1.f) * *p.k_scale;
     for (int j = 0; j < n && ok; ++j) {
       if (!__all_sync(0xffffffffu, mbar_wait(&s_full[X], j & 1, abort_flag, 0x331))) {
         ok = false;
@@ -358,7 +414,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           mx3 = fmaxf(mx3, __uint_as_float(sb[c + 1]));
         }
       }
-      const float tmax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2;
+      const float tmax = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sc;
       // Raise the running max only when it grows by more than 2^8 (the final
       // 1/l keeps this exact).  Decided per warp: TMEM accesses are
       // warp-collective.  PV_X(j-1) is complete because S_X(j) is.
@@ -382,8 +438,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       const float neg_m = (m == -INFINITY) ? 0.f : -m;
       float rs0 = 0.f, rs1 = 0.f, rs2 = 0.f, rs3 = 0.f;
-      // pass 2: re-read S in halves, exponentiate, pack P (bf16 pairs) over
-      // the consumed columns
+      // pass 2: re-read S in halves, exponentiate, pack P (bf16 pairs, or
+      // e4m3 quadruples) over the consumed columns
 #pragma unroll
       for (int h2 = 0; h2 < 2; ++h2) {
         uint32_t sa[64];
@@ -399,24 +455,43 @@ __global__ void __launch_bounds__(THREADS, 1)
           for (int c = 0; c < 64; ++c)
             if (h2 * 64 + c > lim) sa[c] = __float_as_uint(-INFINITY);
         }
-#pragma unroll
-        for (int q2 = 0; q2 < 2; ++q2) {
+        if constexpr (F8) {
+          // 64 keys -> 16 columns; the normaliser sums the unrounded values
           uint32_t pk[16];
 #pragma unroll
-          for (int c = 0; c < 16; c += 2) {
-            const int k0 = q2 * 32 + 2 * c;
-            const float p0 = fast_exp2(fmaf(__uint_as_float(sa[k0]), p.scale_log2, neg_m));
-            const float p1 = fast_exp2(fmaf(__uint_as_float(sa[k0 + 1]), p.scale_log2, neg_m));
-            const float p2 = fast_exp2(fmaf(__uint_as_float(sa[k0 + 2]), p.scale_log2, neg_m));
-            const float p3 = fast_exp2(fmaf(__uint_as_float(sa[k0 + 3]), p.scale_log2, neg_m));
+          for (int c = 0; c < 16; ++c) {
+            const int k0 = 4 * c;
+            const float p0 = fast_exp2(fmaf(__uint_as_float(sa[k0]), sc, neg_m));
+            const float p1 = fast_exp2(fmaf(__uint_as_float(sa[k0 + 1]), sc, neg_m));
+            const float p2 = fast_exp2(fmaf(__uint_as_float(sa[k0 + 2]), sc, neg_m));
+            const float p3 = fast_exp2(fmaf(__uint_as_float(sa[k0 + 3]), sc, neg_m));
             rs0 += p0;
             rs1 += p1;
             rs2 += p2;
             rs3 += p3;
-            pk[c] = pack_bf16x2(p0, p1);
-            pk[c + 1] = pack_bf16x2(p2, p3);
+            pk[c] = pack_e4m3x4(p0, p1, p2, p3);
           }
-          tmem_st16(tS + h2 * 32 + q2 * 16, pk);
+          tmem_st16(tS + h2 * 16, pk);
+        } else {
+#pragma unroll
+          for (int q2 = 0; q2 < 2; ++q2) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int c = 0; c < 16; c += 2) {
+              const int k0 = q2 * 32 + 2 * c;
+              const float p0 = fast_exp2(fmaf(__uint_as_float(sa[k0]), sc, neg_m));
+              const float p1 = fast_exp2(fmaf(__uint_as_float(sa[k0 + 1]), sc, neg_m));
+              const float p2 = fast_exp2(fmaf(__uint_as_float(sa[k0 + 2]), sc, neg_m));
+              const float p3 = fast_exp2(fmaf(__uint_as_float(sa[k0 + 3]), sc, neg_m));
+              rs0 += p0;
+              rs1 += p1;
+              rs2 += p2;
+              rs3 += p3;
+              pk[c] = pack_bf16x2(p0, p1);
+              pk[c + 1] = pack_bf16x2(p2, p3);
+            }
+            tmem_st16(tS + h2 * 32 + q2 * 16, pk);
+          }
         }
       }
       l += (rs0 + rs1) + (rs2 + rs3);
@@ -432,7 +507,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     // rows: coalesced stores instead of one 16-byte piece per row per lane.
     float* stage = reinterpret_cast<float*>(sK) + X * (BQ * HD);
     const int h = hX[X];
-    const float inv_l = (l > 0.f) ? 1.f / l : 0.f;
+    float vs = 1.f;
+    if constexpr (F8) vs = *p.v_scale;
+    const float inv_l = (l > 0.f) ? vs / l : 0.f;
     const float lse_nat = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
     if (fin) {
       tc_fence_after();

@@ -233,6 +233,8 @@ int dg_check_device_errors(void* stream, uint32_t* code_out);
  *   lse    fp32 [B, Hq, Lq] natural-log sum of exp of the scaled scores (may be NULL)
  *   cache_len: device [B]; every value must be <= max_prefix (host bound used
  *   to plan the split over keys).
+ * Cached rows from cache_len[b] up to the next multiple of 128 are read and
+ * weighted by zero: they must hold finite values (a zeroed cache does).
  * Requires hd in {64,128}, Hq % Hkv == 0, Lq >= 1, lmax >= max_prefix,
  * ldq/ldkv/ldo multiples of 8.  Workspace: dg_canvas_attn_workspace_bytes().
  */
@@ -242,6 +244,41 @@ int dg_canvas_attn(const void* q, int ldq, const void* k_new, const void* v_new,
                    int B, int Hq, int Hkv, int Lq, int hd, float scale, int mask_mode,
                    void* workspace, size_t workspace_bytes, void* stream);
 size_t dg_canvas_attn_workspace_bytes(int B, int Hq, int Hkv, int Lq, int hd, int max_prefix);
+
+/*
+ * dg_canvas_attn_e4m3 - dg_canvas_attn on e4m3 operands (the FP8 attention of
+ * FP8 serving; aiexpert.news, "Google's DiffusionGemma Atinge 1.000 Tokens por
+ * Segundo", throughput paragraph, quotes FP8 on one H200 without a recipe).
+ * This library's recipe, with the codes of dg_quantize_e4m3:
+ *   s[i, j] = scale * q_scale[b*Lq+i] * k_scale * sum_d dec(q)[d] dec(key_j)[d]
+ *   p[i, j] = exp(s[i, j] - m_i), m_i a running maximum of row i that lags the
+ *             row's by at most a factor 2^8 (p <= 256)
+ *   out[b,i,h,:] = v_scale * sum_j e4m3(p[i, j]) dec(value_j) / sum_j p[i, j]
+ * i.e. both products are 8-bit MMAs with fp32 accumulation, the probabilities
+ * enter the value product as e4m3 values and the normaliser unrounded.  Keys,
+ * mask, GQA mapping, split plan and lse are those of dg_canvas_attn.
+ * Layouts (one byte per e4m3 code):
+ *   q        [B, Lq, ldq]        head h at columns h*128; q_scale device fp32
+ *                                [B*Lq], one per token (dg_quantize_e4m3 per row)
+ *   k_new    [B, Lq, ldkv]       kv head g at columns g*128
+ *   vt_new   [B, Hkv, 128, ldvt] V of the new rows transposed: row (b, g, d)
+ *                                holds d of keys 0..Lq-1
+ *   k_cache  [B, Hkv, lmax, 128]
+ *   vt_cache [B, Hkv, 128, lmax] the cached V transposed the same way
+ *   k_scale, v_scale: device fp32 scalars, one for prefix and new rows together
+ *   out      bf16 [B, Lq, ldo]; lse fp32 [B, Hq, Lq] or NULL
+ * Every scale must be positive and finite.  Cached keys from cache_len[b] up to
+ * the next multiple of 128 are read and weighted by zero: they must hold finite
+ * codes (a zeroed cache does).  Requires hd == 128, ldq, ldkv, ldvt and lmax
+ * multiples of 16, ldvt >= Lq, ldo a multiple of 8.  Workspace:
+ * dg_canvas_attn_workspace_bytes(B, Hq, Hkv, Lq, 128, max_prefix).
+ */
+int dg_canvas_attn_e4m3(const uint8_t* q, int ldq, const float* q_scale, const uint8_t* k_new,
+                        int ldkv, const uint8_t* vt_new, int ldvt, const uint8_t* k_cache,
+                        const uint8_t* vt_cache, const float* k_scale, const float* v_scale,
+                        const int32_t* cache_len, int max_prefix, int lmax, void* out, int ldo,
+                        float* lse, int B, int Hq, int Hkv, int Lq, int hd, float scale,
+                        int mask_mode, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * dg_unembed - vocabulary logits of the normalised final hidden states (the
