@@ -647,11 +647,26 @@ int launch_attn_e4m3(const uint8_t* q, int ldq, const float* q_scale, const uint
 // ---------------------------------------------------------------------------
 // Sampler
 // ---------------------------------------------------------------------------
-int sample_chunking(int V, int* chunk) {
-  // chunks of >= 65536 elements (>= 256 per thread: the CTA's closing
-  // reduction is then a small share of its work), at most 64 per row, in
-  // multiples of 4 elements
-  int nchunk = std::max(1, std::min(64, V / 65536));
+// Row pass chunks: >= 65536 elements (>= 256 per thread: the CTA's closing
+// reduction is then a small share of its work), at most 64 per row, in
+// multiples of 4 elements.  When the rows are few (fewer than 16 waves of
+// resident CTAs), up to twice as many chunks are taken if that fills the last
+// wave better.  The plan depends on the shape only.
+int sample_chunking(int rows, int V, int* chunk) {
+  const int n0 = std::max(1, std::min(64, V / 65536));
+  const long slots = (long)kNumSMs * dg::RP_CTAS_PER_SM;
+  int nchunk = n0;
+  if ((long)rows * n0 < 16 * slots) {
+    double best = 0.0;
+    for (int n = n0; n <= std::min(64, 2 * n0); ++n) {
+      const long ctas = (long)rows * n;
+      const double fill = (double)ctas / (double)(cdiv(ctas, slots) * slots);
+      if (fill > best + 1e-9) {
+        best = fill;
+        nchunk = n;
+      }
+    }
+  }
   int c = cdiv(V, nchunk);
   c = (c + 3) / 4 * 4;
   nchunk = cdiv(V, c);
@@ -661,7 +676,7 @@ int sample_chunking(int V, int* chunk) {
 
 size_t sample_ws_bytes(int B, int C, int V) {
   int chunk;
-  const int nchunk = sample_chunking(V, &chunk);
+  const int nchunk = sample_chunking(B * C, V, &chunk);
   return align_up((size_t)B * C * nchunk * sizeof(dg::RowPartial), 256);
 }
 
@@ -677,7 +692,7 @@ dg::SampleParams make_sample_params(const dg_sampler_cfg& cfg, uint32_t seed, in
                                     const int32_t* step_ptr, int step, int B, int C, int V) {
   dg::SampleParams p;
   p.B = B; p.C = C; p.V = V;
-  p.nchunk = sample_chunking(V, &p.chunk);
+  p.nchunk = sample_chunking(B * C, V, &p.chunk);
   p.seed = seed;
   p.block = block;
   p.step_ptr = step_ptr;
@@ -695,12 +710,19 @@ dg::SampleParams make_sample_params(const dg_sampler_cfg& cfg, uint32_t seed, in
   return p;
 }
 
+PerDeviceFlag rowpass_attr_done;
+
 int launch_sample(const float* logits, int32_t* tok, uint8_t* committed, int32_t* prev_argmax,
                   int32_t* seq_status, const dg::SampleParams& p, const dg_step_out* out,
                   void* ws, cudaStream_t s) {
   dg::RowPartial* part = (dg::RowPartial*)ws;
+  if (!rowpass_attr_done()) {
+    DG_CUDA(cudaFuncSetAttribute(dg::sample_rowpass_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, dg::RP_SMEM));
+    rowpass_attr_done() = true;
+  }
   DG_CUDA(launch_ex(dg::sample_rowpass_kernel, dim3(p.B * p.C * p.nchunk), dim3(dg::RP_THREADS),
-                    0, s, 1, logits, (const int32_t*)seq_status, p, part));
+                    dg::RP_SMEM, s, 1, logits, (const int32_t*)seq_status, p, part));
   count_launch();
   const int threads = (p.C + 31) / 32 * 32;
   dg::SampleParams pc = p;

@@ -19,6 +19,8 @@
 // z - ln(E).  Ties resolve to the lowest vocabulary index / position.
 #pragma once
 
+#include <type_traits>
+
 #include "dg_common.cuh"
 
 namespace dg {
@@ -272,15 +274,59 @@ __device__ __forceinline__ void merge_best(float& v, int& i, float v2, int i2) {
 }
 
 // Grid: B * C * nchunk CTAs of RP_THREADS threads.  Chunk length is a multiple
-// of 4.  Each thread runs a RowState over its interleaved groups of 4.
+// of 4.  The chunk streams through a ring of RP_STAGES shared-memory batches of
+// RP_THREADS * 16 entries, filled by bulk async copies (thread 0 keeps three
+// batches in flight while the CTA works on the fourth); thread t takes the
+// float4 groups at t*4 + u*RP_THREADS*4, u < 4, so each thread meets its
+// entries in ascending order.
+//
+// Every entry enters the softmax sums (one FFMA and one ex2 against the
+// warp's running maximum m).  Few can win the Gumbel race, and two exact
+// bounds on the exponential variate E = -ln(u) of an entry's draw word keep
+// the rest out of it:
+//   * E >= w = 1 - u (exact from the word's bits): with S the best race score
+//     known to the warp (log2 units, a real entry's), an entry whose
+//     2^(zl - m) < 2^(S - m - kTieSlack) w cannot beat that entry, so its
+//     variate and race step are skipped;
+//   * E >= E_min ~ 2^-24 for every word: a group of four whose largest zl lies
+//     more than kRaceSlack below S cannot win whatever its draws; when no lane
+//     of the warp holds such a group, its Philox block is skipped too.
+// S is shared across the CTA through an order-preserving integer max, read
+// without a barrier (a stale value is only a weaker bound), after batches
+// 0, 1, 3, 7, ... .  When every group of a batch needs its Philox block, the
+// four blocks run as one straight-line piece (four independent round chains).
+// The race keeps (pe, E) of the leader; its score is log2(pe) + m - log2(E).
 constexpr int RP_THREADS = 256;
-constexpr int RP_UNROLL = 4;
+constexpr int RP_CTAS_PER_SM = 3;   // guaranteed by the launch bounds; sets the chunking
+constexpr int RP_STAGES = 4;
+constexpr int RP_BATCH = RP_THREADS * 16;              // entries per batch (16 KB)
+constexpr int RP_SMEM = RP_STAGES * RP_BATCH * 4;       // dynamic shared memory
+constexpr float kRaceSlack = 24.5f;   // > -log2(E_min) = 24
+constexpr float kTieSlack = 1e-3f;    // far above the rounding of a score
 
-__global__ void __launch_bounds__(RP_THREADS) sample_rowpass_kernel(
+__device__ __forceinline__ int ordered_bits(float f) {
+  const int b = __float_as_int(f);
+  return b ^ ((b >> 31) & 0x7FFFFFFF);
+}
+__device__ __forceinline__ float ordered_float(int k) {
+  return __int_as_float(k ^ ((k >> 31) & 0x7FFFFFFF));
+}
+
+// u of the draw word r as in exp_variate (exact); E >= 1 - u.
+__device__ __forceinline__ float draw_uniform(uint32_t r) {
+  return __uint_as_float(0x3F800000u | (r >> 9)) - 0.999999940395355224609375f;
+}
+
+__global__ void __launch_bounds__(RP_THREADS, RP_CTAS_PER_SM) sample_rowpass_kernel(
     const float* __restrict__ logits, const int32_t* __restrict__ seq_status, SampleParams p,
     RowPartial* __restrict__ part) {
   griddep_wait();
   griddep_launch();
+  extern __shared__ __align__(128) uint8_t rp_smem[];
+  float* ring = reinterpret_cast<float*>(rp_smem);  // [RP_STAGES][RP_BATCH]
+  __shared__ uint64_t full_bar[RP_STAGES], empty_bar[RP_STAGES];
+  __shared__ int s_best;  // the CTA's best race score so far, ordered bits
+  __shared__ int s_abort;
   const int row = blockIdx.x / p.nchunk;
   const int ck = blockIdx.x - row * p.nchunk;
   const int b = row / p.C;
@@ -294,31 +340,184 @@ __global__ void __launch_bounds__(RP_THREADS) sample_rowpass_kernel(
   const int v1 = min(p.V, v0 + p.chunk);
   const uint32_t c1 = (static_cast<uint32_t>(pos) & 0xFFFFFFu) | (kTagGumbel << 24);
   const uint2 key = make_uint2(p.seed, static_cast<uint32_t>(b));
+  const int lane = threadIdx.x & 31;
+  const int nb = (v1 - v0 + RP_BATCH - 1) / RP_BATCH;
+  if (threadIdx.x == 0) {
+    s_best = ordered_bits(-INFINITY);
+    s_abort = 0;
+    for (int st = 0; st < RP_STAGES; ++st) {
+      mbar_init(&full_bar[st], 1);
+      mbar_init(&empty_bar[st], RP_THREADS / 32);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  int issued = 0;  // batches requested (thread 0)
+  auto issue = [&](int bt) {
+    const int st = bt % RP_STAGES;
+    const int bs = v0 + bt * RP_BATCH;
+    const uint32_t bytes = static_cast<uint32_t>(min(RP_BATCH, v1 - bs)) * 4u;
+    mbar_expect_tx(&full_bar[st], bytes);
+    bulk_load(ring + st * RP_BATCH, x + bs, bytes, &full_bar[st]);
+    issued = bt + 1;
+  };
+  if (threadIdx.x == 0)
+    for (int bt = 0; bt < min(RP_STAGES, nb); ++bt) issue(bt);
 
-  RowState st;
-  st.reset();
-  for (int base = v0 + threadIdx.x * 4; base < v1; base += RP_THREADS * 4 * RP_UNROLL) {
-    float l[4 * RP_UNROLL];
-    int vg[RP_UNROLL];
-    int n_valid = 0;
+  float m = -INFINITY, s = 0.f, q = 0.f;     // m is warp-uniform
+  float amax = -INFINITY;
+  int aidx = 0x7FFFFFFF;
+  float pb = 0.f, eb = 1.f;                  // race leader of this thread: pe, E
+  int bidx = 0x7FFFFFFF;
+  auto leader_score = [&]() {
+    return (bidx == 0x7FFFFFFF || pb == 0.f) ? -INFINITY : sfu_log2(pb) + m - sfu_log2(eb);
+  };
+  float S = -INFINITY;                       // best score known to the warp (log2 units)
+  float theta = 0.f;                         // 2^(S - m - kTieSlack)
+
+  // One batch; PAD: the batch runs past v1 (only the last one can), whose
+  // missing entries read as -inf.  There the exponent is clamped at -256
+  // (where ex2 is 0 already) so that a missing entry adds 0 to both sums.
+  auto batch = [&](int bt, int bstart, auto pad_tag) {
+    constexpr bool PAD = decltype(pad_tag)::value;
+    const int st = bt % RP_STAGES;
+    // thread 0 refills the stage read one batch ago, once every warp has read it
+    if (threadIdx.x == 0 && bt >= 1 && bt - 1 + RP_STAGES < nb) {
+      const int sp = (bt - 1) % RP_STAGES;
+      mbar_wait(&empty_bar[sp], ((bt - 1) / RP_STAGES) & 1, &s_abort, 0x611);
+      issue(bt - 1 + RP_STAGES);
+    }
+    mbar_wait(&full_bar[st], (bt / RP_STAGES) & 1, &s_abort, 0x612);
+    const float4* src = reinterpret_cast<const float4*>(ring + st * RP_BATCH);
+    float l[16];
+    int vg[4];
+    float gmax[4];
 #pragma unroll
-    for (int u = 0; u < RP_UNROLL; ++u) {
-      const int v = base + u * RP_THREADS * 4;
+    for (int u = 0; u < 4; ++u) {
+      const int v = bstart + u * RP_THREADS * 4 + threadIdx.x * 4;
       vg[u] = v;
-      const float4 l4 = (v < v1) ? __ldcs(reinterpret_cast<const float4*>(x + v))
-                                 : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      const float4 l4 = (!PAD || v < v1)
+                            ? src[u * RP_THREADS + threadIdx.x]
+                            : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
       l[4 * u] = l4.x;
       l[4 * u + 1] = l4.y;
       l[4 * u + 2] = l4.z;
       l[4 * u + 3] = l4.w;
-      n_valid += (v < v1) ? 1 : 0;
+      gmax[u] = fmaxf(fmaxf(l4.x, l4.y), fmaxf(l4.z, l4.w));
     }
-    st.update<RP_UNROLL, false>(l, vg, n_valid, -1, k2, c1, static_cast<uint32_t>(step),
-                                static_cast<uint32_t>(p.block), key);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[st]);
+    const float bm = fmaxf(fmaxf(gmax[0], gmax[1]), fmaxf(gmax[2], gmax[3]));
+    if (bm > amax) {
+      // new raw maximum in this batch: first index holding it (ascending order)
+      amax = bm;
+#pragma unroll
+      for (int u = 3; u >= 0; --u)
+#pragma unroll
+        for (int e = 3; e >= 0; --e)
+          if (l[4 * u + e] == bm) aidx = vg[u] + e;
+    }
+    float wm = bm;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, o));
+    const float wmz = wm * k2;
+    if (wmz > m) {
+      if (m != -INFINITY) {
+        const float d = m - wmz, f = sfu_exp2(d);
+        q = f * (q + d * s);
+        s *= f;
+        pb *= f;
+        theta *= f;
+      }
+      m = wmz;
+    }
+    const float neg_m = (PAD && m == -INFINITY) ? 0.f : -m;
+    float pe[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float t = fmaf(l[i], k2, neg_m);
+      if (PAD) t = fmaxf(t, -256.f);
+      pe[i] = sfu_exp2(t);
+      s += pe[i];
+      q = fmaf(pe[i], t, q);
+    }
+    const float thr = S - kRaceSlack;
+    bool cand[4];
+    unsigned need = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      cand[u] = (!PAD || vg[u] < v1) && gmax[u] * k2 >= thr;
+      if (__any_sync(0xffffffffu, cand[u])) need |= 1u << u;
+    }
+    if (need != 0) {
+      uint32_t rw[16];
+      auto draw = [&](int u) {
+        const uint4 r = philox4x32_10(
+            make_uint4(static_cast<uint32_t>(vg[u] >> 2), c1, static_cast<uint32_t>(step),
+                       static_cast<uint32_t>(p.block)), key);
+        rw[4 * u] = r.x;
+        rw[4 * u + 1] = r.y;
+        rw[4 * u + 2] = r.z;
+        rw[4 * u + 3] = r.w;
+      };
+      if (need == 0xFu) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) draw(u);
+      } else {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (need & (1u << u)) {
+            draw(u);
+          } else {
+            rw[4 * u] = rw[4 * u + 1] = rw[4 * u + 2] = rw[4 * u + 3] = 0u;
+          }
+        }
+      }
+      // pe < theta (1 - u) <= theta E: the entry cannot beat the best known one
+      bool pass[16];
+      bool any = false;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        pass[i] = cand[i >> 2] && !(pe[i] < fmaf(-theta, draw_uniform(rw[i]), theta));
+        any |= pass[i];
+      }
+      if (__any_sync(0xffffffffu, any)) {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (!pass[i]) continue;
+          const float ev = exp_variate(rw[i]);
+          if (pe[i] * eb > pb * ev) {
+            pb = pe[i];
+            eb = ev;
+            bidx = vg[i >> 2] + (i & 3);
+          }
+        }
+      }
+    }
+    if ((bt & (bt + 1)) == 0) {
+      // share the best score: this warp's, then the CTA's
+      float sc = leader_score();
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) sc = fmaxf(sc, __shfl_xor_sync(0xffffffffu, sc, o));
+      if (lane == 0 && sc > S) atomicMax(&s_best, ordered_bits(sc));
+      const float cta = ordered_float(*reinterpret_cast<volatile int*>(&s_best));
+      const float s_new = fmaxf(fmaxf(S, sc), __shfl_sync(0xffffffffu, cta, 0));
+      if (s_new > S) {
+        S = s_new;
+        theta = sfu_exp2(S - m - kTieSlack);
+      }
+    }
+  };
+  const int nfull = (v1 - v0) / (RP_THREADS * 16);
+  for (int bt = 0; bt < nfull; ++bt) batch(bt, v0 + bt * RP_THREADS * 16, std::false_type{});
+  if (v0 + nfull * RP_THREADS * 16 < v1)
+    batch(nfull, v0 + nfull * RP_THREADS * 16, std::true_type{});
+  if (threadIdx.x == 0 && s_abort) {
+    // a wait gave up: let every requested copy land before the CTA exits
+    for (int bt = max(0, issued - RP_STAGES); bt < issued; ++bt)
+      mbar_wait(&full_bar[bt % RP_STAGES], (bt / RP_STAGES) & 1, nullptr, 0x613);
   }
-  float m = st.m, s = st.s, q = st.q, amax = st.amax;
-  int aidx = st.aidx, bidx = st.bidx;
-  float best = st.best_score(k2);
+  float best = leader_score();
 
   // CTA reduction: warp shuffles, then across warps through shared memory.
 #pragma unroll
