@@ -46,6 +46,32 @@ __host__ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint2 k) {
   return c;
 }
 
+// The same generator with its ten round keys computed once by the caller
+// (ks[2r], ks[2r+1] = the key after r Weyl bumps).
+struct PhiloxKeys {
+  uint32_t k[20];
+  __device__ __forceinline__ explicit PhiloxKeys(uint2 key) {
+#pragma unroll
+    for (int r = 0; r < 10; ++r) {
+      k[2 * r] = key.x;
+      k[2 * r + 1] = key.y;
+      key.x += 0x9E3779B9u;
+      key.y += 0xBB67AE85u;
+    }
+  }
+};
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, const PhiloxKeys& ks) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * c.x;
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * c.z;
+    const uint32_t hi0 = static_cast<uint32_t>(p0 >> 32), lo0 = static_cast<uint32_t>(p0);
+    const uint32_t hi1 = static_cast<uint32_t>(p1 >> 32), lo1 = static_cast<uint32_t>(p1);
+    c = make_uint4(hi1 ^ c.y ^ ks.k[2 * r], lo1, hi0 ^ c.w ^ ks.k[2 * r + 1], lo0);
+  }
+  return c;
+}
+
 __device__ __forceinline__ uint32_t position_word(uint32_t seed, uint32_t b, uint32_t block,
                                                   uint32_t step, uint32_t pos, uint32_t tag) {
   return philox4x32_10(make_uint4(0u, (pos & 0xFFFFFFu) | (tag << 24), step, block),
@@ -312,9 +338,23 @@ __device__ __forceinline__ float ordered_float(int k) {
   return __int_as_float(k ^ ((k >> 31) & 0x7FFFFFFF));
 }
 
-// u of the draw word r as in exp_variate (exact); E >= 1 - u.
+// u of the draw word r as in exp_variate (exact); E >= 1 - u.  The bits
+// 0x3F800000 | (r >> 9) are formed as hi32(r * 2^23) + 0x3F800000 (the two
+// fields do not overlap), one multiply-add instead of a shift and an OR.
 __device__ __forceinline__ float draw_uniform(uint32_t r) {
-  return __uint_as_float(0x3F800000u | (r >> 9)) - 0.999999940395355224609375f;
+  return __uint_as_float(__umulhi(r, 1u << 23) + 0x3F800000u) - 0.999999940395355224609375f;
+}
+
+// any = any || (a >= b), one comparison with a predicate operand.
+__device__ __forceinline__ bool ge_or(float a, float b, bool any) {
+  uint32_t r;
+  asm("{\n\t.reg .pred pi, po;\n\t"
+      "setp.ne.u32 pi, %3, 0;\n\t"
+      "setp.ge.or.f32 po, %1, %2, pi;\n\t"
+      "selp.u32 %0, 1, 0, po;\n\t}"
+      : "=r"(r)
+      : "f"(a), "f"(b), "r"(static_cast<uint32_t>(any)));
+  return r != 0;
 }
 
 __global__ void __launch_bounds__(RP_THREADS, RP_CTAS_PER_SM) sample_rowpass_kernel(
@@ -339,7 +379,7 @@ __global__ void __launch_bounds__(RP_THREADS, RP_CTAS_PER_SM) sample_rowpass_ker
   const int v0 = ck * p.chunk;
   const int v1 = min(p.V, v0 + p.chunk);
   const uint32_t c1 = (static_cast<uint32_t>(pos) & 0xFFFFFFu) | (kTagGumbel << 24);
-  const uint2 key = make_uint2(p.seed, static_cast<uint32_t>(b));
+  const PhiloxKeys keys(make_uint2(p.seed, static_cast<uint32_t>(b)));
   const int lane = threadIdx.x & 31;
   const int nb = (v1 - v0 + RP_BATCH - 1) / RP_BATCH;
   if (threadIdx.x == 0) {
@@ -454,7 +494,7 @@ __global__ void __launch_bounds__(RP_THREADS, RP_CTAS_PER_SM) sample_rowpass_ker
       auto draw = [&](int u) {
         const uint4 r = philox4x32_10(
             make_uint4(static_cast<uint32_t>(vg[u] >> 2), c1, static_cast<uint32_t>(step),
-                       static_cast<uint32_t>(p.block)), key);
+                       static_cast<uint32_t>(p.block)), keys);
         rw[4 * u] = r.x;
         rw[4 * u + 1] = r.y;
         rw[4 * u + 2] = r.z;
@@ -474,17 +514,18 @@ __global__ void __launch_bounds__(RP_THREADS, RP_CTAS_PER_SM) sample_rowpass_ker
         }
       }
       // pe < theta (1 - u) <= theta E: the entry cannot beat the best known one
-      bool pass[16];
+      // (a group that is no candidate gets the bound +inf)
+      float bound[16];
       bool any = false;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        pass[i] = cand[i >> 2] && !(pe[i] < fmaf(-theta, draw_uniform(rw[i]), theta));
-        any |= pass[i];
+        bound[i] = cand[i >> 2] ? fmaf(-theta, draw_uniform(rw[i]), theta) : INFINITY;
+        any = ge_or(pe[i], bound[i], any);
       }
       if (__any_sync(0xffffffffu, any)) {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
-          if (!pass[i]) continue;
+          if (!(pe[i] >= bound[i])) continue;
           const float ev = exp_variate(rw[i]);
           if (pe[i] * eb > pb * ev) {
             pb = pe[i];
