@@ -301,8 +301,8 @@ __device__ __forceinline__ void merge_best(float& v, int& i, float v2, int i2) {
 
 // Grid: B * C * nchunk CTAs of RP_THREADS threads.  Chunk length is a multiple
 // of 4.  The chunk streams through a ring of RP_STAGES shared-memory batches of
-// RP_THREADS * 16 entries, filled by bulk async copies (thread 0 keeps three
-// batches in flight while the CTA works on the fourth); thread t takes the
+// RP_THREADS * 16 entries, filled by bulk async copies (thread 0 keeps the
+// next RP_STAGES - 1 batches in flight while the CTA works on one); thread t takes the
 // float4 groups at t*4 + u*RP_THREADS*4, u < 4, so each thread meets its
 // entries in ascending order.
 //
@@ -323,8 +323,8 @@ __device__ __forceinline__ void merge_best(float& v, int& i, float v2, int i2) {
 // four blocks run as one straight-line piece (four independent round chains).
 // The race keeps (pe, E) of the leader; its score is log2(pe) + m - log2(E).
 constexpr int RP_THREADS = 256;
-constexpr int RP_CTAS_PER_SM = 3;   // guaranteed by the launch bounds; sets the chunking
-constexpr int RP_STAGES = 4;
+constexpr int RP_CTAS_PER_SM = 4;   // guaranteed by the launch bounds; sets the chunking
+constexpr int RP_STAGES = 3;
 constexpr int RP_BATCH = RP_THREADS * 16;              // entries per batch (16 KB)
 constexpr int RP_SMEM = RP_STAGES * RP_BATCH * 4;       // dynamic shared memory
 constexpr float kRaceSlack = 24.5f;   // > -log2(E_min) = 24
@@ -449,13 +449,19 @@ __global__ void __launch_bounds__(RP_THREADS, RP_CTAS_PER_SM) sample_rowpass_ker
     if (lane == 0) mbar_arrive(&empty_bar[st]);
     const float bm = fmaxf(fmaxf(gmax[0], gmax[1]), fmaxf(gmax[2], gmax[3]));
     if (bm > amax) {
-      // new raw maximum in this batch: first index holding it (ascending order)
+      // new raw maximum in this batch: first index holding it (ascending
+      // order): the first group holding it, then the first entry of that group
       amax = bm;
+      float4 g4 = make_float4(l[12], l[13], l[14], l[15]);
+      int gv = vg[3];
 #pragma unroll
-      for (int u = 3; u >= 0; --u)
-#pragma unroll
-        for (int e = 3; e >= 0; --e)
-          if (l[4 * u + e] == bm) aidx = vg[u] + e;
+      for (int u = 2; u >= 0; --u) {
+        if (gmax[u] == bm) {
+          g4 = make_float4(l[4 * u], l[4 * u + 1], l[4 * u + 2], l[4 * u + 3]);
+          gv = vg[u];
+        }
+      }
+      aidx = gv + (g4.x == bm ? 0 : g4.y == bm ? 1 : g4.z == bm ? 2 : 3);
     }
     float wm = bm;
 #pragma unroll
@@ -513,13 +519,15 @@ __global__ void __launch_bounds__(RP_THREADS, RP_CTAS_PER_SM) sample_rowpass_ker
           }
         }
       }
-      // pe < theta (1 - u) <= theta E: the entry cannot beat the best known one
-      // (a group that is no candidate gets the bound +inf)
+      // pe < theta (1 - u) <= theta E: the entry cannot beat the best known one.
+      // The test is exact on its own, so it runs on every entry of the batch: a
+      // group whose block was skipped has words 0 (u = 2^-24, bound ~ theta),
+      // and its entries, more than 24.5 below S, lie far under that bound.
       float bound[16];
       bool any = false;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
-        bound[i] = cand[i >> 2] ? fmaf(-theta, draw_uniform(rw[i]), theta) : INFINITY;
+        bound[i] = fmaf(-theta, draw_uniform(rw[i]), theta);
         any = ge_or(pe[i], bound[i], any);
       }
       if (__any_sync(0xffffffffu, any)) {
