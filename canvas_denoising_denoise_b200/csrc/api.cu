@@ -647,20 +647,20 @@ int launch_attn_e4m3(const uint8_t* q, int ldq, const float* q_scale, const uint
 // ---------------------------------------------------------------------------
 // Sampler
 // ---------------------------------------------------------------------------
-// Row pass chunks: >= 65536 elements (>= 256 per thread: the CTA's closing
-// reduction is then a small share of its work), at most 64 per row, in
-// multiples of 4 elements.  When the rows are few (fewer than 16 waves of
-// resident CTAs), up to twice as many chunks are taken if that fills the last
-// wave better.  The plan depends on the shape only.
+// Row pass chunks: >= 131072 elements (>= 512 per thread: the CTA's closing
+// reduction and its first batches, raced before a best score is known, are
+// then a small share of its work), at most 64 per row, in multiples of 4
+// elements.  When the CTAs would be few (fewer than 16 per SM), up to twice as
+// many chunks are taken if that spreads them more evenly over the SMs.  The
+// plan depends on the shape only.
 int sample_chunking(int rows, int V, int* chunk) {
-  const int n0 = std::max(1, std::min(64, V / 65536));
-  const long slots = (long)kNumSMs * dg::RP_CTAS_PER_SM;
+  const int n0 = std::max(1, std::min(64, V / 131072));
   int nchunk = n0;
-  if ((long)rows * n0 < 16 * slots) {
+  if ((long)rows * n0 < 16L * kNumSMs) {
     double best = 0.0;
     for (int n = n0; n <= std::min(64, 2 * n0); ++n) {
       const long ctas = (long)rows * n;
-      const double fill = (double)ctas / (double)(cdiv(ctas, slots) * slots);
+      const double fill = (double)ctas / (double)(cdiv(ctas, (long)kNumSMs) * kNumSMs);
       if (fill > best + 1e-9) {
         best = fill;
         nchunk = n;

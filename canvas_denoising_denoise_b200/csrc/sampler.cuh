@@ -307,7 +307,7 @@ __device__ __forceinline__ void merge_best(float& v, int& i, float v2, int i2) {
 // entries in ascending order.
 //
 // Every entry enters the softmax sums (one FFMA and one ex2 against the
-// warp's running maximum m).  Few can win the Gumbel race, and two exact
+// thread's running maximum m).  Few can win the Gumbel race, and two exact
 // bounds on the exponential variate E = -ln(u) of an entry's draw word keep
 // the rest out of it:
 //   * E >= w = 1 - u (exact from the word's bits): with S the best race score
@@ -323,7 +323,7 @@ __device__ __forceinline__ void merge_best(float& v, int& i, float v2, int i2) {
 // four blocks run as one straight-line piece (four independent round chains).
 // The race keeps (pe, E) of the leader; its score is log2(pe) + m - log2(E).
 constexpr int RP_THREADS = 256;
-constexpr int RP_CTAS_PER_SM = 4;   // guaranteed by the launch bounds; sets the chunking
+constexpr int RP_CTAS_PER_SM = 4;   // resident CTAs per SM, guaranteed by the launch bounds
 constexpr int RP_STAGES = 3;
 constexpr int RP_BATCH = RP_THREADS * 16;              // entries per batch (16 KB)
 constexpr int RP_SMEM = RP_STAGES * RP_BATCH * 4;       // dynamic shared memory
@@ -404,7 +404,7 @@ __global__ void __launch_bounds__(RP_THREADS, RP_CTAS_PER_SM) sample_rowpass_ker
   if (threadIdx.x == 0)
     for (int bt = 0; bt < min(RP_STAGES, nb); ++bt) issue(bt);
 
-  float m = -INFINITY, s = 0.f, q = 0.f;     // m is warp-uniform
+  float m = -INFINITY, s = 0.f, q = 0.f;     // this thread's running max of zl and sums
   float amax = -INFINITY;
   int aidx = 0x7FFFFFFF;
   float pb = 0.f, eb = 1.f;                  // race leader of this thread: pe, E
@@ -413,7 +413,7 @@ __global__ void __launch_bounds__(RP_THREADS, RP_CTAS_PER_SM) sample_rowpass_ker
     return (bidx == 0x7FFFFFFF || pb == 0.f) ? -INFINITY : sfu_log2(pb) + m - sfu_log2(eb);
   };
   float S = -INFINITY;                       // best score known to the warp (log2 units)
-  float theta = 0.f;                         // 2^(S - m - kTieSlack)
+  float theta = 0.f;                         // 2^(S - m - kTieSlack), this thread's m
 
   // One batch; PAD: the batch runs past v1 (only the last one can), whose
   // missing entries read as -inf.  There the exponent is clamped at -256
@@ -463,19 +463,16 @@ __global__ void __launch_bounds__(RP_THREADS, RP_CTAS_PER_SM) sample_rowpass_ker
       }
       aidx = gv + (g4.x == bm ? 0 : g4.y == bm ? 1 : g4.z == bm ? 2 : 3);
     }
-    float wm = bm;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, o));
-    const float wmz = wm * k2;
-    if (wmz > m) {
+    const float bmz = bm * k2;
+    if (bmz > m) {
       if (m != -INFINITY) {
-        const float d = m - wmz, f = sfu_exp2(d);
+        const float d = m - bmz, f = sfu_exp2(d);
         q = f * (q + d * s);
         s *= f;
         pb *= f;
         theta *= f;
       }
-      m = wmz;
+      m = bmz;
     }
     const float neg_m = (PAD && m == -INFINITY) ? 0.f : -m;
     float pe[16];

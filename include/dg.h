@@ -413,15 +413,16 @@ int dg_unembed_sample_commit_e4m3(const uint8_t* h_q, const float* h_scale, cons
 
 /*
  * dg_sample_commit_noalloc - dg_sample_commit without a workspace argument.
- * The paper has no counterpart: this is a library convenience.  It serves
+ * No page describes it: this is a library convenience.  It serves
  * callers that cannot allocate device memory - a plugin whose host owns every
  * device allocation, or code enqueueing work during stream capture, where
  * cudaMalloc is not permitted.  Its scratch lives in a fixed 4 MiB static
  * device array that every GPU loading the library keeps until process exit;
  * nothing is allocated per call (no cudaMalloc, cudaFree or allocating library
  * routine).  Sizes whose scratch exceeds 4 MiB (dg_sample_commit_workspace_bytes
- * of B, C, V: 32 bytes per position and 65536-entry vocabulary chunk, so at
- * C = 256, V = 262144 up to B = 128) return DG_ERR_UNSUPPORTED_SHAPE.  The
+ * of B, C, V: 32 bytes per position and vocabulary chunk, the chunks 131072
+ * entries once there are 16 or more per SM, so at C = 256, V = 262144 up to
+ * B = 256) return DG_ERR_UNSUPPORTED_SHAPE.  The
  * first call on a device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current and keeps it for the life
  * of the process; make that first call before any stream capture.  A device

@@ -84,10 +84,11 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     lib = _lib.load()
     cfg = _lib.SamplerCfg()
     lib.dg_sampler_defaults(ctypes.byref(cfg))
-    # four 32-byte chunk partials per position at V = 262144: the fixed 4 MiB
-    # holds 128 canvases of 256 positions exactly
-    assert lib.dg_sample_commit_workspace_bytes(128, 256, 262144) == 4 << 20
-    B, C, V = 129, 256, 262144
+    # two 32-byte chunk partials per position at V = 262144 (131072-entry
+    # chunks with this many rows): the fixed 4 MiB holds 256 canvases of 256
+    # positions exactly
+    assert lib.dg_sample_commit_workspace_bytes(256, 256, 262144) == 4 << 20
+    B, C, V = 257, 256, 262144
     assert lib.dg_sample_commit_workspace_bytes(B, C, V) > (4 << 20)
     p = ctypes.c_void_p(256)
     rc = lib.dg_sample_commit_noalloc(p, p, p, p, p, ctypes.byref(cfg), 0, 0, 0, B, C, V, None,
