@@ -112,6 +112,13 @@ __device__ __forceinline__ float exp_variate(uint32_t r) {
   return w <= 0.0625f ? e_ser : e_log;
 }
 
+// u of the draw word r as in exp_variate (exact); E >= 1 - u.  The bits
+// 0x3F800000 | (r >> 9) are formed as hi32(r * 2^23) + 0x3F800000 (the two
+// fields do not overlap), one multiply-add instead of a shift and an OR.
+__device__ __forceinline__ float draw_uniform(uint32_t r) {
+  return __uint_as_float(__umulhi(r, 1u << 23) + 0x3F800000u) - 0.999999940395355224609375f;
+}
+
 __device__ __forceinline__ float step_temperature(int step, int max_steps, float t0, float t1) {
   if (max_steps <= 1) return t0;
   return t0 + (t1 - t0) * (static_cast<float>(step) / static_cast<float>(max_steps - 1));
@@ -216,12 +223,18 @@ struct RowState {
         const float pe = sfu_exp2(t);
         s += pe;
         q = fmaf(pe, t, q);
-        const float ev = exp_variate(rw[e]);
-        if (pe * eb > pb * ev) {
-          pb = pe;
-          eb = ev;
-          lb = lv;
-          bidx = vg[g] + e;
+        // E >= 1 - u: when pe eb <= pb (1 - u) the race step below cannot take
+        // the lead, so the variate is only computed for entries that might
+        // (the outcome is bit for bit that of the plain race)
+        const float lhs = pe * eb;
+        if (lhs > fmaf(-pb, draw_uniform(rw[e]), pb)) {
+          const float ev = exp_variate(rw[e]);
+          if (lhs > pb * ev) {
+            pb = pe;
+            eb = ev;
+            lb = lv;
+            bidx = vg[g] + e;
+          }
         }
         if (TRACK_CUR && vg[g] + e == cur) lcur = lv;
       }
@@ -338,12 +351,6 @@ __device__ __forceinline__ float ordered_float(int k) {
   return __int_as_float(k ^ ((k >> 31) & 0x7FFFFFFF));
 }
 
-// u of the draw word r as in exp_variate (exact); E >= 1 - u.  The bits
-// 0x3F800000 | (r >> 9) are formed as hi32(r * 2^23) + 0x3F800000 (the two
-// fields do not overlap), one multiply-add instead of a shift and an OR.
-__device__ __forceinline__ float draw_uniform(uint32_t r) {
-  return __uint_as_float(__umulhi(r, 1u << 23) + 0x3F800000u) - 0.999999940395355224609375f;
-}
 
 // any = any || (a >= b), one comparison with a predicate operand.
 __device__ __forceinline__ bool ge_or(float a, float b, bool any) {
