@@ -278,14 +278,6 @@ cudaError_t gemm_set_attrs() {
   return cudaSuccess;
 }
 
-bool gemm_plan_known(const GemmPlan& pl) {
-#define DG_X(S_, BN_, R_) \
-  if (pl.splits == S_ && pl.bn == BN_ && pl.ring_kb == R_) return true;
-  DG_GEMM_VARIANTS(DG_X)
-#undef DG_X
-  return false;
-}
-
 template <bool F8>
 cudaError_t launch_gemm_plan(const GemmPlan& pl, dim3 grid, cudaStream_t s, const CUtensorMap& tw,
                              const CUtensorMap& tx, const dg::gemm::Params& p) {

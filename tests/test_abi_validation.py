@@ -112,6 +112,25 @@ def test_canvas_attn_rejects_bad_arguments(lib):
     assert call(q=NULL) == INVALID
 
 
+def test_canvas_attn_e4m3_rejects_bad_arguments(lib):
+    def call(hd=128, Hq=16, Hkv=8, mask=0, ldq=16 * 128, ldkv=8 * 128, ldvt=256, lmax=4352,
+             q=P, qs=P, maxp=4096, ws_bytes=1 << 30):
+        return lib.dg_canvas_attn_e4m3(q, ldq, qs, P, ldkv, P, ldvt, P, P, P, P, P, maxp, lmax,
+                                       P, 16 * 128, None, 1, Hq, Hkv, 256, hd, 0.088, mask, P,
+                                       ws_bytes, None)
+    assert call(hd=64) == SHAPE                   # e4m3 attention is hd = 128 only
+    assert call(Hq=12, Hkv=8) == INVALID          # Hq % Hkv
+    assert call(mask=5) == INVALID
+    assert call(maxp=5000) == INVALID             # prefix beyond the cache
+    assert call(ldvt=200) == ALIGN                # ldvt below Lq
+    assert call(ldvt=264) == ALIGN                # ldvt not a multiple of 16
+    assert call(lmax=4360) == ALIGN               # lmax not a multiple of 16
+    assert call(ldq=16 * 128 - 16) == ALIGN       # leading dimension below Hq * 128
+    assert call(q=MIS) == ALIGN
+    assert call(qs=NULL) == INVALID               # the per-token scales are required
+    assert call(ws_bytes=16) == WS                # the split plan needs its partials
+
+
 def test_workspace_queries(lib, L):
     assert lib.dg_sample_commit_workspace_bytes(0, 256, 512) == 0
     assert lib.dg_unembed_sample_commit_workspace_bytes(1, 256, 1000) == 0         # V % 256
